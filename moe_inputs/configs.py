@@ -1,0 +1,145 @@
+"""The five named workloads of the MoE-layer forward and their input recipes.
+
+Shapes and value distributions follow the workloads this library is measured on:
+
+* ``tiny_shazeer_f32``   - Shazeer-style MoE, fp32, T=128, d=64, n=8, k=2, experts 64->128 ReLU->64,
+  router weights scaled x4 so logits are well separated (seed 0).
+* ``shazeer_bf16``       - Shazeer-style MoE, bf16, T=8192, d=512, n=256, k=4, experts
+  512->1024 ReLU->512, inputs and weights ~ N(0, 1/fan_in) (seed 1).
+* ``muse_decode``        - Muse-shape latent MoE, T=64, hidden 8192, latent 4096, 256 SwiGLU
+  experts (4096->4096->4096), top-8, per-expert input-scaled RMSNorm, residual gate (seed 2).
+* ``muse_prefill``       - the same layer at T=16384 (seed 3).
+* ``muse_imbalanced``    - the same layer at T=32768 with a Zipf(s=1.2) per-expert router bias
+  scaled so the hottest expert receives about 20x the mean load (seed 4).
+
+The Muse layer is the latent MoE block described in "Muse Spark Open: Norm-Preserving Gates Are
+Not a Norm Guarantee" (flozi.net, sections "Latent experts: normalization happens before the
+weighted sum" and "Residual gates"); the Shazeer layer is the one of "816 billion parameters, and
+only 42 billion show up for each token" (bobbyburns.tech, sections "The math" and "The gate").
+
+This module holds no layer arithmetic: only sizes, seeds and distributions.
+"""
+from __future__ import annotations
+
+import dataclasses
+import math
+
+# Stream identifiers: one independent counter stream per tensor (any distinct integers work).
+STREAM_X = 1
+STREAM_W_ROUTER = 2
+STREAM_P_DOWN = 3
+STREAM_P_UP = 4
+STREAM_W_GU = 5
+STREAM_W_DOWN = 6
+STREAM_GAMMA_PRE = 7
+STREAM_GAMMA_EXPERT = 8
+STREAM_RESID_G = 9
+STREAM_RESID_H = 10
+STREAM_ZIPF = 11
+STREAM_SUBSAMPLE = 12
+
+ACT_RELU = 0
+ACT_SWIGLU = 1
+RESID_NONE = 0
+RESID_MUSE_GATE = 1
+RESID_LITERAL = 2
+
+# Scale c of the Zipf router bias  bias_e = -c * s * ln(rank_e)  (s = 1.2) for the imbalanced
+# workload.  Calibrated by tests/golden/calibrate_zipf_bias.py, which bisects c with the CPU
+# oracle's router on a seeded 2048-token calibration sample until the hottest expert's load is
+# 20x the mean; the script's output is tests/golden/zipf_bias_scale.json and a CPU test keeps the
+# two equal.
+ZIPF_S = 1.2
+ZIPF_BIAS_SCALE = 0.46277
+
+
+@dataclasses.dataclass(frozen=True)
+class MoEConfig:
+    name: str
+    T: int
+    d_model: int
+    n_experts: int
+    top_k: int
+    d_ff: int                 # expert hidden width (ReLU hidden, or SwiGLU intermediate I)
+    d_latent: int = 0         # 0: no latent projections (Shazeer layer)
+    dtype: str = "bf16"       # "f32" or "bf16"
+    act: int = ACT_SWIGLU
+    pre_norm: int = 0         # centred RMSNorm after the latent down-projection
+    expert_norm: int = 0      # per-expert input-scaled RMSNorm before the weighted sum
+    resid_mode: int = RESID_NONE
+    eps: float = 1e-6
+    tau: float = 0.3
+    resid_floor: float = 1e-3
+    routed_scale: float = 1.0
+    seed: int = 0
+    x_sigma: float = 1.0      # std of the layer input u (and of the residual h = u)
+    router_gain: float = 1.0  # extra factor on the router weights' std
+    zipf_bias: bool = False
+    gamma_sigma: float = 0.02
+
+    @property
+    def latent(self) -> bool:
+        return self.d_latent > 0
+
+    @property
+    def expert_in(self) -> int:
+        """Width of an expert's input (latent width, or the model width without latent)."""
+        return self.d_latent if self.latent else self.d_model
+
+    @property
+    def gu_rows(self) -> int:
+        """Rows of one expert's first weight matrix: 2*I (gate rows, then up rows) or h."""
+        return 2 * self.d_ff if self.act == ACT_SWIGLU else self.d_ff
+
+    def replace(self, **kw) -> "MoEConfig":
+        return dataclasses.replace(self, **kw)
+
+    # ---- std of each generated tensor (N(0, 1/fan_in) weights) ----
+    def sigma_router(self) -> float:
+        return self.router_gain / math.sqrt(self.d_model)
+
+    def sigma_p_down(self) -> float:
+        return 1.0 / math.sqrt(self.d_model)
+
+    def sigma_p_up(self) -> float:
+        return 1.0 / math.sqrt(self.d_latent)
+
+    def sigma_w_gu(self) -> float:
+        return 1.0 / math.sqrt(self.expert_in)
+
+    def sigma_w_down(self) -> float:
+        return 1.0 / math.sqrt(self.d_ff)
+
+
+TINY_SHAZEER_F32 = MoEConfig(
+    name="tiny_shazeer_f32", T=128, d_model=64, n_experts=8, top_k=2, d_ff=128, dtype="f32",
+    act=ACT_RELU, seed=0, x_sigma=1.0, router_gain=4.0)
+
+SHAZEER_BF16 = MoEConfig(
+    name="shazeer_bf16", T=8192, d_model=512, n_experts=256, top_k=4, d_ff=1024, dtype="bf16",
+    act=ACT_RELU, seed=1, x_sigma=1.0 / math.sqrt(512))
+
+MUSE_DECODE = MoEConfig(
+    name="muse_decode", T=64, d_model=8192, d_latent=4096, n_experts=256, top_k=8, d_ff=4096,
+    dtype="bf16", act=ACT_SWIGLU, pre_norm=1, expert_norm=1, resid_mode=RESID_MUSE_GATE,
+    eps=1e-6, seed=2, x_sigma=1.0)
+
+MUSE_PREFILL = MUSE_DECODE.replace(name="muse_prefill", T=16384, seed=3)
+
+MUSE_IMBALANCED = MUSE_DECODE.replace(name="muse_imbalanced", T=32768, seed=4, zipf_bias=True)
+
+CONFIGS = {c.name: c for c in (TINY_SHAZEER_F32, SHAZEER_BF16, MUSE_DECODE, MUSE_PREFILL,
+                               MUSE_IMBALANCED)}
+
+
+def small_muse(T: int = 37, d: int = 256, L: int = 128, I: int = 128, n: int = 16, k: int = 4,
+               seed: int = 7, **kw) -> MoEConfig:
+    """A Muse-structured layer at sizes the oracle finishes in well under a second."""
+    return MUSE_DECODE.replace(name=f"small_muse_T{T}", T=T, d_model=d, d_latent=L, d_ff=I,
+                               n_experts=n, top_k=k, seed=seed, **kw)
+
+
+def small_shazeer(T: int = 45, d: int = 128, h: int = 256, n: int = 16, k: int = 4,
+                  seed: int = 5, **kw) -> MoEConfig:
+    return SHAZEER_BF16.replace(name=f"small_shazeer_T{T}", T=T, d_model=d, d_ff=h, n_experts=n,
+                                top_k=k, seed=seed, x_sigma=1.0 / math.sqrt(d), **kw)
