@@ -1,0 +1,178 @@
+/*
+ * moe.h - C ABI of the B200 (sm_100a) forward pass of a top-k softmax-routed (latent)
+ * mixture-of-experts layer:  y = sum_i G(x)_i E_i(x)  with the Muse latent-expert structure.
+ *
+ * The operations and where they are defined:
+ *   [SHAZEER] "816 billion parameters, and only 42 billion show up for each token"
+ *             (bobbyburns.tech), sections "The math" (y = sum_i G(x)_i E_i(x), ReLU experts,
+ *             experts with G_i = 0 are not evaluated) and "The gate" (Softmax(KeepTopK)).
+ *   [MUSE]    "Muse Spark Open: Norm-Preserving Gates Are Not a Norm Guarantee" (flozi.net),
+ *             sections "Two normalization orders implement different functions" (R_eps, C_gamma,
+ *             I_gamma), "Latent experts: normalization happens before the weighted sum" (latent
+ *             8192->4096 projection, C_pre, dispatch, SwiGLU experts, per-expert I_gamma before the
+ *             weighted sum), "Residual gates: derive the advertised intuition carefully" (learned
+ *             residual gate) and "What this means for serving and kernel work" (precision
+ *             contract, legal fusions).
+ *   [ARCHDB]  "Muse-Spark-Open-816B-A42B" model sheet: renormalised top-k weights,
+ *             routed_scaling_factor, latent width 4096, residual gate formula, no FFN biases.
+ *
+ * Conventions shared by every call:
+ *   - Every call returns a moe_status_t.  Argument, size, alignment and workspace errors are
+ *     detected on the host before anything is launched, and nothing is launched then.
+ *   - Pointers are DEVICE pointers owned by the caller.  The library allocates no device memory;
+ *     calls that need scratch take a caller-provided workspace (size from moe_workspace_size).
+ *   - Calls are asynchronous on the given CUDA stream (cudaStream_t passed as void*; NULL is the
+ *     legacy default stream).  Buffers must stay valid until the stream reaches the call.
+ *   - Tensors are dense row-major.  bf16 values are passed as their 16-bit patterns.  Every
+ *     pointer must be 16-byte aligned (MOE_ERR_ALIGNMENT otherwise).
+ *   - Inputs are never written.  Outputs must not alias inputs, except that the residual r of
+ *     moe_layer_forward may be the same buffer as u.
+ *   - Device-side consistency checks (an out-of-range expert index, a bounded wait that ran out)
+ *     latch an error code in a per-device status word instead of trapping; the computation is
+ *     skipped for the offending element.  moe_get_device_status synchronises the stream, reads
+ *     and clears it.
+ *   - Supported shapes: bf16 with d_model, d_latent, d_ff multiples of 64, 1 <= n_experts <= 256,
+ *     1 <= top_k <= min(8, n_experts); fp32 (CUDA-core path, for small layers) with no latent
+ *     projection.  Anything else returns MOE_ERR_UNSUPPORTED.
+ */
+#ifndef MOE_H
+#define MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,   /* NULL where a buffer is required, inconsistent sizes */
+  MOE_ERR_UNSUPPORTED = 2,   /* shape or mode outside the supported set */
+  MOE_ERR_ALIGNMENT = 3,     /* a pointer not 16-byte aligned */
+  MOE_ERR_WORKSPACE = 4,     /* workspace missing or smaller than moe_workspace_size */
+  MOE_ERR_CUDA = 5,          /* a CUDA runtime/driver call failed (launch, tensor map) */
+  MOE_ERR_TIMEOUT = 6,       /* device: a bounded wait inside a kernel ran out */
+  MOE_ERR_DEVICE_CHECK = 7   /* device: an index failed its range check */
+} moe_status_t;
+
+enum { MOE_F32 = 0, MOE_BF16 = 1 };
+enum { MOE_ACT_RELU = 0, MOE_ACT_SWIGLU = 1 };
+enum { MOE_RESID_NONE = 0, MOE_RESID_MUSE_GATE = 1, MOE_RESID_LITERAL = 2 };
+
+typedef struct {
+  int32_t T;            /* tokens */
+  int32_t d_model;      /* width of u, r and the layer output */
+  int32_t d_latent;     /* latent width L of the expert path; 0 = no latent projections */
+  int32_t d_ff;         /* expert hidden width: ReLU hidden h, or SwiGLU intermediate I */
+  int32_t n_experts;    /* n */
+  int32_t top_k;        /* k */
+  int32_t dtype;        /* MOE_F32 | MOE_BF16 (activations and weights; accumulation is fp32) */
+  int32_t expert_act;   /* MOE_ACT_RELU (E(x) = W2 ReLU(W1 x)) | MOE_ACT_SWIGLU */
+  int32_t pre_norm;     /* 1: z = C_pre(P_down u) (centred RMSNorm, gain 1+gamma_pre) */
+  int32_t expert_norm;  /* 1: each expert output goes through I_gamma before weighting */
+  int32_t resid_mode;   /* MOE_RESID_NONE | MOE_RESID_MUSE_GATE | MOE_RESID_LITERAL */
+  float eps;            /* RMSNorm epsilon (both norms) */
+  float tau;            /* residual gate temperature */
+  float resid_floor;    /* residual gate floor delta on alpha^2 */
+  float routed_scale;   /* routed_scaling_factor applied to the renormalised weights */
+} moe_config_t;
+
+typedef struct {
+  const void* w_router;     /* [n, d_model]                          dtype */
+  const void* p_down;       /* [d_latent, d_model]  (latent only)     dtype */
+  const void* p_up;         /* [d_model, d_latent]  (latent only)     dtype */
+  const void* w_gu;         /* [n, 2*d_ff, E_in] SwiGLU: rows [0, d_ff) gate, [d_ff, 2*d_ff) up;
+                               [n, d_ff, E_in] ReLU.  E_in = d_latent, or d_model without latent */
+  const void* w_down;       /* [n, E_in, d_ff]                        dtype */
+  const float* gamma_pre;   /* [d_latent] (pre_norm only) */
+  const float* gamma_expert;/* [E_in] one gain shared by all experts (expert_norm only) */
+  const float* resid_g;     /* [d_model] residual gate parameter g (resid_mode != NONE) */
+  const float* logit_bias;  /* [n] added to every token's router logits, or NULL */
+} moe_weights_t;
+
+/* Human-readable name of a status code (static storage). */
+MOE_API const char* moe_status_string(moe_status_t s);
+
+/* Bytes of workspace moe_layer_forward needs for this configuration (also an upper bound for
+ * moe_permute and moe_expert_ffn).  Only host arithmetic. */
+MOE_API moe_status_t moe_workspace_size(const moe_config_t* cfg, size_t* bytes);
+
+/* Router [SHAZEER "The gate"; ARCHDB gating fields]:
+ *   l = u W_router^T (+ logit_bias), fp32 accumulation;  the k largest logits are selected
+ *   (ties to the lower expert index) in descending order; w_j = exp(l_j - l_1) / sum_sel exp(.)
+ *   times routed_scale, which equals softmax-then-renormalise over the kept experts.
+ * u: [T, d_model]; topk_idx: [T, k] int32; topk_w: [T, k] fp32; logits_out: [T, n] fp32 with
+ * the bias included, or NULL. */
+MOE_API moe_status_t moe_route(const moe_config_t* cfg, const void* u, const void* w_router,
+                       const float* logit_bias, float* logits_out, int32_t* topk_idx,
+                       float* topk_w, void* stream);
+
+/* Dispatch [MUSE "Latent experts"; SHAZEER "The math"]: groups the T*k routed slots by expert
+ * in the canonical order (experts ascending; within an expert, tokens ascending), so that every
+ * index output is unique and bit-exact:
+ *   expert_offsets [n+1] (exclusive prefix sum of per-expert counts), perm_token [T*k]
+ *   (row -> token), inv_perm [T*k] (slot t*k+j -> row).
+ * If x is not NULL it also gathers rows: x_perm[inv_perm[t*k+j]] = f(x[t]) where x is [T, E_in]
+ * and f is C_pre with gain 1+gamma_pre when gamma_pre is not NULL (cfg->pre_norm), else the
+ * identity.  workspace: at least moe_workspace_size bytes.  An index outside [0, n) latches
+ * MOE_ERR_DEVICE_CHECK and that slot is dropped. */
+MOE_API moe_status_t moe_permute(const moe_config_t* cfg, const int32_t* topk_idx,
+                         int32_t* expert_offsets, int32_t* perm_token, int32_t* inv_perm,
+                         const void* x, const float* gamma_pre, void* x_perm, void* workspace,
+                         size_t workspace_bytes, void* stream);
+
+/* Experts on their routed rows only [MUSE "Latent experts"; SHAZEER "The math"]: for each expert
+ * e, rows [expert_offsets[e], expert_offsets[e+1]) of x_perm [T*k, E_in]:
+ *   SwiGLU: a = SiLU(x W_gate^T) * (x W_up^T) stored in dtype;  ReLU: a = ReLU(x W1^T);
+ *   o = a W_down^T stored in dtype;  with expert_norm: out = dtype((1+gamma_expert) * o), the
+ *   scaled vector that I_gamma reduces ([MUSE "Two normalization orders"]), else out = o.
+ * out_perm: [T*k, E_in].  workspace holds the activation a. */
+MOE_API moe_status_t moe_expert_ffn(const moe_config_t* cfg, const void* x_perm,
+                            const int32_t* expert_offsets, const void* w_gu, const void* w_down,
+                            const float* gamma_expert, void* out_perm, void* workspace,
+                            size_t workspace_bytes, void* stream);
+
+/* Normalise and combine [MUSE "Latent experts" (normalise each expert output, then weight and
+ * accumulate); SHAZEER "The math"]: for each token t,
+ *   y_t = dtype( sum_j topk_w[t,j] * n_j ),  n_j = dtype(s_j / sqrt(mean(s_j^2) + eps)) with
+ *   s_j = out_perm[inv_perm[t*k+j]] when expert_norm, else n_j = s_j;  fp32 accumulation in slot
+ *   order.  y: [T, E_in]. */
+MOE_API moe_status_t moe_combine(const moe_config_t* cfg, const void* out_perm, const int32_t* inv_perm,
+                         const float* topk_w, void* y, void* stream);
+
+/* Latent down-projection [MUSE "Latent experts"]: z_raw = dtype(u P_down^T), [T, d_latent]. */
+MOE_API moe_status_t moe_latent_down(const moe_config_t* cfg, const void* u, const void* p_down,
+                             void* z_raw, void* stream);
+
+/* Latent up-projection and residual update [MUSE "Residual gates"; ARCHDB residual field]:
+ *   b = dtype(y P_up^T); out = dtype(alpha*r + beta*b) with beta = sigmoid(g/tau),
+ *   alpha = sqrt(max(sigmoid(-g/tau)*(1+beta), resid_floor)) per channel (MUSE_GATE), or
+ *   dtype(r + g*b) (LITERAL), or b (NONE).  y: [T, d_latent]; r, out: [T, d_model]. */
+MOE_API moe_status_t moe_latent_up(const moe_config_t* cfg, const void* y, const void* p_up,
+                           const void* r, const float* resid_g, void* out, void* stream);
+
+/* The whole layer: route -> latent down (+C_pre) -> dispatch -> experts (+I_gamma prep) ->
+ * normalise and combine -> latent up -> residual update.  u: [T, d_model] is the branch input
+ * (router and down-projection read it), r: [T, d_model] the residual stream (may equal u;
+ * ignored when resid_mode is NONE), out: [T, d_model].  logits_out [T, n], topk_idx_out [T, k]
+ * and topk_w_out [T, k] are optional copies of the routing. */
+MOE_API moe_status_t moe_layer_forward(const moe_config_t* cfg, const moe_weights_t* w, const void* u,
+                               const void* r, void* out, float* logits_out,
+                               int32_t* topk_idx_out, float* topk_w_out, void* workspace,
+                               size_t workspace_bytes, void* stream);
+
+/* Synchronises the stream, returns and clears the device status word of the current device
+ * (MOE_OK if no kernel latched an error since the last call). */
+MOE_API moe_status_t moe_get_device_status(void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif

@@ -1,0 +1,200 @@
+"""Python binding of libmoe.so, the sm_100a forward pass of a top-k softmax-routed (latent)
+mixture-of-experts layer.
+
+The binding only marshals arguments: every step of the layer runs in the library's CUDA kernels.
+PyTorch is used for device memory and streams.  There is no fallback: if libmoe.so is missing or
+cannot be loaded, importing ``lib()`` raises.
+
+C entry points (same names as in include/moe.h): moe_route, moe_permute, moe_expert_ffn,
+moe_combine, moe_latent_down, moe_latent_up, moe_layer_forward, moe_workspace_size,
+moe_get_device_status, moe_status_string.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmoe.so")
+
+MOE_F32, MOE_BF16 = 0, 1
+MOE_ACT_RELU, MOE_ACT_SWIGLU = 0, 1
+MOE_RESID_NONE, MOE_RESID_MUSE_GATE, MOE_RESID_LITERAL = 0, 1, 2
+STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED", 3: "MOE_ERR_ALIGNMENT",
+          4: "MOE_ERR_WORKSPACE", 5: "MOE_ERR_CUDA", 6: "MOE_ERR_TIMEOUT",
+          7: "MOE_ERR_DEVICE_CHECK"}
+STATUS_CODES = {v: k for k, v in STATUS.items()}
+EXPORTS = ("moe_status_string", "moe_workspace_size", "moe_route", "moe_permute",
+           "moe_expert_ffn", "moe_combine", "moe_latent_down", "moe_latent_up",
+           "moe_layer_forward", "moe_get_device_status")
+
+
+class MoeError(RuntimeError):
+    def __init__(self, fn: str, code: int):
+        super().__init__(f"{fn} returned {STATUS.get(code, code)}")
+        self.code = code
+
+
+class Config(ctypes.Structure):
+    """moe_config_t"""
+    _fields_ = [(n, ctypes.c_int32) for n in ("T", "d_model", "d_latent", "d_ff", "n_experts",
+                                              "top_k", "dtype", "expert_act", "pre_norm",
+                                              "expert_norm", "resid_mode")] + \
+               [(n, ctypes.c_float) for n in ("eps", "tau", "resid_floor", "routed_scale")]
+
+
+class Weights(ctypes.Structure):
+    """moe_weights_t"""
+    _fields_ = [(n, ctypes.c_void_p) for n in ("w_router", "p_down", "p_up", "w_gu", "w_down",
+                                               "gamma_pre", "gamma_expert", "resid_g",
+                                               "logit_bias")]
+
+
+_lib = None
+
+
+def lib():
+    """The loaded libmoe.so (built in place by ``build.build()``)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"libmoe.so not built ({LIB_PATH}); run "
+                              "python sparse_moe_layer_softmax_b200/build.py")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i32, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+        cp, wp = ctypes.POINTER(Config), ctypes.POINTER(Weights)
+        L.moe_status_string.restype = ctypes.c_char_p
+        L.moe_status_string.argtypes = [i32]
+        sigs = {
+            "moe_workspace_size": [cp, ctypes.POINTER(sz)],
+            "moe_route": [cp, vp, vp, vp, vp, vp, vp, vp],
+            "moe_permute": [cp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp],
+            "moe_expert_ffn": [cp, vp, vp, vp, vp, vp, vp, vp, sz, vp],
+            "moe_combine": [cp, vp, vp, vp, vp, vp],
+            "moe_latent_down": [cp, vp, vp, vp, vp],
+            "moe_latent_up": [cp, vp, vp, vp, vp, vp, vp],
+            "moe_layer_forward": [cp, wp, vp, vp, vp, vp, vp, vp, vp, sz, vp],
+            "moe_get_device_status": [vp],
+        }
+        for name, args in sigs.items():
+            f = getattr(L, name)
+            f.restype = i32
+            f.argtypes = args
+        _lib = L
+    return _lib
+
+
+def make_config(T, d_model, n_experts, top_k, d_ff, d_latent=0, dtype=MOE_BF16,
+                expert_act=MOE_ACT_SWIGLU, pre_norm=0, expert_norm=0, resid_mode=MOE_RESID_NONE,
+                eps=1e-6, tau=0.3, resid_floor=1e-3, routed_scale=1.0) -> Config:
+    return Config(T=T, d_model=d_model, d_latent=d_latent, d_ff=d_ff, n_experts=n_experts,
+                  top_k=top_k, dtype=dtype, expert_act=expert_act, pre_norm=pre_norm,
+                  expert_norm=expert_norm, resid_mode=resid_mode, eps=eps, tau=tau,
+                  resid_floor=resid_floor, routed_scale=routed_scale)
+
+
+def _ptr(t) -> int | None:
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    return stream if isinstance(stream, int) else stream.cuda_stream
+
+
+def _check(name: str, code: int):
+    if code != 0:
+        raise MoeError(name, code)
+
+
+def workspace_size(cfg: Config) -> int:
+    n = ctypes.c_size_t()
+    _check("moe_workspace_size", lib().moe_workspace_size(ctypes.byref(cfg), ctypes.byref(n)))
+    return n.value
+
+
+def moe_route(cfg, u, w_router, logit_bias, logits_out, topk_idx, topk_w, stream=None):
+    _check("moe_route", lib().moe_route(ctypes.byref(cfg), _ptr(u), _ptr(w_router),
+                                        _ptr(logit_bias), _ptr(logits_out), _ptr(topk_idx),
+                                        _ptr(topk_w), _stream(stream)))
+
+
+def moe_permute(cfg, topk_idx, expert_offsets, perm_token, inv_perm, x=None, gamma_pre=None,
+                x_perm=None, workspace=None, workspace_bytes=0, stream=None):
+    if workspace is not None and not workspace_bytes:
+        workspace_bytes = workspace.numel() * workspace.element_size()
+    _check("moe_permute", lib().moe_permute(ctypes.byref(cfg), _ptr(topk_idx), _ptr(expert_offsets),
+                                            _ptr(perm_token), _ptr(inv_perm), _ptr(x),
+                                            _ptr(gamma_pre), _ptr(x_perm), _ptr(workspace),
+                                            workspace_bytes, _stream(stream)))
+
+
+def moe_expert_ffn(cfg, x_perm, expert_offsets, w_gu, w_down, gamma_expert, out_perm,
+                   workspace=None, workspace_bytes=0, stream=None):
+    if workspace is not None and not workspace_bytes:
+        workspace_bytes = workspace.numel() * workspace.element_size()
+    _check("moe_expert_ffn", lib().moe_expert_ffn(ctypes.byref(cfg), _ptr(x_perm),
+                                                  _ptr(expert_offsets), _ptr(w_gu), _ptr(w_down),
+                                                  _ptr(gamma_expert), _ptr(out_perm),
+                                                  _ptr(workspace), workspace_bytes,
+                                                  _stream(stream)))
+
+
+def moe_combine(cfg, out_perm, inv_perm, topk_w, y, stream=None):
+    _check("moe_combine", lib().moe_combine(ctypes.byref(cfg), _ptr(out_perm), _ptr(inv_perm),
+                                            _ptr(topk_w), _ptr(y), _stream(stream)))
+
+
+def moe_latent_down(cfg, u, p_down, z_raw, stream=None):
+    _check("moe_latent_down", lib().moe_latent_down(ctypes.byref(cfg), _ptr(u), _ptr(p_down),
+                                                    _ptr(z_raw), _stream(stream)))
+
+
+def moe_latent_up(cfg, y, p_up, r, resid_g, out, stream=None):
+    _check("moe_latent_up", lib().moe_latent_up(ctypes.byref(cfg), _ptr(y), _ptr(p_up), _ptr(r),
+                                                _ptr(resid_g), _ptr(out), _stream(stream)))
+
+
+def make_weights(w: dict) -> Weights:
+    """moe_weights_t from a dict of CUDA tensors (missing entries are NULL)."""
+    return Weights(**{k: _ptr(w.get(k)) for k, _ in Weights._fields_})
+
+
+def moe_layer_forward(cfg, weights: Weights, u, r, out, logits_out=None, topk_idx_out=None,
+                      topk_w_out=None, workspace=None, workspace_bytes=0, stream=None):
+    if workspace is not None and not workspace_bytes:
+        workspace_bytes = workspace.numel() * workspace.element_size()
+    _check("moe_layer_forward", lib().moe_layer_forward(
+        ctypes.byref(cfg), ctypes.byref(weights), _ptr(u), _ptr(r), _ptr(out), _ptr(logits_out),
+        _ptr(topk_idx_out), _ptr(topk_w_out), _ptr(workspace), workspace_bytes, _stream(stream)))
+
+
+def moe_get_device_status(stream=None) -> int:
+    return lib().moe_get_device_status(_stream(stream))
+
+
+class MoELayer:
+    """A layer instance holding its device weights and a workspace, with a forward() that takes
+    device or pinned-host inputs.  Nothing here computes: forward() is one moe_layer_forward."""
+
+    def __init__(self, cfg: Config, weights: dict):
+        import torch
+        self.cfg = cfg
+        self.weights = weights
+        self._w = make_weights(weights)
+        self.workspace = torch.empty(workspace_size(cfg), dtype=torch.uint8, device="cuda")
+
+    def forward(self, u, r=None, out=None, logits_out=None, topk_idx_out=None, topk_w_out=None,
+                stream=None):
+        import torch
+        if out is None:
+            out = torch.empty_like(u)
+        moe_layer_forward(self.cfg, self._w, u, r if r is not None else u, out, logits_out,
+                          topk_idx_out, topk_w_out, self.workspace, stream=stream)
+        return out

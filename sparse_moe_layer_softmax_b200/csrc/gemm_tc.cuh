@@ -1,0 +1,444 @@
+// Grouped GEMM on the 5th-generation tensor cores (tcgen05.mma, accumulators in TMEM, operands
+// staged by TMA with the 128-byte swizzle), persistent and warp-specialised, with the MoE
+// layer's epilogues fused in.
+//
+//   out[r, c] = epi( sum_k X[r, k] * W[g*Nw + c', k] )      for r in group g's row segment
+//
+// X is the activation matrix (rows grouped by expert, or one group for a dense projection) and
+// W the stacked weights of all groups, both K-major bf16.  Two orientations:
+//   normal : tcgen05 M = 128 rows of X, N = BN rows of W    (prefill-sized groups)
+//   swap   : tcgen05 M = 128 rows of W, N = BN rows of X    (decode: a few tokens per expert;
+//            the weights fill the 128-wide M side and the tokens the narrow N side)
+// Tiles are ordered (group, feature tile, row chunk) with the row chunk fastest, so the CTAs
+// working at one time share weight tiles through L2 and each weight tile leaves HBM about once.
+//
+// Warp roles (192 threads): warp 0 = TMA producer, warp 1 = TMEM allocator + MMA issuer,
+// warps 2..5 = epilogue (TMEM -> registers -> fused math -> global).  The accumulator is double
+// buffered in TMEM so the epilogue of one tile overlaps the MMAs of the next.
+#pragma once
+
+#include "common.cuh"
+
+namespace moe {
+
+enum EpiKind : int {
+  EPI_STORE = 0,    // dtype(acc), optionally dtype(dtype(acc) * (1 + gamma[col]))
+  EPI_RELU = 1,     // dtype(max(acc, 0))
+  EPI_SWIGLU = 2,   // dtype(SiLU(gate) * up), gate/up W rows paired (rows c and Nw/2 + c)
+  EPI_RESGATE = 3,  // residual update of the latent up-projection
+  EPI_ROUTER = 4,   // top-k selection and renormalised weights over the row's logits
+};
+
+struct GemmParams {
+  const int* seg;   // [G+1] row offsets of the groups in X, or nullptr: one group of M rows
+  int G;            // groups
+  int M;            // rows of X when seg == nullptr
+  int K;            // reduction length, multiple of 64
+  int Nw;           // W rows per group
+  int Nout;         // output columns (= row stride of out)
+  void* out;        // [rows, Nout]: bf16 bits
+  const float* gamma;        // EPI_STORE: optional gain (1 + gamma[col])
+  const uint16_t* resid;     // EPI_RESGATE: residual r [rows, Nout]
+  const float* gparam;       // EPI_RESGATE: g [Nout]
+  float tau, floor_;
+  int resid_mode;            // MOE_RESID_*
+  float* logits;             // EPI_ROUTER: [rows, Nout] fp32 or nullptr
+  int32_t* topk_idx;         // EPI_ROUTER: [rows, top_k]
+  float* topk_w;             // EPI_ROUTER: [rows, top_k]
+  const float* bias;         // EPI_ROUTER: [Nout] or nullptr
+  int top_k;
+  float routed_scale;
+};
+
+template <bool kSwap, int BN, int kEpi>
+struct GemmShape {
+  static constexpr bool kDual = (kEpi == EPI_SWIGLU);
+  static constexpr int kBK = 64;                                  // 128 bytes of bf16
+  static constexpr int kABytes = 128 * 128 * ((kSwap && kDual) ? 2 : 1);
+  static constexpr int kBBytes = BN * 128;
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kFO = kSwap ? 128 : (kDual ? BN / 2 : BN);  // output features per tile
+  static constexpr int kCH = kSwap ? BN : 128;                     // X rows per tile
+  static constexpr int kAccCols = (kSwap && kDual) ? 2 * BN : BN;  // fp32 TMEM columns
+  static constexpr int kTmemCols = (2 * kAccCols <= 32)    ? 32
+                                   : (2 * kAccCols <= 64)  ? 64
+                                   : (2 * kAccCols <= 128) ? 128
+                                   : (2 * kAccCols <= 256) ? 256
+                                                           : 512;
+  static constexpr int kXBoxRows = kSwap ? BN : 128;
+  static constexpr int kWBoxRows = kSwap ? 128 : (kDual ? BN / 2 : BN);
+  static constexpr uint32_t kIdesc = idesc_bf16_f32(128, BN);
+  static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "tcgen05 M=128 needs N % 16 == 0");
+  static_assert(2 * kAccCols <= 512, "two accumulators must fit in TMEM");
+};
+
+constexpr int kMaxGroups = 256;
+constexpr int kGemmThreads = 192;
+constexpr int kSmemMisc = 4096;
+
+template <bool kSwap, int BN, int kEpi, int kStages>
+constexpr int gemm_smem_bytes() {
+  return kStages * GemmShape<kSwap, BN, kEpi>::kStageBytes + 1024 + kSmemMisc;
+}
+
+struct TileCoord {
+  int g, ft, row0, nrows;
+};
+
+__device__ __forceinline__ TileCoord decode_tile(int t, const int* s_seg, const int* s_pref,
+                                                 int G, int FT, int CH) {
+  int lo = 0, hi = G;
+  while (lo < hi) {  // last g with s_pref[g] <= t
+    int mid = (lo + hi + 1) >> 1;
+    if (s_pref[mid] <= t) lo = mid; else hi = mid - 1;
+  }
+  TileCoord c;
+  c.g = lo;
+  int chunks = (s_pref[lo + 1] - s_pref[lo]) / FT;
+  int local = t - s_pref[lo];
+  c.ft = local / chunks;
+  int chunk = local - c.ft * chunks;
+  c.row0 = s_seg[lo] + chunk * CH;
+  int rem = s_seg[lo + 1] - c.row0;
+  c.nrows = rem < CH ? rem : CH;
+  return c;
+}
+
+template <int kMaxK>
+struct TopK {
+  float v[kMaxK];
+  int i[kMaxK];
+  __device__ __forceinline__ void init() {
+#pragma unroll
+    for (int j = 0; j < kMaxK; ++j) { v[j] = -INFINITY; i[j] = -1; }
+  }
+  // Columns arrive in ascending index order; strict comparisons keep the lower index first
+  // among equal values.  Insertion into the sorted list of the k best (k <= kMaxK).
+  __device__ __forceinline__ void push(float x, int idx, int k) {
+    if (i[k - 1] >= 0 && !(x > v[k - 1])) return;
+#pragma unroll
+    for (int j = kMaxK - 1; j >= 0; --j) {
+      if (j >= k) continue;
+      const bool above = (j > 0) && (i[j - 1] < 0 || x > v[j - 1]);
+      if (above) {
+        v[j] = v[j - 1];
+        i[j] = i[j - 1];
+      } else {
+        v[j] = x;
+        i[j] = idx;
+        break;
+      }
+    }
+  }
+};
+
+template <bool kSwap, int BN, int kEpi, int kStages>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
+                   const GemmParams p) {
+  using S = GemmShape<kSwap, BN, kEpi>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* tiles = smem;
+  uint64_t* full = reinterpret_cast<uint64_t*>(tiles + kStages * S::kStageBytes);
+  uint64_t* empty = full + kStages;
+  uint64_t* tfull = empty + kStages;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* done = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+  int* s_seg = reinterpret_cast<int*>(tmem_slot + 4);
+  int* s_pref = s_seg + (kMaxGroups + 4);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int G = p.G;
+  const int FT = (p.Nout + S::kFO - 1) / S::kFO;  // the router's last tile may be partial
+  const int KB = p.K / S::kBK;
+
+  // ---- group segments and the per-group tile prefix (warp 0)
+  if (warp == 0) {
+    const int per = (G + 31) / 32;
+    int local = 0;
+    for (int j = 0; j < per; ++j) {
+      int g = lane * per + j;
+      if (g < G) {
+        int a = p.seg ? p.seg[g] : 0, b = p.seg ? p.seg[g + 1] : p.M;
+        if (b < a) { latch_status(MOE_ERR_DEVICE_CHECK); b = a; }
+        s_seg[g] = a;
+        if (g == G - 1) s_seg[G] = b;
+        local += ((b - a + S::kCH - 1) / S::kCH) * FT;
+      }
+    }
+    int incl = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    int run = incl - local;
+    for (int j = 0; j < per; ++j) {
+      int g = lane * per + j;
+      if (g < G) {
+        int a = p.seg ? p.seg[g] : 0, b = p.seg ? p.seg[g + 1] : p.M;
+        if (b < a) b = a;
+        s_pref[g] = run;
+        run += ((b - a + S::kCH - 1) / S::kCH) * FT;
+      }
+    }
+    if (lane == 31) s_pref[G] = incl;
+  }
+  if (threadIdx.x == 32) {
+    for (int s = 0; s < kStages; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+    for (int a = 0; a < 2; ++a) { mbar_init(&tfull[a], 1); mbar_init(&tempty[a], 128); }
+    mbar_init(done, 1);
+    fence_barrier_init();
+  }
+  if (warp == 1) tmem_alloc(tmem_slot, S::kTmemCols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int total = s_pref[G];
+
+  if (warp == 0 && lane == 0) {
+    // ------------------------------------------------------------ TMA producer
+    tma_prefetch_desc(&tmX);
+    tma_prefetch_desc(&tmW);
+    uint32_t stage = 0, phase = 0;
+    uint32_t last_parity[kStages];
+    bool issued[kStages];
+#pragma unroll
+    for (int s = 0; s < kStages; ++s) { issued[s] = false; last_parity[s] = 0; }
+    bool ok = true;
+    for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+      TileCoord c = decode_tile(t, s_seg, s_pref, G, FT, S::kCH);
+      const int wrow = c.g * p.Nw + c.ft * S::kFO;
+      for (int kb = 0; kb < KB; ++kb) {
+        if (!mbar_wait(&empty[stage], phase ^ 1)) { ok = false; break; }
+        uint8_t* sa = tiles + stage * S::kStageBytes;
+        uint8_t* sb = sa + S::kABytes;
+        mbar_arrive_expect_tx(&full[stage], S::kStageBytes);
+        const int kx = kb * S::kBK;
+        if (!kSwap) {
+          tma_load_2d(&tmX, &full[stage], sa, kx, c.row0);
+          tma_load_2d(&tmW, &full[stage], sb, kx, wrow);
+          if (S::kDual) tma_load_2d(&tmW, &full[stage], sb + (BN / 2) * 128, kx, wrow + p.Nw / 2);
+        } else {
+          tma_load_2d(&tmW, &full[stage], sa, kx, wrow);
+          if (S::kDual) tma_load_2d(&tmW, &full[stage], sa + 128 * 128, kx, wrow + p.Nw / 2);
+          tma_load_2d(&tmX, &full[stage], sb, kx, c.row0);
+        }
+        issued[stage] = true;
+        last_parity[stage] = phase;
+        if (++stage == kStages) { stage = 0; phase ^= 1; }
+      }
+    }
+    // No copy may still be landing in shared memory when the CTA exits.
+    for (int s = 0; s < kStages; ++s)
+      if (issued[s]) mbar_wait(&full[s], last_parity[s]);
+  } else if (warp == 1 && lane == 0) {
+    // ------------------------------------------------------------ MMA issuer
+    uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+      if (!mbar_wait(&tempty[acc], acc_phase ^ 1)) break;
+      tc_fence_after();
+      const uint32_t d = tmem_base + acc * S::kAccCols;
+      for (int kb = 0; kb < KB; ++kb) {
+        if (!mbar_wait(&full[stage], phase)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t a_addr = smem_u32(tiles + stage * S::kStageBytes);
+        const uint32_t b_addr = a_addr + S::kABytes;
+#pragma unroll
+        for (int k = 0; k < S::kBK / 16; ++k) {
+          const uint32_t accum = (kb | k) != 0;
+          const uint64_t bdesc = smem_desc_k128(b_addr + 32 * k);
+          tc_mma_bf16(d, smem_desc_k128(a_addr + 32 * k), bdesc, S::kIdesc, accum);
+          if (kSwap && S::kDual)
+            tc_mma_bf16(d + BN, smem_desc_k128(a_addr + 128 * 128 + 32 * k), bdesc, S::kIdesc,
+                        accum);
+        }
+        tc_commit(&empty[stage]);
+        if (++stage == kStages) { stage = 0; phase ^= 1; }
+      }
+      if (!ok) break;
+      tc_commit(&tfull[acc]);
+      if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+    }
+    // Every MMA of this CTA has finished before TMEM is released.
+    tc_commit(done);
+    mbar_wait(done, 0);
+  } else if (warp >= 2) {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    uint32_t acc = 0, acc_phase = 0;
+    for (int t = blockIdx.x; t < total; t += gridDim.x) {
+      TileCoord c = decode_tile(t, s_seg, s_pref, G, FT, S::kCH);
+      if (!mbar_wait(&tfull[acc], acc_phase)) break;
+      tc_fence_after();
+      const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * S::kAccCols;
+      const int f0 = c.ft * S::kFO;
+      if constexpr (!kSwap) {
+        const int rl = q * 32 + lane;
+        const bool valid = rl < c.nrows;
+        const size_t row = static_cast<size_t>(c.row0 + rl);
+        if constexpr (kEpi == EPI_ROUTER) {
+          TopK<8> tk;
+          tk.init();
+          for (int c0 = 0; c0 < BN; c0 += 16) {
+            float v[16];
+            tmem_ld16(tbase + c0, v);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const int col = c0 + i;
+              if (col < p.Nout) {
+                float l = v[i] + (p.bias ? p.bias[col] : 0.0f);
+                v[i] = l;
+                tk.push(l, col, p.top_k);
+              }
+            }
+            if (valid && p.logits) {
+              float* dst = p.logits + row * p.Nout + c0;
+              if (c0 + 16 <= p.Nout && (p.Nout & 3) == 0) {
+#pragma unroll
+                for (int i = 0; i < 16; i += 4)
+                  *reinterpret_cast<float4*>(dst + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+              } else {
+                for (int i = 0; c0 + i < p.Nout; ++i) dst[i] = v[i];
+              }
+            }
+          }
+          if (valid) {
+            float sum = 0.0f;
+            float e[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              e[j] = (j < p.top_k) ? __expf(tk.v[j] - tk.v[0]) : 0.0f;
+              sum += e[j];
+            }
+            const float scale = p.routed_scale / sum;
+            for (int j = 0; j < p.top_k; ++j) {
+              p.topk_idx[row * p.top_k + j] = tk.i[j];
+              p.topk_w[row * p.top_k + j] = e[j] * scale;
+            }
+          }
+        } else if constexpr (kEpi == EPI_SWIGLU) {
+          uint16_t* out = static_cast<uint16_t*>(p.out) + row * p.Nout + f0;
+          for (int c0 = 0; c0 < BN / 2; c0 += 16) {
+            float gv[16], uv[16];
+            tmem_ld16(tbase + c0, gv);
+            tmem_ld16(tbase + BN / 2 + c0, uv);
+            uint32_t pk[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              pk[i] = pack_bf16x2(silu(gv[2 * i]) * uv[2 * i], silu(gv[2 * i + 1]) * uv[2 * i + 1]);
+            if (valid) {
+              uint4* dst = reinterpret_cast<uint4*>(out + c0);
+              dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+              dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+            }
+          }
+        } else {
+          uint16_t* out = static_cast<uint16_t*>(p.out) + row * p.Nout + f0;
+          for (int c0 = 0; c0 < BN; c0 += 16) {
+            float v[16];
+            tmem_ld16(tbase + c0, v);
+            if constexpr (kEpi == EPI_RELU) {
+#pragma unroll
+              for (int i = 0; i < 16; ++i) v[i] = fmaxf(v[i], 0.0f);
+            } else if constexpr (kEpi == EPI_STORE) {
+              if (p.gamma) {
+#pragma unroll
+                for (int i = 0; i < 16; ++i) v[i] = round_bf16(v[i]) * (1.0f + p.gamma[f0 + c0 + i]);
+              }
+            } else if constexpr (kEpi == EPI_RESGATE) {
+              if (valid) {
+                const uint4* hp = reinterpret_cast<const uint4*>(p.resid + row * p.Nout + f0 + c0);
+                uint4 h0 = hp[0], h1 = hp[1];
+                const uint16_t* hs0 = reinterpret_cast<const uint16_t*>(&h0);
+                const uint16_t* hs1 = reinterpret_cast<const uint16_t*>(&h1);
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                  const float b = round_bf16(v[i]);
+                  const float h = bf16_to_f32(i < 8 ? hs0[i] : hs1[i - 8]);
+                  const float g = p.gparam ? p.gparam[f0 + c0 + i] : 0.0f;
+                  if (p.resid_mode == MOE_RESID_MUSE_GATE) {
+                    const float beta = sigmoidf_(g / p.tau);
+                    const float a2 = fmaxf(sigmoidf_(-g / p.tau) * (1.0f + beta), p.floor_);
+                    v[i] = sqrtf(a2) * h + beta * b;
+                  } else if (p.resid_mode == MOE_RESID_LITERAL) {
+                    v[i] = h + g * b;
+                  } else {
+                    v[i] = b;
+                  }
+                }
+              }
+            }
+            if (valid) {
+              uint32_t pk[8];
+#pragma unroll
+              for (int i = 0; i < 8; ++i) pk[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
+              uint4* dst = reinterpret_cast<uint4*>(out + c0);
+              dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+              dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+            }
+          }
+        }
+      } else {
+        // swap orientation: this thread owns output feature f for the BN rows of the chunk
+        const int f = f0 + q * 32 + lane;
+        float coefA = 1.0f, coefB = 0.0f, gsc = 1.0f;
+        if constexpr (kEpi == EPI_STORE) gsc = p.gamma ? (1.0f + p.gamma[f]) : 1.0f;
+        if constexpr (kEpi == EPI_RESGATE) {
+          const float g = p.gparam ? p.gparam[f] : 0.0f;
+          if (p.resid_mode == MOE_RESID_MUSE_GATE) {
+            coefB = sigmoidf_(g / p.tau);
+            coefA = sqrtf(fmaxf(sigmoidf_(-g / p.tau) * (1.0f + coefB), p.floor_));
+          } else if (p.resid_mode == MOE_RESID_LITERAL) {
+            coefA = 1.0f;
+            coefB = g;
+          }
+        }
+        uint16_t* out = static_cast<uint16_t*>(p.out);
+        for (int j0 = 0; j0 < BN; j0 += 16) {
+          float v[16];
+          tmem_ld16(tbase + j0, v);
+          if constexpr (kEpi == EPI_SWIGLU) {
+            float uv[16];
+            tmem_ld16(tbase + BN + j0, uv);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) v[i] = silu(v[i]) * uv[i];
+          }
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const int j = j0 + i;
+            if (j < c.nrows) {
+              const size_t row = static_cast<size_t>(c.row0 + j);
+              float x = v[i];
+              if constexpr (kEpi == EPI_RELU) x = fmaxf(x, 0.0f);
+              if constexpr (kEpi == EPI_STORE) { if (p.gamma) x = round_bf16(x) * gsc; }
+              if constexpr (kEpi == EPI_RESGATE) {
+                const float b = round_bf16(x);
+                if (p.resid_mode == MOE_RESID_NONE) x = b;
+                else x = coefA * bf16_to_f32(p.resid[row * p.Nout + f]) + coefB * b;
+              }
+              out[row * p.Nout + f] = f32_to_bf16(x);
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&tempty[acc]);
+      if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) {
+    __syncwarp();
+    tmem_dealloc(tmem_base, S::kTmemCols);
+  }
+}
+
+}  // namespace moe

@@ -1,0 +1,375 @@
+// CUDA-core kernels of the MoE layer: the canonical dispatch permutation (integer, bit-exact),
+// the token-major row scatter with the fused centred RMSNorm, the fused per-expert
+// normalisation + weighted combine, and the fp32 path (router, experts) for small layers.
+#pragma once
+
+#include "common.cuh"
+
+namespace moe {
+
+constexpr int kPermChunk = 128;  // tokens per CTA in the permutation kernels
+constexpr int kMaxTopK = 8;
+constexpr int kMaxExperts = 256;
+
+__device__ __forceinline__ float block_sum_256(float v, float* red) {
+  // Sum over a block of blockDim.x (multiple of 32, <= 256) threads; red: >= 8 floats.
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  const int w = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  __syncthreads();
+  if ((threadIdx.x & 31) == 0) red[w] = v;
+  __syncthreads();
+  float s = 0.0f;
+  for (int i = 0; i < nw; ++i) s += red[i];
+  return s;
+}
+
+// ------------------------------------------------------------------ dispatch permutation
+//
+// Canonical order: rows grouped by expert ascending, within an expert by token ascending.
+// Every token holds an expert at most once, so this order is unique; it is built without
+// atomics-order dependence: per-chunk histograms -> per-expert prefix over chunks and an
+// exclusive scan over experts -> each expert's rows of a chunk handed out in token order.
+
+__global__ void perm_count_kernel(const int32_t* __restrict__ idx, int T, int k, int n,
+                                  int32_t* __restrict__ counts) {
+  __shared__ int h[kMaxExperts];
+  for (int e = threadIdx.x; e < n; e += blockDim.x) h[e] = 0;
+  __syncthreads();
+  const long t0 = static_cast<long>(blockIdx.x) * kPermChunk;
+  const long t1 = min(static_cast<long>(T), t0 + kPermChunk);
+  for (long i = t0 * k + threadIdx.x; i < t1 * k; i += blockDim.x) {
+    const int e = idx[i];
+    if (e < 0 || e >= n) latch_status(MOE_ERR_DEVICE_CHECK);
+    else atomicAdd(&h[e], 1);
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < n; e += blockDim.x) counts[blockIdx.x * n + e] = h[e];
+}
+
+// One CTA of kMaxExperts threads: counts[c][e] becomes the number of rows of expert e in chunks
+// before c; offsets = exclusive scan of the per-expert totals.
+__global__ void perm_scan_kernel(int32_t* __restrict__ counts, int nchunks, int n,
+                                 int32_t* __restrict__ offsets) {
+  __shared__ int warp_tot[kMaxExperts / 32];
+  const int e = threadIdx.x;
+  int run = 0;
+  if (e < n) {
+    for (int c = 0; c < nchunks; ++c) {
+      const int v = counts[c * n + e];
+      counts[c * n + e] = run;
+      run += v;
+    }
+  }
+  // block-wide exclusive scan of run over e
+  int incl = run;
+  const int lane = e & 31, w = e >> 5;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) warp_tot[w] = incl;
+  __syncthreads();
+  int base = 0;
+  for (int i = 0; i < w; ++i) base += warp_tot[i];
+  if (e < n) offsets[e] = base + incl - run;
+  if (e == n - 1) offsets[n] = base + incl;
+}
+
+__global__ void perm_rank_kernel(const int32_t* __restrict__ idx, int T, int k, int n,
+                                 const int32_t* __restrict__ chunk_base,
+                                 const int32_t* __restrict__ offsets,
+                                 int32_t* __restrict__ perm_token, int32_t* __restrict__ inv_perm) {
+  __shared__ int s_idx[kPermChunk * kMaxTopK];
+  const int t0 = blockIdx.x * kPermChunk;
+  const int cnt = (min(T, t0 + kPermChunk) - t0) * k;
+  for (int i = threadIdx.x; i < cnt; i += blockDim.x) {
+    const int e = idx[static_cast<long>(t0) * k + i];
+    s_idx[i] = e;
+    if (e < 0 || e >= n) inv_perm[static_cast<long>(t0) * k + i] = -1;  // dropped slot
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < n; e += blockDim.x) {
+    int row = offsets[e] + chunk_base[blockIdx.x * n + e];
+    for (int i = 0; i < cnt; ++i) {
+      if (s_idx[i] == e) {
+        perm_token[row] = t0 + i / k;
+        inv_perm[static_cast<long>(t0) * k + i] = row;
+        ++row;
+      }
+    }
+  }
+}
+
+// ------------------------------------------------------------------ row scatter (+ C_pre)
+//
+// One CTA per token: the row is read once, optionally normalised with the output-scaled centred
+// RMSNorm  z = dtype((1 + gamma) * x / sqrt(mean(x^2) + eps))  (fp32 reduction), and written to
+// each of the token's k dispatch rows.  VEC 16-byte vectors per thread.
+template <int VEC>
+__global__ void scatter_rows_bf16_kernel(const uint16_t* __restrict__ x, int E, int k,
+                                         const int32_t* __restrict__ inv_perm,
+                                         const float* __restrict__ gamma, float eps,
+                                         uint16_t* __restrict__ x_perm) {
+  __shared__ float red[8];
+  const int t = blockIdx.x;
+  const int nvec = E / 8;
+  const uint4* src = reinterpret_cast<const uint4*>(x + static_cast<size_t>(t) * E);
+  uint4 r[VEC];
+  float ss = 0.0f;
+#pragma unroll
+  for (int v = 0; v < VEC; ++v) {
+    const int vi = threadIdx.x + v * blockDim.x;
+    r[v] = vi < nvec ? src[vi] : make_uint4(0, 0, 0, 0);
+    if (gamma) {
+      const uint16_t* h = reinterpret_cast<const uint16_t*>(&r[v]);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) { const float f = bf16_to_f32(h[i]); ss += f * f; }
+    }
+  }
+  if (gamma) {
+    const float tot = block_sum_256(ss, red);
+    const float rinv = rsqrtf(tot / static_cast<float>(E) + eps);
+#pragma unroll
+    for (int v = 0; v < VEC; ++v) {
+      const int vi = threadIdx.x + v * blockDim.x;
+      if (vi < nvec) {
+        uint16_t* h = reinterpret_cast<uint16_t*>(&r[v]);
+        const float4 g0 = reinterpret_cast<const float4*>(gamma)[2 * vi];
+        const float4 g1 = reinterpret_cast<const float4*>(gamma)[2 * vi + 1];
+        const float gg[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+#pragma unroll
+        for (int i = 0; i < 8; ++i) h[i] = f32_to_bf16((1.0f + gg[i]) * (bf16_to_f32(h[i]) * rinv));
+      }
+    }
+  }
+  for (int j = 0; j < k; ++j) {
+    const int row = inv_perm[static_cast<size_t>(t) * k + j];
+    if (row < 0) continue;
+    uint4* dst = reinterpret_cast<uint4*>(x_perm + static_cast<size_t>(row) * E);
+#pragma unroll
+    for (int v = 0; v < VEC; ++v) {
+      const int vi = threadIdx.x + v * blockDim.x;
+      if (vi < nvec) dst[vi] = r[v];
+    }
+  }
+}
+
+template <typename Tv>
+__global__ void scatter_rows_f32_kernel(const float* __restrict__ x, int E, int k,
+                                        const int32_t* __restrict__ inv_perm,
+                                        float* __restrict__ x_perm) {
+  const int t = blockIdx.x;
+  for (int j = 0; j < k; ++j) {
+    const int row = inv_perm[static_cast<size_t>(t) * k + j];
+    if (row < 0) continue;
+    for (int c = threadIdx.x; c < E; c += blockDim.x)
+      x_perm[static_cast<size_t>(row) * E + c] = x[static_cast<size_t>(t) * E + c];
+  }
+}
+
+// ------------------------------------------------------------------ normalise + combine
+//
+// One CTA per token: for each slot j the expert row s_j = out_perm[inv_perm[t,k+j]] is loaded,
+// its I_gamma denominator sqrt(mean(s_j^2) + eps) reduced in fp32, n_j = dtype(s_j / denom)
+// (when expert_norm), and y = dtype(sum_j w_j n_j) accumulated in fp32 in slot order.
+template <int VEC>
+__global__ void combine_bf16_kernel(const uint16_t* __restrict__ s, int E, int k,
+                                    const int32_t* __restrict__ inv_perm,
+                                    const float* __restrict__ topk_w, int expert_norm, float eps,
+                                    uint16_t* __restrict__ y) {
+  __shared__ float red[8][kMaxTopK];
+  const int t = blockIdx.x;
+  const int nvec = E / 8;
+  uint4 r[kMaxTopK][VEC];
+  float ss[kMaxTopK];
+#pragma unroll
+  for (int j = 0; j < kMaxTopK; ++j) {
+    ss[j] = 0.0f;
+    const int row = j < k ? inv_perm[static_cast<size_t>(t) * k + j] : -1;
+#pragma unroll
+    for (int v = 0; v < VEC; ++v) {
+      const int vi = threadIdx.x + v * blockDim.x;
+      r[j][v] = (row >= 0 && vi < nvec)
+                    ? reinterpret_cast<const uint4*>(s + static_cast<size_t>(row) * E)[vi]
+                    : make_uint4(0, 0, 0, 0);
+      const uint16_t* h = reinterpret_cast<const uint16_t*>(&r[j][v]);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) { const float f = bf16_to_f32(h[i]); ss[j] += f * f; }
+    }
+  }
+  float rinv[kMaxTopK];
+  if (expert_norm) {
+    const int w = threadIdx.x >> 5, nw = blockDim.x >> 5;
+#pragma unroll
+    for (int j = 0; j < kMaxTopK; ++j) {
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) ss[j] += __shfl_xor_sync(0xffffffffu, ss[j], o);
+      if ((threadIdx.x & 31) == 0) red[w][j] = ss[j];
+    }
+    __syncthreads();
+#pragma unroll
+    for (int j = 0; j < kMaxTopK; ++j) {
+      float tot = 0.0f;
+      for (int i = 0; i < nw; ++i) tot += red[i][j];
+      rinv[j] = rsqrtf(tot / static_cast<float>(E) + eps);
+    }
+  }
+  float wt[kMaxTopK];
+#pragma unroll
+  for (int j = 0; j < kMaxTopK; ++j) {
+    const int row = j < k ? inv_perm[static_cast<size_t>(t) * k + j] : -1;
+    wt[j] = row >= 0 ? topk_w[static_cast<size_t>(t) * k + j] : 0.0f;
+  }
+#pragma unroll
+  for (int v = 0; v < VEC; ++v) {
+    const int vi = threadIdx.x + v * blockDim.x;
+    if (vi >= nvec) continue;
+    float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+#pragma unroll
+    for (int j = 0; j < kMaxTopK; ++j) {
+      if (j >= k) break;
+      const uint16_t* h = reinterpret_cast<const uint16_t*>(&r[j][v]);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float sv = bf16_to_f32(h[i]);
+        const float nv = expert_norm ? round_bf16(sv * rinv[j]) : sv;
+        acc[i] += wt[j] * nv;
+      }
+    }
+    uint4 o;
+    o.x = pack_bf16x2(acc[0], acc[1]);
+    o.y = pack_bf16x2(acc[2], acc[3]);
+    o.z = pack_bf16x2(acc[4], acc[5]);
+    o.w = pack_bf16x2(acc[6], acc[7]);
+    reinterpret_cast<uint4*>(y + static_cast<size_t>(t) * E)[vi] = o;
+  }
+}
+
+__global__ void combine_f32_kernel(const float* __restrict__ s, int E, int k,
+                                   const int32_t* __restrict__ inv_perm,
+                                   const float* __restrict__ topk_w, int expert_norm, float eps,
+                                   float* __restrict__ y) {
+  __shared__ float red[8];
+  const int t = blockIdx.x;
+  for (int c0 = 0; c0 < E; c0 += blockDim.x) {
+    const int c = c0 + threadIdx.x;
+    float acc = 0.0f;
+    for (int j = 0; j < k; ++j) {
+      const int row = inv_perm[static_cast<size_t>(t) * k + j];
+      if (row < 0) continue;
+      const float* sr = s + static_cast<size_t>(row) * E;
+      float rinv = 1.0f;
+      if (expert_norm) {
+        float ss = 0.0f;
+        for (int i = threadIdx.x; i < E; i += blockDim.x) ss += sr[i] * sr[i];
+        rinv = rsqrtf(block_sum_256(ss, red) / static_cast<float>(E) + eps);
+      }
+      if (c < E) acc += topk_w[static_cast<size_t>(t) * k + j] * (sr[c] * rinv);
+    }
+    if (c < E) y[static_cast<size_t>(t) * E + c] = acc;
+  }
+}
+
+// ------------------------------------------------------------------ fp32 path
+
+// Router: one warp per token; logits in fp32 FMA, the k best selected by repeated warp argmax
+// (ties to the lower index), weights renormalised over the kept experts.
+__global__ void router_f32_kernel(const float* __restrict__ u, const float* __restrict__ w,
+                                  const float* __restrict__ bias, int T, int d, int n, int k,
+                                  float routed_scale, float* __restrict__ logits_out,
+                                  int32_t* __restrict__ topk_idx, float* __restrict__ topk_w) {
+  const int warps = blockDim.x >> 5;
+  const int t = blockIdx.x * warps + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (t >= T) return;
+  float l[kMaxExperts / 32];
+#pragma unroll
+  for (int i = 0; i < kMaxExperts / 32; ++i) {
+    const int e = lane + 32 * i;
+    float acc = -INFINITY;
+    if (e < n) {
+      acc = 0.0f;
+      for (int c = 0; c < d; ++c) acc = fmaf(u[static_cast<size_t>(t) * d + c], w[static_cast<size_t>(e) * d + c], acc);
+      if (bias) acc += bias[e];
+      if (logits_out) logits_out[static_cast<size_t>(t) * n + e] = acc;
+    }
+    l[i] = acc;
+  }
+  float top_v[kMaxTopK];
+  int top_i[kMaxTopK];
+  for (int j = 0; j < k; ++j) {
+    float bv = -INFINITY;
+    int bi = 0x7fffffff;
+#pragma unroll
+    for (int i = 0; i < kMaxExperts / 32; ++i) {
+      const int e = lane + 32 * i;
+      if (e < n && (l[i] > bv || (l[i] == bv && e < bi))) { bv = l[i]; bi = e; }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+      if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
+    }
+    top_v[j] = bv;
+    top_i[j] = bi;
+#pragma unroll
+    for (int i = 0; i < kMaxExperts / 32; ++i)
+      if (lane + 32 * i == bi) l[i] = -INFINITY;
+  }
+  if (lane == 0) {
+    float sum = 0.0f;
+    for (int j = 0; j < k; ++j) sum += expf(top_v[j] - top_v[0]);
+    for (int j = 0; j < k; ++j) {
+      topk_idx[static_cast<size_t>(t) * k + j] = top_i[j];
+      topk_w[static_cast<size_t>(t) * k + j] = expf(top_v[j] - top_v[0]) / sum * routed_scale;
+    }
+  }
+}
+
+// Experts in fp32: one CTA per dispatched row; hidden activation in shared memory.
+__global__ void expert_ffn_f32_kernel(const float* __restrict__ x_perm,
+                                      const int32_t* __restrict__ offsets, int n, int E, int H,
+                                      int act, const float* __restrict__ w_gu,
+                                      const float* __restrict__ w_down,
+                                      const float* __restrict__ gamma,
+                                      float* __restrict__ out_perm) {
+  extern __shared__ float sm[];  // [E] input row, [H] hidden
+  float* xr = sm;
+  float* hid = sm + E;
+  const int row = blockIdx.x;
+  if (row >= offsets[n]) return;
+  int lo = 0, hi = n - 1;  // expert owning this row: last e with offsets[e] <= row
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (offsets[mid] <= row) lo = mid; else hi = mid - 1;
+  }
+  const int e = lo;
+  const int gu_rows = act == MOE_ACT_SWIGLU ? 2 * H : H;
+  const float* W1 = w_gu + static_cast<size_t>(e) * gu_rows * E;
+  const float* W2 = w_down + static_cast<size_t>(e) * E * H;
+  for (int c = threadIdx.x; c < E; c += blockDim.x) xr[c] = x_perm[static_cast<size_t>(row) * E + c];
+  __syncthreads();
+  for (int i = threadIdx.x; i < H; i += blockDim.x) {
+    float a = 0.0f;
+    for (int c = 0; c < E; ++c) a = fmaf(xr[c], W1[static_cast<size_t>(i) * E + c], a);
+    if (act == MOE_ACT_SWIGLU) {
+      float b = 0.0f;
+      for (int c = 0; c < E; ++c) b = fmaf(xr[c], W1[static_cast<size_t>(H + i) * E + c], b);
+      hid[i] = a / (1.0f + expf(-a)) * b;
+    } else {
+      hid[i] = fmaxf(a, 0.0f);
+    }
+  }
+  __syncthreads();
+  for (int c = threadIdx.x; c < E; c += blockDim.x) {
+    float o = 0.0f;
+    for (int i = 0; i < H; ++i) o = fmaf(hid[i], W2[static_cast<size_t>(c) * H + i], o);
+    if (gamma) o *= 1.0f + gamma[c];
+    out_perm[static_cast<size_t>(row) * E + c] = o;
+  }
+}
+
+}  // namespace moe

@@ -1,0 +1,549 @@
+// Host side of the C ABI declared in include/moe.h: argument checks, workspace layout, TMA
+// descriptors and the launch sequence of the MoE-layer forward on the caller's stream.
+#include <cudaTypedefs.h>
+
+#include <initializer_list>
+#include <mutex>
+
+#include "common.cuh"
+#include "gemm_tc.cuh"
+#include "kernels_simt.cuh"
+
+namespace moe {
+namespace {
+
+// ------------------------------------------------------------------ small helpers
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline bool all_aligned(std::initializer_list<const void*> ps) {
+  for (const void* p : ps)
+    if (!aligned16(p)) return false;
+  return true;
+}
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+inline int cdiv(long a, long b) { return static_cast<int>((a + b - 1) / b); }
+
+struct DeviceInfo {
+  int sms = 0;
+};
+
+DeviceInfo& device_info() {
+  static std::mutex mu;
+  static DeviceInfo info[64];
+  int dev = 0;
+  cudaGetDevice(&dev);
+  std::lock_guard<std::mutex> lk(mu);
+  DeviceInfo& d = info[dev & 63];
+  if (d.sms == 0) cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev);
+  return d;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    cudaDriverEntryPointQueryResult q;
+    void* p = nullptr;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 2-D bf16 row-major [rows, cols] tensor, boxes of 64 columns x box_rows rows, 128-byte swizzle.
+bool make_tmap(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+moe_status_t last_launch() {
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+// ------------------------------------------------------------------ GEMM launcher
+
+template <bool kSwap, int BN, int kEpi, int kStages>
+moe_status_t launch_gemm(const void* X, long x_rows, const void* W, long w_rows,
+                         const GemmParams& p, long max_tiles, cudaStream_t st) {
+  using S = GemmShape<kSwap, BN, kEpi>;
+  constexpr int smem = gemm_smem_bytes<kSwap, BN, kEpi, kStages>();
+  static_assert(smem <= 232448, "shared memory budget");
+  auto kern = gemm_tc_kernel<kSwap, BN, kEpi, kStages>;
+  static std::once_flag once;  // the attribute is per function; set it once per process
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [&] {
+    attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  });
+  if (attr_err != cudaSuccess) return MOE_ERR_CUDA;
+  CUtensorMap tx, tw;
+  if (!make_tmap(&tx, X, static_cast<uint64_t>(x_rows), static_cast<uint64_t>(p.K), S::kXBoxRows))
+    return MOE_ERR_CUDA;
+  if (!make_tmap(&tw, W, static_cast<uint64_t>(w_rows), static_cast<uint64_t>(p.K), S::kWBoxRows))
+    return MOE_ERR_CUDA;
+  long grid = device_info().sms;
+  if (max_tiles < grid) grid = max_tiles;
+  if (grid <= 0) return MOE_OK;
+  kern<<<static_cast<unsigned>(grid), kGemmThreads, smem, st>>>(tx, tw, p);
+  return last_launch();
+}
+
+// Upper bound of the tile count of a grouped GEMM (each group adds at most one partial chunk).
+long tile_bound(long rows, int G, int ch, int ft) { return (static_cast<long>(cdiv(rows, ch)) + G) * ft; }
+
+enum class Orient { kNormal, kSwap };
+
+// Output-feature tile choice of the normal orientation: the widest of 256/128/64 dividing Nout
+// (for SwiGLU the tile holds gate and up halves, so the output width per tile is BN/2).
+int pick_bn_normal(int nout, bool dual) {
+  const int div = dual ? 2 : 1;
+  for (int bn : {256, 128, 64})
+    if (!(dual && bn < 128) && nout % (bn / div) == 0) return bn;
+  return 0;
+}
+
+// Grouped expert GEMM (or dense projection when seg == nullptr).
+moe_status_t run_gemm(int epi, Orient o, int bn, const void* X, long x_rows, const void* W,
+                      long w_rows, const GemmParams& p, cudaStream_t st) {
+  const bool dual = epi == EPI_SWIGLU;
+  if (o == Orient::kSwap) {
+    const int ft = p.Nout / 128;
+    const long mt = tile_bound(x_rows, p.G, bn, ft);
+#define SW(BN_, E_, ST_) \
+  if (bn == BN_ && epi == E_) return launch_gemm<true, BN_, E_, ST_>(X, x_rows, W, w_rows, p, mt, st);
+    SW(16, EPI_SWIGLU, 6) SW(32, EPI_SWIGLU, 6) SW(64, EPI_SWIGLU, 5)
+    SW(16, EPI_STORE, 10) SW(32, EPI_STORE, 9) SW(64, EPI_STORE, 8)
+    SW(16, EPI_RELU, 10) SW(32, EPI_RELU, 9) SW(64, EPI_RELU, 8)
+#undef SW
+    return MOE_ERR_UNSUPPORTED;
+  }
+  const int fo = dual ? bn / 2 : bn;
+  const long mt = tile_bound(x_rows, p.G, 128, cdiv(p.Nout, fo));
+#define NM(BN_, E_, ST_) \
+  if (bn == BN_ && epi == E_) return launch_gemm<false, BN_, E_, ST_>(X, x_rows, W, w_rows, p, mt, st);
+  NM(256, EPI_SWIGLU, 4) NM(128, EPI_SWIGLU, 6)
+  NM(256, EPI_STORE, 4) NM(128, EPI_STORE, 6) NM(64, EPI_STORE, 8)
+  NM(256, EPI_RELU, 4) NM(128, EPI_RELU, 6) NM(64, EPI_RELU, 8)
+  NM(256, EPI_RESGATE, 4) NM(128, EPI_RESGATE, 6) NM(64, EPI_RESGATE, 8)
+  NM(256, EPI_ROUTER, 4) NM(128, EPI_ROUTER, 6) NM(64, EPI_ROUTER, 8) NM(32, EPI_ROUTER, 8)
+#undef NM
+  return MOE_ERR_UNSUPPORTED;
+}
+
+// ------------------------------------------------------------------ configuration checks
+
+int expert_in(const moe_config_t& c) { return c.d_latent > 0 ? c.d_latent : c.d_model; }
+int gu_rows(const moe_config_t& c) { return c.expert_act == MOE_ACT_SWIGLU ? 2 * c.d_ff : c.d_ff; }
+
+moe_status_t check_cfg(const moe_config_t* c) {
+  if (!c) return MOE_ERR_INVALID_ARG;
+  if (c->T < 0 || c->d_model <= 0 || c->d_latent < 0 || c->d_ff <= 0 || c->n_experts <= 0 ||
+      c->top_k <= 0)
+    return MOE_ERR_INVALID_ARG;
+  if (c->top_k > c->n_experts) return MOE_ERR_INVALID_ARG;
+  if (c->n_experts > kMaxExperts || c->top_k > kMaxTopK) return MOE_ERR_UNSUPPORTED;
+  if (c->dtype != MOE_F32 && c->dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
+  if (c->expert_act != MOE_ACT_RELU && c->expert_act != MOE_ACT_SWIGLU) return MOE_ERR_UNSUPPORTED;
+  if (c->resid_mode < MOE_RESID_NONE || c->resid_mode > MOE_RESID_LITERAL) return MOE_ERR_UNSUPPORTED;
+  if (!(c->eps >= 0.0f) || !(c->tau > 0.0f) || !(c->resid_floor >= 0.0f)) return MOE_ERR_INVALID_ARG;
+  if (static_cast<long>(c->T) * c->top_k > 0x7fffffffL / 2) return MOE_ERR_UNSUPPORTED;
+  if (c->dtype == MOE_BF16) {
+    if (c->d_model % 64 || c->d_latent % 64 || c->d_ff % 64) return MOE_ERR_UNSUPPORTED;
+    if (expert_in(*c) > 8192) return MOE_ERR_UNSUPPORTED;  // row kernels hold a row in registers
+    if (c->d_latent == 0 && c->resid_mode != MOE_RESID_NONE) return MOE_ERR_UNSUPPORTED;
+    if (c->pre_norm && c->d_latent == 0) return MOE_ERR_UNSUPPORTED;
+  } else {
+    if (c->d_latent != 0 || c->pre_norm || c->resid_mode != MOE_RESID_NONE) return MOE_ERR_UNSUPPORTED;
+  }
+  return MOE_OK;
+}
+
+size_t dsize(const moe_config_t& c) { return c.dtype == MOE_BF16 ? 2 : 4; }
+int nchunks(const moe_config_t& c) { return cdiv(c.T, kPermChunk); }
+
+struct Workspace {
+  size_t idx, w, z_raw, offsets, perm, inv, counts, x_perm, act, y, total;
+};
+
+Workspace layout(const moe_config_t& c) {
+  Workspace L{};
+  const size_t TK = static_cast<size_t>(c.T) * c.top_k, E = expert_in(c), ds = dsize(c);
+  size_t o = 0;
+  auto take = [&](size_t bytes) { size_t at = o; o = align_up(o + bytes, 256); return at; };
+  L.idx = take(TK * 4);
+  L.w = take(TK * 4);
+  L.z_raw = take(c.d_latent > 0 ? static_cast<size_t>(c.T) * c.d_latent * ds : 0);
+  L.offsets = take((c.n_experts + 1) * 4);
+  L.perm = take(TK * 4);
+  L.inv = take(TK * 4);
+  L.counts = take(static_cast<size_t>(nchunks(c)) * c.n_experts * 4);
+  L.x_perm = take(TK * E * ds);
+  L.act = take(TK * c.d_ff * ds);
+  L.y = take(c.d_latent > 0 ? static_cast<size_t>(c.T) * E * ds : 0);
+  L.total = o;
+  return L;
+}
+
+template <typename T>
+T* at(void* base, size_t off) { return reinterpret_cast<T*>(static_cast<char*>(base) + off); }
+
+// Grouped-GEMM orientation for the experts from the mean rows per expert.
+void pick_expert_orient(const moe_config_t& c, int nout, bool dual, Orient* o, int* bn) {
+  const double mean_rows = static_cast<double>(c.T) * c.top_k / c.n_experts;
+  if (nout % 128 == 0 && mean_rows <= 48.0) {
+    *o = Orient::kSwap;
+    *bn = mean_rows <= 12.0 ? 16 : (mean_rows <= 24.0 ? 32 : 64);
+  } else {
+    *o = Orient::kNormal;
+    *bn = pick_bn_normal(nout, dual);
+  }
+}
+
+// ------------------------------------------------------------------ steps
+
+moe_status_t do_route(const moe_config_t& c, const void* u, const void* w_router,
+                      const float* bias, float* logits, int32_t* idx, float* w, cudaStream_t st) {
+  if (c.T == 0) return MOE_OK;
+  if (c.dtype == MOE_F32) {
+    const int warps = 4;
+    router_f32_kernel<<<cdiv(c.T, warps), 32 * warps, 0, st>>>(
+        static_cast<const float*>(u), static_cast<const float*>(w_router), bias, c.T, c.d_model,
+        c.n_experts, c.top_k, c.routed_scale, logits, idx, w);
+    return last_launch();
+  }
+  GemmParams p{};
+  p.G = 1;
+  p.M = c.T;
+  p.K = c.d_model;
+  p.Nw = c.n_experts;
+  p.Nout = c.n_experts;
+  p.logits = logits;
+  p.topk_idx = idx;
+  p.topk_w = w;
+  p.bias = bias;
+  p.top_k = c.top_k;
+  p.routed_scale = c.routed_scale;
+  const int bn = c.n_experts <= 32 ? 32 : c.n_experts <= 64 ? 64 : c.n_experts <= 128 ? 128 : 256;
+  return run_gemm(EPI_ROUTER, Orient::kNormal, bn, u, c.T, w_router, c.n_experts, p, st);
+}
+
+moe_status_t do_permute(const moe_config_t& c, const int32_t* idx, int32_t* offsets,
+                        int32_t* perm, int32_t* inv, const void* x, const float* gamma_pre,
+                        void* x_perm, int32_t* counts, cudaStream_t st) {
+  const int n = c.n_experts, k = c.top_k, nc = nchunks(c);
+  if (c.T == 0) {
+    cudaMemsetAsync(offsets, 0, (n + 1) * sizeof(int32_t), st);
+    return last_launch();
+  }
+  perm_count_kernel<<<nc, 256, 0, st>>>(idx, c.T, k, n, counts);
+  perm_scan_kernel<<<1, kMaxExperts, 0, st>>>(counts, nc, n, offsets);
+  perm_rank_kernel<<<nc, 256, 0, st>>>(idx, c.T, k, n, counts, offsets, perm, inv);
+  moe_status_t s = last_launch();
+  if (s != MOE_OK || !x) return s;
+  const int E = c.d_latent > 0 ? c.d_latent : c.d_model;
+  if (c.dtype == MOE_F32) {
+    scatter_rows_f32_kernel<float><<<c.T, 128, 0, st>>>(static_cast<const float*>(x), E, k, inv,
+                                                        static_cast<float*>(x_perm));
+    return last_launch();
+  }
+  const int nvec = E / 8;
+  const int threads = nvec >= 256 ? 256 : ((nvec + 31) / 32) * 32;
+  const int vec = cdiv(nvec, threads);
+  const uint16_t* xs = static_cast<const uint16_t*>(x);
+  uint16_t* xp = static_cast<uint16_t*>(x_perm);
+  switch (vec) {
+    case 1: scatter_rows_bf16_kernel<1><<<c.T, threads, 0, st>>>(xs, E, k, inv, gamma_pre, c.eps, xp); break;
+    case 2: scatter_rows_bf16_kernel<2><<<c.T, threads, 0, st>>>(xs, E, k, inv, gamma_pre, c.eps, xp); break;
+    case 3:
+    case 4: scatter_rows_bf16_kernel<4><<<c.T, threads, 0, st>>>(xs, E, k, inv, gamma_pre, c.eps, xp); break;
+    default: return MOE_ERR_UNSUPPORTED;
+  }
+  return last_launch();
+}
+
+moe_status_t do_experts(const moe_config_t& c, const void* x_perm, const int32_t* offsets,
+                        const void* w_gu, const void* w_down, const float* gamma_e,
+                        void* out_perm, void* act, cudaStream_t st) {
+  const long TK = static_cast<long>(c.T) * c.top_k;
+  if (TK == 0) return MOE_OK;
+  const int E = expert_in(c), H = c.d_ff, n = c.n_experts;
+  if (c.dtype == MOE_F32) {
+    const size_t smem = static_cast<size_t>(E + H) * sizeof(float);
+    if (smem > 48 * 1024) return MOE_ERR_UNSUPPORTED;
+    expert_ffn_f32_kernel<<<static_cast<unsigned>(TK), 128, smem, st>>>(
+        static_cast<const float*>(x_perm), offsets, n, E, H, c.expert_act,
+        static_cast<const float*>(w_gu), static_cast<const float*>(w_down),
+        c.expert_norm ? gamma_e : nullptr, static_cast<float*>(out_perm));
+    return last_launch();
+  }
+  const bool swiglu = c.expert_act == MOE_ACT_SWIGLU;
+  // first GEMM: x_perm [TK, E] x W_gu[e]^T -> act [TK, H]
+  GemmParams p1{};
+  p1.seg = offsets;
+  p1.G = n;
+  p1.K = E;
+  p1.Nw = gu_rows(c);
+  p1.Nout = H;
+  p1.out = act;
+  Orient o1;
+  int bn1;
+  pick_expert_orient(c, H, swiglu, &o1, &bn1);
+  if (bn1 == 0) return MOE_ERR_UNSUPPORTED;
+  moe_status_t s = run_gemm(swiglu ? EPI_SWIGLU : EPI_RELU, o1, bn1, x_perm, TK, w_gu,
+                            static_cast<long>(n) * p1.Nw, p1, st);
+  if (s != MOE_OK) return s;
+  // second GEMM: act [TK, H] x W_down[e]^T -> out [TK, E] (scaled by 1 + gamma for I_gamma)
+  GemmParams p2{};
+  p2.seg = offsets;
+  p2.G = n;
+  p2.K = H;
+  p2.Nw = E;
+  p2.Nout = E;
+  p2.out = out_perm;
+  p2.gamma = c.expert_norm ? gamma_e : nullptr;
+  Orient o2;
+  int bn2;
+  pick_expert_orient(c, E, false, &o2, &bn2);
+  if (bn2 == 0) return MOE_ERR_UNSUPPORTED;
+  return run_gemm(EPI_STORE, o2, bn2, act, TK, w_down, static_cast<long>(n) * E, p2, st);
+}
+
+moe_status_t do_combine(const moe_config_t& c, const void* s, const int32_t* inv,
+                        const float* w, void* y, cudaStream_t st) {
+  if (c.T == 0) return MOE_OK;
+  const int E = expert_in(c);
+  if (c.dtype == MOE_F32) {
+    combine_f32_kernel<<<c.T, 128, 0, st>>>(static_cast<const float*>(s), E, c.top_k, inv, w,
+                                            c.expert_norm, c.eps, static_cast<float*>(y));
+    return last_launch();
+  }
+  const int nvec = E / 8;
+  const int threads = nvec >= 256 ? 256 : ((nvec + 31) / 32) * 32;
+  const int vec = cdiv(nvec, threads);
+  const uint16_t* sp = static_cast<const uint16_t*>(s);
+  uint16_t* yp = static_cast<uint16_t*>(y);
+  switch (vec) {
+    case 1: combine_bf16_kernel<1><<<c.T, threads, 0, st>>>(sp, E, c.top_k, inv, w, c.expert_norm, c.eps, yp); break;
+    case 2: combine_bf16_kernel<2><<<c.T, threads, 0, st>>>(sp, E, c.top_k, inv, w, c.expert_norm, c.eps, yp); break;
+    case 3:
+    case 4: combine_bf16_kernel<4><<<c.T, threads, 0, st>>>(sp, E, c.top_k, inv, w, c.expert_norm, c.eps, yp); break;
+    default: return MOE_ERR_UNSUPPORTED;
+  }
+  return last_launch();
+}
+
+moe_status_t do_latent_down(const moe_config_t& c, const void* u, const void* p_down, void* z,
+                            cudaStream_t st) {
+  if (c.T == 0) return MOE_OK;
+  GemmParams p{};
+  p.G = 1;
+  p.M = c.T;
+  p.K = c.d_model;
+  p.Nw = c.d_latent;
+  p.Nout = c.d_latent;
+  p.out = z;
+  return run_gemm(EPI_STORE, Orient::kNormal, pick_bn_normal(c.d_latent, false), u, c.T, p_down,
+                  c.d_latent, p, st);
+}
+
+moe_status_t do_latent_up(const moe_config_t& c, const void* y, const void* p_up, const void* r,
+                          const float* g, void* out, cudaStream_t st) {
+  if (c.T == 0) return MOE_OK;
+  GemmParams p{};
+  p.G = 1;
+  p.M = c.T;
+  p.K = c.d_latent;
+  p.Nw = c.d_model;
+  p.Nout = c.d_model;
+  p.out = out;
+  p.resid = static_cast<const uint16_t*>(r);
+  p.gparam = g;
+  p.tau = c.tau;
+  p.floor_ = c.resid_floor;
+  p.resid_mode = c.resid_mode;
+  return run_gemm(EPI_RESGATE, Orient::kNormal, pick_bn_normal(c.d_model, false), y, c.T, p_up,
+                  c.d_model, p, st);
+}
+
+}  // namespace
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+const char* moe_status_string(moe_status_t s) {
+  switch (s) {
+    case MOE_OK: return "MOE_OK";
+    case MOE_ERR_INVALID_ARG: return "MOE_ERR_INVALID_ARG: invalid argument";
+    case MOE_ERR_UNSUPPORTED: return "MOE_ERR_UNSUPPORTED: shape or mode not supported";
+    case MOE_ERR_ALIGNMENT: return "MOE_ERR_ALIGNMENT: pointer not 16-byte aligned";
+    case MOE_ERR_WORKSPACE: return "MOE_ERR_WORKSPACE: workspace missing or too small";
+    case MOE_ERR_CUDA: return "MOE_ERR_CUDA: CUDA call failed";
+    case MOE_ERR_TIMEOUT: return "MOE_ERR_TIMEOUT: a bounded wait inside a kernel ran out";
+    case MOE_ERR_DEVICE_CHECK: return "MOE_ERR_DEVICE_CHECK: device-side index check failed";
+  }
+  return "unknown moe_status_t";
+}
+
+moe_status_t moe_workspace_size(const moe_config_t* cfg, size_t* bytes) {
+  moe_status_t s = check_cfg(cfg);
+  if (s != MOE_OK) return s;
+  if (!bytes) return MOE_ERR_INVALID_ARG;
+  *bytes = layout(*cfg).total;
+  return MOE_OK;
+}
+
+moe_status_t moe_route(const moe_config_t* cfg, const void* u, const void* w_router,
+                       const float* logit_bias, float* logits_out, int32_t* topk_idx,
+                       float* topk_w, void* stream) {
+  moe_status_t s = check_cfg(cfg);
+  if (s != MOE_OK) return s;
+  if (cfg->T > 0 && (!u || !w_router || !topk_idx || !topk_w)) return MOE_ERR_INVALID_ARG;
+  if (!all_aligned({u, w_router, static_cast<const void*>(logit_bias),
+                        static_cast<const void*>(logits_out), static_cast<const void*>(topk_idx),
+                        static_cast<const void*>(topk_w)})) return MOE_ERR_ALIGNMENT;
+  return do_route(*cfg, u, w_router, logit_bias, logits_out, topk_idx, topk_w,
+                  static_cast<cudaStream_t>(stream));
+}
+
+moe_status_t moe_permute(const moe_config_t* cfg, const int32_t* topk_idx,
+                         int32_t* expert_offsets, int32_t* perm_token, int32_t* inv_perm,
+                         const void* x, const float* gamma_pre, void* x_perm, void* workspace,
+                         size_t workspace_bytes, void* stream) {
+  moe_status_t s = check_cfg(cfg);
+  if (s != MOE_OK) return s;
+  if (!expert_offsets || (cfg->T > 0 && (!topk_idx || !perm_token || !inv_perm)))
+    return MOE_ERR_INVALID_ARG;
+  if (x && !x_perm) return MOE_ERR_INVALID_ARG;
+  if (gamma_pre && (cfg->dtype != MOE_BF16 || cfg->d_latent == 0)) return MOE_ERR_UNSUPPORTED;
+  if (!all_aligned({static_cast<const void*>(topk_idx), static_cast<const void*>(expert_offsets),
+                        static_cast<const void*>(perm_token), static_cast<const void*>(inv_perm), x,
+                        static_cast<const void*>(gamma_pre), x_perm, workspace})) return MOE_ERR_ALIGNMENT;
+  const size_t need = static_cast<size_t>(nchunks(*cfg)) * cfg->n_experts * 4;
+  if (cfg->T > 0 && (!workspace || workspace_bytes < need)) return MOE_ERR_WORKSPACE;
+  return do_permute(*cfg, topk_idx, expert_offsets, perm_token, inv_perm, x, gamma_pre, x_perm,
+                    static_cast<int32_t*>(workspace), static_cast<cudaStream_t>(stream));
+}
+
+moe_status_t moe_expert_ffn(const moe_config_t* cfg, const void* x_perm,
+                            const int32_t* expert_offsets, const void* w_gu, const void* w_down,
+                            const float* gamma_expert, void* out_perm, void* workspace,
+                            size_t workspace_bytes, void* stream) {
+  moe_status_t s = check_cfg(cfg);
+  if (s != MOE_OK) return s;
+  const size_t TK = static_cast<size_t>(cfg->T) * cfg->top_k;
+  if (TK > 0 && (!x_perm || !expert_offsets || !w_gu || !w_down || !out_perm))
+    return MOE_ERR_INVALID_ARG;
+  if (cfg->expert_norm && TK > 0 && !gamma_expert) return MOE_ERR_INVALID_ARG;
+  if (!all_aligned({x_perm, static_cast<const void*>(expert_offsets), w_gu, w_down,
+                        static_cast<const void*>(gamma_expert), out_perm, workspace})) return MOE_ERR_ALIGNMENT;
+  const size_t need = TK * cfg->d_ff * dsize(*cfg);
+  if (cfg->dtype == MOE_BF16 && TK > 0 && (!workspace || workspace_bytes < need))
+    return MOE_ERR_WORKSPACE;
+  return do_experts(*cfg, x_perm, expert_offsets, w_gu, w_down, gamma_expert, out_perm, workspace,
+                    static_cast<cudaStream_t>(stream));
+}
+
+moe_status_t moe_combine(const moe_config_t* cfg, const void* out_perm, const int32_t* inv_perm,
+                         const float* topk_w, void* y, void* stream) {
+  moe_status_t s = check_cfg(cfg);
+  if (s != MOE_OK) return s;
+  if (cfg->T > 0 && (!out_perm || !inv_perm || !topk_w || !y)) return MOE_ERR_INVALID_ARG;
+  if (!all_aligned({out_perm, static_cast<const void*>(inv_perm),
+                        static_cast<const void*>(topk_w), static_cast<const void*>(y)})) return MOE_ERR_ALIGNMENT;
+  return do_combine(*cfg, out_perm, inv_perm, topk_w, y, static_cast<cudaStream_t>(stream));
+}
+
+moe_status_t moe_latent_down(const moe_config_t* cfg, const void* u, const void* p_down,
+                             void* z_raw, void* stream) {
+  moe_status_t s = check_cfg(cfg);
+  if (s != MOE_OK) return s;
+  if (cfg->d_latent == 0 || cfg->dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
+  if (cfg->T > 0 && (!u || !p_down || !z_raw)) return MOE_ERR_INVALID_ARG;
+  if (!all_aligned({u, p_down, static_cast<const void*>(z_raw)})) return MOE_ERR_ALIGNMENT;
+  return do_latent_down(*cfg, u, p_down, z_raw, static_cast<cudaStream_t>(stream));
+}
+
+moe_status_t moe_latent_up(const moe_config_t* cfg, const void* y, const void* p_up,
+                           const void* r, const float* resid_g, void* out, void* stream) {
+  moe_status_t s = check_cfg(cfg);
+  if (s != MOE_OK) return s;
+  if (cfg->d_latent == 0 || cfg->dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
+  if (cfg->T > 0 && (!y || !p_up || !out)) return MOE_ERR_INVALID_ARG;
+  if (cfg->T > 0 && cfg->resid_mode != MOE_RESID_NONE && (!r || !resid_g)) return MOE_ERR_INVALID_ARG;
+  if (!all_aligned({y, p_up, r, static_cast<const void*>(resid_g), static_cast<const void*>(out)})) return MOE_ERR_ALIGNMENT;
+  return do_latent_up(*cfg, y, p_up, r, resid_g, out, static_cast<cudaStream_t>(stream));
+}
+
+moe_status_t moe_layer_forward(const moe_config_t* cfg, const moe_weights_t* w, const void* u,
+                               const void* r, void* out, float* logits_out,
+                               int32_t* topk_idx_out, float* topk_w_out, void* workspace,
+                               size_t workspace_bytes, void* stream) {
+  moe_status_t s = check_cfg(cfg);
+  if (s != MOE_OK) return s;
+  const moe_config_t& c = *cfg;
+  if (!w) return MOE_ERR_INVALID_ARG;
+  if (c.T == 0) return MOE_OK;
+  const bool latent = c.d_latent > 0;
+  if (!u || !out || !w->w_router || !w->w_gu || !w->w_down) return MOE_ERR_INVALID_ARG;
+  if (latent && (!w->p_down || !w->p_up)) return MOE_ERR_INVALID_ARG;
+  if (c.pre_norm && !w->gamma_pre) return MOE_ERR_INVALID_ARG;
+  if (c.expert_norm && !w->gamma_expert) return MOE_ERR_INVALID_ARG;
+  if (c.resid_mode != MOE_RESID_NONE && (!r || !w->resid_g)) return MOE_ERR_INVALID_ARG;
+  if (!all_aligned({u, r, static_cast<const void*>(out), static_cast<const void*>(logits_out),
+                        static_cast<const void*>(topk_idx_out), static_cast<const void*>(topk_w_out),
+                        workspace, w->w_router, w->p_down, w->p_up, w->w_gu, w->w_down,
+                        static_cast<const void*>(w->gamma_pre),
+                        static_cast<const void*>(w->gamma_expert),
+                        static_cast<const void*>(w->resid_g), static_cast<const void*>(w->logit_bias)})) return MOE_ERR_ALIGNMENT;
+  const Workspace L = layout(c);
+  if (!workspace || workspace_bytes < L.total) return MOE_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int32_t* idx = topk_idx_out ? topk_idx_out : at<int32_t>(workspace, L.idx);
+  float* wt = topk_w_out ? topk_w_out : at<float>(workspace, L.w);
+  int32_t* offsets = at<int32_t>(workspace, L.offsets);
+  int32_t* perm = at<int32_t>(workspace, L.perm);
+  int32_t* inv = at<int32_t>(workspace, L.inv);
+  void* x_perm = at<void>(workspace, L.x_perm);
+  void* act = at<void>(workspace, L.act);
+
+  if ((s = do_route(c, u, w->w_router, w->logit_bias, logits_out, idx, wt, st)) != MOE_OK) return s;
+  const void* xin = u;
+  if (latent) {
+    void* z = at<void>(workspace, L.z_raw);
+    if ((s = do_latent_down(c, u, w->p_down, z, st)) != MOE_OK) return s;
+    xin = z;
+  }
+  if ((s = do_permute(c, idx, offsets, perm, inv, xin, c.pre_norm ? w->gamma_pre : nullptr, x_perm,
+                      at<int32_t>(workspace, L.counts), st)) != MOE_OK)
+    return s;
+  // The expert output overwrites the dispatched input rows (no longer needed after GEMM 1).
+  if ((s = do_experts(c, x_perm, offsets, w->w_gu, w->w_down, w->gamma_expert, x_perm, act, st)) !=
+      MOE_OK)
+    return s;
+  if (!latent) return do_combine(c, x_perm, inv, wt, out, st);
+  void* y = at<void>(workspace, L.y);
+  if ((s = do_combine(c, x_perm, inv, wt, y, st)) != MOE_OK) return s;
+  return do_latent_up(c, y, w->p_up, r, w->resid_g, out, st);
+}
+
+moe_status_t moe_get_device_status(void* stream) {
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return MOE_ERR_CUDA;
+  int v = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&v, g_status, sizeof(int)) != cudaSuccess) return MOE_ERR_CUDA;
+  if (v != 0 && cudaMemcpyToSymbol(g_status, &zero, sizeof(int)) != cudaSuccess) return MOE_ERR_CUDA;
+  return static_cast<moe_status_t>(v);
+}
+
+}  // extern "C"

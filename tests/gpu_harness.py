@@ -1,0 +1,113 @@
+"""Helpers shared by the GPU parity tests, the smoke check and the benchmark.
+
+Inputs come from the seeded generator only (device copies generated on the device, host copies
+on the host, bit-identical).  Expected values come from the CPU oracle only.  The CUDA path is
+called through the C ABI (the ctypes binding of libmoe.so).
+"""
+from __future__ import annotations
+
+import numpy as np
+
+import moe_inputs
+import sparse_moe_layer_softmax_b200 as moe
+from moe_inputs import configs
+
+BF16_TOL = 2e-2   # max over tokens of |out - ref|_inf / |ref|_inf, bf16 storage
+F32_TOL = 1e-4    # same for fp32 storage
+
+
+def abi_config(cfg, T: int | None = None):
+    return moe.make_config(
+        T=cfg.T if T is None else T, d_model=cfg.d_model, n_experts=cfg.n_experts,
+        top_k=cfg.top_k, d_ff=cfg.d_ff, d_latent=cfg.d_latent,
+        dtype=moe.MOE_BF16 if cfg.dtype == "bf16" else moe.MOE_F32, expert_act=cfg.act,
+        pre_norm=cfg.pre_norm, expert_norm=cfg.expert_norm, resid_mode=cfg.resid_mode,
+        eps=cfg.eps, tau=cfg.tau, resid_floor=cfg.resid_floor, routed_scale=cfg.routed_scale)
+
+
+def host_values(a: np.ndarray, dtype: str) -> np.ndarray:
+    """float64 values of host tensors (bf16 codes or float32)."""
+    if dtype == "bf16":
+        return (a.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    return a.astype(np.float64)
+
+
+def device_values(t) -> np.ndarray:
+    """float64 values of a CUDA tensor (bf16 or fp32)."""
+    import torch
+    return t.detach().to(torch.float32).cpu().numpy().astype(np.float64)
+
+
+def row_rel_err(got: np.ndarray, ref: np.ndarray) -> np.ndarray:
+    """Per-row |got - ref|_inf / |ref|_inf."""
+    num = np.max(np.abs(got - ref), axis=-1)
+    den = np.maximum(np.max(np.abs(ref), axis=-1), 1e-30)
+    return num / den
+
+
+def tolerance(cfg) -> float:
+    return BF16_TOL if cfg.dtype == "bf16" else F32_TOL
+
+
+def run_layer(cfg, dev: dict, want_logits: bool = True):
+    """moe_layer_forward through the C ABI on device inputs; returns torch tensors."""
+    import torch
+    c = abi_config(cfg)
+    layer = moe.MoELayer(c, dev)
+    u = dev["u"]
+    out = torch.empty_like(u)
+    logits = torch.empty((cfg.T, cfg.n_experts), dtype=torch.float32, device="cuda") \
+        if want_logits else None
+    idx = torch.empty((cfg.T, cfg.top_k), dtype=torch.int32, device="cuda")
+    w = torch.empty((cfg.T, cfg.top_k), dtype=torch.float32, device="cuda")
+    layer.forward(u, u, out=out, logits_out=logits, topk_idx_out=idx, topk_w_out=w)
+    status = moe.moe_get_device_status()
+    assert status == 0, f"device status {moe.STATUS.get(status, status)}"
+    return {"out": out, "logits": logits, "idx": idx, "w": w, "layer": layer}
+
+
+def oracle_reference(cfg, tokens=None):
+    """Oracle layer outputs for the listed tokens (all by default).  Small workloads hold every
+    tensor on the host; large ones evaluate one expert's weights at a time."""
+    import oracle
+    big = cfg.n_experts * cfg.gu_rows * cfg.expert_in > 64 * 1024 * 1024
+    if not big:
+        inp = moe_inputs.host_inputs(cfg)
+        return oracle.layer_forward(cfg, inp, tokens=tokens)
+    tokens = np.arange(cfg.T) if tokens is None else np.asarray(tokens)
+
+    def get_inputs(tk):
+        d = {"u": moe_inputs.host_rows(cfg, "u", rows=tk)}
+        for name in moe_inputs.tensor_specs(cfg):
+            if name not in ("u", "w_gu", "w_down"):
+                d[name] = moe_inputs.host_rows(cfg, name)
+        if cfg.zipf_bias:
+            d["logit_bias"] = moe_inputs.zipf_bias(cfg)
+        return d
+
+    def get_expert(e):
+        return (moe_inputs.host_rows(cfg, "w_gu", lead=e), moe_inputs.host_rows(cfg, "w_down", lead=e))
+
+    return oracle.layer_forward_staged(cfg, tokens, get_inputs, get_expert)
+
+
+def check_routing(cfg, logits_gpu: np.ndarray, idx_gpu: np.ndarray, w_gpu: np.ndarray):
+    """Bit-exact routing on every token: the oracle's selection run on the GPU's fp32 logits must
+    equal the GPU's indices; weights within 1e-6 relative; permutation bit-exact."""
+    import oracle
+    sel, wref = oracle.softmax_topk(logits_gpu.astype(np.float32), cfg.top_k, cfg.routed_scale)
+    np.testing.assert_array_equal(idx_gpu, sel)
+    np.testing.assert_allclose(w_gpu, wref, rtol=1e-6, atol=1e-7)
+    np.testing.assert_allclose(w_gpu.sum(1), cfg.routed_scale, rtol=2e-6)
+
+
+def near_tie_tokens(logits_ref: np.ndarray, k: int, rel: float = 1e-4) -> np.ndarray:
+    """Tokens whose k-th and (k+1)-th largest oracle logits are closer than rel * rms(logits):
+    fp32 and double accumulation may order them differently, so their selection is not unique."""
+    n = logits_ref.shape[1]
+    if k >= n:
+        return np.zeros(len(logits_ref), dtype=bool)
+    s = -np.sort(-logits_ref, axis=1)
+    margin = s[:, k - 1] - s[:, k]
+    rms = np.sqrt(np.mean(logits_ref ** 2, axis=1))
+    return margin < rel * rms

@@ -1,0 +1,277 @@
+"""Parity of the CUDA path (called through the C ABI) with the CPU oracle on seeded inputs.
+
+Routing indices and the dispatch permutation are compared bit for bit; values within the
+tolerance of the storage dtype (max over tokens of |out - ref|_inf / |ref|_inf <= 2e-2 for bf16,
+1e-4 for fp32, against the double-accumulating oracle).
+"""
+import numpy as np
+import pytest
+
+import moe_inputs
+import oracle
+from moe_inputs import configs
+
+from gpu_harness import (abi_config, check_routing, device_values, host_values, near_tie_tokens,
+                         oracle_reference, row_rel_err, run_layer, tolerance)
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+moe = pytest.importorskip("sparse_moe_layer_softmax_b200")
+
+
+@pytest.fixture(autouse=True)
+def _cuda_cleanup():
+    yield
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+
+
+# ------------------------------------------------------------------ input generator
+
+
+def test_generator_device_matches_host():
+    for seed, stream, first, count, sigma in ((0, 1, 0, 100003, 1.0), (3, 5, 12345, 4099, 0.02),
+                                              (4, 6, 1 << 33, 777, 0.5)):
+        t = torch.empty(count, dtype=torch.bfloat16, device="cuda")
+        moe_inputs.normal_device(t, seed, stream, first, sigma)
+        h = moe_inputs.normal_host(seed, stream, first, count, sigma, "bf16")
+        np.testing.assert_array_equal(t.view(torch.int16).cpu().numpy().view(np.uint16), h)
+        f = torch.empty(count, dtype=torch.float32, device="cuda")
+        moe_inputs.normal_device(f, seed, stream, first, sigma)
+        np.testing.assert_array_equal(f.cpu().numpy(), moe_inputs.normal_host(seed, stream, first,
+                                                                             count, sigma, "f32"))
+        moe_inputs.uniform_device(f, seed, stream, first)
+        np.testing.assert_array_equal(f.cpu().numpy(), moe_inputs.uniform_host(seed, stream, first,
+                                                                              count))
+
+
+# ------------------------------------------------------------------ whole layer, small shapes
+
+SMALL = [
+    # normal orientation, ragged T, several M tiles, Muse structure
+    configs.small_muse(T=300, d=512, L=256, I=256, n=16, k=4, seed=11),
+    # swap orientation (few rows per expert), max experts and top-k
+    configs.small_muse(T=40, d=256, L=128, I=128, n=256, k=8, seed=12),
+    configs.small_muse(T=77, d=256, L=256, I=128, n=64, k=8, seed=13),
+    # residual variants and no pre-norm
+    configs.small_muse(T=130, d=256, L=128, I=192, n=8, k=2, seed=14,
+                       resid_mode=configs.RESID_LITERAL),
+    configs.small_muse(T=65, d=192, L=128, I=128, n=8, k=3, seed=15, pre_norm=0,
+                       resid_mode=configs.RESID_NONE),
+    # k = 1 (one-hot gate) and k = n (dense softmax mixture)
+    configs.small_muse(T=129, d=256, L=128, I=128, n=8, k=1, seed=16),
+    configs.small_muse(T=50, d=256, L=128, I=128, n=8, k=8, seed=17),
+    # Shazeer structure in bf16 (ReLU experts, no latent, no norm)
+    configs.small_shazeer(T=257, d=128, h=256, n=16, k=4, seed=18),
+    configs.small_shazeer(T=33, d=256, h=512, n=64, k=2, seed=19),
+    # fp32 CUDA-core path
+    configs.TINY_SHAZEER_F32.replace(T=45, seed=20),
+    configs.TINY_SHAZEER_F32.replace(T=64, top_k=8, seed=21),
+]
+
+
+@pytest.mark.parametrize("cfg", SMALL, ids=lambda c: f"{c.name}-n{c.n_experts}k{c.top_k}-{c.dtype}"
+                         f"-r{c.resid_mode}p{c.pre_norm}")
+def test_layer_small(cfg):
+    dev = moe_inputs.device_inputs(cfg)
+    res = run_layer(cfg, dev)
+    ref = oracle_reference(cfg)
+    logits = res["logits"].cpu().numpy()
+    idx = res["idx"].cpu().numpy()
+    check_routing(cfg, logits, idx, res["w"].cpu().numpy())
+    ties = near_tie_tokens(ref["logits"], cfg.top_k)
+    assert ties.sum() <= max(1, cfg.T // 100)
+    np.testing.assert_array_equal(idx[~ties], ref["idx"][~ties])
+    np.testing.assert_allclose(logits, ref["logits"], rtol=0,
+                               atol=1e-5 * max(1.0, np.abs(ref["logits"]).max()))
+    err = row_rel_err(device_values(res["out"])[~ties], ref["out"][~ties])
+    assert err.max() <= tolerance(cfg), f"max row error {err.max():.3e}"
+
+
+# ------------------------------------------------------------------ individual entry points
+
+
+def _rand_routing(T, n, k, seed, hot=None):
+    rng = np.random.default_rng(seed)
+    p = None
+    if hot is not None:
+        p = np.full(n, (1 - hot) / (n - 1))
+        p[0] = hot
+    return np.stack([rng.choice(n, size=k, replace=False, p=p) for _ in range(T)]).astype(np.int32)
+
+
+@pytest.mark.parametrize("T,n,k,hot", [(1, 4, 2, None), (129, 16, 4, None), (1000, 256, 8, None),
+                                       (513, 64, 3, 0.9), (300, 256, 1, None), (64, 8, 8, None)])
+def test_permute_bit_exact(T, n, k, hot):
+    cfg = configs.small_muse(T=T, n=n, k=k)
+    c = abi_config(cfg)
+    idx = _rand_routing(T, n, k, seed=T + n, hot=hot)
+    d_idx = torch.from_numpy(idx).cuda()
+    off = torch.full((n + 1,), -7, dtype=torch.int32, device="cuda")
+    perm = torch.full((T * k,), -7, dtype=torch.int32, device="cuda")
+    inv = torch.full((T * k,), -7, dtype=torch.int32, device="cuda")
+    ws = torch.empty(moe.workspace_size(c), dtype=torch.uint8, device="cuda")
+    moe.moe_permute(c, d_idx, off, perm, inv, workspace=ws)
+    assert moe.moe_get_device_status() == 0
+    r_off, r_perm, r_inv = oracle.permutation(T, k, n, idx)
+    np.testing.assert_array_equal(off.cpu().numpy(), r_off)
+    np.testing.assert_array_equal(perm.cpu().numpy(), r_perm)
+    np.testing.assert_array_equal(inv.cpu().numpy(), r_inv)
+
+
+def test_permute_empty_and_bad_index():
+    cfg = configs.small_muse(T=0, n=16, k=4)
+    c = abi_config(cfg)
+    off = torch.full((17,), -7, dtype=torch.int32, device="cuda")
+    ws = torch.empty(64, dtype=torch.uint8, device="cuda")
+    moe.moe_permute(c, None, off, None, None, workspace=ws)
+    assert moe.moe_get_device_status() == 0
+    assert (off.cpu().numpy() == 0).all()
+    # an out-of-range expert index is latched as a device check error and the slot dropped
+    cfg = configs.small_muse(T=3, n=4, k=2)
+    c = abi_config(cfg)
+    idx = torch.tensor([[0, 1], [2, 9], [3, 0]], dtype=torch.int32, device="cuda")
+    off = torch.zeros(5, dtype=torch.int32, device="cuda")
+    perm = torch.zeros(6, dtype=torch.int32, device="cuda")
+    inv = torch.zeros(6, dtype=torch.int32, device="cuda")
+    ws = torch.empty(moe.workspace_size(c), dtype=torch.uint8, device="cuda")
+    moe.moe_permute(c, idx, off, perm, inv, workspace=ws)
+    assert moe.moe_get_device_status() == moe.STATUS_CODES["MOE_ERR_DEVICE_CHECK"]
+    assert moe.moe_get_device_status() == 0  # cleared by the read
+    assert off.cpu().numpy().tolist() == [0, 2, 3, 4, 5]
+    assert inv.cpu().numpy()[3] == -1
+
+
+@pytest.mark.parametrize("E,gamma", [(256, True), (4096, True), (512, False), (8192, True)])
+def test_scatter_rows_with_centred_norm(E, gamma):
+    T, n, k = 37, 8, 3
+    cfg = configs.small_muse(T=T, d=E, L=E, I=128, n=n, k=k)
+    c = abi_config(cfg)
+    x_h = moe_inputs.normal_host(5, 40, 0, T * E, 1.7, "bf16").reshape(T, E)
+    g_h = moe_inputs.normal_host(5, 41, 0, E, 0.3, "f32")
+    idx = _rand_routing(T, n, k, seed=E)
+    x = torch.from_numpy(x_h.view(np.int16)).view(torch.bfloat16).cuda()
+    g = torch.from_numpy(g_h).cuda()
+    off = torch.empty(n + 1, dtype=torch.int32, device="cuda")
+    perm = torch.empty(T * k, dtype=torch.int32, device="cuda")
+    inv = torch.empty(T * k, dtype=torch.int32, device="cuda")
+    xp = torch.empty((T * k, E), dtype=torch.bfloat16, device="cuda")
+    ws = torch.empty(moe.workspace_size(c), dtype=torch.uint8, device="cuda")
+    moe.moe_permute(c, torch.from_numpy(idx).cuda(), off, perm, inv, x=x,
+                    gamma_pre=g if gamma else None, x_perm=xp, workspace=ws)
+    assert moe.moe_get_device_status() == 0
+    xv = host_values(x_h, "bf16")
+    _, _, r_inv = oracle.permutation(T, k, n, idx)
+    got = device_values(xp)
+    for t in range(T):
+        ref = oracle.centered_rmsnorm(xv[t], g_h.astype(np.float64), cfg.eps) if gamma else xv[t]
+        ref = oracle.bf16_round(ref)
+        for j in range(k):
+            row = got[r_inv[t * k + j]]
+            if gamma:
+                assert row_rel_err(row, ref) <= 1e-2
+            else:
+                np.testing.assert_array_equal(row, ref)
+
+
+@pytest.mark.parametrize("cfg", [
+    configs.small_muse(T=200, d=256, L=256, I=384, n=8, k=2, seed=31),    # normal orientation
+    configs.small_muse(T=24, d=256, L=256, I=256, n=64, k=8, seed=32),    # swap orientation
+    configs.small_shazeer(T=300, d=128, h=256, n=8, k=2, seed=33),
+    configs.small_shazeer(T=20, d=128, h=256, n=64, k=4, seed=34),
+], ids=lambda c: f"{c.name}-n{c.n_experts}k{c.top_k}-act{c.act}")
+def test_expert_ffn(cfg):
+    """Experts on dispatched rows (inputs from the generator, routing synthetic)."""
+    c = abi_config(cfg)
+    T, k, n, E, H = cfg.T, cfg.top_k, cfg.n_experts, cfg.expert_in, cfg.d_ff
+    idx = _rand_routing(T, n, k, seed=cfg.seed)
+    off, perm, inv = oracle.permutation(T, k, n, idx)
+    xh = moe_inputs.normal_host(cfg.seed, 50, 0, T * k * E, 1.0, "bf16").reshape(T * k, E)
+    gam = moe_inputs.host_rows(cfg, "gamma_expert") if cfg.expert_norm else None
+    w_gu = moe_inputs.host_rows(cfg, "w_gu")
+    w_dn = moe_inputs.host_rows(cfg, "w_down")
+    dev = moe_inputs.device_inputs(cfg)
+    x = torch.from_numpy(xh.view(np.int16)).view(torch.bfloat16).cuda()
+    out = torch.empty((T * k, E), dtype=torch.bfloat16, device="cuda")
+    ws = torch.empty(moe.workspace_size(c), dtype=torch.uint8, device="cuda")
+    moe.moe_expert_ffn(c, x, torch.from_numpy(off).cuda(), dev["w_gu"], dev["w_down"],
+                       dev.get("gamma_expert"), out, workspace=ws)
+    assert moe.moe_get_device_status() == 0
+    got = device_values(out)
+    oc = oracle.make_cfg(cfg.replace(expert_norm=0))
+    xv = host_values(xh, "bf16")
+    errs = []
+    for e in range(n):
+        rows = np.arange(off[e], off[e + 1])
+        if len(rows) == 0:
+            continue
+        ref = np.zeros((len(rows), E))
+        wg = np.ascontiguousarray(w_gu[e])
+        wd = np.ascontiguousarray(w_dn[e])
+        zr = np.ascontiguousarray(xv[rows])
+        oracle.lib().orc_expert_batch(oracle.ctypes.byref(oc), wg.ctypes.data, wd.ctypes.data, None,
+                                      zr.ctypes.data, len(rows), ref.ctypes.data, 4)
+        if gam is not None:  # the kernel stores dtype((1 + gamma) * o), the vector I_gamma reduces
+            ref = oracle.bf16_round(ref * (1.0 + gam.astype(np.float64)))
+        errs.append(row_rel_err(got[rows], ref))
+    assert np.concatenate(errs).max() <= 2e-2
+
+
+@pytest.mark.parametrize("E,k,norm", [(128, 4, 1), (4096, 8, 1), (512, 4, 0), (1024, 1, 1)])
+def test_combine(E, k, norm):
+    T, n = 45, 16
+    cfg = configs.small_muse(T=T, d=E, L=E, I=128, n=n, k=k, expert_norm=norm)
+    c = abi_config(cfg)
+    idx = _rand_routing(T, n, k, seed=E + k)
+    _, _, inv = oracle.permutation(T, k, n, idx)
+    sh = moe_inputs.normal_host(9, 60, 0, T * k * E, 0.8, "bf16").reshape(T * k, E)
+    wr = moe_inputs.uniform_host(9, 61, 0, T * k).reshape(T, k).astype(np.float64) + 0.05
+    wr = (wr / wr.sum(1, keepdims=True)).astype(np.float32)
+    y = torch.empty((T, E), dtype=torch.bfloat16, device="cuda")
+    moe.moe_combine(c, torch.from_numpy(sh.view(np.int16)).view(torch.bfloat16).cuda(),
+                    torch.from_numpy(inv).cuda(), torch.from_numpy(wr).cuda(), y)
+    assert moe.moe_get_device_status() == 0
+    sv = host_values(sh, "bf16")
+    oc = oracle.make_cfg(cfg)
+    got = device_values(y)
+    zero = np.zeros(E)
+    for t in range(T):
+        ns = np.zeros((k, E))
+        for j in range(k):
+            s = sv[inv[t * k + j]]
+            ns[j] = oracle.bf16_round(oracle.input_scaled_rmsnorm(s, zero, cfg.eps, 1)) if norm else s
+        ref = np.zeros(E)
+        wj = wr[t].astype(np.float64)
+        oracle.lib().orc_combine_token(oracle.ctypes.byref(oc), np.ascontiguousarray(ns).ctypes.data,
+                                       wj.ctypes.data, ref.ctypes.data)
+        assert row_rel_err(got[t], ref) <= 1e-2
+
+
+def test_latent_down_and_up():
+    cfg = configs.small_muse(T=150, d=512, L=256, I=128, n=8, k=2, seed=41)
+    c = abi_config(cfg)
+    dev = moe_inputs.device_inputs(cfg)
+    inp = moe_inputs.host_inputs(cfg)
+    z = torch.empty((cfg.T, cfg.d_latent), dtype=torch.bfloat16, device="cuda")
+    moe.moe_latent_down(c, dev["u"], dev["p_down"], z)
+    yh = moe_inputs.normal_host(41, 70, 0, cfg.T * cfg.d_latent, 0.7, "bf16").reshape(cfg.T, -1)
+    out = torch.empty_like(dev["u"])
+    moe.moe_latent_up(c, torch.from_numpy(yh.view(np.int16)).view(torch.bfloat16).cuda(),
+                      dev["p_up"], dev["u"], dev["resid_g"], out)
+    assert moe.moe_get_device_status() == 0
+    oc = oracle.make_cfg(cfg.replace(pre_norm=0))
+    keep = oracle._Keep()
+    x = oracle.make_tensors(cfg, inp, keep)
+    zg, og = device_values(z), device_values(out)
+    yv = host_values(yh, "bf16")
+    for t in range(cfg.T):
+        zr = np.zeros(cfg.d_latent)
+        oracle.lib().orc_expert_input_token(oracle.ctypes.byref(oc), oracle.ctypes.byref(x), t,
+                                            zr.ctypes.data)
+        assert row_rel_err(zg[t], zr) <= 1e-2
+        o = np.zeros(cfg.d_model)
+        yt = np.ascontiguousarray(yv[t])
+        oracle.lib().orc_output_token(oracle.ctypes.byref(oc), oracle.ctypes.byref(x), t,
+                                      yt.ctypes.data, o.ctypes.data)
+        assert row_rel_err(og[t], o) <= 1e-2
