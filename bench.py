@@ -1,0 +1,484 @@
+#!/usr/bin/env python
+"""Throughput of the top-k softmax-routed latent MoE-layer forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step is one moe_layer_forward over one batch of synthetic tokens: route, latent
+down-projection, dispatch, expert gate/up and down GEMMs, normalise + combine, latent
+up-projection with the residual gate.  Rank 0 prints one JSON line.
+
+* value: tokens/s over all ranks (each rank processes the full workload: weak scaling, no
+  data-path collective), from CUDA events around K steps, max over ranks;
+* e2e: the same through the host-memory API (pinned host input -> device -> layer -> host);
+* roofline: the dominant kernel (expert gate/up GEMM) timed live with the library's stage events;
+* cpu_baseline: the CPU oracle on a bounded token sample of the same workload (rank 0, N=1);
+* decode: the T=64 Muse decode workload measured the same way (secondary line item).
+
+--impl reference times the CPU oracle (the only reference this path has) on the same workload,
+metric and unit, a bounded token sample per step.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+sys.path.insert(0, os.path.join(ROOT, "tests"))
+
+METRIC = "MoE-layer tokens/s (Muse shape, T=64 & T=16K) and % of HBM/BF16 roofline"
+UNIT = "tokens/s"
+DEFAULT_WORKLOAD = "muse_prefill"
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--no-decode", action="store_true", help="skip the secondary decode item")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-sample", type=int, default=0, help="tokens in the CPU oracle sample")
+    a = ap.parse_args(argv)
+    if a.warmup < 3:
+        ap.error("at least 3 warm-up steps")
+    return a
+
+
+# ------------------------------------------------------------------ ranks
+
+def dist_env():
+    return (int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)),
+            int(os.environ.get("LOCAL_RANK", 0)))
+
+
+def init_dist(backend: str):
+    import datetime
+    import torch.distributed as dist
+    rank, world, _ = dist_env()
+    if world > 1 and not dist.is_initialized():
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return rank, world
+
+
+def barrier():
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        dist.barrier()
+
+
+def reduce_max(x: float, device=None) -> float:
+    """Max of a float over ranks (identity on one rank)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------ clocks during the timed region
+
+class ClockSampler:
+    """nvidia-smi sampling every 200 ms while the timed region runs."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.3)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        return self.parse(open(self.path).read())
+
+    @staticmethod
+    def parse(text: str) -> dict:
+        sm, mx, reasons, power = [], [], set(), []
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for line in text.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+                power.append(float(f[3]))
+            except ValueError:
+                continue
+            for name, val in zip(names, f[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        busy = [s for s in sm if s > 0.5 * max(sm)] or sm
+        return {"sm_mhz": statistics.median(busy), "sm_max_mhz": max(mx),
+                "power_w_max": max(power), "samples": len(sm), "reasons": sorted(reasons)}
+
+
+def measured_peaks() -> dict:
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": p["hbm_gbs"], "bf16_tflops": p["bf16_tflops"],
+                "bf16_tflops_sustained": p.get("bf16_tflops_sustained", p["bf16_tflops"]),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+# ------------------------------------------------------------------ algorithmic work
+
+def work_model(cfg, distinct_experts: int) -> dict:
+    """Algorithmic FLOPs and HBM bytes of one layer forward and of its expert gate/up GEMM:
+    the contractions the method must do, the weights it must read (only the distinct experts
+    routed), the input read once and the output written once; intermediates that a fused
+    design could keep on chip are not counted."""
+    T, d, n, k, H = cfg.T, cfg.d_model, cfg.n_experts, cfg.top_k, cfg.d_ff
+    E = cfg.expert_in
+    b = 2 if cfg.dtype == "bf16" else 4
+    gu = cfg.gu_rows
+    expert_w = gu * E + E * H                      # elements of one expert's two matrices
+    flops = 2 * T * (d * n + k * expert_w)
+    wbytes = (n * d + distinct_experts * expert_w) * b
+    if cfg.latent:
+        flops += 2 * T * (d * cfg.d_latent * 2)
+        wbytes += 2 * cfg.d_latent * d * b
+    act_bytes = 2 * T * d * b                       # u in, out back
+    gate_up = {"flops": 2 * T * k * E * gu,
+               "bytes": distinct_experts * gu * E * b + T * k * E * b + T * k * H * b}
+    return {"flops": flops, "bytes": wbytes + act_bytes, "gate_up": gate_up}
+
+
+def roofline_entry(bound: str, work: float, seconds: float, peaks: dict, sustained: bool,
+                   traffic=None) -> dict:
+    if bound == "tensor":
+        peak = peaks["bf16_tflops_sustained" if sustained else "bf16_tflops"]
+        achieved = work / seconds / 1e12
+        unit = "TFLOP/s"
+    else:
+        peak = peaks["hbm_gbs"]
+        achieved = work / seconds / 1e9
+        unit = "GB/s"
+    return {"bound": bound, "achieved": round(achieved, 2), "peak": peak, "unit": unit,
+            "frac": round(achieved / peak, 4), "traffic": traffic,
+            "peak_source": peaks["source"] + (" sustained" if sustained and bound == "tensor"
+                                              else "")}
+
+
+# ------------------------------------------------------------------ our arm
+
+def measure_ours(cfg, steps: int, warmup: int, device, peaks: dict, with_e2e: bool = True,
+                 sampler=None) -> dict:
+    import torch
+    import moe_inputs
+    import sparse_moe_layer_softmax_b200 as moe
+    from gpu_harness import abi_config
+
+    dev = moe_inputs.device_inputs(cfg, device=device)
+    layer = moe.MoELayer(abi_config(cfg), dev)
+    u = dev["u"]
+    out = torch.empty_like(u)
+    idx = torch.empty((cfg.T, cfg.top_k), dtype=torch.int32, device=device)
+    stream = torch.cuda.current_stream()
+    for _ in range(warmup):
+        layer.forward(u, u, out=out, topk_idx_out=idx)
+    status = moe.moe_get_device_status()
+    if status != 0:
+        raise RuntimeError(f"device status {moe.STATUS.get(status, status)} after warm-up")
+    distinct = int(torch.unique(idx).numel())
+    loads = torch.bincount(idx.flatten().long(), minlength=cfg.n_experts)
+    max_over_mean = float(loads.max().item()) / (cfg.T * cfg.top_k / cfg.n_experts)
+
+    # ---- device-resident timed region
+    barrier()
+    torch.cuda.synchronize()
+    if sampler:
+        sampler.start()
+    launches0 = moe.launch_count()
+    moe.profile_begin(steps)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        layer.forward(u, u, out=out, topk_idx_out=idx)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    stage_ms, calls = moe.profile_end()
+    launches = moe.launch_count() - launches0
+    clocks = sampler.stop() if sampler else None
+    barrier()
+    ms = e0.elapsed_time(e1) / steps
+    ms_max = reduce_max(ms, device)
+    status = moe.moe_get_device_status()
+    if status != 0:
+        raise RuntimeError(f"device status {moe.STATUS.get(status, status)} after timing")
+
+    work = work_model(cfg, distinct)
+    gate_up_s = stage_ms["expert_gate_up"] / max(calls, 1) / 1e3
+    tensor_bound = work["flops"] / (peaks["bf16_tflops_sustained"] * 1e12) > \
+        work["bytes"] / (peaks["hbm_gbs"] * 1e9)
+    if tensor_bound:
+        roof = roofline_entry("tensor", work["gate_up"]["flops"], gate_up_s, peaks, True)
+    else:
+        roof = roofline_entry("hbm", work["gate_up"]["bytes"], gate_up_s, peaks, False)
+    roof["kernel"] = "expert gate/up GEMM (gemm_tc_kernel, SwiGLU epilogue)"
+    roof["ms_per_launch"] = round(gate_up_s * 1e3, 4)
+    t_roof = max(work["flops"] / (peaks["bf16_tflops_sustained"] * 1e12),
+                 work["bytes"] / (peaks["hbm_gbs"] * 1e9))
+    res = {"ms_per_step": ms_max, "tokens_per_step": cfg.T, "roofline": roof,
+           "layer_roofline": {"bound": "tensor" if tensor_bound else "hbm",
+                              "flops": work["flops"], "bytes": work["bytes"],
+                              "roofline_ms": round(t_roof * 1e3, 4),
+                              "frac": round(t_roof * 1e3 / ms_max, 4)},
+           "stage_ms": {k: round(v / max(calls, 1), 4) for k, v in stage_ms.items()},
+           "distinct_experts": distinct, "max_over_mean_load": round(max_over_mean, 3),
+           "gpu_launches": int(launches), "clocks": clocks}
+
+    # ---- end to end through the host-memory API: pinned host in, pinned host out
+    if with_e2e:
+        u_host = u.cpu().pin_memory()
+        out_host = torch.empty_like(u_host).pin_memory()
+        u_dev = torch.empty_like(u)
+        for _ in range(2):
+            layer.forward_host(u_host, out_host, u_dev, out)
+        barrier()
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(steps):
+            layer.forward_host(u_host, out_host, u_dev, out)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        res["e2e_ms"] = reduce_max(e0.elapsed_time(e1) / steps, device)
+        res["h2d_bytes"] = u_host.numel() * u_host.element_size()
+        res["d2h_bytes"] = out_host.numel() * out_host.element_size()
+    del layer, dev
+    torch.cuda.empty_cache()
+    return res
+
+
+# ------------------------------------------------------------------ the CPU oracle as a baseline
+
+class OracleRunner:
+    """The CPU oracle on sampled tokens of a workload.  Weights are generated on the host once
+    (they are the layer's parameters, resident like the GPU's); each run routes, evaluates the
+    experts and projects the listed tokens with the oracle's own threads."""
+
+    def __init__(self, cfg):
+        import moe_inputs
+        self.cfg = cfg
+        self.dense = {name: moe_inputs.host_rows(cfg, name) for name in moe_inputs.tensor_specs(cfg)
+                      if name not in ("u", "w_gu", "w_down")}
+        if cfg.zipf_bias:
+            self.dense["logit_bias"] = moe_inputs.zipf_bias(cfg)
+        self.experts = {}
+
+    def _inputs(self, tokens):
+        import moe_inputs
+        d = dict(self.dense)
+        d["u"] = moe_inputs.host_rows(self.cfg, "u", rows=tokens)
+        return d
+
+    def _expert(self, e):
+        import moe_inputs
+        if e not in self.experts:
+            self.experts[e] = (moe_inputs.host_rows(self.cfg, "w_gu", lead=e),
+                               moe_inputs.host_rows(self.cfg, "w_down", lead=e))
+        return self.experts[e]
+
+    def prepare(self):
+        """Untimed: generate the host weights of every expert."""
+        for e in range(self.cfg.n_experts):
+            self._expert(e)
+
+    def run(self, tokens) -> float:
+        """Seconds of wall time for the oracle on these tokens."""
+        import oracle
+        t0 = time.perf_counter()
+        oracle.layer_forward_staged(self.cfg, tokens, self._inputs, self._expert)
+        return time.perf_counter() - t0
+
+
+def cpu_sample_tokens(cfg, count: int, salt: int = 0):
+    import moe_inputs
+    from moe_inputs import configs
+    toks = moe_inputs.fisher_yates(cfg.seed + 1000 * (salt + 1), configs.STREAM_SUBSAMPLE,
+                                   cfg.T, count)
+    return np.sort(toks)
+
+
+def default_cpu_sample(cfg) -> int:
+    """Tokens per CPU-oracle sample: about 10-30 s of work on the host's cores."""
+    per_token_gmac = (cfg.d_model * cfg.n_experts + cfg.top_k * (cfg.gu_rows * cfg.expert_in +
+                      cfg.expert_in * cfg.d_ff) + 2 * cfg.d_model * cfg.d_latent) / 1e9
+    cores = os.cpu_count() or 1
+    n = int(15.0 * cores * 0.25 / max(per_token_gmac, 1e-6))  # ~0.25 GMAC/s per core
+    return int(max(cores, min(n, cfg.T, 4096)))
+
+
+def cpu_baseline(cfg, sample: int) -> dict:
+    runner = OracleRunner(cfg)
+    toks = cpu_sample_tokens(cfg, sample)
+    runner.prepare()
+    secs = runner.run(toks)
+    return {"value": round(len(toks) / secs, 3), "unit": UNIT, "cores": os.cpu_count(),
+            "kind": "oracle",
+            "sample": f"{len(toks)} seeded tokens of {cfg.name} (T={cfg.T}); full layer per token "
+                      f"in double on {os.cpu_count()} threads; host weights generated untimed",
+            "seconds": round(secs, 3)}
+
+
+def config_block(cfg, world: int) -> dict:
+    return {"workload": cfg.name, "T": cfg.T, "d_model": cfg.d_model, "d_latent": cfg.d_latent,
+            "d_ff": cfg.d_ff, "n_experts": cfg.n_experts, "top_k": cfg.top_k, "seed": cfg.seed,
+            "global_batch": cfg.T * world,
+            "parallelism": f"replicas x{world}: every rank runs the full workload",
+            "l2": "no flush: every step streams the routed experts' weights (GBs) and activations "
+                  "far larger than the 126 MB L2"}
+
+
+# ------------------------------------------------------------------ reference arm: the CPU oracle
+
+def run_reference(args) -> int:
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    from moe_inputs import configs
+    cfg = configs.CONFIGS[args.workload]
+    runner = OracleRunner(cfg)
+    runner.prepare()
+    per_step = args.cpu_sample or (os.cpu_count() or 1)
+    for s in range(args.warmup):
+        runner.run(cpu_sample_tokens(cfg, per_step, salt=100 + s))
+    secs = 0.0
+    for s in range(args.steps):
+        secs += runner.run(cpu_sample_tokens(cfg, per_step, salt=s))
+    value = per_step * args.steps / secs
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": UNIT,
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(secs / args.steps * 1e3, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": config_block(cfg, 1),
+            "cpu_baseline": {"value": round(value, 3), "unit": UNIT, "cores": os.cpu_count(),
+                             "kind": "oracle",
+                             "sample": f"{per_step} seeded tokens of {cfg.name} per step"},
+            "e2e": {"value": round(value, 3), "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ main
+
+def visible_gpu_index(local: int) -> str:
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if vis:
+        ids = [x.strip() for x in vis.split(",") if x.strip()]
+        if local < len(ids):
+            return ids[local]
+    return str(local)
+
+
+BAD_REASONS = {"hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown"}
+
+
+def measure_checked(cfg, args, device, peaks, rank, local, with_e2e=True) -> dict:
+    """Measure; re-measure once if the clocks record shows a rejected throttle reason."""
+    for attempt in range(2):
+        sampler = ClockSampler(visible_gpu_index(local)) if rank == 0 else None
+        res = measure_ours(cfg, args.steps, args.warmup, device, peaks, with_e2e, sampler)
+        clk = res.get("clocks") or {}
+        bad = BAD_REASONS & set(clk.get("reasons") or [])
+        if not bad:
+            break
+        res["remeasured_after"] = sorted(bad)
+    return res
+
+
+def main(argv=None) -> int:
+    args = parse_args(argv)
+    if args.impl == "reference":
+        return run_reference(args)
+    import torch
+    from moe_inputs import configs
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    init_dist("nccl")
+    peaks = measured_peaks()
+    cfg = configs.CONFIGS[args.workload]
+    res = measure_checked(cfg, args, device, peaks, rank, local)
+    value = cfg.T * world / (res["ms_per_step"] / 1e3)
+    line = {"metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(res["ms_per_step"], 4), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded counter-based generator; random-init weights)",
+            "config": config_block(cfg, world),
+            "roofline": res["roofline"], "layer_roofline": res["layer_roofline"],
+            "e2e": {"value": round(cfg.T * world / (res["e2e_ms"] / 1e3), 2), "unit": UNIT,
+                    "h2d_bytes_per_step": res["h2d_bytes"], "d2h_bytes_per_step": res["d2h_bytes"],
+                    "ms_per_step": round(res["e2e_ms"], 4)},
+            "gpu_launches": res["gpu_launches"], "clocks": res["clocks"],
+            "stage_ms": res["stage_ms"], "distinct_experts": res["distinct_experts"],
+            "max_over_mean_load": res["max_over_mean_load"]}
+    if "remeasured_after" in res:
+        line["remeasured_after"] = res["remeasured_after"]
+    if not args.no_decode and cfg.name != "muse_decode":
+        dres = measure_checked(configs.MUSE_DECODE, args, device, peaks, rank, local)
+        line["decode"] = {
+            "workload": "muse_decode", "value": round(64 * world / (dres["ms_per_step"] / 1e3), 2),
+            "unit": UNIT, "ms_per_step": round(dres["ms_per_step"], 4),
+            "roofline": dres["roofline"], "layer_roofline": dres["layer_roofline"],
+            "e2e": {"value": round(64 * world / (dres["e2e_ms"] / 1e3), 2), "unit": UNIT,
+                    "h2d_bytes_per_step": dres["h2d_bytes"],
+                    "d2h_bytes_per_step": dres["d2h_bytes"]},
+            "stage_ms": dres["stage_ms"], "distinct_experts": dres["distinct_experts"],
+            "gpu_launches": dres["gpu_launches"], "clocks": dres["clocks"]}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(cfg, args.cpu_sample or default_cpu_sample(cfg))
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    import torch.distributed as dist
+    if dist.is_initialized():
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())
+

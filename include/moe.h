@@ -172,6 +172,25 @@ MOE_API moe_status_t moe_layer_forward(const moe_config_t* cfg, const moe_weight
  * (MOE_OK if no kernel latched an error since the last call). */
 MOE_API moe_status_t moe_get_device_status(void* stream);
 
+/* Stage timing of moe_layer_forward, for measurement (not part of the layer's definition).
+ * moe_profile_begin(max_calls) creates CUDA events for up to max_calls forward calls on the
+ * current device; each following moe_layer_forward call records MOE_PROFILE_STAGES + 1 events on
+ * its stream around its stages, in this order:
+ *   0 route, 1 latent down-projection, 2 dispatch (permute + row scatter), 3 expert gate/up (or
+ *   ReLU) GEMM, 4 expert down GEMM, 5 normalise + combine, 6 latent up-projection + residual.
+ * Stages a configuration does not have take zero time.  moe_profile_end synchronises on the
+ * last recorded event, writes the summed milliseconds of each stage over the recorded calls to
+ * stage_ms[MOE_PROFILE_STAGES] and the number of recorded calls to *calls, destroys the events
+ * and stops recording.  Calls beyond max_calls are not recorded.  Not thread-safe: one profiling
+ * session per process at a time. */
+#define MOE_PROFILE_STAGES 7
+MOE_API moe_status_t moe_profile_begin(int32_t max_calls);
+MOE_API moe_status_t moe_profile_end(float* stage_ms, int32_t* calls);
+
+/* Number of CUDA kernels this library has launched in this process (host-side counter, for
+ * measurement: the difference across a region is the kernels that region launched). */
+MOE_API unsigned long long moe_launch_count(void);
+
 #ifdef __cplusplus
 }
 #endif

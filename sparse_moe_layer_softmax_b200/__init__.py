@@ -26,7 +26,10 @@ STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED", 3: "M
 STATUS_CODES = {v: k for k, v in STATUS.items()}
 EXPORTS = ("moe_status_string", "moe_workspace_size", "moe_route", "moe_permute",
            "moe_expert_ffn", "moe_combine", "moe_latent_down", "moe_latent_up",
-           "moe_layer_forward", "moe_get_device_status")
+           "moe_layer_forward", "moe_get_device_status", "moe_profile_begin", "moe_profile_end",
+           "moe_launch_count")
+PROFILE_STAGES = ("route", "latent_down", "dispatch", "expert_gate_up", "expert_down", "combine",
+                  "latent_up_resgate")
 
 
 class MoeError(RuntimeError):
@@ -75,11 +78,15 @@ def lib():
             "moe_latent_up": [cp, vp, vp, vp, vp, vp, vp],
             "moe_layer_forward": [cp, wp, vp, vp, vp, vp, vp, vp, vp, sz, vp],
             "moe_get_device_status": [vp],
+            "moe_profile_begin": [ctypes.c_int32],
+            "moe_profile_end": [vp, vp],
         }
         for name, args in sigs.items():
             f = getattr(L, name)
             f.restype = i32
             f.argtypes = args
+        L.moe_launch_count.restype = ctypes.c_ulonglong
+        L.moe_launch_count.argtypes = []
         _lib = L
     return _lib
 
@@ -179,6 +186,24 @@ def moe_get_device_status(stream=None) -> int:
     return lib().moe_get_device_status(_stream(stream))
 
 
+def launch_count() -> int:
+    """Kernels libmoe.so has launched in this process."""
+    return int(lib().moe_launch_count())
+
+
+def profile_begin(max_calls: int):
+    """Start recording per-stage CUDA events in the next ``max_calls`` moe_layer_forward calls."""
+    _check("moe_profile_begin", lib().moe_profile_begin(max_calls))
+
+
+def profile_end() -> tuple[dict, int]:
+    """Stop recording; returns ({stage: summed ms}, recorded calls)."""
+    ms = (ctypes.c_float * len(PROFILE_STAGES))()
+    calls = ctypes.c_int32()
+    _check("moe_profile_end", lib().moe_profile_end(ms, ctypes.byref(calls)))
+    return {k: float(v) for k, v in zip(PROFILE_STAGES, ms)}, calls.value
+
+
 class MoELayer:
     """A layer instance holding its device weights and a workspace, with a forward() that takes
     device or pinned-host inputs.  Nothing here computes: forward() is one moe_layer_forward."""
@@ -198,3 +223,15 @@ class MoELayer:
         moe_layer_forward(self.cfg, self._w, u, r if r is not None else u, out, logits_out,
                           topk_idx_out, topk_w_out, self.workspace, stream=stream)
         return out
+
+    def forward_host(self, u_host, out_host, u_dev, out_dev, stream=None):
+        """One forward from pinned host memory to pinned host memory: the input is copied to the
+        device, the layer runs, and the output is copied back, all queued on one stream (the
+        residual is the input).  u_dev / out_dev are the device staging buffers."""
+        import torch
+        s = stream if stream is not None else torch.cuda.current_stream()
+        with torch.cuda.stream(s):
+            u_dev.copy_(u_host, non_blocking=True)
+            self.forward(u_dev, u_dev, out=out_dev, stream=s)
+            out_host.copy_(out_dev, non_blocking=True)
+        return out_host

@@ -2,8 +2,10 @@
 // descriptors and the launch sequence of the MoE-layer forward on the caller's stream.
 #include <cudaTypedefs.h>
 
+#include <atomic>
 #include <initializer_list>
 #include <mutex>
+#include <vector>
 
 #include "common.cuh"
 #include "gemm_tc.cuh"
@@ -66,7 +68,11 @@ bool make_tmap(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, u
   return r == CUDA_SUCCESS;
 }
 
-moe_status_t last_launch() {
+std::atomic<unsigned long long> g_launches{0};  // kernels this library has launched
+
+// Status of the kernel launch(es) just issued; counts `n` launches.
+moe_status_t last_launch(int n = 1) {
+  g_launches.fetch_add(static_cast<unsigned long long>(n), std::memory_order_relaxed);
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
@@ -242,12 +248,12 @@ moe_status_t do_permute(const moe_config_t& c, const int32_t* idx, int32_t* offs
   const int n = c.n_experts, k = c.top_k, nc = nchunks(c);
   if (c.T == 0) {
     cudaMemsetAsync(offsets, 0, (n + 1) * sizeof(int32_t), st);
-    return last_launch();
+    return last_launch(0);
   }
   perm_count_kernel<<<nc, 256, 0, st>>>(idx, c.T, k, n, counts);
   perm_scan_kernel<<<1, kMaxExperts, 0, st>>>(counts, nc, n, offsets);
   perm_rank_kernel<<<nc, 256, 0, st>>>(idx, c.T, k, n, counts, offsets, perm, inv);
-  moe_status_t s = last_launch();
+  moe_status_t s = last_launch(3);
   if (s != MOE_OK || !x) return s;
   const int E = c.d_latent > 0 ? c.d_latent : c.d_model;
   if (c.dtype == MOE_F32) {
@@ -270,9 +276,34 @@ moe_status_t do_permute(const moe_config_t& c, const int32_t* idx, int32_t* offs
   return last_launch();
 }
 
+// ------------------------------------------------------------------ stage timing
+
+struct Profiler {
+  std::vector<cudaEvent_t> ev;  // max_calls x (MOE_PROFILE_STAGES + 1)
+  int max_calls = 0, calls = 0;
+  bool active = false;
+};
+
+Profiler& prof() {
+  static Profiler p;
+  return p;
+}
+
+constexpr int kMarks = MOE_PROFILE_STAGES + 1;
+
+void prof_mark(cudaStream_t st, int i) {
+  Profiler& p = prof();
+  if (p.active && p.calls < p.max_calls) cudaEventRecord(p.ev[p.calls * kMarks + i], st);
+}
+
+void prof_next_call() {
+  Profiler& p = prof();
+  if (p.active && p.calls < p.max_calls) ++p.calls;
+}
+
 moe_status_t do_experts(const moe_config_t& c, const void* x_perm, const int32_t* offsets,
                         const void* w_gu, const void* w_down, const float* gamma_e,
-                        void* out_perm, void* act, cudaStream_t st) {
+                        void* out_perm, void* act, cudaStream_t st, bool mark = false) {
   const long TK = static_cast<long>(c.T) * c.top_k;
   if (TK == 0) return MOE_OK;
   const int E = expert_in(c), H = c.d_ff, n = c.n_experts;
@@ -301,6 +332,7 @@ moe_status_t do_experts(const moe_config_t& c, const void* x_perm, const int32_t
   moe_status_t s = run_gemm(swiglu ? EPI_SWIGLU : EPI_RELU, o1, bn1, x_perm, TK, w_gu,
                             static_cast<long>(n) * p1.Nw, p1, st);
   if (s != MOE_OK) return s;
+  if (mark) prof_mark(st, 4);
   // second GEMM: act [TK, H] x W_down[e]^T -> out [TK, E] (scaled by 1 + gamma for I_gamma)
   GemmParams p2{};
   p2.seg = offsets;
@@ -517,24 +549,78 @@ moe_status_t moe_layer_forward(const moe_config_t* cfg, const moe_weights_t* w, 
   void* x_perm = at<void>(workspace, L.x_perm);
   void* act = at<void>(workspace, L.act);
 
+  prof_mark(st, 0);
   if ((s = do_route(c, u, w->w_router, w->logit_bias, logits_out, idx, wt, st)) != MOE_OK) return s;
+  prof_mark(st, 1);
   const void* xin = u;
   if (latent) {
     void* z = at<void>(workspace, L.z_raw);
     if ((s = do_latent_down(c, u, w->p_down, z, st)) != MOE_OK) return s;
     xin = z;
   }
+  prof_mark(st, 2);
   if ((s = do_permute(c, idx, offsets, perm, inv, xin, c.pre_norm ? w->gamma_pre : nullptr, x_perm,
                       at<int32_t>(workspace, L.counts), st)) != MOE_OK)
     return s;
+  prof_mark(st, 3);
   // The expert output overwrites the dispatched input rows (no longer needed after GEMM 1).
-  if ((s = do_experts(c, x_perm, offsets, w->w_gu, w->w_down, w->gamma_expert, x_perm, act, st)) !=
-      MOE_OK)
+  if ((s = do_experts(c, x_perm, offsets, w->w_gu, w->w_down, w->gamma_expert, x_perm, act, st,
+                      true)) != MOE_OK)
     return s;
-  if (!latent) return do_combine(c, x_perm, inv, wt, out, st);
-  void* y = at<void>(workspace, L.y);
+  if (c.dtype == MOE_F32) prof_mark(st, 4);  // one fused kernel: all time in stage 3
+  prof_mark(st, 5);
+  void* y = latent ? at<void>(workspace, L.y) : out;
   if ((s = do_combine(c, x_perm, inv, wt, y, st)) != MOE_OK) return s;
-  return do_latent_up(c, y, w->p_up, r, w->resid_g, out, st);
+  prof_mark(st, 6);
+  if (latent && (s = do_latent_up(c, y, w->p_up, r, w->resid_g, out, st)) != MOE_OK) return s;
+  prof_mark(st, 7);
+  prof_next_call();
+  return MOE_OK;
+}
+
+unsigned long long moe_launch_count(void) { return g_launches.load(); }
+
+moe_status_t moe_profile_begin(int32_t max_calls) {
+  if (max_calls <= 0 || max_calls > 100000) return MOE_ERR_INVALID_ARG;
+  Profiler& p = prof();
+  if (p.active) return MOE_ERR_INVALID_ARG;
+  p.ev.assign(static_cast<size_t>(max_calls) * kMarks, nullptr);
+  for (auto& e : p.ev)
+    if (cudaEventCreate(&e) != cudaSuccess) {
+      for (auto& f : p.ev)
+        if (f) cudaEventDestroy(f);
+      p.ev.clear();
+      return MOE_ERR_CUDA;
+    }
+  p.max_calls = max_calls;
+  p.calls = 0;
+  p.active = true;
+  return MOE_OK;
+}
+
+moe_status_t moe_profile_end(float* stage_ms, int32_t* calls) {
+  Profiler& p = prof();
+  if (!p.active || !stage_ms) return MOE_ERR_INVALID_ARG;
+  moe_status_t s = MOE_OK;
+  for (int i = 0; i < MOE_PROFILE_STAGES; ++i) stage_ms[i] = 0.0f;
+  if (p.calls > 0 && cudaEventSynchronize(p.ev[(p.calls - 1) * kMarks + MOE_PROFILE_STAGES]) !=
+                         cudaSuccess)
+    s = MOE_ERR_CUDA;
+  for (int c = 0; c < p.calls && s == MOE_OK; ++c)
+    for (int i = 0; i < MOE_PROFILE_STAGES; ++i) {
+      float ms = 0.0f;
+      if (cudaEventElapsedTime(&ms, p.ev[c * kMarks + i], p.ev[c * kMarks + i + 1]) != cudaSuccess) {
+        s = MOE_ERR_CUDA;
+        break;
+      }
+      stage_ms[i] += ms;
+    }
+  if (calls) *calls = p.calls;
+  for (auto& e : p.ev) cudaEventDestroy(e);
+  p.ev.clear();
+  p.active = false;
+  p.calls = p.max_calls = 0;
+  return s;
 }
 
 moe_status_t moe_get_device_status(void* stream) {

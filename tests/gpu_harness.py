@@ -49,6 +49,14 @@ def tolerance(cfg) -> float:
     return BF16_TOL if cfg.dtype == "bf16" else F32_TOL
 
 
+def logit_atol(cfg, logits: np.ndarray) -> float:
+    """Absolute tolerance of fp32-accumulated router logits against double: the products of two
+    bf16 (or fp32-rounded) values are summed in fp32 over K = d_model terms; rounding errors of
+    a K-term sum grow like sqrt(K) * 2^-24 * |partial sums|, so allow 16 sqrt(K) 2^-24 times the
+    largest logit magnitude (at least 1)."""
+    return 16.0 * np.sqrt(cfg.d_model) * 2.0 ** -24 * max(1.0, float(np.abs(logits).max()))
+
+
 def run_layer(cfg, dev: dict, want_logits: bool = True):
     """moe_layer_forward through the C ABI on device inputs; returns torch tensors."""
     import torch
@@ -99,6 +107,29 @@ def check_routing(cfg, logits_gpu: np.ndarray, idx_gpu: np.ndarray, w_gpu: np.nd
     np.testing.assert_array_equal(idx_gpu, sel)
     np.testing.assert_allclose(w_gpu, wref, rtol=1e-6, atol=1e-7)
     np.testing.assert_allclose(w_gpu.sum(1), cfg.routed_scale, rtol=2e-6)
+
+
+def order_tie_tokens(logits_ref: np.ndarray, k: int, rel: float = 1e-4) -> np.ndarray:
+    """Tokens with two of their k selected oracle logits closer than rel * rms(logits): the set
+    of selected experts is unique but their slot order is not (fp32 and double may differ)."""
+    s = -np.sort(-logits_ref, axis=1)[:, :k]
+    if k < 2:
+        return np.zeros(len(logits_ref), dtype=bool)
+    gaps = np.min(s[:, :-1] - s[:, 1:], axis=1)
+    rms = np.sqrt(np.mean(logits_ref ** 2, axis=1))
+    return gaps < rel * rms
+
+
+def compare_selection(idx_gpu: np.ndarray, ref_logits: np.ndarray, ref_idx: np.ndarray, k: int):
+    """GPU selection vs the oracle's (double-logit) selection, comparing what is unique: tokens
+    with a near tie at the k-th place are skipped (their selected set is not unique), tokens with
+    a near tie inside the selection are compared as sets.  Returns the boundary-tie mask."""
+    ties = near_tie_tokens(ref_logits, k)
+    ot = order_tie_tokens(ref_logits, k) & ~ties
+    exact = ~ties & ~ot
+    np.testing.assert_array_equal(idx_gpu[exact], ref_idx[exact])
+    np.testing.assert_array_equal(np.sort(idx_gpu[ot], axis=1), np.sort(ref_idx[ot], axis=1))
+    return ties
 
 
 def near_tie_tokens(logits_ref: np.ndarray, k: int, rel: float = 1e-4) -> np.ndarray:
