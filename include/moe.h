@@ -128,6 +128,28 @@ MOE_API moe_status_t moe_permute(const moe_config_t* cfg, const int32_t* topk_id
                          const void* x, const float* gamma_pre, void* x_perm, void* workspace,
                          size_t workspace_bytes, void* stream);
 
+/* moe_permute without a workspace argument, for callers that cannot allocate device memory: a
+ * plugin or embedding host that hands the library only its input and output buffers (no
+ * allocator handle, no scratch pool), or code that may not call cudaMalloc on its path because
+ * that call can synchronise the device.  The pages describe no such variant: it exists for this
+ * library's callers only.
+ *
+ * Same arguments, outputs and errors as moe_permute, minus workspace/workspace_bytes.  Its
+ * scratch (the per-chunk expert histograms, ceil(T/128) * n_experts int32 values) lives in one
+ * device array inside the library of MOE_PERMUTE_STATIC_MAX_COUNTS int32 (256 KB), which every
+ * GPU that loads the library keeps until the process exits; it covers T <= 32768 tokens with 256
+ * experts (ceil(T/128) * n_experts <= 65536).  Larger sizes return MOE_ERR_WORKSPACE before any
+ * launch.  The call allocates nothing.  The first call on each device looks up the array's
+ * device address (cudaGetSymbolAddress, with that device current); make that first call before
+ * any stream capture on the device.  All calls share the one array and leave their histograms in
+ * it: calls that can overlap on the GPU (on different streams, or from several host threads
+ * without ordering) race and produce wrong offsets; order them on one stream. */
+#define MOE_PERMUTE_STATIC_MAX_COUNTS 65536
+MOE_API moe_status_t moe_permute_static(const moe_config_t* cfg, const int32_t* topk_idx,
+                                        int32_t* expert_offsets, int32_t* perm_token,
+                                        int32_t* inv_perm, const void* x, const float* gamma_pre,
+                                        void* x_perm, void* stream);
+
 /* Experts on their routed rows only [MUSE "Latent experts"; SHAZEER "The math"]: for each expert
  * e, rows [expert_offsets[e], expert_offsets[e+1]) of x_perm [T*k, E_in]:
  *   SwiGLU: a = SiLU(x W_gate^T) * (x W_up^T) stored in dtype;  ReLU: a = ReLU(x W1^T);

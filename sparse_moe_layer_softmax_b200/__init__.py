@@ -27,7 +27,7 @@ STATUS_CODES = {v: k for k, v in STATUS.items()}
 EXPORTS = ("moe_status_string", "moe_workspace_size", "moe_route", "moe_permute",
            "moe_expert_ffn", "moe_combine", "moe_latent_down", "moe_latent_up",
            "moe_layer_forward", "moe_get_device_status", "moe_profile_begin", "moe_profile_end",
-           "moe_launch_count")
+           "moe_launch_count", "moe_permute_static")
 PROFILE_STAGES = ("route", "latent_down", "dispatch", "expert_gate_up", "expert_down", "combine",
                   "latent_up_resgate")
 
@@ -80,6 +80,7 @@ def lib():
             "moe_get_device_status": [vp],
             "moe_profile_begin": [ctypes.c_int32],
             "moe_profile_end": [vp, vp],
+            "moe_permute_static": [cp, vp, vp, vp, vp, vp, vp, vp, vp],
         }
         for name, args in sigs.items():
             f = getattr(L, name)
@@ -140,6 +141,16 @@ def moe_permute(cfg, topk_idx, expert_offsets, perm_token, inv_perm, x=None, gam
                                             _ptr(perm_token), _ptr(inv_perm), _ptr(x),
                                             _ptr(gamma_pre), _ptr(x_perm), _ptr(workspace),
                                             workspace_bytes, _stream(stream)))
+
+
+def moe_permute_static(cfg, topk_idx, expert_offsets, perm_token, inv_perm, x=None,
+                       gamma_pre=None, x_perm=None, stream=None):
+    """moe_permute for callers that cannot allocate: the scratch is a fixed 256 KB array inside
+    the library (ceil(T/128) * n_experts <= 65536), shared by all calls, so calls must not
+    overlap on the GPU."""
+    _check("moe_permute_static", lib().moe_permute_static(
+        ctypes.byref(cfg), _ptr(topk_idx), _ptr(expert_offsets), _ptr(perm_token),
+        _ptr(inv_perm), _ptr(x), _ptr(gamma_pre), _ptr(x_perm), _stream(stream)))
 
 
 def moe_expert_ffn(cfg, x_perm, expert_offsets, w_gu, w_down, gamma_expert, out_perm,

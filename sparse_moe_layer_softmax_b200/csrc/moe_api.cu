@@ -467,6 +467,61 @@ moe_status_t moe_permute(const moe_config_t* cfg, const int32_t* topk_idx,
                     static_cast<int32_t*>(workspace), static_cast<cudaStream_t>(stream));
 }
 
+}  // extern "C"
+
+// ------------------------------------------------------------------ allocation-free dispatch
+//
+// Scratch of moe_permute_static: the per-chunk expert histograms of the dispatch permutation
+// (ceil(T/128) x n int32), held in a file-scope device array instead of a caller workspace.  Every
+// device that loads the library holds these 256 KB until the process exits.  Host code must not
+// pass the symbol itself to a kernel (on the host it names a host-side stand-in); its device
+// address is taken once per device with cudaGetSymbolAddress and passed as a plain pointer.
+static __device__ __align__(256) int32_t g_permute_scratch[MOE_PERMUTE_STATIC_MAX_COUNTS];
+
+namespace {
+
+// Device address of g_permute_scratch on the current device, looked up on the first call on
+// that device (nullptr if the lookup fails).
+int32_t* permute_scratch_ptr() {
+  static std::mutex mu;
+  static int32_t* ptr[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lk(mu);
+  if (!ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_permute_scratch) != cudaSuccess) return nullptr;
+    ptr[dev] = static_cast<int32_t*>(p);
+  }
+  return ptr[dev];
+}
+
+}  // namespace
+
+extern "C" {
+
+moe_status_t moe_permute_static(const moe_config_t* cfg, const int32_t* topk_idx,
+                                int32_t* expert_offsets, int32_t* perm_token, int32_t* inv_perm,
+                                const void* x, const float* gamma_pre, void* x_perm, void* stream) {
+  moe_status_t s = check_cfg(cfg);
+  if (s != MOE_OK) return s;
+  if (!expert_offsets || (cfg->T > 0 && (!topk_idx || !perm_token || !inv_perm)))
+    return MOE_ERR_INVALID_ARG;
+  if (x && !x_perm) return MOE_ERR_INVALID_ARG;
+  if (gamma_pre && (cfg->dtype != MOE_BF16 || cfg->d_latent == 0)) return MOE_ERR_UNSUPPORTED;
+  if (!all_aligned({static_cast<const void*>(topk_idx), static_cast<const void*>(expert_offsets),
+                    static_cast<const void*>(perm_token), static_cast<const void*>(inv_perm), x,
+                    static_cast<const void*>(gamma_pre), x_perm}))
+    return MOE_ERR_ALIGNMENT;
+  const long need = static_cast<long>(nchunks(*cfg)) * cfg->n_experts;
+  if (need > MOE_PERMUTE_STATIC_MAX_COUNTS) return MOE_ERR_WORKSPACE;
+  int32_t* scratch = permute_scratch_ptr();
+  if (!scratch) return MOE_ERR_CUDA;
+  // The count kernel overwrites every histogram entry this call uses, so no clearing is needed.
+  return do_permute(*cfg, topk_idx, expert_offsets, perm_token, inv_perm, x, gamma_pre, x_perm,
+                    scratch, static_cast<cudaStream_t>(stream));
+}
+
 moe_status_t moe_expert_ffn(const moe_config_t* cfg, const void* x_perm,
                             const int32_t* expert_offsets, const void* w_gu, const void* w_down,
                             const float* gamma_expert, void* out_perm, void* workspace,
