@@ -160,6 +160,38 @@ def measured_peaks() -> dict:
             "source": "fallback"}
 
 
+# ------------------------------------------------------------------ measured DRAM traffic
+
+# DRAM bytes (read + write) per launch of the expert gate/up GEMM from one ncu capture of each
+# reduced-expert case (profiles/gemm_gateup_muse_*_n32.md), with the units it processed.  A full
+# launch scales by the same units: prefill by routed rows and experts (both 8x), decode by routed
+# experts.  Valid only for the kernel source the capture was taken on (fingerprint below).
+TRAFFIC_CAPTURES = {
+    "kernel_sha256_16": "d5d8668a842fecc0",
+    "muse_prefill": {"bytes": 2.300616e9 + 0.13310336e9, "experts": 32, "rows": 2048 * 8},
+    "muse_decode": {"bytes": 1.947401e9 + 0.004740864e9, "experts": 29, "rows": 8 * 8},
+}
+
+
+def kernel_fingerprint() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for f in ("common.cuh", "gemm_tc.cuh"):
+        with open(os.path.join(ROOT, "sparse_moe_layer_softmax_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def gate_up_traffic(cfg, distinct_experts: int):
+    """Measured traffic scaled to this launch, or None if the kernel changed since the capture."""
+    cap = TRAFFIC_CAPTURES.get(cfg.name)
+    if cap is None or kernel_fingerprint() != TRAFFIC_CAPTURES["kernel_sha256_16"]:
+        return None
+    if cfg.name == "muse_prefill":
+        return round(cap["bytes"] * (cfg.T * cfg.top_k) / cap["rows"])
+    return round(cap["bytes"] * distinct_experts / cap["experts"])
+
+
 # ------------------------------------------------------------------ algorithmic work
 
 def work_model(cfg, distinct_experts: int) -> dict:
@@ -254,6 +286,8 @@ def measure_ours(cfg, steps: int, warmup: int, device, peaks: dict, with_e2e: bo
         roof = roofline_entry("tensor", work["gate_up"]["flops"], gate_up_s, peaks, True)
     else:
         roof = roofline_entry("hbm", work["gate_up"]["bytes"], gate_up_s, peaks, False)
+    roof["traffic"] = gate_up_traffic(cfg, distinct)
+    roof["algorithmic_bytes"] = work["gate_up"]["bytes"]
     roof["kernel"] = "expert gate/up GEMM (gemm_tc_kernel, SwiGLU epilogue)"
     roof["ms_per_launch"] = round(gate_up_s * 1e3, 4)
     t_roof = max(work["flops"] / (peaks["bf16_tflops_sustained"] * 1e12),
@@ -377,7 +411,7 @@ def run_reference(args) -> int:
     if rank != 0:
         return 0
     from moe_inputs import configs
-    cfg = configs.CONFIGS[args.workload]
+    cfg = configs.ALL_CONFIGS[args.workload]
     runner = OracleRunner(cfg)
     runner.prepare()
     per_step = args.cpu_sample or (os.cpu_count() or 1)
@@ -439,7 +473,7 @@ def main(argv=None) -> int:
     device = torch.device("cuda", local)
     init_dist("nccl")
     peaks = measured_peaks()
-    cfg = configs.CONFIGS[args.workload]
+    cfg = configs.ALL_CONFIGS[args.workload]
     res = measure_checked(cfg, args, device, peaks, rank, local)
     value = cfg.T * world / (res["ms_per_step"] / 1e3)
     line = {"metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,

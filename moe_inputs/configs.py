@@ -131,6 +131,14 @@ MUSE_IMBALANCED = MUSE_DECODE.replace(name="muse_imbalanced", T=32768, seed=4, z
 CONFIGS = {c.name: c for c in (TINY_SHAZEER_F32, SHAZEER_BF16, MUSE_DECODE, MUSE_PREFILL,
                                MUSE_IMBALANCED)}
 
+# Profiler capture cases: the Muse layer with 32 experts instead of 256, so that a capture holds a
+# few GB of weights, at the same rows per expert as the full workloads (prefill: 512 per expert;
+# decode: 2 per expert), i.e. the same per-tile work in every kernel.
+MUSE_PREFILL_N32 = MUSE_PREFILL.replace(name="muse_prefill_n32", T=2048, n_experts=32, seed=5)
+MUSE_DECODE_N32 = MUSE_DECODE.replace(name="muse_decode_n32", T=8, n_experts=32, seed=6)
+PROFILE_CONFIGS = {c.name: c for c in (MUSE_PREFILL_N32, MUSE_DECODE_N32)}
+ALL_CONFIGS = {**CONFIGS, **PROFILE_CONFIGS}
+
 
 def small_muse(T: int = 37, d: int = 256, L: int = 128, I: int = 128, n: int = 16, k: int = 4,
                seed: int = 7, **kw) -> MoEConfig:
