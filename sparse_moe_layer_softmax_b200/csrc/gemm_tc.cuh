@@ -74,7 +74,10 @@ struct GemmShape {
 
 constexpr int kMaxGroups = 256;
 constexpr int kGemmThreads = 192;
-constexpr int kSmemMisc = 4096;
+constexpr int kSmemMisc = 8192;  // barriers, TMEM slot, group tables, residual-gate coefficients
+
+// Barrier 1 among the 128 epilogue threads only (barrier 0 is __syncthreads).
+__device__ __forceinline__ void epilogue_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
 template <bool kSwap, int BN, int kEpi, int kStages>
 constexpr int gemm_smem_bytes() {
@@ -149,6 +152,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
   int* s_seg = reinterpret_cast<int*>(tmem_slot + 4);
   int* s_pref = s_seg + (kMaxGroups + 4);
+  float* s_coef = reinterpret_cast<float*>(s_pref + (kMaxGroups + 4));  // [2][BN] alpha, beta
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = p.G;
@@ -338,6 +342,55 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
               dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
             }
           }
+        } else if constexpr (kEpi == EPI_RESGATE) {
+          // Per-column coefficients of this tile, computed once by the 128 epilogue threads:
+          // out = alpha * r + beta * b  (MUSE gate: beta = sigmoid(g/tau), alpha =
+          // sqrt(max(sigmoid(-g/tau)(1+beta), floor)); literal: alpha = 1, beta = g; none: 0, 1).
+          epilogue_bar();  // the previous tile's readers are done with s_coef
+          for (int cc = static_cast<int>(threadIdx.x) - 64; cc < BN; cc += 128) {
+            const float g = p.gparam ? p.gparam[f0 + cc] : 0.0f;
+            float a = 0.0f, b = 1.0f;
+            if (p.resid_mode == MOE_RESID_MUSE_GATE) {
+              b = sigmoidf_(g / p.tau);
+              a = sqrtf(fmaxf(sigmoidf_(-g / p.tau) * (1.0f + b), p.floor_));
+            } else if (p.resid_mode == MOE_RESID_LITERAL) {
+              a = 1.0f;
+              b = g;
+            }
+            s_coef[cc] = a;
+            s_coef[BN + cc] = b;
+          }
+          epilogue_bar();
+          const bool has_r = p.resid_mode != MOE_RESID_NONE;
+          uint16_t* out = static_cast<uint16_t*>(p.out) + row * p.Nout + f0;
+          const uint16_t* hrow = has_r ? p.resid + row * p.Nout + f0 : nullptr;
+          for (int c0 = 0; c0 < BN; c0 += 64) {
+            uint4 hv[8];  // 64 residual values, loaded together so their latency overlaps
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              hv[i] = (valid && has_r) ? reinterpret_cast<const uint4*>(hrow + c0)[i]
+                                       : make_uint4(0, 0, 0, 0);
+#pragma unroll
+            for (int qq = 0; qq < 4; ++qq) {
+              float v[16];
+              tmem_ld16(tbase + c0 + 16 * qq, v);
+              const uint16_t* hs = reinterpret_cast<const uint16_t*>(&hv[2 * qq]);
+              uint32_t pk[8];
+#pragma unroll
+              for (int i = 0; i < 16; i += 2) {
+                const int col = c0 + 16 * qq + i;
+                const float o0 = s_coef[col] * bf16_to_f32(hs[i]) + s_coef[BN + col] * round_bf16(v[i]);
+                const float o1 =
+                    s_coef[col + 1] * bf16_to_f32(hs[i + 1]) + s_coef[BN + col + 1] * round_bf16(v[i + 1]);
+                pk[i / 2] = pack_bf16x2(o0, o1);
+              }
+              if (valid) {
+                uint4* dst = reinterpret_cast<uint4*>(out + c0 + 16 * qq);
+                dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+              }
+            }
+          }
         } else {
           uint16_t* out = static_cast<uint16_t*>(p.out) + row * p.Nout + f0;
           for (int c0 = 0; c0 < BN; c0 += 16) {
@@ -350,28 +403,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
               if (p.gamma) {
 #pragma unroll
                 for (int i = 0; i < 16; ++i) v[i] = round_bf16(v[i]) * (1.0f + p.gamma[f0 + c0 + i]);
-              }
-            } else if constexpr (kEpi == EPI_RESGATE) {
-              if (valid) {
-                const uint4* hp = reinterpret_cast<const uint4*>(p.resid + row * p.Nout + f0 + c0);
-                uint4 h0 = hp[0], h1 = hp[1];
-                const uint16_t* hs0 = reinterpret_cast<const uint16_t*>(&h0);
-                const uint16_t* hs1 = reinterpret_cast<const uint16_t*>(&h1);
-#pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                  const float b = round_bf16(v[i]);
-                  const float h = bf16_to_f32(i < 8 ? hs0[i] : hs1[i - 8]);
-                  const float g = p.gparam ? p.gparam[f0 + c0 + i] : 0.0f;
-                  if (p.resid_mode == MOE_RESID_MUSE_GATE) {
-                    const float beta = sigmoidf_(g / p.tau);
-                    const float a2 = fmaxf(sigmoidf_(-g / p.tau) * (1.0f + beta), p.floor_);
-                    v[i] = sqrtf(a2) * h + beta * b;
-                  } else if (p.resid_mode == MOE_RESID_LITERAL) {
-                    v[i] = h + g * b;
-                  } else {
-                    v[i] = b;
-                  }
-                }
               }
             }
             if (valid) {

@@ -179,28 +179,41 @@ __global__ void combine_bf16_kernel(const uint16_t* __restrict__ s, int E, int k
                                     const int32_t* __restrict__ inv_perm,
                                     const float* __restrict__ topk_w, int expert_norm, float eps,
                                     uint16_t* __restrict__ y) {
+  // Two passes over the k rows so that few registers are live and several CTAs share an SM:
+  // pass 1 reduces each row's sum of squares, pass 2 re-reads the rows (now in L1/L2) and
+  // accumulates the weighted, normalised values.
   __shared__ float red[8][kMaxTopK];
+  __shared__ int s_row[kMaxTopK];
+  __shared__ float s_w[kMaxTopK], s_rinv[kMaxTopK];
   const int t = blockIdx.x;
   const int nvec = E / 8;
-  uint4 r[kMaxTopK][VEC];
-  float ss[kMaxTopK];
-#pragma unroll
-  for (int j = 0; j < kMaxTopK; ++j) {
-    ss[j] = 0.0f;
+  if (threadIdx.x < kMaxTopK) {
+    const int j = threadIdx.x;
     const int row = j < k ? inv_perm[static_cast<size_t>(t) * k + j] : -1;
-#pragma unroll
-    for (int v = 0; v < VEC; ++v) {
-      const int vi = threadIdx.x + v * blockDim.x;
-      r[j][v] = (row >= 0 && vi < nvec)
-                    ? reinterpret_cast<const uint4*>(s + static_cast<size_t>(row) * E)[vi]
-                    : make_uint4(0, 0, 0, 0);
-      const uint16_t* h = reinterpret_cast<const uint16_t*>(&r[j][v]);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) { const float f = bf16_to_f32(h[i]); ss[j] += f * f; }
-    }
+    s_row[j] = row;
+    s_w[j] = row >= 0 ? topk_w[static_cast<size_t>(t) * k + j] : 0.0f;
+    s_rinv[j] = 1.0f;
   }
-  float rinv[kMaxTopK];
+  __syncthreads();
   if (expert_norm) {
+    float ss[kMaxTopK];
+#pragma unroll
+    for (int j = 0; j < kMaxTopK; ++j) {
+      ss[j] = 0.0f;
+      const int row = s_row[j];
+      if (row < 0) continue;
+      const uint4* src = reinterpret_cast<const uint4*>(s + static_cast<size_t>(row) * E);
+#pragma unroll
+      for (int v = 0; v < VEC; ++v) {
+        const int vi = threadIdx.x + v * blockDim.x;
+        if (vi < nvec) {
+          const uint4 q = src[vi];
+          const uint16_t* h = reinterpret_cast<const uint16_t*>(&q);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) { const float f = bf16_to_f32(h[i]); ss[j] += f * f; }
+        }
+      }
+    }
     const int w = threadIdx.x >> 5, nw = blockDim.x >> 5;
 #pragma unroll
     for (int j = 0; j < kMaxTopK; ++j) {
@@ -209,33 +222,29 @@ __global__ void combine_bf16_kernel(const uint16_t* __restrict__ s, int E, int k
       if ((threadIdx.x & 31) == 0) red[w][j] = ss[j];
     }
     __syncthreads();
-#pragma unroll
-    for (int j = 0; j < kMaxTopK; ++j) {
+    if (threadIdx.x < kMaxTopK) {
       float tot = 0.0f;
-      for (int i = 0; i < nw; ++i) tot += red[i][j];
-      rinv[j] = rsqrtf(tot / static_cast<float>(E) + eps);
+      for (int i = 0; i < nw; ++i) tot += red[i][threadIdx.x];
+      s_rinv[threadIdx.x] = rsqrtf(tot / static_cast<float>(E) + eps);
     }
-  }
-  float wt[kMaxTopK];
-#pragma unroll
-  for (int j = 0; j < kMaxTopK; ++j) {
-    const int row = j < k ? inv_perm[static_cast<size_t>(t) * k + j] : -1;
-    wt[j] = row >= 0 ? topk_w[static_cast<size_t>(t) * k + j] : 0.0f;
+    __syncthreads();
   }
 #pragma unroll
   for (int v = 0; v < VEC; ++v) {
     const int vi = threadIdx.x + v * blockDim.x;
     if (vi >= nvec) continue;
     float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-#pragma unroll
-    for (int j = 0; j < kMaxTopK; ++j) {
-      if (j >= k) break;
-      const uint16_t* h = reinterpret_cast<const uint16_t*>(&r[j][v]);
+    for (int j = 0; j < k; ++j) {
+      const int row = s_row[j];
+      if (row < 0) continue;
+      const uint4 q = reinterpret_cast<const uint4*>(s + static_cast<size_t>(row) * E)[vi];
+      const uint16_t* h = reinterpret_cast<const uint16_t*>(&q);
+      const float rj = s_rinv[j], wj = s_w[j];
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         const float sv = bf16_to_f32(h[i]);
-        const float nv = expert_norm ? round_bf16(sv * rinv[j]) : sv;
-        acc[i] += wt[j] * nv;
+        const float nv = expert_norm ? round_bf16(sv * rj) : sv;
+        acc[i] += wj * nv;
       }
     }
     uint4 o;
@@ -269,6 +278,113 @@ __global__ void combine_f32_kernel(const float* __restrict__ s, int E, int k,
       if (c < E) acc += topk_w[static_cast<size_t>(t) * k + j] * (sr[c] * rinv);
     }
     if (c < E) y[static_cast<size_t>(t) * E + c] = acc;
+  }
+}
+
+// ------------------------------------------------------------------ router for few tokens
+//
+// With a few dozen tokens the router is a 4 MB weight stream that one GEMM tile cannot spread over
+// the GPU.  Here a CTA takes kRouterTok tokens (staged in shared memory) and kRouterExp experts;
+// each warp owns experts, lanes stride the model width in 16-byte vectors, and the fp32 sums of
+// the exact bf16 products are reduced across the warp.  A second kernel selects the top k.
+constexpr int kRouterTok = 8;
+constexpr int kRouterExp = 16;
+
+__global__ void __launch_bounds__(256) router_logits_small_kernel(
+    const uint16_t* __restrict__ u, const uint16_t* __restrict__ w, const float* __restrict__ bias,
+    int T, int d, int n, float* __restrict__ logits) {
+  extern __shared__ uint4 s_u[];  // [kRouterTok][d/8]
+  const int t0 = blockIdx.y * kRouterTok;
+  const int nt = min(kRouterTok, T - t0);
+  const int nvec = d / 8;
+  for (int i = threadIdx.x; i < kRouterTok * nvec; i += blockDim.x) {
+    const int tt = i / nvec, v = i - tt * nvec;
+    s_u[i] = tt < nt ? reinterpret_cast<const uint4*>(u + static_cast<size_t>(t0 + tt) * d)[v]
+                     : make_uint4(0, 0, 0, 0);
+  }
+  __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
+  for (int el = warp; el < kRouterExp; el += nwarps) {
+    const int e = blockIdx.x * kRouterExp + el;
+    if (e >= n) break;
+    const uint4* wr = reinterpret_cast<const uint4*>(w + static_cast<size_t>(e) * d);
+    float acc[kRouterTok];
+#pragma unroll
+    for (int tt = 0; tt < kRouterTok; ++tt) acc[tt] = 0.0f;
+    for (int v = lane; v < nvec; v += 32) {
+      const uint4 wq = wr[v];
+      const uint16_t* wh = reinterpret_cast<const uint16_t*>(&wq);
+      float wf[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) wf[i] = bf16_to_f32(wh[i]);
+#pragma unroll
+      for (int tt = 0; tt < kRouterTok; ++tt) {
+        const uint4 uq = s_u[tt * nvec + v];
+        const uint16_t* uh = reinterpret_cast<const uint16_t*>(&uq);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[tt] = fmaf(bf16_to_f32(uh[i]), wf[i], acc[tt]);
+      }
+    }
+#pragma unroll
+    for (int tt = 0; tt < kRouterTok; ++tt) {
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) acc[tt] += __shfl_xor_sync(0xffffffffu, acc[tt], o);
+    }
+    if (lane < nt) {
+      float l = acc[0];
+#pragma unroll
+      for (int tt = 1; tt < kRouterTok; ++tt)
+        if (lane == tt) l = acc[tt];
+      logits[static_cast<size_t>(t0 + lane) * n + e] = l + (bias ? bias[e] : 0.0f);
+    }
+  }
+}
+
+// One warp per token: the k largest logits (ties to the lower index), in descending order, and
+// the weights exp(l_j - l_1) / sum_sel exp(l - l_1) * routed_scale.
+__global__ void topk_rows_kernel(const float* __restrict__ logits, int T, int n, int k,
+                                 float routed_scale, int32_t* __restrict__ topk_idx,
+                                 float* __restrict__ topk_w) {
+  const int warps = blockDim.x >> 5;
+  const int t = blockIdx.x * warps + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (t >= T) return;
+  float l[kMaxExperts / 32];
+#pragma unroll
+  for (int i = 0; i < kMaxExperts / 32; ++i) {
+    const int e = lane + 32 * i;
+    l[i] = e < n ? logits[static_cast<size_t>(t) * n + e] : -INFINITY;
+  }
+  float top_v[kMaxTopK];
+  int top_i[kMaxTopK];
+  for (int j = 0; j < k; ++j) {
+    float bv = -INFINITY;
+    int bi = 0x7fffffff;
+#pragma unroll
+    for (int i = 0; i < kMaxExperts / 32; ++i) {
+      const int e = lane + 32 * i;
+      if (e < n && (l[i] > bv || (l[i] == bv && e < bi))) { bv = l[i]; bi = e; }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+      if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
+    }
+    top_v[j] = bv;
+    top_i[j] = bi;
+#pragma unroll
+    for (int i = 0; i < kMaxExperts / 32; ++i)
+      if (lane + 32 * i == bi) l[i] = -INFINITY;
+  }
+  if (lane == 0) {
+    float sum = 0.0f;
+    for (int j = 0; j < k; ++j) sum += __expf(top_v[j] - top_v[0]);
+    const float scale = routed_scale / sum;
+    for (int j = 0; j < k; ++j) {
+      topk_idx[static_cast<size_t>(t) * k + j] = top_i[j];
+      topk_w[static_cast<size_t>(t) * k + j] = __expf(top_v[j] - top_v[0]) * scale;
+    }
   }
 }
 

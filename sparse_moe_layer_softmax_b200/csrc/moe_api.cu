@@ -177,7 +177,7 @@ size_t dsize(const moe_config_t& c) { return c.dtype == MOE_BF16 ? 2 : 4; }
 int nchunks(const moe_config_t& c) { return cdiv(c.T, kPermChunk); }
 
 struct Workspace {
-  size_t idx, w, z_raw, offsets, perm, inv, counts, x_perm, act, y, total;
+  size_t idx, w, logits, z_raw, offsets, perm, inv, counts, x_perm, act, y, total;
 };
 
 Workspace layout(const moe_config_t& c) {
@@ -187,6 +187,7 @@ Workspace layout(const moe_config_t& c) {
   auto take = [&](size_t bytes) { size_t at = o; o = align_up(o + bytes, 256); return at; };
   L.idx = take(TK * 4);
   L.w = take(TK * 4);
+  L.logits = take(static_cast<size_t>(c.T) * c.n_experts * 4);
   L.z_raw = take(c.d_latent > 0 ? static_cast<size_t>(c.T) * c.d_latent * ds : 0);
   L.offsets = take((c.n_experts + 1) * 4);
   L.perm = take(TK * 4);
@@ -216,8 +217,13 @@ void pick_expert_orient(const moe_config_t& c, int nout, bool dual, Orient* o, i
 
 // ------------------------------------------------------------------ steps
 
+// Tokens up to which the router runs as a many-CTA logits kernel + a top-k kernel (a single
+// GEMM tile would leave most SMs idle while it streams the router weights).
+constexpr int kSmallRouterMaxT = 256;
+
 moe_status_t do_route(const moe_config_t& c, const void* u, const void* w_router,
-                      const float* bias, float* logits, int32_t* idx, float* w, cudaStream_t st) {
+                      const float* bias, float* logits, int32_t* idx, float* w, cudaStream_t st,
+                      float* logits_scratch = nullptr) {
   if (c.T == 0) return MOE_OK;
   if (c.dtype == MOE_F32) {
     const int warps = 4;
@@ -225,6 +231,24 @@ moe_status_t do_route(const moe_config_t& c, const void* u, const void* w_router
         static_cast<const float*>(u), static_cast<const float*>(w_router), bias, c.T, c.d_model,
         c.n_experts, c.top_k, c.routed_scale, logits, idx, w);
     return last_launch();
+  }
+  float* lbuf = logits ? logits : logits_scratch;
+  const size_t small_smem = static_cast<size_t>(kRouterTok) * c.d_model * 2;
+  if (c.T <= kSmallRouterMaxT && lbuf && small_smem <= 200 * 1024) {
+    static std::once_flag once;
+    static cudaError_t attr = cudaSuccess;
+    std::call_once(once, [] {
+      attr = cudaFuncSetAttribute(router_logits_small_kernel,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+    });
+    if (attr != cudaSuccess) return MOE_ERR_CUDA;
+    dim3 grid(cdiv(c.n_experts, kRouterExp), cdiv(c.T, kRouterTok));
+    router_logits_small_kernel<<<grid, 256, small_smem, st>>>(
+        static_cast<const uint16_t*>(u), static_cast<const uint16_t*>(w_router), bias, c.T,
+        c.d_model, c.n_experts, lbuf);
+    topk_rows_kernel<<<cdiv(c.T, 8), 256, 0, st>>>(lbuf, c.T, c.n_experts, c.top_k,
+                                                    c.routed_scale, idx, w);
+    return last_launch(2);
   }
   GemmParams p{};
   p.G = 1;
@@ -605,7 +629,9 @@ moe_status_t moe_layer_forward(const moe_config_t* cfg, const moe_weights_t* w, 
   void* act = at<void>(workspace, L.act);
 
   prof_mark(st, 0);
-  if ((s = do_route(c, u, w->w_router, w->logit_bias, logits_out, idx, wt, st)) != MOE_OK) return s;
+  if ((s = do_route(c, u, w->w_router, w->logit_bias, logits_out, idx, wt, st,
+                    at<float>(workspace, L.logits))) != MOE_OK)
+    return s;
   prof_mark(st, 1);
   const void* xin = u;
   if (latent) {
