@@ -148,6 +148,67 @@ class ClockSampler:
                 "power_w_max": max(power), "samples": len(sm), "reasons": sorted(reasons)}
 
 
+class NvmlClockSampler:
+    """Reads the SM clock, power and clock-event reasons of one GPU every 20 ms through NVML
+    (read-only queries) on a background thread while the timed region runs."""
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"))
+
+    def __init__(self, device_index: int):
+        import threading
+        import pynvml
+        import torch
+        self.nv = pynvml
+        pynvml.nvmlInit()
+        props = torch.cuda.get_device_properties(device_index)
+        bus = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
+        self.handle = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+        self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.handle, pynvml.NVML_CLOCK_SM)
+        self.samples = []
+        self.stop_evt = threading.Event()
+        self.thread = threading.Thread(target=self._run, daemon=True)
+
+    def _run(self):
+        nv = self.nv
+        while not self.stop_evt.is_set():
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(self.handle, nv.NVML_CLOCK_SM)
+                pw = nv.nvmlDeviceGetPowerUsage(self.handle) / 1000.0
+                rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self.handle)
+                self.samples.append((sm, pw, rs))
+            except nv.NVMLError:
+                pass
+            self.stop_evt.wait(0.02)
+
+    def start(self):
+        self.thread.start()
+
+    def stop(self) -> dict:
+        self.stop_evt.set()
+        self.thread.join(timeout=5)
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["no samples"]}
+        reasons = set()
+        for _, _, rs in self.samples:
+            for name, const in self.REASONS:
+                if rs & getattr(self.nv, const):
+                    reasons.add(name)
+        sm = [s for s, _, _ in self.samples]
+        return {"sm_mhz": statistics.median(sm), "sm_min_mhz": min(sm), "sm_max_mhz": self.max_mhz,
+                "power_w_median": round(statistics.median(p for _, p, _ in self.samples), 1),
+                "power_w_max": round(max(p for _, p, _ in self.samples), 1),
+                "samples": len(self.samples), "source": "nvml 20 ms", "reasons": sorted(reasons)}
+
+
+def make_sampler(local: int):
+    try:
+        return NvmlClockSampler(local)
+    except Exception:  # no NVML: fall back to nvidia-smi sampling
+        return ClockSampler(visible_gpu_index(local))
+
+
 def measured_peaks() -> dict:
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -452,7 +513,7 @@ BAD_REASONS = {"hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown"}
 def measure_checked(cfg, args, device, peaks, rank, local, with_e2e=True) -> dict:
     """Measure; re-measure once if the clocks record shows a rejected throttle reason."""
     for attempt in range(2):
-        sampler = ClockSampler(visible_gpu_index(local)) if rank == 0 else None
+        sampler = make_sampler(local) if rank == 0 else None
         res = measure_ours(cfg, args.steps, args.warmup, device, peaks, with_e2e, sampler)
         clk = res.get("clocks") or {}
         bad = BAD_REASONS & set(clk.get("reasons") or [])

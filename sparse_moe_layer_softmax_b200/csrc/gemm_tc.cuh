@@ -79,6 +79,22 @@ constexpr int kSmemMisc = 8192;  // barriers, TMEM slot, group tables, residual-
 // Barrier 1 among the 128 epilogue threads only (barrier 0 is __syncthreads).
 __device__ __forceinline__ void epilogue_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
+// Barrier 1 with an AND over the 128 epilogue threads: every thread gets the same answer, so a
+// bounded wait that ran out in one thread makes all of them leave together (none is left
+// waiting at a later barrier for threads that already left).
+__device__ __forceinline__ bool epilogue_all(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, 1, 128, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(v))
+      : "memory");
+  return r != 0;
+}
+
 template <bool kSwap, int BN, int kEpi, int kStages>
 constexpr int gemm_smem_bytes() {
   return kStages * GemmShape<kSwap, BN, kEpi>::kStageBytes + 1024 + kSmemMisc;
@@ -134,6 +150,145 @@ struct TopK {
     }
   }
 };
+
+// Epilogue of the normal orientation: this thread owns row row0 + 32*q + lane of the tile (valid
+// if below nrows) and the tile's BN accumulator columns (output features f0 ...).
+template <int BN, int kEpi>
+__device__ __forceinline__ void epilogue_rows(const GemmParams& p, int row0, int nrows, int f0,
+                                              uint32_t tbase, int q, int lane, float* s_coef) {
+    const int rl = q * 32 + lane;
+    const bool valid = rl < nrows;
+    const size_t row = static_cast<size_t>(row0 + rl);
+    if constexpr (kEpi == EPI_ROUTER) {
+      TopK<8> tk;
+      tk.init();
+      for (int c0 = 0; c0 < BN; c0 += 16) {
+        float v[16];
+        tmem_ld16(tbase + c0, v);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int col = c0 + i;
+          if (col < p.Nout) {
+            float l = v[i] + (p.bias ? p.bias[col] : 0.0f);
+            v[i] = l;
+            tk.push(l, col, p.top_k);
+          }
+        }
+        if (valid && p.logits) {
+          float* dst = p.logits + row * p.Nout + c0;
+          if (c0 + 16 <= p.Nout && (p.Nout & 3) == 0) {
+#pragma unroll
+            for (int i = 0; i < 16; i += 4)
+              *reinterpret_cast<float4*>(dst + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+          } else {
+            for (int i = 0; c0 + i < p.Nout; ++i) dst[i] = v[i];
+          }
+        }
+      }
+      if (valid) {
+        float sum = 0.0f;
+        float e[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          e[j] = (j < p.top_k) ? __expf(tk.v[j] - tk.v[0]) : 0.0f;
+          sum += e[j];
+        }
+        const float scale = p.routed_scale / sum;
+        for (int j = 0; j < p.top_k; ++j) {
+          p.topk_idx[row * p.top_k + j] = tk.i[j];
+          p.topk_w[row * p.top_k + j] = e[j] * scale;
+        }
+      }
+    } else if constexpr (kEpi == EPI_SWIGLU) {
+      uint16_t* out = static_cast<uint16_t*>(p.out) + row * p.Nout + f0;
+      for (int c0 = 0; c0 < BN / 2; c0 += 16) {
+        float gv[16], uv[16];
+        tmem_ld16(tbase + c0, gv);
+        tmem_ld16(tbase + BN / 2 + c0, uv);
+        uint32_t pk[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          pk[i] = pack_bf16x2(silu(gv[2 * i]) * uv[2 * i], silu(gv[2 * i + 1]) * uv[2 * i + 1]);
+        if (valid) {
+          uint4* dst = reinterpret_cast<uint4*>(out + c0);
+          dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+        }
+      }
+    } else if constexpr (kEpi == EPI_RESGATE) {
+      // Per-column coefficients of this tile, computed once by the 128 epilogue threads:
+      // out = alpha * r + beta * b  (MUSE gate: beta = sigmoid(g/tau), alpha =
+      // sqrt(max(sigmoid(-g/tau)(1+beta), floor)); literal: alpha = 1, beta = g; none: 0, 1).
+      epilogue_bar();  // the previous tile's readers are done with s_coef
+      for (int cc = static_cast<int>(threadIdx.x) - 64; cc < BN; cc += 128) {
+        const float g = p.gparam ? p.gparam[f0 + cc] : 0.0f;
+        float a = 0.0f, b = 1.0f;
+        if (p.resid_mode == MOE_RESID_MUSE_GATE) {
+          b = sigmoidf_(g / p.tau);
+          a = sqrtf(fmaxf(sigmoidf_(-g / p.tau) * (1.0f + b), p.floor_));
+        } else if (p.resid_mode == MOE_RESID_LITERAL) {
+          a = 1.0f;
+          b = g;
+        }
+        s_coef[cc] = a;
+        s_coef[BN + cc] = b;
+      }
+      epilogue_bar();
+      const bool has_r = p.resid_mode != MOE_RESID_NONE;
+      uint16_t* out = static_cast<uint16_t*>(p.out) + row * p.Nout + f0;
+      const uint16_t* hrow = has_r ? p.resid + row * p.Nout + f0 : nullptr;
+      for (int c0 = 0; c0 < BN; c0 += 64) {
+        uint4 hv[8];  // 64 residual values, loaded together so their latency overlaps
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          hv[i] = (valid && has_r) ? reinterpret_cast<const uint4*>(hrow + c0)[i]
+                                   : make_uint4(0, 0, 0, 0);
+#pragma unroll
+        for (int qq = 0; qq < 4; ++qq) {
+          float v[16];
+          tmem_ld16(tbase + c0 + 16 * qq, v);
+          const uint16_t* hs = reinterpret_cast<const uint16_t*>(&hv[2 * qq]);
+          uint32_t pk[8];
+#pragma unroll
+          for (int i = 0; i < 16; i += 2) {
+            const int col = c0 + 16 * qq + i;
+            const float o0 = s_coef[col] * bf16_to_f32(hs[i]) + s_coef[BN + col] * round_bf16(v[i]);
+            const float o1 =
+                s_coef[col + 1] * bf16_to_f32(hs[i + 1]) + s_coef[BN + col + 1] * round_bf16(v[i + 1]);
+            pk[i / 2] = pack_bf16x2(o0, o1);
+          }
+          if (valid) {
+            uint4* dst = reinterpret_cast<uint4*>(out + c0 + 16 * qq);
+            dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+          }
+        }
+      }
+    } else {
+      uint16_t* out = static_cast<uint16_t*>(p.out) + row * p.Nout + f0;
+      for (int c0 = 0; c0 < BN; c0 += 16) {
+        float v[16];
+        tmem_ld16(tbase + c0, v);
+        if constexpr (kEpi == EPI_RELU) {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) v[i] = fmaxf(v[i], 0.0f);
+        } else if constexpr (kEpi == EPI_STORE) {
+          if (p.gamma) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) v[i] = round_bf16(v[i]) * (1.0f + p.gamma[f0 + c0 + i]);
+          }
+        }
+        if (valid) {
+          uint32_t pk[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) pk[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
+          uint4* dst = reinterpret_cast<uint4*>(out + c0);
+          dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+        }
+      }
+    }
+}
 
 template <bool kSwap, int BN, int kEpi, int kStages>
 __global__ void __launch_bounds__(kGemmThreads, 1)
@@ -278,143 +433,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     uint32_t acc = 0, acc_phase = 0;
     for (int t = blockIdx.x; t < total; t += gridDim.x) {
       TileCoord c = decode_tile(t, s_seg, s_pref, G, FT, S::kCH);
-      if (!mbar_wait(&tfull[acc], acc_phase)) break;
+      if (!epilogue_all(mbar_wait(&tfull[acc], acc_phase))) break;
       tc_fence_after();
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * S::kAccCols;
       const int f0 = c.ft * S::kFO;
       if constexpr (!kSwap) {
-        const int rl = q * 32 + lane;
-        const bool valid = rl < c.nrows;
-        const size_t row = static_cast<size_t>(c.row0 + rl);
-        if constexpr (kEpi == EPI_ROUTER) {
-          TopK<8> tk;
-          tk.init();
-          for (int c0 = 0; c0 < BN; c0 += 16) {
-            float v[16];
-            tmem_ld16(tbase + c0, v);
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const int col = c0 + i;
-              if (col < p.Nout) {
-                float l = v[i] + (p.bias ? p.bias[col] : 0.0f);
-                v[i] = l;
-                tk.push(l, col, p.top_k);
-              }
-            }
-            if (valid && p.logits) {
-              float* dst = p.logits + row * p.Nout + c0;
-              if (c0 + 16 <= p.Nout && (p.Nout & 3) == 0) {
-#pragma unroll
-                for (int i = 0; i < 16; i += 4)
-                  *reinterpret_cast<float4*>(dst + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
-              } else {
-                for (int i = 0; c0 + i < p.Nout; ++i) dst[i] = v[i];
-              }
-            }
-          }
-          if (valid) {
-            float sum = 0.0f;
-            float e[8];
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              e[j] = (j < p.top_k) ? __expf(tk.v[j] - tk.v[0]) : 0.0f;
-              sum += e[j];
-            }
-            const float scale = p.routed_scale / sum;
-            for (int j = 0; j < p.top_k; ++j) {
-              p.topk_idx[row * p.top_k + j] = tk.i[j];
-              p.topk_w[row * p.top_k + j] = e[j] * scale;
-            }
-          }
-        } else if constexpr (kEpi == EPI_SWIGLU) {
-          uint16_t* out = static_cast<uint16_t*>(p.out) + row * p.Nout + f0;
-          for (int c0 = 0; c0 < BN / 2; c0 += 16) {
-            float gv[16], uv[16];
-            tmem_ld16(tbase + c0, gv);
-            tmem_ld16(tbase + BN / 2 + c0, uv);
-            uint32_t pk[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i)
-              pk[i] = pack_bf16x2(silu(gv[2 * i]) * uv[2 * i], silu(gv[2 * i + 1]) * uv[2 * i + 1]);
-            if (valid) {
-              uint4* dst = reinterpret_cast<uint4*>(out + c0);
-              dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-              dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-            }
-          }
-        } else if constexpr (kEpi == EPI_RESGATE) {
-          // Per-column coefficients of this tile, computed once by the 128 epilogue threads:
-          // out = alpha * r + beta * b  (MUSE gate: beta = sigmoid(g/tau), alpha =
-          // sqrt(max(sigmoid(-g/tau)(1+beta), floor)); literal: alpha = 1, beta = g; none: 0, 1).
-          epilogue_bar();  // the previous tile's readers are done with s_coef
-          for (int cc = static_cast<int>(threadIdx.x) - 64; cc < BN; cc += 128) {
-            const float g = p.gparam ? p.gparam[f0 + cc] : 0.0f;
-            float a = 0.0f, b = 1.0f;
-            if (p.resid_mode == MOE_RESID_MUSE_GATE) {
-              b = sigmoidf_(g / p.tau);
-              a = sqrtf(fmaxf(sigmoidf_(-g / p.tau) * (1.0f + b), p.floor_));
-            } else if (p.resid_mode == MOE_RESID_LITERAL) {
-              a = 1.0f;
-              b = g;
-            }
-            s_coef[cc] = a;
-            s_coef[BN + cc] = b;
-          }
-          epilogue_bar();
-          const bool has_r = p.resid_mode != MOE_RESID_NONE;
-          uint16_t* out = static_cast<uint16_t*>(p.out) + row * p.Nout + f0;
-          const uint16_t* hrow = has_r ? p.resid + row * p.Nout + f0 : nullptr;
-          for (int c0 = 0; c0 < BN; c0 += 64) {
-            uint4 hv[8];  // 64 residual values, loaded together so their latency overlaps
-#pragma unroll
-            for (int i = 0; i < 8; ++i)
-              hv[i] = (valid && has_r) ? reinterpret_cast<const uint4*>(hrow + c0)[i]
-                                       : make_uint4(0, 0, 0, 0);
-#pragma unroll
-            for (int qq = 0; qq < 4; ++qq) {
-              float v[16];
-              tmem_ld16(tbase + c0 + 16 * qq, v);
-              const uint16_t* hs = reinterpret_cast<const uint16_t*>(&hv[2 * qq]);
-              uint32_t pk[8];
-#pragma unroll
-              for (int i = 0; i < 16; i += 2) {
-                const int col = c0 + 16 * qq + i;
-                const float o0 = s_coef[col] * bf16_to_f32(hs[i]) + s_coef[BN + col] * round_bf16(v[i]);
-                const float o1 =
-                    s_coef[col + 1] * bf16_to_f32(hs[i + 1]) + s_coef[BN + col + 1] * round_bf16(v[i + 1]);
-                pk[i / 2] = pack_bf16x2(o0, o1);
-              }
-              if (valid) {
-                uint4* dst = reinterpret_cast<uint4*>(out + c0 + 16 * qq);
-                dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-                dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-              }
-            }
-          }
-        } else {
-          uint16_t* out = static_cast<uint16_t*>(p.out) + row * p.Nout + f0;
-          for (int c0 = 0; c0 < BN; c0 += 16) {
-            float v[16];
-            tmem_ld16(tbase + c0, v);
-            if constexpr (kEpi == EPI_RELU) {
-#pragma unroll
-              for (int i = 0; i < 16; ++i) v[i] = fmaxf(v[i], 0.0f);
-            } else if constexpr (kEpi == EPI_STORE) {
-              if (p.gamma) {
-#pragma unroll
-                for (int i = 0; i < 16; ++i) v[i] = round_bf16(v[i]) * (1.0f + p.gamma[f0 + c0 + i]);
-              }
-            }
-            if (valid) {
-              uint32_t pk[8];
-#pragma unroll
-              for (int i = 0; i < 8; ++i) pk[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
-              uint4* dst = reinterpret_cast<uint4*>(out + c0);
-              dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-              dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-            }
-          }
-        }
+        epilogue_rows<BN, kEpi>(p, c.row0, c.nrows, f0, tbase, q, lane, s_coef);
       } else {
         // swap orientation: this thread owns output feature f for the BN rows of the chunk
         const int f = f0 + q * 32 + lane;
@@ -469,6 +493,205 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   if (warp == 1) {
     __syncwarp();
     tmem_dealloc(tmem_base, S::kTmemCols);
+  }
+}
+
+// ==================================================================== CTA-pair variant
+//
+// Normal orientation with a 256 x BN tile computed by the two CTAs of a cluster:
+// tcgen05.mma.cta_group::2 (M = 256) issued by the leader, each CTA holding 128 rows of X and
+// BN/2 rows of W in its own shared memory, each CTA's TMEM holding the accumulator of its 128
+// rows.  Per SM this halves the W bytes staged and read per MMA, which is what bounds the 1-SM
+// 128 x 256 tile (its TMA fill plus operand reads exceed the shared-memory bandwidth).
+//   - Both CTAs load their halves with cta_group::2 TMA (no multicast); the bytes complete on
+//     the leader's full barrier, whose expected count the leader sets for both halves.
+//   - The leader's MMA commits arrive on both CTAs' empty / tmem-full barriers (multicast commit).
+//   - Each CTA's epilogue drains its own TMEM lanes; one thread per CTA then arrives on the
+//     leader's tmem-empty barrier (count 2).
+//   - For SwiGLU the leader loads the 128 gate rows and the peer the 128 up rows, so accumulator
+//     columns [0, 128) are the gate and [128, 256) the up projection, as in the 1-SM tile.
+
+template <int BN, int kEpi>
+struct PairShape {
+  static constexpr bool kDual = (kEpi == EPI_SWIGLU);
+  static constexpr int kBK = 64;
+  static constexpr int kABytes = 128 * 128;
+  static constexpr int kBBytes = (BN / 2) * 128;
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kFO = kDual ? BN / 2 : BN;
+  static constexpr int kCH = 256;
+  static constexpr int kTmemCols = 2 * BN <= 256 ? 256 : 512;
+  static constexpr uint32_t kIdesc = idesc_bf16_f32(256, BN);
+  static_assert(BN == 128 || BN == 256, "pair tile width");
+};
+
+template <int BN, int kEpi, int kStages>
+constexpr int gemm_pair_smem_bytes() {
+  return kStages * PairShape<BN, kEpi>::kStageBytes + 1024 + kSmemMisc;
+}
+
+template <int BN, int kEpi, int kStages>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
+    gemm_tc_pair_kernel(const __grid_constant__ CUtensorMap tmX,
+                        const __grid_constant__ CUtensorMap tmW, const GemmParams p) {
+  using S = PairShape<BN, kEpi>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* tiles = smem;
+  uint64_t* full = reinterpret_cast<uint64_t*>(tiles + kStages * S::kStageBytes);
+  uint64_t* empty = full + kStages;
+  uint64_t* tfull = empty + kStages;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* done = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+  int* s_seg = reinterpret_cast<int*>(tmem_slot + 4);
+  int* s_pref = s_seg + (kMaxGroups + 4);
+  float* s_coef = reinterpret_cast<float*>(s_pref + (kMaxGroups + 4));
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+  const int G = p.G;
+  const int FT = p.Nout / S::kFO;
+  const int KB = p.K / S::kBK;
+
+  if (warp == 0) {  // group segments and tile prefix, as in the 1-SM kernel (256-row chunks)
+    const int per = (G + 31) / 32;
+    int local = 0;
+    for (int j = 0; j < per; ++j) {
+      int g = lane * per + j;
+      if (g < G) {
+        int a = p.seg ? p.seg[g] : 0, b = p.seg ? p.seg[g + 1] : p.M;
+        if (b < a) { latch_status(MOE_ERR_DEVICE_CHECK); b = a; }
+        s_seg[g] = a;
+        if (g == G - 1) s_seg[G] = b;
+        local += ((b - a + S::kCH - 1) / S::kCH) * FT;
+      }
+    }
+    int incl = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    int run = incl - local;
+    for (int j = 0; j < per; ++j) {
+      int g = lane * per + j;
+      if (g < G) {
+        int a = p.seg ? p.seg[g] : 0, b = p.seg ? p.seg[g + 1] : p.M;
+        if (b < a) b = a;
+        s_pref[g] = run;
+        run += ((b - a + S::kCH - 1) / S::kCH) * FT;
+      }
+    }
+    if (lane == 31) s_pref[G] = incl;
+  }
+  if (threadIdx.x == 32) {
+    for (int s = 0; s < kStages; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+    for (int a = 0; a < 2; ++a) { mbar_init(&tfull[a], 1); mbar_init(&tempty[a], 2); }
+    mbar_init(done, 1);
+    fence_barrier_init();
+  }
+  if (warp == 1) tmem_alloc_pair(tmem_slot, S::kTmemCols);
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();  // the peer's barriers exist before any remote arrive or TMA completion
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int total = s_pref[G];
+
+  if (warp == 0 && lane == 0) {
+    // ------------------------------------------------------------ TMA producer (both CTAs)
+    tma_prefetch_desc(&tmX);
+    tma_prefetch_desc(&tmW);
+    uint32_t stage = 0, phase = 0;
+    uint32_t last_parity[kStages];
+    bool issued[kStages];
+#pragma unroll
+    for (int s = 0; s < kStages; ++s) { issued[s] = false; last_parity[s] = 0; }
+    bool ok = true;
+    for (int t = pair; t < total && ok; t += npairs) {
+      TileCoord c = decode_tile(t, s_seg, s_pref, G, FT, S::kCH);
+      const int xrow = c.row0 + 128 * static_cast<int>(rank);
+      const int wrow = S::kDual ? c.g * p.Nw + (leader ? 0 : p.Nw / 2) + c.ft * (BN / 2)
+                                : c.g * p.Nw + c.ft * BN + static_cast<int>(rank) * (BN / 2);
+      for (int kb = 0; kb < KB; ++kb) {
+        if (!mbar_wait(&empty[stage], phase ^ 1)) { ok = false; break; }
+        uint8_t* sa = tiles + stage * S::kStageBytes;
+        uint8_t* sb = sa + S::kABytes;
+        if (leader) mbar_arrive_expect_tx(&full[stage], 2 * S::kStageBytes);
+        const uint32_t fb = cluster_addr(&full[stage], 0);
+        const int kx = kb * S::kBK;
+        tma_load_2d_pair(&tmX, fb, sa, kx, xrow);
+        tma_load_2d_pair(&tmW, fb, sb, kx, wrow);
+        issued[stage] = true;
+        last_parity[stage] = phase;
+        if (++stage == kStages) { stage = 0; phase ^= 1; }
+      }
+    }
+    // The leader's full barriers count both CTAs' bytes: no copy is still landing afterwards.
+    if (leader)
+      for (int s = 0; s < kStages; ++s)
+        if (issued[s]) mbar_wait(&full[s], last_parity[s]);
+  } else if (warp == 1 && lane == 0) {
+    // ------------------------------------------------------------ MMA issuer (leader only)
+    if (leader) {
+      uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
+      bool ok = true;
+      for (int t = pair; t < total && ok; t += npairs) {
+        if (!mbar_wait(&tempty[acc], acc_phase ^ 1)) break;
+        tc_fence_after();
+        const uint32_t d = tmem_base + acc * BN;
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!mbar_wait(&full[stage], phase)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(tiles + stage * S::kStageBytes);
+          const uint32_t b_addr = a_addr + S::kABytes;
+#pragma unroll
+          for (int k = 0; k < S::kBK / 16; ++k)
+            tc_mma_bf16_pair(d, smem_desc_k128(a_addr + 32 * k), smem_desc_k128(b_addr + 32 * k),
+                             S::kIdesc, (kb | k) != 0);
+          tc_commit_pair(&empty[stage], 0x3);
+          if (++stage == kStages) { stage = 0; phase ^= 1; }
+        }
+        if (!ok) break;
+        tc_commit_pair(&tfull[acc], 0x3);
+        if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+      }
+      tc_commit_pair(done, 0x3);  // both CTAs learn that every pair MMA has finished
+    }
+    mbar_wait(done, 0);
+  } else if (warp >= 2) {
+    // ------------------------------------------------------------ epilogue (both CTAs)
+    const int q = warp & 3;
+    uint32_t acc = 0, acc_phase = 0;
+    const uint32_t tempty_leader = cluster_addr(&tempty[0], 0);
+    for (int t = pair; t < total; t += npairs) {
+      TileCoord c = decode_tile(t, s_seg, s_pref, G, FT, S::kCH);
+      const int row0 = c.row0 + 128 * static_cast<int>(rank);
+      const int nrows = max(0, min(128, c.nrows - 128 * static_cast<int>(rank)));
+      if (!epilogue_all(mbar_wait(&tfull[acc], acc_phase))) break;
+      tc_fence_after();
+      const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * BN;
+      epilogue_rows<BN, kEpi>(p, row0, nrows, c.ft * S::kFO, tbase, q, lane, s_coef);
+      tc_fence_before();
+      epilogue_bar();  // all 128 epilogue threads have finished reading this accumulator
+      if (threadIdx.x == 64) {
+        if (leader) mbar_arrive(&tempty[acc]);
+        else mbar_arrive_cluster(tempty_leader + acc * static_cast<uint32_t>(sizeof(uint64_t)));
+      }
+      if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();  // neither CTA leaves while the pair's MMAs may still use its memory
+  tc_fence_after();
+  if (warp == 1) {
+    __syncwarp();
+    tmem_dealloc_pair(tmem_base, S::kTmemCols);
   }
 }
 

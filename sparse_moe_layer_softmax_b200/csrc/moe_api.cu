@@ -103,10 +103,35 @@ moe_status_t launch_gemm(const void* X, long x_rows, const void* W, long w_rows,
   return last_launch();
 }
 
+// CTA-pair variant: grid of whole clusters of 2.
+template <int BN, int kEpi, int kStages>
+moe_status_t launch_gemm_pair(const void* X, long x_rows, const void* W, long w_rows,
+                              const GemmParams& p, long max_tiles, cudaStream_t st) {
+  constexpr int smem = gemm_pair_smem_bytes<BN, kEpi, kStages>();
+  static_assert(smem <= 232448, "shared memory budget");
+  auto kern = gemm_tc_pair_kernel<BN, kEpi, kStages>;
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [&] {
+    attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  });
+  if (attr_err != cudaSuccess) return MOE_ERR_CUDA;
+  CUtensorMap tx, tw;
+  if (!make_tmap(&tx, X, static_cast<uint64_t>(x_rows), static_cast<uint64_t>(p.K), 128))
+    return MOE_ERR_CUDA;
+  if (!make_tmap(&tw, W, static_cast<uint64_t>(w_rows), static_cast<uint64_t>(p.K), BN / 2))
+    return MOE_ERR_CUDA;
+  long pairs = device_info().sms / 2;
+  if (max_tiles < pairs) pairs = max_tiles;
+  if (pairs <= 0) return MOE_OK;
+  kern<<<static_cast<unsigned>(2 * pairs), kGemmThreads, smem, st>>>(tx, tw, p);
+  return last_launch();
+}
+
 // Upper bound of the tile count of a grouped GEMM (each group adds at most one partial chunk).
 long tile_bound(long rows, int G, int ch, int ft) { return (static_cast<long>(cdiv(rows, ch)) + G) * ft; }
 
-enum class Orient { kNormal, kSwap };
+enum class Orient { kNormal, kSwap, kPair };
 
 // Output-feature tile choice of the normal orientation: the widest of 256/128/64 dividing Nout
 // (for SwiGLU the tile holds gate and up halves, so the output width per tile is BN/2).
@@ -133,6 +158,14 @@ moe_status_t run_gemm(int epi, Orient o, int bn, const void* X, long x_rows, con
     return MOE_ERR_UNSUPPORTED;
   }
   const int fo = dual ? bn / 2 : bn;
+  if (o == Orient::kPair) {
+    const long pt = tile_bound(x_rows, p.G, 256, cdiv(p.Nout, fo));
+#define PR(BN_, E_, ST_) \
+  if (bn == BN_ && epi == E_) return launch_gemm_pair<BN_, E_, ST_>(X, x_rows, W, w_rows, p, pt, st);
+    PR(256, EPI_SWIGLU, 6) PR(256, EPI_STORE, 6) PR(256, EPI_RELU, 6) PR(256, EPI_RESGATE, 6)
+#undef PR
+    return MOE_ERR_UNSUPPORTED;
+  }
   const long mt = tile_bound(x_rows, p.G, 128, cdiv(p.Nout, fo));
 #define NM(BN_, E_, ST_) \
   if (bn == BN_ && epi == E_) return launch_gemm<false, BN_, E_, ST_>(X, x_rows, W, w_rows, p, mt, st);
@@ -203,6 +236,15 @@ Workspace layout(const moe_config_t& c) {
 template <typename T>
 T* at(void* base, size_t off) { return reinterpret_cast<T*>(static_cast<char*>(base) + off); }
 
+// Tuning knob: MOE_GEMM_PAIR=1 in the environment selects CTA-pair 256-row tiles for large groups
+// and dense projections (same values as the 1-SM tiles).  Off by default: on this power-capped
+// part the pair kernel keeps the tensor pipe busier per clock but runs at lower clocks and reads
+// more DRAM, and its steps measured slower than the 1-SM 128 x 256 tiles.
+bool pair_tiles_enabled() {
+  const char* v = getenv("MOE_GEMM_PAIR");
+  return v && v[0] == '1';
+}
+
 // Grouped-GEMM orientation for the experts from the mean rows per expert.
 void pick_expert_orient(const moe_config_t& c, int nout, bool dual, Orient* o, int* bn) {
   const double mean_rows = static_cast<double>(c.T) * c.top_k / c.n_experts;
@@ -210,9 +252,16 @@ void pick_expert_orient(const moe_config_t& c, int nout, bool dual, Orient* o, i
     *o = Orient::kSwap;
     *bn = mean_rows <= 12.0 ? 16 : (mean_rows <= 24.0 ? 32 : 64);
   } else {
-    *o = Orient::kNormal;
     *bn = pick_bn_normal(nout, dual);
+    // 256-row CTA-pair tiles once groups are large enough to fill them
+    *o = (pair_tiles_enabled() && *bn == 256 && mean_rows >= 192.0) ? Orient::kPair
+                                                                     : Orient::kNormal;
   }
+}
+
+// Dense projections: CTA-pair tiles for at least 256 rows and a 256-wide feature tile.
+Orient dense_orient(int rows, int bn) {
+  return (pair_tiles_enabled() && bn == 256 && rows >= 256) ? Orient::kPair : Orient::kNormal;
 }
 
 // ------------------------------------------------------------------ steps
@@ -407,7 +456,8 @@ moe_status_t do_latent_down(const moe_config_t& c, const void* u, const void* p_
   p.Nw = c.d_latent;
   p.Nout = c.d_latent;
   p.out = z;
-  return run_gemm(EPI_STORE, Orient::kNormal, pick_bn_normal(c.d_latent, false), u, c.T, p_down,
+  const int bn = pick_bn_normal(c.d_latent, false);
+  return run_gemm(EPI_STORE, dense_orient(c.T, bn), bn, u, c.T, p_down,
                   c.d_latent, p, st);
 }
 
@@ -426,7 +476,8 @@ moe_status_t do_latent_up(const moe_config_t& c, const void* y, const void* p_up
   p.tau = c.tau;
   p.floor_ = c.resid_floor;
   p.resid_mode = c.resid_mode;
-  return run_gemm(EPI_RESGATE, Orient::kNormal, pick_bn_normal(c.d_model, false), y, c.T, p_up,
+  const int bn = pick_bn_normal(c.d_model, false);
+  return run_gemm(EPI_RESGATE, dense_orient(c.T, bn), bn, y, c.T, p_up,
                   c.d_model, p, st);
 }
 

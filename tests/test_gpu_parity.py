@@ -51,6 +51,10 @@ def test_generator_device_matches_host():
 SMALL = [
     # normal orientation, ragged T, several M tiles, Muse structure
     configs.small_muse(T=300, d=512, L=256, I=256, n=16, k=4, seed=11),
+    # CTA-pair tiles (>= 192 rows per expert; dense projections with T >= 256), ragged groups
+    configs.small_muse(T=517, d=512, L=256, I=256, n=4, k=2, seed=22),
+    configs.small_muse(T=1100, d=256, L=256, I=512, n=8, k=2, seed=23,
+                       resid_mode=configs.RESID_LITERAL),
     # swap orientation (few rows per expert), max experts and top-k
     configs.small_muse(T=40, d=256, L=128, I=128, n=256, k=8, seed=12),
     configs.small_muse(T=77, d=256, L=256, I=128, n=64, k=8, seed=13),
@@ -71,9 +75,23 @@ SMALL = [
 ]
 
 
+PAIR_CASES = [c for c in SMALL if c.T in (517, 1100)]
+
+
 @pytest.mark.parametrize("cfg", SMALL, ids=lambda c: f"{c.name}-n{c.n_experts}k{c.top_k}-{c.dtype}"
                          f"-r{c.resid_mode}p{c.pre_norm}")
 def test_layer_small(cfg):
+    _check_layer(cfg)
+
+
+@pytest.mark.parametrize("cfg", PAIR_CASES, ids=lambda c: c.name)
+def test_layer_small_pair_tiles(cfg, monkeypatch):
+    """The same layers with the CTA-pair 256-row GEMM tiles selected (MOE_GEMM_PAIR=1)."""
+    monkeypatch.setenv("MOE_GEMM_PAIR", "1")
+    _check_layer(cfg)
+
+
+def _check_layer(cfg):
     dev = moe_inputs.device_inputs(cfg)
     res = run_layer(cfg, dev)
     ref = oracle_reference(cfg)
@@ -176,11 +194,16 @@ def test_scatter_rows_with_centred_norm(E, gamma):
 @pytest.mark.parametrize("cfg", [
     configs.small_muse(T=200, d=256, L=256, I=384, n=8, k=2, seed=31),    # normal orientation
     configs.small_muse(T=24, d=256, L=256, I=256, n=64, k=8, seed=32),    # swap orientation
+    configs.small_muse(T=700, d=256, L=256, I=256, n=4, k=2, seed=35),    # CTA-pair tiles
+    configs.small_shazeer(T=900, d=256, h=512, n=4, k=2, seed=36),        # pair tiles, ReLU
     configs.small_shazeer(T=300, d=128, h=256, n=8, k=2, seed=33),
     configs.small_shazeer(T=20, d=128, h=256, n=64, k=4, seed=34),
 ], ids=lambda c: f"{c.name}-n{c.n_experts}k{c.top_k}-act{c.act}")
-def test_expert_ffn(cfg):
-    """Experts on dispatched rows (inputs from the generator, routing synthetic)."""
+def test_expert_ffn(cfg, monkeypatch):
+    """Experts on dispatched rows (inputs from the generator, routing synthetic); the large-group
+    cases run with the CTA-pair tiles selected."""
+    if cfg.T in (700, 900):
+        monkeypatch.setenv("MOE_GEMM_PAIR", "1")
     c = abi_config(cfg)
     T, k, n, E, H = cfg.T, cfg.top_k, cfg.n_experts, cfg.expert_in, cfg.d_ff
     idx = _rand_routing(T, n, k, seed=cfg.seed)
