@@ -213,6 +213,14 @@ MOE_API moe_status_t moe_profile_end(float* stage_ms, int32_t* calls);
  * measurement: the difference across a region is the kernels that region launched). */
 MOE_API unsigned long long moe_launch_count(void);
 
+/* Self-test of the device-side failure detection (not part of the layer): one thread waits, with
+ * the bounded wait the GEMM pipeline uses and a budget of budget_clocks SM clocks (1 .. about 2e9),
+ * on an mbarrier that nothing arrives at.  The wait runs out, latches MOE_ERR_TIMEOUT in the
+ * device status word (read it with moe_get_device_status) and writes 1 to *gave_up (device
+ * int32); the kernel then returns normally and the context stays usable. */
+MOE_API moe_status_t moe_selftest_wait_timeout(long long budget_clocks, int32_t* gave_up,
+                                               void* stream);
+
 #ifdef __cplusplus
 }
 #endif

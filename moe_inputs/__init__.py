@@ -165,7 +165,8 @@ def tensor_specs(cfg: MoEConfig):
     n, d, L, I = cfg.n_experts, cfg.d_model, cfg.d_latent, cfg.d_ff
     specs = {
         "u": ((cfg.T, d), configs.STREAM_X, "act", cfg.x_sigma),
-        "w_router": ((n, d), configs.STREAM_W_ROUTER, "w", cfg.sigma_router()),
+        "w_router": ((n, d), configs.STREAM_W_ROUTER, "f32n" if cfg.router_f32 else "w",
+                     cfg.sigma_router()),
         "w_gu": ((n, cfg.gu_rows, cfg.expert_in), configs.STREAM_W_GU, "w", cfg.sigma_w_gu()),
         "w_down": ((n, cfg.expert_in, I), configs.STREAM_W_DOWN, "w", cfg.sigma_w_down()),
     }
@@ -177,6 +178,8 @@ def tensor_specs(cfg: MoEConfig):
     if cfg.expert_norm:
         specs["gamma_expert"] = ((cfg.expert_in,), configs.STREAM_GAMMA_EXPERT, "f32n",
                                  cfg.gamma_sigma)
+    if cfg.gate_mode == configs.GATE_SIGMOID:
+        specs["correction_bias"] = ((n,), configs.STREAM_CORR_BIAS, "f32n", cfg.corr_sigma)
     if cfg.resid_mode != configs.RESID_NONE:
         specs["resid_g"] = ((d,), configs.STREAM_RESID_G, "f32u", 0.0)
     return specs

@@ -43,6 +43,9 @@ ACT_SWIGLU = 1
 RESID_NONE = 0
 RESID_MUSE_GATE = 1
 RESID_LITERAL = 2
+GATE_SOFTMAX = 0
+GATE_SIGMOID = 1
+STREAM_CORR_BIAS = 13
 
 # Scale c of the Zipf router bias  bias_e = -c * s * ln(rank_e)  (s = 1.2) for the imbalanced
 # workload.  Calibrated by tests/golden/calibrate_zipf_bias.py, which bisects c with the CPU
@@ -76,6 +79,10 @@ class MoEConfig:
     router_gain: float = 1.0  # extra factor on the router weights' std
     zipf_bias: bool = False
     gamma_sigma: float = 0.02
+    gate_mode: int = GATE_SOFTMAX
+    router_f32: int = 0         # router weights stored in fp32
+    logit_mult: float = 1.0     # output_multiplier of the sigmoid gate
+    corr_sigma: float = 0.05    # std of the sigmoid gate's selection-only correction bias
 
     @property
     def latent(self) -> bool:
@@ -137,7 +144,16 @@ CONFIGS = {c.name: c for c in (TINY_SHAZEER_F32, SHAZEER_BF16, MUSE_DECODE, MUSE
 MUSE_PREFILL_N32 = MUSE_PREFILL.replace(name="muse_prefill_n32", T=2048, n_experts=32, seed=5)
 MUSE_DECODE_N32 = MUSE_DECODE.replace(name="muse_decode_n32", T=8, n_experts=32, seed=6)
 PROFILE_CONFIGS = {c.name: c for c in (MUSE_PREFILL_N32, MUSE_DECODE_N32)}
-ALL_CONFIGS = {**CONFIGS, **PROFILE_CONFIGS}
+
+# The Muse router as the Muse audit describes it ("Latent experts"): fp32 router weights, sigmoid
+# scores, a selection-only correction bias ~ N(0, 0.05^2) (values not given on the pages),
+# output_multiplier 1 (value not given) and routed_scaling_factor 1 (model sheet).
+MUSE_DECODE_SIGMOID = MUSE_DECODE.replace(name="muse_decode_sigmoid", gate_mode=GATE_SIGMOID,
+                                          router_f32=1, seed=8)
+MUSE_PREFILL_SIGMOID = MUSE_PREFILL.replace(name="muse_prefill_sigmoid", gate_mode=GATE_SIGMOID,
+                                            router_f32=1, seed=9)
+VARIANT_CONFIGS = {c.name: c for c in (MUSE_DECODE_SIGMOID, MUSE_PREFILL_SIGMOID)}
+ALL_CONFIGS = {**CONFIGS, **PROFILE_CONFIGS, **VARIANT_CONFIGS}
 
 
 def small_muse(T: int = 37, d: int = 256, L: int = 128, I: int = 128, n: int = 16, k: int = 4,

@@ -33,7 +33,9 @@ class OrcCfg(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int) for n in ("T", "d_model", "d_latent", "d_ff", "n_experts",
                                             "top_k", "is_bf16", "act", "pre_norm",
                                             "expert_norm", "resid_mode")] + \
-               [(n, ctypes.c_double) for n in ("eps", "tau", "resid_floor", "routed_scale")]
+               [(n, ctypes.c_double) for n in ("eps", "tau", "resid_floor", "routed_scale")] + \
+               [("gate_mode", ctypes.c_int), ("router_f32", ctypes.c_int),
+                ("logit_mult", ctypes.c_double)]
 
 
 class OrcTensors(ctypes.Structure):
@@ -41,7 +43,8 @@ class OrcTensors(ctypes.Structure):
                 ("logit_bias", ctypes.c_void_p), ("p_down", ctypes.c_void_p),
                 ("p_up", ctypes.c_void_p), ("w_gu", ctypes.POINTER(ctypes.c_void_p)),
                 ("w_down", ctypes.POINTER(ctypes.c_void_p)), ("gamma_pre", ctypes.c_void_p),
-                ("gamma_expert", ctypes.c_void_p), ("resid_g", ctypes.c_void_p)]
+                ("gamma_expert", ctypes.c_void_p), ("resid_g", ctypes.c_void_p),
+                ("correction_bias", ctypes.c_void_p)]
 
 
 def lib():
@@ -70,6 +73,10 @@ def lib():
         L.orc_expert_batch.argtypes = [cp, vp, vp, vp, vp, i32, vp, i32]
         L.orc_permutation.restype = i32
         L.orc_permutation.argtypes = [i32, i32, i32, vp, vp, vp, vp]
+        L.orc_sigmoid_topk.argtypes = [vp, vp, i32, i32, dbl, vp, vp, vp]
+        L.orc_sigmoid_topk.restype = None
+        L.orc_sigmoid_topk_scores_f32.argtypes = [vp, vp, i32, i32, dbl, vp, vp]
+        L.orc_sigmoid_topk_scores_f32.restype = None
         for f in ("orc_rms_normalize", "orc_centered_rmsnorm", "orc_input_scaled_rmsnorm",
                   "orc_softmax_topk", "orc_softmax_topk_f32", "orc_resid_gate_coeffs",
                   "orc_router_token", "orc_expert_input_token", "orc_expert_token",
@@ -94,7 +101,8 @@ def make_cfg(cfg, T: int | None = None) -> OrcCfg:
                   d_ff=cfg.d_ff, n_experts=cfg.n_experts, top_k=cfg.top_k,
                   is_bf16=1 if cfg.dtype == "bf16" else 0, act=cfg.act, pre_norm=cfg.pre_norm,
                   expert_norm=cfg.expert_norm, resid_mode=cfg.resid_mode, eps=cfg.eps,
-                  tau=cfg.tau, resid_floor=cfg.resid_floor, routed_scale=cfg.routed_scale)
+                  tau=cfg.tau, resid_floor=cfg.resid_floor, routed_scale=cfg.routed_scale,
+                  gate_mode=cfg.gate_mode, router_f32=cfg.router_f32, logit_mult=cfg.logit_mult)
 
 
 class _Keep:
@@ -137,7 +145,8 @@ def make_tensors(cfg, inp: dict, keep: _Keep, experts: dict | None = None) -> Or
                       p_up=keep.ptr(inp.get("p_up")), w_gu=gu, w_down=dn,
                       gamma_pre=keep.ptr(inp.get("gamma_pre")),
                       gamma_expert=keep.ptr(inp.get("gamma_expert")),
-                      resid_g=keep.ptr(inp.get("resid_g")))
+                      resid_g=keep.ptr(inp.get("resid_g")),
+                      correction_bias=keep.ptr(inp.get("correction_bias")))
 
 
 def layer_forward(cfg, inp: dict, tokens=None, nthreads: int | None = None) -> dict:
@@ -226,6 +235,34 @@ def softmax_topk(logits: np.ndarray, k: int, routed_scale: float = 1.0):
     for i in range(rows.shape[0]):
         fn(_p(rows[i]), n, k, routed_scale, _p(idx[i]), _p(w[i]))
     return idx.reshape(logits.shape[:-1] + (k,)), w.reshape(logits.shape[:-1] + (k,))
+
+
+def sigmoid_topk(logits: np.ndarray, k: int, correction_bias=None, routed_scale: float = 1.0):
+    """Muse sigmoid gate on double logits: (idx, w, scores) per row."""
+    n = logits.shape[-1]
+    rows = np.ascontiguousarray(logits.reshape(-1, n), dtype=np.float64)
+    cb = None if correction_bias is None else np.ascontiguousarray(correction_bias, np.float32)
+    idx = np.zeros((rows.shape[0], k), dtype=np.int32)
+    w = np.zeros((rows.shape[0], k))
+    s = np.zeros_like(rows)
+    for i in range(rows.shape[0]):
+        lib().orc_sigmoid_topk(_p(rows[i]), None if cb is None else _p(cb), n, k, routed_scale,
+                               _p(idx[i]), _p(w[i]), _p(s[i]))
+    return idx, w, s
+
+
+def sigmoid_topk_scores_f32(scores: np.ndarray, k: int, correction_bias=None,
+                            routed_scale: float = 1.0):
+    """Selection of the sigmoid gate taken in fp32 on given fp32 scores: (idx, w) per row."""
+    n = scores.shape[-1]
+    rows = np.ascontiguousarray(scores.reshape(-1, n), dtype=np.float32)
+    cb = None if correction_bias is None else np.ascontiguousarray(correction_bias, np.float32)
+    idx = np.zeros((rows.shape[0], k), dtype=np.int32)
+    w = np.zeros((rows.shape[0], k))
+    for i in range(rows.shape[0]):
+        lib().orc_sigmoid_topk_scores_f32(_p(rows[i]), None if cb is None else _p(cb), n, k,
+                                          routed_scale, _p(idx[i]), _p(w[i]))
+    return idx, w
 
 
 def rms_normalize(x, eps=0.0):

@@ -148,6 +148,55 @@ void orc_softmax_topk_f32(const float* logits, int n, int k, double routed_scale
   free(l);
 }
 
+/* Muse sigmoid gate [MUSE "Latent experts": fp32 logits times output_multiplier, sigmoid; a
+ * correction bias affects top-k selection only; weights gather the original sigmoid scores,
+ * divide by their selected sum plus 1e-15 and apply routed_scaling_factor]. */
+void orc_sigmoid_topk(const double* logits, const float* correction_bias, int n, int k,
+                      double routed_scale, int* idx, double* w, double* scores) {
+  double* s = (double*)malloc(sizeof(double) * (size_t)n);
+  char* taken = (char*)calloc((size_t)n, 1);
+  for (int e = 0; e < n; ++e) s[e] = sigmoid(logits[e]);
+  double sel = 0.0;
+  for (int j = 0; j < k; ++j) {
+    int best = -1;
+    double best_key = 0.0;
+    for (int e = 0; e < n; ++e) {
+      if (taken[e]) continue;
+      double key = s[e] + (correction_bias ? (double)correction_bias[e] : 0.0);
+      if (best < 0 || key > best_key) { best = e; best_key = key; }
+    }
+    taken[best] = 1;
+    idx[j] = best;
+    w[j] = s[best];
+    sel += s[best];
+  }
+  for (int j = 0; j < k; ++j) w[j] = w[j] / (sel + 1e-15) * routed_scale;
+  if (scores) memcpy(scores, s, sizeof(double) * (size_t)n);
+  free(taken);
+  free(s);
+}
+
+void orc_sigmoid_topk_scores_f32(const float* scores, const float* correction_bias, int n, int k,
+                                 double routed_scale, int* idx, double* w) {
+  char* taken = (char*)calloc((size_t)n, 1);
+  double sel = 0.0;
+  for (int j = 0; j < k; ++j) {
+    int best = -1;
+    float best_key = 0.0f;
+    for (int e = 0; e < n; ++e) {
+      if (taken[e]) continue;
+      float key = scores[e] + (correction_bias ? correction_bias[e] : 0.0f);
+      if (best < 0 || key > best_key) { best = e; best_key = key; }
+    }
+    taken[best] = 1;
+    idx[j] = best;
+    w[j] = (double)scores[best];
+    sel += (double)scores[best];
+  }
+  for (int j = 0; j < k; ++j) w[j] = w[j] / (sel + 1e-15) * routed_scale;
+  free(taken);
+}
+
 /* beta = sigmoid(g/tau), alpha = sqrt(max(sigmoid(-g/tau) * (1 + beta), delta))
  * [MUSE "Residual gates"; ARCHDB residual field].  Not rewritten as 1 - beta^2. */
 void orc_resid_gate_coeffs(double g, double tau, double floor_, double* alpha, double* beta) {
@@ -167,11 +216,19 @@ void orc_router_token(const orc_cfg* c, const orc_tensors* x, int64_t t, double*
   int d = c->d_model, n = c->n_experts;
   double* ut = (double*)malloc(sizeof(double) * (size_t)d);
   for (int i = 0; i < d; ++i) ut[i] = ld(x->u, (size_t)t * d + i, c->is_bf16);
+  /* fp32 router weights are read as fp32 whatever the other tensors' dtype */
+  const int w_is_bf16 = c->router_f32 ? 0 : c->is_bf16;
   for (int e = 0; e < n; ++e) {
-    logits[e] = dot_row(x->w_router, (size_t)e, d, ut, c->is_bf16);
+    logits[e] = dot_row(x->w_router, (size_t)e, d, ut, w_is_bf16);
+    if (c->gate_mode == 1) logits[e] *= c->logit_mult;
     if (x->logit_bias) logits[e] += (double)x->logit_bias[e];
   }
-  orc_softmax_topk(logits, n, c->top_k, c->routed_scale, idx, w);
+  if (c->gate_mode == 1) {
+    /* logits[] returns the sigmoid scores in this mode (what the weights are made of) */
+    orc_sigmoid_topk(logits, x->correction_bias, n, c->top_k, c->routed_scale, idx, w, logits);
+  } else {
+    orc_softmax_topk(logits, n, c->top_k, c->routed_scale, idx, w);
+  }
   free(ut);
 }
 

@@ -38,6 +38,11 @@ typedef struct {
   int expert_norm; /* input-scaled RMSNorm I_gamma on each expert output, before weighting */
   int resid_mode;  /* 0: none, 1: Muse residual gate, 2: literal h + g*b */
   double eps, tau, resid_floor, routed_scale;
+  int gate_mode;     /* 0: softmax over all n then renormalise over the kept k;
+                        1: Muse sigmoid gate (scores sigmoid(l), selection by score + correction
+                           bias, weights score / (sum_sel score + 1e-15)) */
+  int router_f32;    /* 1: router weights are fp32 (whatever the tensors' dtype) */
+  double logit_mult; /* output_multiplier applied to the router logits (sigmoid gate) */
 } orc_cfg;
 
 typedef struct {
@@ -52,6 +57,7 @@ typedef struct {
   const float* gamma_pre;   /* [d_latent] */
   const float* gamma_expert;/* [E_in], one gain shared by every expert */
   const float* resid_g;     /* [d_model] */
+  const float* correction_bias; /* [n] sigmoid gate: added to the scores for selection only */
 } orc_tensors;
 
 /* storage rounding of the configured dtype (bf16 RNE, or fp32) */
@@ -75,6 +81,16 @@ void orc_softmax_topk_f32(const float* logits, int n, int k, double routed_scale
 
 /* Residual gate coefficients for one channel. */
 void orc_resid_gate_coeffs(double g, double tau, double floor_, double* alpha, double* beta);
+
+/* Muse sigmoid gate on logits l (already multiplied by output_multiplier):
+ * s = sigmoid(l); the k experts with the largest s + correction_bias (ties to the lower index),
+ * in that order; w_j = s_j / (sum_sel s + 1e-15) * routed_scale.  scores (may be NULL) gets s. */
+void orc_sigmoid_topk(const double* logits, const float* correction_bias, int n, int k,
+                      double routed_scale, int* idx, double* w, double* scores);
+/* The same selection taken in fp32 on given fp32 scores: key = (float)(s + bias) (an exact
+ * IEEE fp32 addition), ties to the lower index; weights from the given scores in double. */
+void orc_sigmoid_topk_scores_f32(const float* scores, const float* correction_bias, int n, int k,
+                                 double routed_scale, int* idx, double* w);
 
 /* Per-token steps. */
 void orc_router_token(const orc_cfg* c, const orc_tensors* x, int64_t t, double* logits, int* idx,

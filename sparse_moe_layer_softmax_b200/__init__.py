@@ -27,7 +27,7 @@ STATUS_CODES = {v: k for k, v in STATUS.items()}
 EXPORTS = ("moe_status_string", "moe_workspace_size", "moe_route", "moe_permute",
            "moe_expert_ffn", "moe_combine", "moe_latent_down", "moe_latent_up",
            "moe_layer_forward", "moe_get_device_status", "moe_profile_begin", "moe_profile_end",
-           "moe_launch_count", "moe_permute_static")
+           "moe_launch_count", "moe_permute_static", "moe_selftest_wait_timeout")
 PROFILE_STAGES = ("route", "latent_down", "dispatch", "expert_gate_up", "expert_down", "combine",
                   "latent_up_resgate")
 
@@ -81,6 +81,7 @@ def lib():
             "moe_profile_begin": [ctypes.c_int32],
             "moe_profile_end": [vp, vp],
             "moe_permute_static": [cp, vp, vp, vp, vp, vp, vp, vp, vp],
+            "moe_selftest_wait_timeout": [ctypes.c_longlong, vp, vp],
         }
         for name, args in sigs.items():
             f = getattr(L, name)

@@ -68,11 +68,12 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 // Returns false (and latches MOE_ERR_TIMEOUT) if the phase did not complete within the budget.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
+                                          long long budget = kWaitBudgetClocks) {
   if (mbar_try_wait(bar, parity)) return true;
   long long t0 = clock64();
   while (!mbar_try_wait(bar, parity)) {
-    if (clock64() - t0 > kWaitBudgetClocks) {
+    if (clock64() - t0 > budget) {
       latch_status(MOE_ERR_TIMEOUT);
       return false;
     }

@@ -388,6 +388,20 @@ __global__ void topk_rows_kernel(const float* __restrict__ logits, int T, int n,
   }
 }
 
+// ------------------------------------------------------------------ failure-detection self-test
+//
+// One thread initialises an mbarrier that expects one arrival which never comes and waits on
+// it with the same bounded wait the GEMM pipeline uses; the wait runs out after `budget` clocks,
+// latches MOE_ERR_TIMEOUT in the status word and the kernel returns normally.
+__global__ void wait_timeout_selftest_kernel(long long budget, int* gave_up) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x != 0) return;
+  mbar_init(&bar, 1);
+  fence_barrier_init();
+  const bool ok = mbar_wait(&bar, 0, budget);
+  *gave_up = ok ? 0 : 1;
+}
+
 // ------------------------------------------------------------------ fp32 path
 
 // Router: one warp per token; logits in fp32 FMA, the k best selected by repeated warp argmax

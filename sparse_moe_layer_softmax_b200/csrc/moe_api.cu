@@ -712,6 +712,14 @@ moe_status_t moe_layer_forward(const moe_config_t* cfg, const moe_weights_t* w, 
 
 unsigned long long moe_launch_count(void) { return g_launches.load(); }
 
+moe_status_t moe_selftest_wait_timeout(long long budget_clocks, int32_t* gave_up, void* stream) {
+  if (!gave_up || budget_clocks <= 0 || budget_clocks > kWaitBudgetClocks) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(gave_up)) return MOE_ERR_ALIGNMENT;
+  wait_timeout_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(budget_clocks,
+                                                                                gave_up);
+  return last_launch();
+}
+
 moe_status_t moe_profile_begin(int32_t max_calls) {
   if (max_calls <= 0 || max_calls > 100000) return MOE_ERR_INVALID_ARG;
   Profiler& p = prof();

@@ -296,3 +296,21 @@ def test_latent_down_and_up():
         oracle.lib().orc_output_token(oracle.ctypes.byref(oc), oracle.ctypes.byref(x), t,
                                       yt.ctypes.data, o.ctypes.data)
         assert row_rel_err(og[t], o) <= 1e-2
+
+
+# ------------------------------------------------------------------ failure detection
+
+
+def test_bounded_wait_runs_out_and_reports():
+    """A wait on a barrier nothing arrives at gives up after its budget, latches MOE_ERR_TIMEOUT
+    in the status word, and the context stays usable."""
+    gave_up = torch.zeros(4, dtype=torch.int32, device="cuda")
+    rc = moe.lib().moe_selftest_wait_timeout(2_000_000, gave_up.data_ptr(),
+                                             torch.cuda.current_stream().cuda_stream)
+    assert rc == 0
+    assert moe.moe_get_device_status() == moe.STATUS_CODES["MOE_ERR_TIMEOUT"]
+    assert gave_up[0].item() == 1
+    assert moe.moe_get_device_status() == 0
+    # the device still runs work correctly afterwards
+    cfg = configs.small_muse(T=40, d=256, L=128, I=128, n=16, k=4, seed=77)
+    _check_layer(cfg)

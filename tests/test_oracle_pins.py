@@ -224,15 +224,25 @@ def dense_bruteforce(cfg, inp):
     """Every expert evaluated on every token with numpy matmuls, then gathered by the gate."""
     dt = cfg.dtype
     u = _val(inp["u"], dt)
-    wr = _val(inp["w_router"], dt)
+    wr = _val(inp["w_router"], "f32" if cfg.router_f32 else dt)
     logits = u @ wr.T
+    if cfg.gate_mode == configs.GATE_SIGMOID:
+        logits = logits * cfg.logit_mult
     if "logit_bias" in inp:
         logits = logits + inp["logit_bias"].astype(np.float64)
-    p = np.exp(logits - logits.max(1, keepdims=True))
-    p /= p.sum(1, keepdims=True)
-    top = np.argsort(-logits, axis=1, kind="stable")[:, :cfg.top_k]
-    w = np.take_along_axis(p, top, 1)
-    w = w / w.sum(1, keepdims=True) * cfg.routed_scale
+    if cfg.gate_mode == configs.GATE_SIGMOID:
+        s = 1.0 / (1.0 + np.exp(-logits))
+        key = s + inp["correction_bias"].astype(np.float64)
+        top = np.argsort(-key, axis=1, kind="stable")[:, :cfg.top_k]
+        w = np.take_along_axis(s, top, 1)
+        w = w / (w.sum(1, keepdims=True) + 1e-15) * cfg.routed_scale
+        logits = s  # the oracle reports the scores in this mode
+    else:
+        p = np.exp(logits - logits.max(1, keepdims=True))
+        p /= p.sum(1, keepdims=True)
+        top = np.argsort(-logits, axis=1, kind="stable")[:, :cfg.top_k]
+        w = np.take_along_axis(p, top, 1)
+        w = w / w.sum(1, keepdims=True) * cfg.routed_scale
     if cfg.latent:
         zr = _rnd(u @ _val(inp["p_down"], dt).T, dt)
         if cfg.pre_norm:
@@ -285,6 +295,12 @@ BRUTE_CASES = [
     configs.small_muse(T=11, d=32, L=16, I=24, n=4, k=2, resid_mode=configs.RESID_LITERAL,
                        gamma_sigma=0.3),
     configs.small_muse(T=7, d=32, L=16, I=16, n=4, k=2, pre_norm=0, resid_mode=configs.RESID_NONE),
+    # Muse sigmoid gate with fp32 router weights, output_multiplier and routed_scaling_factor
+    configs.small_muse(T=15, d=48, L=32, I=24, n=8, k=3, gamma_sigma=0.3,
+                       gate_mode=configs.GATE_SIGMOID, router_f32=1, logit_mult=2.0,
+                       corr_sigma=0.3, routed_scale=1.5),
+    configs.small_muse(T=10, d=40, L=24, I=16, n=6, k=2, dtype="f32",
+                       gate_mode=configs.GATE_SIGMOID, router_f32=1),
 ]
 
 
@@ -363,3 +379,48 @@ def test_zipf_bias_imbalance_recipe():
     b = moe_inputs.zipf_bias(cfg, scale=1.0)
     np.testing.assert_allclose(b, -1.2 * np.log(r), rtol=1e-6)
     assert b.max() == 0.0
+
+
+# ------------------------------------------------------------------ Muse sigmoid gate
+# sigmoid(ln 3) = 3/4 and sigmoid(-ln 3) = 1/4 exactly, so these weights have closed forms.
+
+
+def test_sigmoid_gate_closed_form():
+    l = np.array([[0.0, math.log(3.0), -math.log(3.0)]])
+    idx, w, s = oracle.sigmoid_topk(l, 2)
+    np.testing.assert_allclose(s[0], [0.5, 0.75, 0.25], rtol=1e-15)
+    assert idx[0].tolist() == [1, 0]
+    np.testing.assert_allclose(w[0], [0.75 / 1.25, 0.5 / 1.25], rtol=1e-14)
+    # the correction bias changes the selection, not the weights' source (the original scores)
+    idx, w, _ = oracle.sigmoid_topk(l, 2, correction_bias=np.array([0.0, 0.0, 1.0]))
+    assert idx[0].tolist() == [2, 1]
+    np.testing.assert_allclose(w[0], [0.25, 0.75], rtol=1e-14)
+    # routed_scaling_factor multiplies the renormalised weights
+    _, w2, _ = oracle.sigmoid_topk(l, 2, routed_scale=2.5)
+    np.testing.assert_allclose(w2[0], 2.5 * np.array([0.6, 0.4]), rtol=1e-14)
+
+
+def test_sigmoid_gate_invariants():
+    rng = np.random.default_rng(5)
+    l = rng.normal(size=(40, 16)) * 3
+    cb = rng.normal(size=16).astype(np.float32) * 0.5
+    # k = n: every expert kept, weights are the scores over their sum, whatever the bias
+    idx, w, s = oracle.sigmoid_topk(l, 16, correction_bias=cb)
+    for r in range(40):
+        np.testing.assert_allclose(w[r], s[r, idx[r]] / s[r].sum(), rtol=1e-13)
+    # selection follows score + bias, weights sum to routed_scale
+    idx, w, s = oracle.sigmoid_topk(l, 4, correction_bias=cb)
+    for r in range(40):
+        key = s[r] + cb.astype(np.float64)
+        assert idx[r].tolist() == np.argsort(-key, kind="stable")[:4].tolist()
+        assert abs(w[r].sum() - 1.0) < 1e-13
+    # the 1e-15 in the denominator only matters for vanishing scores
+    idx, w, s = oracle.sigmoid_topk(np.full((1, 8), -100.0), 2)
+    np.testing.assert_allclose(w[0], s[0, idx[0]] / (2 * s[0, 0] + 1e-15), rtol=1e-12)
+    assert w[0].sum() < 1e-20
+    # the fp32 selection on fp32 scores agrees when keys are distinct
+    sf = s.astype(np.float32)
+    i32, _ = oracle.sigmoid_topk_scores_f32(oracle.sigmoid_topk(l, 4, cb)[2].astype(np.float32),
+                                            4, cb)
+    np.testing.assert_array_equal(i32, oracle.sigmoid_topk(l, 4, cb)[0])
+    del sf
