@@ -266,7 +266,7 @@ def work_model(cfg, distinct_experts: int) -> dict:
     gu = cfg.gu_rows
     expert_w = gu * E + E * H                      # elements of one expert's two matrices
     flops = 2 * T * (d * n + k * expert_w)
-    wbytes = (n * d + distinct_experts * expert_w) * b
+    wbytes = n * d * (4 if cfg.router_f32 else b) + distinct_experts * expert_w * b
     if cfg.latent:
         flops += 2 * T * (d * cfg.d_latent * 2)
         wbytes += 2 * cfg.d_latent * d * b
@@ -563,6 +563,15 @@ def main(argv=None) -> int:
                     "d2h_bytes_per_step": dres["d2h_bytes"]},
             "stage_ms": dres["stage_ms"], "distinct_experts": dres["distinct_experts"],
             "gpu_launches": dres["gpu_launches"], "clocks": dres["clocks"]}
+    if not args.no_decode and cfg.name != "muse_decode":
+        # the Muse router as the Muse audit describes it (fp32 weights, sigmoid gate) on decode
+        vcfg = configs.MUSE_DECODE_SIGMOID
+        vres = measure_checked(vcfg, args, device, peaks, rank, local, with_e2e=False)
+        line["variants"] = {vcfg.name: {
+            "value": round(vcfg.T * world / (vres["ms_per_step"] / 1e3), 2), "unit": UNIT,
+            "ms_per_step": round(vres["ms_per_step"], 4),
+            "route_ms": vres["stage_ms"]["route"],
+            "layer_roofline": vres["layer_roofline"], "clocks": vres["clocks"]}}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(cfg, args.cpu_sample or default_cpu_sample(cfg))
     if rank == 0:

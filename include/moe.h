@@ -65,6 +65,7 @@ typedef enum {
 enum { MOE_F32 = 0, MOE_BF16 = 1 };
 enum { MOE_ACT_RELU = 0, MOE_ACT_SWIGLU = 1 };
 enum { MOE_RESID_NONE = 0, MOE_RESID_MUSE_GATE = 1, MOE_RESID_LITERAL = 2 };
+enum { MOE_GATE_SOFTMAX = 0, MOE_GATE_SIGMOID = 1 };
 
 typedef struct {
   int32_t T;            /* tokens */
@@ -82,6 +83,12 @@ typedef struct {
   float tau;            /* residual gate temperature */
   float resid_floor;    /* residual gate floor delta on alpha^2 */
   float routed_scale;   /* routed_scaling_factor applied to the renormalised weights */
+  int32_t gate_mode;    /* MOE_GATE_SOFTMAX (softmax, keep top k, renormalise) |
+                           MOE_GATE_SIGMOID (Muse: sigmoid scores, selection by score + correction
+                           bias, weights = score / (sum of selected scores + 1e-15)) */
+  int32_t router_f32;   /* 1: the router weights are fp32, passed as their exact bf16 split
+                           [n, 3*d_model] (hi, mid, lo; see moe_router_split_weights) */
+  float logit_mult;     /* output_multiplier on the router logits (sigmoid gate) */
 } moe_config_t;
 
 typedef struct {
@@ -95,6 +102,7 @@ typedef struct {
   const float* gamma_expert;/* [E_in] one gain shared by all experts (expert_norm only) */
   const float* resid_g;     /* [d_model] residual gate parameter g (resid_mode != NONE) */
   const float* logit_bias;  /* [n] added to every token's router logits, or NULL */
+  const float* correction_bias; /* [n] sigmoid gate: added to the scores for selection only */
 } moe_weights_t;
 
 /* Human-readable name of a status code (static storage). */
@@ -104,15 +112,28 @@ MOE_API const char* moe_status_string(moe_status_t s);
  * moe_permute and moe_expert_ffn).  Only host arithmetic. */
 MOE_API moe_status_t moe_workspace_size(const moe_config_t* cfg, size_t* bytes);
 
-/* Router [SHAZEER "The gate"; ARCHDB gating fields]:
- *   l = u W_router^T (+ logit_bias), fp32 accumulation;  the k largest logits are selected
- *   (ties to the lower expert index) in descending order; w_j = exp(l_j - l_1) / sum_sel exp(.)
- *   times routed_scale, which equals softmax-then-renormalise over the kept experts.
- * u: [T, d_model]; topk_idx: [T, k] int32; topk_w: [T, k] fp32; logits_out: [T, n] fp32 with
- * the bias included, or NULL. */
+/* Router [SHAZEER "The gate"; ARCHDB gating fields; MUSE "Latent experts" for the sigmoid gate]:
+ *   l = u W_router^T, fp32 accumulation of exact products (bf16 weights, or the exact
+ *   hi/mid/lo split of fp32 weights when cfg->router_f32).
+ *   Softmax gate: l += logit_bias; the k largest l are selected (ties to the lower expert
+ *   index) in descending order; w_j = exp(l_j - l_1) / sum_sel exp(.) * routed_scale, which
+ *   equals softmax-then-renormalise over the kept experts.  logits_out returns l.
+ *   Sigmoid gate: s = sigmoid(logit_mult * l + logit_bias); the k largest keys
+ *   s + correction_bias (one fp32 addition; ties to the lower index) are selected in descending
+ *   key order; w_j = s_j / (sum_sel s + 1e-15) * routed_scale.  logits_out returns s.
+ * u: [T, d_model]; topk_idx: [T, k] int32; topk_w: [T, k] fp32; logits_out: [T, n] fp32 or
+ * NULL; logit_bias, correction_bias: [n] fp32 or NULL. */
 MOE_API moe_status_t moe_route(const moe_config_t* cfg, const void* u, const void* w_router,
-                       const float* logit_bias, float* logits_out, int32_t* topk_idx,
-                       float* topk_w, void* stream);
+                       const float* logit_bias, const float* correction_bias, float* logits_out,
+                       int32_t* topk_idx, float* topk_w, void* stream);
+
+/* Prepares fp32 router weights w [n, d] for the tensor-core router: w_split [n, 3*d] bf16 holds
+ * per row the bf16 parts hi = bf16(w), mid = bf16(w - hi), lo = bf16(w - hi - mid) (each
+ * subtraction exact in fp32), so hi + mid + lo = w exactly for every normal fp32 w with a normal
+ * lo part (zero remainders stay exact).  Run once per weight load.  Device pointers, d a
+ * multiple of 64. */
+MOE_API moe_status_t moe_router_split_weights(const float* w, int32_t n, int32_t d, void* w_split,
+                                              void* stream);
 
 /* Dispatch [MUSE "Latent experts"; SHAZEER "The math"]: groups the T*k routed slots by expert
  * in the canonical order (experts ascending; within an expert, tokens ascending), so that every

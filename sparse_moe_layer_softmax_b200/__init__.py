@@ -20,6 +20,7 @@ LIB_PATH = os.path.join(_HERE, "libmoe.so")
 MOE_F32, MOE_BF16 = 0, 1
 MOE_ACT_RELU, MOE_ACT_SWIGLU = 0, 1
 MOE_RESID_NONE, MOE_RESID_MUSE_GATE, MOE_RESID_LITERAL = 0, 1, 2
+MOE_GATE_SOFTMAX, MOE_GATE_SIGMOID = 0, 1
 STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED", 3: "MOE_ERR_ALIGNMENT",
           4: "MOE_ERR_WORKSPACE", 5: "MOE_ERR_CUDA", 6: "MOE_ERR_TIMEOUT",
           7: "MOE_ERR_DEVICE_CHECK"}
@@ -27,7 +28,8 @@ STATUS_CODES = {v: k for k, v in STATUS.items()}
 EXPORTS = ("moe_status_string", "moe_workspace_size", "moe_route", "moe_permute",
            "moe_expert_ffn", "moe_combine", "moe_latent_down", "moe_latent_up",
            "moe_layer_forward", "moe_get_device_status", "moe_profile_begin", "moe_profile_end",
-           "moe_launch_count", "moe_permute_static", "moe_selftest_wait_timeout")
+           "moe_launch_count", "moe_permute_static", "moe_selftest_wait_timeout",
+           "moe_router_split_weights")
 PROFILE_STAGES = ("route", "latent_down", "dispatch", "expert_gate_up", "expert_down", "combine",
                   "latent_up_resgate")
 
@@ -43,14 +45,16 @@ class Config(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in ("T", "d_model", "d_latent", "d_ff", "n_experts",
                                               "top_k", "dtype", "expert_act", "pre_norm",
                                               "expert_norm", "resid_mode")] + \
-               [(n, ctypes.c_float) for n in ("eps", "tau", "resid_floor", "routed_scale")]
+               [(n, ctypes.c_float) for n in ("eps", "tau", "resid_floor", "routed_scale")] + \
+               [("gate_mode", ctypes.c_int32), ("router_f32", ctypes.c_int32),
+                ("logit_mult", ctypes.c_float)]
 
 
 class Weights(ctypes.Structure):
     """moe_weights_t"""
     _fields_ = [(n, ctypes.c_void_p) for n in ("w_router", "p_down", "p_up", "w_gu", "w_down",
                                                "gamma_pre", "gamma_expert", "resid_g",
-                                               "logit_bias")]
+                                               "logit_bias", "correction_bias")]
 
 
 _lib = None
@@ -70,7 +74,8 @@ def lib():
         L.moe_status_string.argtypes = [i32]
         sigs = {
             "moe_workspace_size": [cp, ctypes.POINTER(sz)],
-            "moe_route": [cp, vp, vp, vp, vp, vp, vp, vp],
+            "moe_route": [cp, vp, vp, vp, vp, vp, vp, vp, vp],
+            "moe_router_split_weights": [vp, ctypes.c_int32, ctypes.c_int32, vp, vp],
             "moe_permute": [cp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp],
             "moe_expert_ffn": [cp, vp, vp, vp, vp, vp, vp, vp, sz, vp],
             "moe_combine": [cp, vp, vp, vp, vp, vp],
@@ -95,11 +100,13 @@ def lib():
 
 def make_config(T, d_model, n_experts, top_k, d_ff, d_latent=0, dtype=MOE_BF16,
                 expert_act=MOE_ACT_SWIGLU, pre_norm=0, expert_norm=0, resid_mode=MOE_RESID_NONE,
-                eps=1e-6, tau=0.3, resid_floor=1e-3, routed_scale=1.0) -> Config:
+                eps=1e-6, tau=0.3, resid_floor=1e-3, routed_scale=1.0, gate_mode=MOE_GATE_SOFTMAX,
+                router_f32=0, logit_mult=1.0) -> Config:
     return Config(T=T, d_model=d_model, d_latent=d_latent, d_ff=d_ff, n_experts=n_experts,
                   top_k=top_k, dtype=dtype, expert_act=expert_act, pre_norm=pre_norm,
                   expert_norm=expert_norm, resid_mode=resid_mode, eps=eps, tau=tau,
-                  resid_floor=resid_floor, routed_scale=routed_scale)
+                  resid_floor=resid_floor, routed_scale=routed_scale, gate_mode=gate_mode,
+                  router_f32=router_f32, logit_mult=logit_mult)
 
 
 def _ptr(t) -> int | None:
@@ -128,10 +135,25 @@ def workspace_size(cfg: Config) -> int:
     return n.value
 
 
-def moe_route(cfg, u, w_router, logit_bias, logits_out, topk_idx, topk_w, stream=None):
+def moe_route(cfg, u, w_router, logit_bias, logits_out, topk_idx, topk_w, stream=None,
+              correction_bias=None):
     _check("moe_route", lib().moe_route(ctypes.byref(cfg), _ptr(u), _ptr(w_router),
-                                        _ptr(logit_bias), _ptr(logits_out), _ptr(topk_idx),
-                                        _ptr(topk_w), _stream(stream)))
+                                        _ptr(logit_bias), _ptr(correction_bias), _ptr(logits_out),
+                                        _ptr(topk_idx), _ptr(topk_w), _stream(stream)))
+
+
+def moe_router_split_weights(w, w_split, stream=None):
+    """fp32 router weights w [n, d] -> their exact bf16 hi/mid/lo split w_split [n, 3d]."""
+    n, d = w.shape
+    _check("moe_router_split_weights",
+           lib().moe_router_split_weights(_ptr(w), n, d, _ptr(w_split), _stream(stream)))
+
+
+def router_split(w, stream=None):
+    import torch
+    out = torch.empty((w.shape[0], 3 * w.shape[1]), dtype=torch.bfloat16, device=w.device)
+    moe_router_split_weights(w, out, stream)
+    return out
 
 
 def moe_permute(cfg, topk_idx, expert_offsets, perm_token, inv_perm, x=None, gamma_pre=None,
@@ -224,6 +246,10 @@ class MoELayer:
         import torch
         self.cfg = cfg
         self.weights = weights
+        if cfg.router_f32 and cfg.dtype == MOE_BF16 and weights["w_router"].dtype == torch.float32:
+            # fp32 router weights go to the tensor cores as their exact bf16 split (once)
+            weights = dict(weights, w_router=router_split(weights["w_router"]))
+            self.weights = weights
         self._w = make_weights(weights)
         self.workspace = torch.empty(workspace_size(cfg), dtype=torch.uint8, device="cuda")
 

@@ -48,6 +48,11 @@ struct GemmParams {
   const float* bias;         // EPI_ROUTER: [Nout] or nullptr
   int top_k;
   float routed_scale;
+  int gate_mode;             // EPI_ROUTER: MOE_GATE_SOFTMAX | MOE_GATE_SIGMOID
+  float logit_mult;          // EPI_ROUTER (sigmoid): output_multiplier
+  const float* sel_bias;     // EPI_ROUTER (sigmoid): selection-only correction bias [Nout]
+  int x_k_period;            // > 0: X's k coordinate wraps every x_k_period columns (W's K is
+                             // a multiple: the fp32 router weights' hi/mid/lo bf16 parts)
 };
 
 template <bool kSwap, int BN, int kEpi>
@@ -125,15 +130,16 @@ __device__ __forceinline__ TileCoord decode_tile(int t, const int* s_seg, const 
 
 template <int kMaxK>
 struct TopK {
-  float v[kMaxK];
+  float v[kMaxK];  // selection keys, descending
+  float s[kMaxK];  // payload carried with each key (the sigmoid score, or the logit)
   int i[kMaxK];
   __device__ __forceinline__ void init() {
 #pragma unroll
-    for (int j = 0; j < kMaxK; ++j) { v[j] = -INFINITY; i[j] = -1; }
+    for (int j = 0; j < kMaxK; ++j) { v[j] = -INFINITY; s[j] = 0.0f; i[j] = -1; }
   }
   // Columns arrive in ascending index order; strict comparisons keep the lower index first
   // among equal values.  Insertion into the sorted list of the k best (k <= kMaxK).
-  __device__ __forceinline__ void push(float x, int idx, int k) {
+  __device__ __forceinline__ void push(float x, float payload, int idx, int k) {
     if (i[k - 1] >= 0 && !(x > v[k - 1])) return;
 #pragma unroll
     for (int j = kMaxK - 1; j >= 0; --j) {
@@ -141,15 +147,36 @@ struct TopK {
       const bool above = (j > 0) && (i[j - 1] < 0 || x > v[j - 1]);
       if (above) {
         v[j] = v[j - 1];
+        s[j] = s[j - 1];
         i[j] = i[j - 1];
       } else {
         v[j] = x;
+        s[j] = payload;
         i[j] = idx;
         break;
       }
     }
   }
 };
+
+// Routing weights of the selected k: softmax over the kept logits (= softmax over all, then
+// renormalised), or the Muse sigmoid gate's scores / (their sum + 1e-15); times routed_scale.
+template <int kMaxK>
+__device__ __forceinline__ void topk_weights(const TopK<kMaxK>& tk, int k, int gate_mode,
+                                             float routed_scale, float* w) {
+  float sum = 0.0f;
+#pragma unroll
+  for (int j = 0; j < kMaxK; ++j) {
+    float e = 0.0f;
+    if (j < k) e = gate_mode == MOE_GATE_SIGMOID ? tk.s[j] : __expf(tk.s[j] - tk.s[0]);
+    w[j] = e;
+    sum += e;
+  }
+  const float scale = gate_mode == MOE_GATE_SIGMOID ? routed_scale / (sum + 1e-15f)
+                                                    : routed_scale / sum;
+#pragma unroll
+  for (int j = 0; j < kMaxK; ++j) w[j] *= scale;
+}
 
 // Epilogue of the normal orientation: this thread owns row row0 + 32*q + lane of the tile (valid
 // if below nrows) and the tile's BN accumulator columns (output features f0 ...).
@@ -169,9 +196,20 @@ __device__ __forceinline__ void epilogue_rows(const GemmParams& p, int row0, int
         for (int i = 0; i < 16; ++i) {
           const int col = c0 + i;
           if (col < p.Nout) {
-            float l = v[i] + (p.bias ? p.bias[col] : 0.0f);
-            v[i] = l;
-            tk.push(l, col, p.top_k);
+            if (p.gate_mode == MOE_GATE_SIGMOID) {
+              // score s = sigmoid(output_multiplier * l (+ bias)); selection key s + correction
+              // bias (one fp32 addition); the score is what the weights are made of and what
+              // logits_out returns in this mode
+              const float l = v[i] * p.logit_mult + (p.bias ? p.bias[col] : 0.0f);
+              const float sc = 1.0f / (1.0f + expf(-l));
+              const float key = sc + (p.sel_bias ? p.sel_bias[col] : 0.0f);
+              v[i] = sc;
+              tk.push(key, sc, col, p.top_k);
+            } else {
+              const float l = v[i] + (p.bias ? p.bias[col] : 0.0f);
+              v[i] = l;
+              tk.push(l, l, col, p.top_k);
+            }
           }
         }
         if (valid && p.logits) {
@@ -186,17 +224,11 @@ __device__ __forceinline__ void epilogue_rows(const GemmParams& p, int row0, int
         }
       }
       if (valid) {
-        float sum = 0.0f;
-        float e[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          e[j] = (j < p.top_k) ? __expf(tk.v[j] - tk.v[0]) : 0.0f;
-          sum += e[j];
-        }
-        const float scale = p.routed_scale / sum;
+        float w[8];
+        topk_weights(tk, p.top_k, p.gate_mode, p.routed_scale, w);
         for (int j = 0; j < p.top_k; ++j) {
           p.topk_idx[row * p.top_k + j] = tk.i[j];
-          p.topk_w[row * p.top_k + j] = e[j] * scale;
+          p.topk_w[row * p.top_k + j] = w[j];
         }
       }
     } else if constexpr (kEpi == EPI_SWIGLU) {
@@ -378,14 +410,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         uint8_t* sb = sa + S::kABytes;
         mbar_arrive_expect_tx(&full[stage], S::kStageBytes);
         const int kx = kb * S::kBK;
+        const int kxx = p.x_k_period > 0 ? kx % p.x_k_period : kx;  // X's k coordinate
         if (!kSwap) {
-          tma_load_2d(&tmX, &full[stage], sa, kx, c.row0);
+          tma_load_2d(&tmX, &full[stage], sa, kxx, c.row0);
           tma_load_2d(&tmW, &full[stage], sb, kx, wrow);
           if (S::kDual) tma_load_2d(&tmW, &full[stage], sb + (BN / 2) * 128, kx, wrow + p.Nw / 2);
         } else {
           tma_load_2d(&tmW, &full[stage], sa, kx, wrow);
           if (S::kDual) tma_load_2d(&tmW, &full[stage], sa + 128 * 128, kx, wrow + p.Nw / 2);
-          tma_load_2d(&tmX, &full[stage], sb, kx, c.row0);
+          tma_load_2d(&tmX, &full[stage], sb, kxx, c.row0);
         }
         issued[stage] = true;
         last_parity[stage] = phase;

@@ -292,7 +292,8 @@ constexpr int kRouterExp = 16;
 
 __global__ void __launch_bounds__(256) router_logits_small_kernel(
     const uint16_t* __restrict__ u, const uint16_t* __restrict__ w, const float* __restrict__ bias,
-    int T, int d, int n, float* __restrict__ logits) {
+    int T, int d, int n, int wk, float mult, float* __restrict__ logits) {
+  // w rows have wk = d (bf16 weights) or 3d (hi/mid/lo parts of fp32 weights; u repeats)
   extern __shared__ uint4 s_u[];  // [kRouterTok][d/8]
   const int t0 = blockIdx.y * kRouterTok;
   const int nt = min(kRouterTok, T - t0);
@@ -307,12 +308,14 @@ __global__ void __launch_bounds__(256) router_logits_small_kernel(
   for (int el = warp; el < kRouterExp; el += nwarps) {
     const int e = blockIdx.x * kRouterExp + el;
     if (e >= n) break;
-    const uint4* wr = reinterpret_cast<const uint4*>(w + static_cast<size_t>(e) * d);
+    const uint4* wr = reinterpret_cast<const uint4*>(w + static_cast<size_t>(e) * wk);
     float acc[kRouterTok];
 #pragma unroll
     for (int tt = 0; tt < kRouterTok; ++tt) acc[tt] = 0.0f;
-    for (int v = lane; v < nvec; v += 32) {
-      const uint4 wq = wr[v];
+    const int wvec = wk / 8;
+    for (int vw = lane; vw < wvec; vw += 32) {
+      const int v = vw % nvec;
+      const uint4 wq = wr[vw];
       const uint16_t* wh = reinterpret_cast<const uint16_t*>(&wq);
       float wf[8];
 #pragma unroll
@@ -335,56 +338,98 @@ __global__ void __launch_bounds__(256) router_logits_small_kernel(
 #pragma unroll
       for (int tt = 1; tt < kRouterTok; ++tt)
         if (lane == tt) l = acc[tt];
-      logits[static_cast<size_t>(t0 + lane) * n + e] = l + (bias ? bias[e] : 0.0f);
+      logits[static_cast<size_t>(t0 + lane) * n + e] = l * mult + (bias ? bias[e] : 0.0f);
     }
   }
 }
 
-// One warp per token: the k largest logits (ties to the lower index), in descending order, and
-// the weights exp(l_j - l_1) / sum_sel exp(l - l_1) * routed_scale.
-__global__ void topk_rows_kernel(const float* __restrict__ logits, int T, int n, int k,
-                                 float routed_scale, int32_t* __restrict__ topk_idx,
-                                 float* __restrict__ topk_w) {
+// One warp per token.  Softmax gate: the k largest logits (ties to the lower index), in
+// descending order, weights exp(l_j - l_1) / sum_sel exp(l - l_1) * routed_scale.  Sigmoid gate:
+// scores s = sigmoid(l) replace the logits in the buffer, the k largest keys s + sel_bias are
+// selected, weights s_j / (sum_sel s + 1e-15) * routed_scale.
+__global__ void topk_rows_kernel(float* __restrict__ logits, int T, int n, int k,
+                                 float routed_scale, int gate_mode,
+                                 const float* __restrict__ sel_bias,
+                                 int32_t* __restrict__ topk_idx, float* __restrict__ topk_w) {
   const int warps = blockDim.x >> 5;
   const int t = blockIdx.x * warps + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (t >= T) return;
-  float l[kMaxExperts / 32];
+  float key[kMaxExperts / 32], pay[kMaxExperts / 32];
 #pragma unroll
   for (int i = 0; i < kMaxExperts / 32; ++i) {
     const int e = lane + 32 * i;
-    l[i] = e < n ? logits[static_cast<size_t>(t) * n + e] : -INFINITY;
+    key[i] = -INFINITY;
+    pay[i] = 0.0f;
+    if (e < n) {
+      const float l = logits[static_cast<size_t>(t) * n + e];
+      if (gate_mode == MOE_GATE_SIGMOID) {
+        const float s = 1.0f / (1.0f + expf(-l));
+        logits[static_cast<size_t>(t) * n + e] = s;
+        key[i] = s + (sel_bias ? sel_bias[e] : 0.0f);
+        pay[i] = s;
+      } else {
+        key[i] = l;
+        pay[i] = l;
+      }
+    }
   }
-  float top_v[kMaxTopK];
+  float top_s[kMaxTopK];
   int top_i[kMaxTopK];
   for (int j = 0; j < k; ++j) {
-    float bv = -INFINITY;
+    float bv = -INFINITY, bs = 0.0f;
     int bi = 0x7fffffff;
 #pragma unroll
     for (int i = 0; i < kMaxExperts / 32; ++i) {
       const int e = lane + 32 * i;
-      if (e < n && (l[i] > bv || (l[i] == bv && e < bi))) { bv = l[i]; bi = e; }
+      if (e < n && (key[i] > bv || (key[i] == bv && e < bi))) { bv = key[i]; bi = e; bs = pay[i]; }
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
       const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
       const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-      if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
+      const float os = __shfl_xor_sync(0xffffffffu, bs, o);
+      if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; bs = os; }
     }
-    top_v[j] = bv;
+    top_s[j] = bs;
     top_i[j] = bi;
 #pragma unroll
     for (int i = 0; i < kMaxExperts / 32; ++i)
-      if (lane + 32 * i == bi) l[i] = -INFINITY;
+      if (lane + 32 * i == bi) key[i] = -INFINITY;
   }
   if (lane == 0) {
+    float e[kMaxTopK];
     float sum = 0.0f;
-    for (int j = 0; j < k; ++j) sum += __expf(top_v[j] - top_v[0]);
-    const float scale = routed_scale / sum;
+    for (int j = 0; j < k; ++j) {
+      e[j] = gate_mode == MOE_GATE_SIGMOID ? top_s[j] : __expf(top_s[j] - top_s[0]);
+      sum += e[j];
+    }
+    const float scale = gate_mode == MOE_GATE_SIGMOID ? routed_scale / (sum + 1e-15f)
+                                                      : routed_scale / sum;
     for (int j = 0; j < k; ++j) {
       topk_idx[static_cast<size_t>(t) * k + j] = top_i[j];
-      topk_w[static_cast<size_t>(t) * k + j] = __expf(top_v[j] - top_v[0]) * scale;
+      topk_w[static_cast<size_t>(t) * k + j] = e[j] * scale;
     }
+  }
+}
+
+// fp32 router weights w [n, d] -> their exact bf16 split [n, 3d]: hi, mid, lo with
+// hi = bf16(w), mid = bf16(w - hi), lo = bf16(w - hi - mid); both subtractions are exact in fp32.
+__global__ void router_split_kernel(const float* __restrict__ w, size_t count, int d,
+                                    uint16_t* __restrict__ out) {
+  const size_t stride = static_cast<size_t>(gridDim.x) * blockDim.x;
+  for (size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < count; i += stride) {
+    const size_t row = i / d, c = i - row * d;
+    const float x = w[i];
+    const uint16_t hi = f32_to_bf16(x);
+    const float r1 = x - bf16_to_f32(hi);
+    const uint16_t mid = f32_to_bf16(r1);
+    const float r2 = r1 - bf16_to_f32(mid);
+    const uint16_t lo = f32_to_bf16(r2);
+    uint16_t* o = out + row * 3 * static_cast<size_t>(d);
+    o[c] = hi;
+    o[d + c] = mid;
+    o[2 * static_cast<size_t>(d) + c] = lo;
   }
 }
 
@@ -408,53 +453,70 @@ __global__ void wait_timeout_selftest_kernel(long long budget, int* gave_up) {
 // (ties to the lower index), weights renormalised over the kept experts.
 __global__ void router_f32_kernel(const float* __restrict__ u, const float* __restrict__ w,
                                   const float* __restrict__ bias, int T, int d, int n, int k,
-                                  float routed_scale, float* __restrict__ logits_out,
+                                  float routed_scale, int gate_mode, float mult,
+                                  const float* __restrict__ sel_bias,
+                                  float* __restrict__ logits_out,
                                   int32_t* __restrict__ topk_idx, float* __restrict__ topk_w) {
   const int warps = blockDim.x >> 5;
   const int t = blockIdx.x * warps + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (t >= T) return;
-  float l[kMaxExperts / 32];
+  float key[kMaxExperts / 32], pay[kMaxExperts / 32];
 #pragma unroll
   for (int i = 0; i < kMaxExperts / 32; ++i) {
     const int e = lane + 32 * i;
-    float acc = -INFINITY;
+    key[i] = -INFINITY;
+    pay[i] = 0.0f;
     if (e < n) {
-      acc = 0.0f;
+      float acc = 0.0f;
       for (int c = 0; c < d; ++c) acc = fmaf(u[static_cast<size_t>(t) * d + c], w[static_cast<size_t>(e) * d + c], acc);
+      if (gate_mode == MOE_GATE_SIGMOID) acc *= mult;
       if (bias) acc += bias[e];
-      if (logits_out) logits_out[static_cast<size_t>(t) * n + e] = acc;
+      if (gate_mode == MOE_GATE_SIGMOID) {
+        const float s = 1.0f / (1.0f + expf(-acc));
+        key[i] = s + (sel_bias ? sel_bias[e] : 0.0f);
+        pay[i] = s;
+      } else {
+        key[i] = acc;
+        pay[i] = acc;
+      }
+      if (logits_out) logits_out[static_cast<size_t>(t) * n + e] = pay[i];
     }
-    l[i] = acc;
   }
-  float top_v[kMaxTopK];
+  float top_s[kMaxTopK];
   int top_i[kMaxTopK];
   for (int j = 0; j < k; ++j) {
-    float bv = -INFINITY;
+    float bv = -INFINITY, bs = 0.0f;
     int bi = 0x7fffffff;
 #pragma unroll
     for (int i = 0; i < kMaxExperts / 32; ++i) {
       const int e = lane + 32 * i;
-      if (e < n && (l[i] > bv || (l[i] == bv && e < bi))) { bv = l[i]; bi = e; }
+      if (e < n && (key[i] > bv || (key[i] == bv && e < bi))) { bv = key[i]; bi = e; bs = pay[i]; }
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
       const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
       const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-      if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
+      const float os = __shfl_xor_sync(0xffffffffu, bs, o);
+      if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; bs = os; }
     }
-    top_v[j] = bv;
+    top_s[j] = bs;
     top_i[j] = bi;
 #pragma unroll
     for (int i = 0; i < kMaxExperts / 32; ++i)
-      if (lane + 32 * i == bi) l[i] = -INFINITY;
+      if (lane + 32 * i == bi) key[i] = -INFINITY;
   }
   if (lane == 0) {
+    float e[kMaxTopK];
     float sum = 0.0f;
-    for (int j = 0; j < k; ++j) sum += expf(top_v[j] - top_v[0]);
+    for (int j = 0; j < k; ++j) {
+      e[j] = gate_mode == MOE_GATE_SIGMOID ? top_s[j] : expf(top_s[j] - top_s[0]);
+      sum += e[j];
+    }
+    const float denom = gate_mode == MOE_GATE_SIGMOID ? sum + 1e-15f : sum;
     for (int j = 0; j < k; ++j) {
       topk_idx[static_cast<size_t>(t) * k + j] = top_i[j];
-      topk_w[static_cast<size_t>(t) * k + j] = expf(top_v[j] - top_v[0]) / sum * routed_scale;
+      topk_w[static_cast<size_t>(t) * k + j] = e[j] / denom * routed_scale;
     }
   }
 }

@@ -2,6 +2,7 @@
 // descriptors and the launch sequence of the MoE-layer forward on the caller's stream.
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <atomic>
 #include <initializer_list>
 #include <mutex>
@@ -92,7 +93,9 @@ moe_status_t launch_gemm(const void* X, long x_rows, const void* W, long w_rows,
   });
   if (attr_err != cudaSuccess) return MOE_ERR_CUDA;
   CUtensorMap tx, tw;
-  if (!make_tmap(&tx, X, static_cast<uint64_t>(x_rows), static_cast<uint64_t>(p.K), S::kXBoxRows))
+  // X is [x_rows, K], or [x_rows, x_k_period] when its k coordinate wraps (W then has K columns)
+  const uint64_t x_cols = static_cast<uint64_t>(p.x_k_period > 0 ? p.x_k_period : p.K);
+  if (!make_tmap(&tx, X, static_cast<uint64_t>(x_rows), x_cols, S::kXBoxRows))
     return MOE_ERR_CUDA;
   if (!make_tmap(&tw, W, static_cast<uint64_t>(w_rows), static_cast<uint64_t>(p.K), S::kWBoxRows))
     return MOE_ERR_CUDA;
@@ -117,6 +120,7 @@ moe_status_t launch_gemm_pair(const void* X, long x_rows, const void* W, long w_
   });
   if (attr_err != cudaSuccess) return MOE_ERR_CUDA;
   CUtensorMap tx, tw;
+  if (p.x_k_period > 0) return MOE_ERR_UNSUPPORTED;  // the pair kernel has no wrapping X
   if (!make_tmap(&tx, X, static_cast<uint64_t>(x_rows), static_cast<uint64_t>(p.K), 128))
     return MOE_ERR_CUDA;
   if (!make_tmap(&tw, W, static_cast<uint64_t>(w_rows), static_cast<uint64_t>(p.K), BN / 2))
@@ -193,6 +197,9 @@ moe_status_t check_cfg(const moe_config_t* c) {
   if (c->dtype != MOE_F32 && c->dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
   if (c->expert_act != MOE_ACT_RELU && c->expert_act != MOE_ACT_SWIGLU) return MOE_ERR_UNSUPPORTED;
   if (c->resid_mode < MOE_RESID_NONE || c->resid_mode > MOE_RESID_LITERAL) return MOE_ERR_UNSUPPORTED;
+  if (c->gate_mode != MOE_GATE_SOFTMAX && c->gate_mode != MOE_GATE_SIGMOID) return MOE_ERR_UNSUPPORTED;
+  if (c->router_f32 != 0 && c->router_f32 != 1) return MOE_ERR_INVALID_ARG;
+  if (c->gate_mode == MOE_GATE_SIGMOID && !(c->logit_mult == c->logit_mult)) return MOE_ERR_INVALID_ARG;
   if (!(c->eps >= 0.0f) || !(c->tau > 0.0f) || !(c->resid_floor >= 0.0f)) return MOE_ERR_INVALID_ARG;
   if (static_cast<long>(c->T) * c->top_k > 0x7fffffffL / 2) return MOE_ERR_UNSUPPORTED;
   if (c->dtype == MOE_BF16) {
@@ -271,16 +278,19 @@ Orient dense_orient(int rows, int bn) {
 constexpr int kSmallRouterMaxT = 256;
 
 moe_status_t do_route(const moe_config_t& c, const void* u, const void* w_router,
-                      const float* bias, float* logits, int32_t* idx, float* w, cudaStream_t st,
-                      float* logits_scratch = nullptr) {
+                      const float* bias, const float* sel_bias, float* logits, int32_t* idx,
+                      float* w, cudaStream_t st, float* logits_scratch = nullptr) {
   if (c.T == 0) return MOE_OK;
+  const bool sig = c.gate_mode == MOE_GATE_SIGMOID;
+  const float mult = sig ? c.logit_mult : 1.0f;
   if (c.dtype == MOE_F32) {
     const int warps = 4;
     router_f32_kernel<<<cdiv(c.T, warps), 32 * warps, 0, st>>>(
         static_cast<const float*>(u), static_cast<const float*>(w_router), bias, c.T, c.d_model,
-        c.n_experts, c.top_k, c.routed_scale, logits, idx, w);
+        c.n_experts, c.top_k, c.routed_scale, c.gate_mode, mult, sel_bias, logits, idx, w);
     return last_launch();
   }
+  const int wk = c.router_f32 ? 3 * c.d_model : c.d_model;  // router weight row length
   float* lbuf = logits ? logits : logits_scratch;
   const size_t small_smem = static_cast<size_t>(kRouterTok) * c.d_model * 2;
   if (c.T <= kSmallRouterMaxT && lbuf && small_smem <= 200 * 1024) {
@@ -294,15 +304,16 @@ moe_status_t do_route(const moe_config_t& c, const void* u, const void* w_router
     dim3 grid(cdiv(c.n_experts, kRouterExp), cdiv(c.T, kRouterTok));
     router_logits_small_kernel<<<grid, 256, small_smem, st>>>(
         static_cast<const uint16_t*>(u), static_cast<const uint16_t*>(w_router), bias, c.T,
-        c.d_model, c.n_experts, lbuf);
+        c.d_model, c.n_experts, wk, mult, lbuf);
     topk_rows_kernel<<<cdiv(c.T, 8), 256, 0, st>>>(lbuf, c.T, c.n_experts, c.top_k,
-                                                    c.routed_scale, idx, w);
+                                                    c.routed_scale, c.gate_mode, sel_bias, idx, w);
     return last_launch(2);
   }
   GemmParams p{};
   p.G = 1;
   p.M = c.T;
-  p.K = c.d_model;
+  p.K = wk;
+  p.x_k_period = c.router_f32 ? c.d_model : 0;
   p.Nw = c.n_experts;
   p.Nout = c.n_experts;
   p.logits = logits;
@@ -311,6 +322,9 @@ moe_status_t do_route(const moe_config_t& c, const void* u, const void* w_router
   p.bias = bias;
   p.top_k = c.top_k;
   p.routed_scale = c.routed_scale;
+  p.gate_mode = c.gate_mode;
+  p.logit_mult = mult;
+  p.sel_bias = sel_bias;
   const int bn = c.n_experts <= 32 ? 32 : c.n_experts <= 64 ? 64 : c.n_experts <= 128 ? 128 : 256;
   return run_gemm(EPI_ROUTER, Orient::kNormal, bn, u, c.T, w_router, c.n_experts, p, st);
 }
@@ -511,16 +525,30 @@ moe_status_t moe_workspace_size(const moe_config_t* cfg, size_t* bytes) {
 }
 
 moe_status_t moe_route(const moe_config_t* cfg, const void* u, const void* w_router,
-                       const float* logit_bias, float* logits_out, int32_t* topk_idx,
-                       float* topk_w, void* stream) {
+                       const float* logit_bias, const float* correction_bias, float* logits_out,
+                       int32_t* topk_idx, float* topk_w, void* stream) {
   moe_status_t s = check_cfg(cfg);
   if (s != MOE_OK) return s;
   if (cfg->T > 0 && (!u || !w_router || !topk_idx || !topk_w)) return MOE_ERR_INVALID_ARG;
   if (!all_aligned({u, w_router, static_cast<const void*>(logit_bias),
-                        static_cast<const void*>(logits_out), static_cast<const void*>(topk_idx),
-                        static_cast<const void*>(topk_w)})) return MOE_ERR_ALIGNMENT;
-  return do_route(*cfg, u, w_router, logit_bias, logits_out, topk_idx, topk_w,
+                    static_cast<const void*>(correction_bias), static_cast<const void*>(logits_out),
+                    static_cast<const void*>(topk_idx), static_cast<const void*>(topk_w)}))
+    return MOE_ERR_ALIGNMENT;
+  return do_route(*cfg, u, w_router, logit_bias, correction_bias, logits_out, topk_idx, topk_w,
                   static_cast<cudaStream_t>(stream));
+}
+
+moe_status_t moe_router_split_weights(const float* w, int32_t n, int32_t d, void* w_split,
+                                      void* stream) {
+  if (!w || !w_split || n <= 0 || d <= 0) return MOE_ERR_INVALID_ARG;
+  if (d % 64) return MOE_ERR_UNSUPPORTED;
+  if (!all_aligned({static_cast<const void*>(w), static_cast<const void*>(w_split)}))
+    return MOE_ERR_ALIGNMENT;
+  const size_t count = static_cast<size_t>(n) * d;
+  const unsigned blocks = static_cast<unsigned>(std::min<size_t>((count + 255) / 256, 148 * 16));
+  router_split_kernel<<<blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      w, count, d, static_cast<uint16_t*>(w_split));
+  return last_launch();
 }
 
 moe_status_t moe_permute(const moe_config_t* cfg, const int32_t* topk_idx,
@@ -667,7 +695,8 @@ moe_status_t moe_layer_forward(const moe_config_t* cfg, const moe_weights_t* w, 
                         workspace, w->w_router, w->p_down, w->p_up, w->w_gu, w->w_down,
                         static_cast<const void*>(w->gamma_pre),
                         static_cast<const void*>(w->gamma_expert),
-                        static_cast<const void*>(w->resid_g), static_cast<const void*>(w->logit_bias)})) return MOE_ERR_ALIGNMENT;
+                        static_cast<const void*>(w->resid_g), static_cast<const void*>(w->logit_bias),
+                        static_cast<const void*>(w->correction_bias)})) return MOE_ERR_ALIGNMENT;
   const Workspace L = layout(c);
   if (!workspace || workspace_bytes < L.total) return MOE_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -680,7 +709,7 @@ moe_status_t moe_layer_forward(const moe_config_t* cfg, const moe_weights_t* w, 
   void* act = at<void>(workspace, L.act);
 
   prof_mark(st, 0);
-  if ((s = do_route(c, u, w->w_router, w->logit_bias, logits_out, idx, wt, st,
+  if ((s = do_route(c, u, w->w_router, w->logit_bias, w->correction_bias, logits_out, idx, wt, st,
                     at<float>(workspace, L.logits))) != MOE_OK)
     return s;
   prof_mark(st, 1);

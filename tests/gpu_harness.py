@@ -22,7 +22,8 @@ def abi_config(cfg, T: int | None = None):
         top_k=cfg.top_k, d_ff=cfg.d_ff, d_latent=cfg.d_latent,
         dtype=moe.MOE_BF16 if cfg.dtype == "bf16" else moe.MOE_F32, expert_act=cfg.act,
         pre_norm=cfg.pre_norm, expert_norm=cfg.expert_norm, resid_mode=cfg.resid_mode,
-        eps=cfg.eps, tau=cfg.tau, resid_floor=cfg.resid_floor, routed_scale=cfg.routed_scale)
+        eps=cfg.eps, tau=cfg.tau, resid_floor=cfg.resid_floor, routed_scale=cfg.routed_scale,
+        gate_mode=cfg.gate_mode, router_f32=cfg.router_f32, logit_mult=cfg.logit_mult)
 
 
 def host_values(a: np.ndarray, dtype: str) -> np.ndarray:
@@ -53,8 +54,12 @@ def logit_atol(cfg, logits: np.ndarray) -> float:
     """Absolute tolerance of fp32-accumulated router logits against double: the products of two
     bf16 (or fp32-rounded) values are summed in fp32 over K = d_model terms; rounding errors of
     a K-term sum grow like sqrt(K) * 2^-24 * |partial sums|, so allow 16 sqrt(K) 2^-24 times the
-    largest logit magnitude (at least 1)."""
-    return 16.0 * np.sqrt(cfg.d_model) * 2.0 ** -24 * max(1.0, float(np.abs(logits).max()))
+    largest logit magnitude (at least 1).  fp32 router weights are summed as three bf16 parts
+    (K = 3 d_model); the sigmoid gate's scores move by at most a quarter of the logit error times
+    the output multiplier, so the same bound scaled by the multiplier covers them."""
+    K = cfg.d_model * (3 if cfg.router_f32 and cfg.dtype == "bf16" else 1)
+    mult = max(1.0, abs(cfg.logit_mult)) if cfg.gate_mode == configs.GATE_SIGMOID else 1.0
+    return 16.0 * np.sqrt(K) * 2.0 ** -24 * mult * max(1.0, float(np.abs(logits).max()))
 
 
 def run_layer(cfg, dev: dict, want_logits: bool = True):
@@ -99,11 +104,30 @@ def oracle_reference(cfg, tokens=None):
     return oracle.layer_forward_staged(cfg, tokens, get_inputs, get_expert)
 
 
+def correction_bias(cfg):
+    """Host copy of the sigmoid gate's selection-only bias (None for the softmax gate)."""
+    if cfg.gate_mode != configs.GATE_SIGMOID:
+        return None
+    return moe_inputs.host_rows(cfg, "correction_bias")
+
+
+def selection_keys(cfg, logits: np.ndarray) -> np.ndarray:
+    """What the top-k is taken on: the logits (softmax gate) or the scores + correction bias."""
+    cb = correction_bias(cfg)
+    return logits if cb is None else logits + cb.astype(np.float64)
+
+
 def check_routing(cfg, logits_gpu: np.ndarray, idx_gpu: np.ndarray, w_gpu: np.ndarray):
-    """Bit-exact routing on every token: the oracle's selection run on the GPU's fp32 logits must
-    equal the GPU's indices; weights within 1e-6 relative; permutation bit-exact."""
+    """Bit-exact routing on every token: the oracle's selection run on the GPU's fp32 logits (or
+    sigmoid scores, with the selection key formed by one fp32 addition of the correction bias)
+    must equal the GPU's indices; weights within 1e-6 relative."""
     import oracle
-    sel, wref = oracle.softmax_topk(logits_gpu.astype(np.float32), cfg.top_k, cfg.routed_scale)
+    if cfg.gate_mode == configs.GATE_SIGMOID:
+        sel, wref = oracle.sigmoid_topk_scores_f32(logits_gpu.astype(np.float32), cfg.top_k,
+                                                   correction_bias(cfg), cfg.routed_scale)
+    else:
+        sel, wref = oracle.softmax_topk(logits_gpu.astype(np.float32), cfg.top_k,
+                                        cfg.routed_scale)
     np.testing.assert_array_equal(idx_gpu, sel)
     np.testing.assert_allclose(w_gpu, wref, rtol=1e-6, atol=1e-7)
     np.testing.assert_allclose(w_gpu.sum(1), cfg.routed_scale, rtol=2e-6)

@@ -64,9 +64,19 @@ def test_bad_config_rejected(lib, field, value, code):
 
 def test_null_and_misaligned_pointers_rejected(lib):
     c = abi_config(configs.MUSE_DECODE)
-    rc = lib.moe_route(ctypes.byref(c), None, None, None, None, None, None, None)
+    rc = lib.moe_route(ctypes.byref(c), None, None, None, None, None, None, None, None)
     assert rc == moe.STATUS_CODES["MOE_ERR_INVALID_ARG"]
-    rc = lib.moe_route(ctypes.byref(c), 0x1001, 0x2000, None, None, 0x3000, 0x4000, None)
+    rc = lib.moe_route(ctypes.byref(c), 0x1001, 0x2000, None, None, None, 0x3000, 0x4000, None)
+    assert rc == moe.STATUS_CODES["MOE_ERR_ALIGNMENT"]
+    # a misaligned correction bias is caught too
+    rc = lib.moe_route(ctypes.byref(c), 0x1000, 0x2000, None, 0x3004, None, 0x3000, 0x4000, None)
+    assert rc == moe.STATUS_CODES["MOE_ERR_ALIGNMENT"]
+    # the split entry point checks its sizes and pointers on the host
+    assert lib.moe_router_split_weights(None, 4, 64, 0x1000, None) == \
+        moe.STATUS_CODES["MOE_ERR_INVALID_ARG"]
+    assert lib.moe_router_split_weights(0x1000, 4, 100, 0x2000, None) == \
+        moe.STATUS_CODES["MOE_ERR_UNSUPPORTED"]
+    rc = lib.moe_route(ctypes.byref(c), 0x1001, 0x2000, None, None, None, 0x3000, 0x4000, None)
     assert rc == moe.STATUS_CODES["MOE_ERR_ALIGNMENT"]
     rc = lib.moe_layer_forward(ctypes.byref(c), None, 0x1000, 0x1000, 0x2000, None, None, None,
                                None, 0, None)

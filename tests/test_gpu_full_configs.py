@@ -15,7 +15,7 @@ import oracle
 from moe_inputs import configs
 
 from gpu_harness import (abi_config, check_routing, compare_selection, device_values, logit_atol,
-                         oracle_reference, row_rel_err, run_layer, tolerance)
+                         oracle_reference, row_rel_err, run_layer, selection_keys, tolerance)
 
 torch = pytest.importorskip("torch")
 moe = pytest.importorskip("sparse_moe_layer_softmax_b200")
@@ -38,9 +38,9 @@ def _permutation_bit_exact(cfg, idx_dev, idx):
     return r_off
 
 
-@pytest.mark.parametrize("name", list(configs.CONFIGS))
+@pytest.mark.parametrize("name", list(configs.CONFIGS) + list(configs.VARIANT_CONFIGS))
 def test_full_workload(name):
-    cfg = configs.CONFIGS[name]
+    cfg = configs.ALL_CONFIGS[name]
     dev = moe_inputs.device_inputs(cfg)
     res = run_layer(cfg, dev)
     logits = res["logits"].cpu().numpy()
@@ -55,7 +55,7 @@ def test_full_workload(name):
     del res, dev
     torch.cuda.empty_cache()
     ref = oracle_reference(cfg, tokens)
-    ties = compare_selection(idx[tokens], ref["logits"], ref["idx"], cfg.top_k)
+    ties = compare_selection(idx[tokens], selection_keys(cfg, ref["logits"]), ref["idx"], cfg.top_k)
     assert ties.sum() <= max(2, len(tokens) // 100)
     lg = logits[tokens]
     np.testing.assert_allclose(lg, ref["logits"], rtol=0, atol=logit_atol(cfg, lg))

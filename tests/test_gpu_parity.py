@@ -12,7 +12,8 @@ import oracle
 from moe_inputs import configs
 
 from gpu_harness import (abi_config, check_routing, compare_selection, device_values, host_values,
-                         logit_atol, oracle_reference, row_rel_err, run_layer, tolerance)
+                         logit_atol, oracle_reference, row_rel_err, run_layer, selection_keys,
+                         tolerance)
 
 torch = pytest.importorskip("torch")
 pytestmark = pytest.mark.gpu
@@ -72,6 +73,16 @@ SMALL = [
     # fp32 CUDA-core path
     configs.TINY_SHAZEER_F32.replace(T=45, seed=20),
     configs.TINY_SHAZEER_F32.replace(T=64, top_k=8, seed=21),
+    # Muse sigmoid gate: fp32 router weights (exact bf16 split) on the GEMM router (T > 256)
+    # and on the few-token router, bf16 router weights, and the fp32 layer
+    configs.small_muse(T=300, d=512, L=256, I=256, n=16, k=4, seed=25, gate_mode=configs.GATE_SIGMOID,
+                       router_f32=1, logit_mult=2.0, corr_sigma=0.3, routed_scale=1.5),
+    configs.small_muse(T=40, d=256, L=128, I=128, n=64, k=8, seed=26,
+                       gate_mode=configs.GATE_SIGMOID, router_f32=1),
+    configs.small_muse(T=96, d=256, L=128, I=128, n=32, k=4, seed=27,
+                       gate_mode=configs.GATE_SIGMOID, corr_sigma=0.2),
+    configs.TINY_SHAZEER_F32.replace(T=50, seed=24, gate_mode=configs.GATE_SIGMOID,
+                                     logit_mult=0.5, router_gain=1.0),
 ]
 
 
@@ -98,7 +109,7 @@ def _check_layer(cfg):
     logits = res["logits"].cpu().numpy()
     idx = res["idx"].cpu().numpy()
     check_routing(cfg, logits, idx, res["w"].cpu().numpy())
-    ties = compare_selection(idx, ref["logits"], ref["idx"], cfg.top_k)
+    ties = compare_selection(idx, selection_keys(cfg, ref["logits"]), ref["idx"], cfg.top_k)
     assert ties.sum() <= max(1, cfg.T // 100)
     np.testing.assert_allclose(logits, ref["logits"], rtol=0, atol=logit_atol(cfg, logits))
     err = row_rel_err(device_values(res["out"])[~ties], ref["out"][~ties])
@@ -106,6 +117,15 @@ def _check_layer(cfg):
 
 
 # ------------------------------------------------------------------ individual entry points
+
+
+def test_router_split_is_exact():
+    """hi + mid + lo reconstructs every fp32 router weight exactly."""
+    w = torch.empty((64, 512), dtype=torch.float32, device="cuda")
+    moe_inputs.normal_device(w, 3, 90, 0, 0.7)
+    w[0, :8] = torch.tensor([0.0, -0.0, 1.0, -3.0e-5, 1.0e4, 1.0 / 3.0, 2.0 ** -100, 65504.0])
+    parts = moe.router_split(w).view(64, 3, 512).double()
+    np.testing.assert_array_equal(parts.sum(1).cpu().numpy(), w.double().cpu().numpy())
 
 
 def _rand_routing(T, n, k, seed, hot=None):
