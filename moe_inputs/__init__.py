@@ -180,6 +180,10 @@ def tensor_specs(cfg: MoEConfig):
                                  cfg.gamma_sigma)
     if cfg.gate_mode == configs.GATE_SIGMOID:
         specs["correction_bias"] = ((n,), configs.STREAM_CORR_BIAS, "f32n", cfg.corr_sigma)
+    if cfg.input_norm:
+        specs["gamma_in"] = ((d,), configs.STREAM_GAMMA_IN, "f32n", cfg.gamma_sigma)
+    if cfg.post_norm:
+        specs["gamma_post"] = ((d,), configs.STREAM_GAMMA_POST, "f32n", cfg.gamma_sigma)
     if cfg.resid_mode != configs.RESID_NONE:
         specs["resid_g"] = ((d,), configs.STREAM_RESID_G, "f32u", 0.0)
     return specs

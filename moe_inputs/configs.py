@@ -46,6 +46,8 @@ RESID_LITERAL = 2
 GATE_SOFTMAX = 0
 GATE_SIGMOID = 1
 STREAM_CORR_BIAS = 13
+STREAM_GAMMA_IN = 14
+STREAM_GAMMA_POST = 15
 
 # Scale c of the Zipf router bias  bias_e = -c * s * ln(rank_e)  (s = 1.2) for the imbalanced
 # workload.  Calibrated by tests/golden/calibrate_zipf_bias.py, which bisects c with the CPU
@@ -83,6 +85,9 @@ class MoEConfig:
     router_f32: int = 0         # router weights stored in fp32
     logit_mult: float = 1.0     # output_multiplier of the sigmoid gate
     corr_sigma: float = 0.05    # std of the sigmoid gate's selection-only correction bias
+    input_norm: int = 0         # decoder wrap: u = C_in(h), centred RMSNorm of the residual stream
+    post_norm: int = 0          # decoder wrap: input-scaled output norm I_post on b before the gate
+    eps_block: float = 1e-5     # epsilon of the decoder-level norms (model sheet: 1e-5)
 
     @property
     def latent(self) -> bool:
@@ -152,7 +157,16 @@ MUSE_DECODE_SIGMOID = MUSE_DECODE.replace(name="muse_decode_sigmoid", gate_mode=
                                           router_f32=1, seed=8)
 MUSE_PREFILL_SIGMOID = MUSE_PREFILL.replace(name="muse_prefill_sigmoid", gate_mode=GATE_SIGMOID,
                                             router_f32=1, seed=9)
-VARIANT_CONFIGS = {c.name: c for c in (MUSE_DECODE_SIGMOID, MUSE_PREFILL_SIGMOID)}
+# The MoE sub-block of the decoder layer as the Muse audit describes it ("The complete layer has
+# two separately normalized residual updates"): the residual stream h is normalised (block norm
+# with a (1 + gamma) gain, eps 1e-5 per the model sheet), the latent MoE runs, its output goes
+# through the FFN's input-scaled output norm, and the residual gate mixes it into h.
+MUSE_DECODE_BLOCK = MUSE_DECODE.replace(name="muse_decode_block", input_norm=1, post_norm=1,
+                                        seed=10)
+MUSE_PREFILL_BLOCK = MUSE_PREFILL.replace(name="muse_prefill_block", input_norm=1, post_norm=1,
+                                          seed=11)
+VARIANT_CONFIGS = {c.name: c for c in (MUSE_DECODE_SIGMOID, MUSE_PREFILL_SIGMOID,
+                                       MUSE_DECODE_BLOCK, MUSE_PREFILL_BLOCK)}
 ALL_CONFIGS = {**CONFIGS, **PROFILE_CONFIGS, **VARIANT_CONFIGS}
 
 

@@ -35,7 +35,8 @@ class OrcCfg(ctypes.Structure):
                                             "expert_norm", "resid_mode")] + \
                [(n, ctypes.c_double) for n in ("eps", "tau", "resid_floor", "routed_scale")] + \
                [("gate_mode", ctypes.c_int), ("router_f32", ctypes.c_int),
-                ("logit_mult", ctypes.c_double)]
+                ("logit_mult", ctypes.c_double), ("input_norm", ctypes.c_int),
+                ("post_norm", ctypes.c_int), ("eps_block", ctypes.c_double)]
 
 
 class OrcTensors(ctypes.Structure):
@@ -44,7 +45,8 @@ class OrcTensors(ctypes.Structure):
                 ("p_up", ctypes.c_void_p), ("w_gu", ctypes.POINTER(ctypes.c_void_p)),
                 ("w_down", ctypes.POINTER(ctypes.c_void_p)), ("gamma_pre", ctypes.c_void_p),
                 ("gamma_expert", ctypes.c_void_p), ("resid_g", ctypes.c_void_p),
-                ("correction_bias", ctypes.c_void_p)]
+                ("correction_bias", ctypes.c_void_p), ("gamma_in", ctypes.c_void_p),
+                ("gamma_post", ctypes.c_void_p)]
 
 
 def lib():
@@ -102,7 +104,8 @@ def make_cfg(cfg, T: int | None = None) -> OrcCfg:
                   is_bf16=1 if cfg.dtype == "bf16" else 0, act=cfg.act, pre_norm=cfg.pre_norm,
                   expert_norm=cfg.expert_norm, resid_mode=cfg.resid_mode, eps=cfg.eps,
                   tau=cfg.tau, resid_floor=cfg.resid_floor, routed_scale=cfg.routed_scale,
-                  gate_mode=cfg.gate_mode, router_f32=cfg.router_f32, logit_mult=cfg.logit_mult)
+                  gate_mode=cfg.gate_mode, router_f32=cfg.router_f32, logit_mult=cfg.logit_mult,
+                  input_norm=cfg.input_norm, post_norm=cfg.post_norm, eps_block=cfg.eps_block)
 
 
 class _Keep:
@@ -146,7 +149,9 @@ def make_tensors(cfg, inp: dict, keep: _Keep, experts: dict | None = None) -> Or
                       gamma_pre=keep.ptr(inp.get("gamma_pre")),
                       gamma_expert=keep.ptr(inp.get("gamma_expert")),
                       resid_g=keep.ptr(inp.get("resid_g")),
-                      correction_bias=keep.ptr(inp.get("correction_bias")))
+                      correction_bias=keep.ptr(inp.get("correction_bias")),
+                      gamma_in=keep.ptr(inp.get("gamma_in")),
+                      gamma_post=keep.ptr(inp.get("gamma_post")))
 
 
 def layer_forward(cfg, inp: dict, tokens=None, nthreads: int | None = None) -> dict:

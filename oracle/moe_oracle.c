@@ -211,11 +211,33 @@ void orc_resid_gate_coeffs(double g, double tau, double floor_, double* alpha, d
 
 static int expert_in(const orc_cfg* c) { return c->d_latent > 0 ? c->d_latent : c->d_model; }
 
+/* The layer's branch input u_t: the given u, or with input_norm the residual stream's centred
+ * RMSNorm dtype(C_in(h_t)) [MUSE "The complete layer has two separately normalized residual
+ * updates": the layer normalizes the residual stream, then runs the latent MoE; ARCHDB: block
+ * norms are RMSNorm with a (1 + w) gain]. */
+static void load_u(const orc_cfg* c, const orc_tensors* x, int64_t t, double* ut) {
+  int d = c->d_model;
+  if (!c->input_norm) {
+    for (int i = 0; i < d; ++i) ut[i] = ld(x->u, (size_t)t * d + i, c->is_bf16);
+    return;
+  }
+  double* h = (double*)malloc(sizeof(double) * (size_t)d);
+  double* g = (double*)malloc(sizeof(double) * (size_t)d);
+  for (int i = 0; i < d; ++i) {
+    h[i] = ld(x->h, (size_t)t * d + i, c->is_bf16);
+    g[i] = (double)x->gamma_in[i];
+  }
+  orc_centered_rmsnorm(h, g, d, c->eps_block, ut);
+  for (int i = 0; i < d; ++i) ut[i] = orc_round(c, ut[i]);
+  free(g);
+  free(h);
+}
+
 void orc_router_token(const orc_cfg* c, const orc_tensors* x, int64_t t, double* logits, int* idx,
                       double* w) {
   int d = c->d_model, n = c->n_experts;
   double* ut = (double*)malloc(sizeof(double) * (size_t)d);
-  for (int i = 0; i < d; ++i) ut[i] = ld(x->u, (size_t)t * d + i, c->is_bf16);
+  load_u(c, x, t, ut);
   /* fp32 router weights are read as fp32 whatever the other tensors' dtype */
   const int w_is_bf16 = c->router_f32 ? 0 : c->is_bf16;
   for (int e = 0; e < n; ++e) {
@@ -235,12 +257,12 @@ void orc_router_token(const orc_cfg* c, const orc_tensors* x, int64_t t, double*
 void orc_expert_input_token(const orc_cfg* c, const orc_tensors* x, int64_t t, double* z) {
   int d = c->d_model, L = c->d_latent;
   if (L <= 0) {
-    for (int i = 0; i < d; ++i) z[i] = ld(x->u, (size_t)t * d + i, c->is_bf16);
+    load_u(c, x, t, z);
     return;
   }
   double* ut = (double*)malloc(sizeof(double) * (size_t)d);
   double* zr = (double*)malloc(sizeof(double) * (size_t)L);
-  for (int i = 0; i < d; ++i) ut[i] = ld(x->u, (size_t)t * d + i, c->is_bf16);
+  load_u(c, x, t, ut);
   for (int i = 0; i < L; ++i) zr[i] = orc_round(c, dot_row(x->p_down, (size_t)i, d, ut, c->is_bf16));
   if (c->pre_norm) {
     double* g = (double*)malloc(sizeof(double) * (size_t)L);
@@ -297,8 +319,22 @@ void orc_combine_token(const orc_cfg* c, const double* n_slots, const double* w,
 void orc_output_token(const orc_cfg* c, const orc_tensors* x, int64_t t, const double* y,
                       double* out) {
   int d = c->d_model, L = c->d_latent;
+  double* bv = (double*)malloc(sizeof(double) * (size_t)d);
+  for (int i = 0; i < d; ++i)
+    bv[i] = (L > 0) ? orc_round(c, dot_row(x->p_up, (size_t)i, L, y, c->is_bf16)) : y[i];
+  if (c->post_norm) {
+    /* the FFN's input-scaled output norm before the residual gate [MUSE "The complete layer
+     * has two separately normalized residual updates"]: b <- dtype(I_post(b)) */
+    double* g = (double*)malloc(sizeof(double) * (size_t)d);
+    double* nb = (double*)malloc(sizeof(double) * (size_t)d);
+    for (int i = 0; i < d; ++i) g[i] = (double)x->gamma_post[i];
+    orc_input_scaled_rmsnorm(c, bv, g, d, c->eps_block, nb);
+    for (int i = 0; i < d; ++i) bv[i] = orc_round(c, nb[i]);
+    free(nb);
+    free(g);
+  }
   for (int i = 0; i < d; ++i) {
-    double b = (L > 0) ? orc_round(c, dot_row(x->p_up, (size_t)i, L, y, c->is_bf16)) : y[i];
+    double b = bv[i];
     double r;
     if (c->resid_mode == 0) {
       r = b;
@@ -314,6 +350,7 @@ void orc_output_token(const orc_cfg* c, const orc_tensors* x, int64_t t, const d
     }
     out[i] = orc_round(c, r);
   }
+  free(bv);
 }
 
 /* ------------------------------------------------------------------ whole layer */

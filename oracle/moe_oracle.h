@@ -43,6 +43,10 @@ typedef struct {
                            bias, weights score / (sum_sel score + 1e-15)) */
   int router_f32;    /* 1: router weights are fp32 (whatever the tensors' dtype) */
   double logit_mult; /* output_multiplier applied to the router logits (sigmoid gate) */
+  int input_norm;    /* decoder wrap: u = C_in(h), the residual stream's centred RMSNorm */
+  int post_norm;     /* decoder wrap: the FFN's input-scaled output norm I_post on b before the
+                        residual gate */
+  double eps_block;  /* epsilon of the two decoder-level norms */
 } orc_cfg;
 
 typedef struct {
@@ -58,6 +62,8 @@ typedef struct {
   const float* gamma_expert;/* [E_in], one gain shared by every expert */
   const float* resid_g;     /* [d_model] */
   const float* correction_bias; /* [n] sigmoid gate: added to the scores for selection only */
+  const float* gamma_in;    /* [d_model] input_norm gain */
+  const float* gamma_post;  /* [d_model] post_norm gain */
 } orc_tensors;
 
 /* storage rounding of the configured dtype (bf16 RNE, or fp32) */

@@ -224,6 +224,10 @@ def dense_bruteforce(cfg, inp):
     """Every expert evaluated on every token with numpy matmuls, then gathered by the gate."""
     dt = cfg.dtype
     u = _val(inp["u"], dt)
+    h = u  # the residual stream
+    if cfg.input_norm:
+        gi = inp["gamma_in"].astype(np.float64)
+        u = _rnd((1 + gi) * h / np.sqrt(np.mean(h * h, 1, keepdims=True) + cfg.eps_block), dt)
     wr = _val(inp["w_router"], "f32" if cfg.router_f32 else dt)
     logits = u @ wr.T
     if cfg.gate_mode == configs.GATE_SIGMOID:
@@ -275,13 +279,16 @@ def dense_bruteforce(cfg, inp):
         b = _rnd(y @ _val(inp["p_up"], dt).T, dt)
     else:
         b = y
+    if cfg.post_norm:
+        sp = _rnd(b * (1 + inp["gamma_post"].astype(np.float64)), dt)
+        b = _rnd(sp / np.sqrt(np.mean(sp * sp, 1, keepdims=True) + cfg.eps_block), dt)
     if cfg.resid_mode == configs.RESID_MUSE_GATE:
         gg = inp["resid_g"].astype(np.float64)
         beta = 1 / (1 + np.exp(-gg / cfg.tau))
         alpha = np.sqrt(np.maximum((1 / (1 + np.exp(gg / cfg.tau))) * (1 + beta), cfg.resid_floor))
-        out = _rnd(alpha * u + beta * b, dt)
+        out = _rnd(alpha * h + beta * b, dt)
     elif cfg.resid_mode == configs.RESID_LITERAL:
-        out = _rnd(u + inp["resid_g"].astype(np.float64) * b, dt)
+        out = _rnd(h + inp["resid_g"].astype(np.float64) * b, dt)
     else:
         out = b
     return out, logits, top, w, y
@@ -301,7 +308,21 @@ BRUTE_CASES = [
                        corr_sigma=0.3, routed_scale=1.5),
     configs.small_muse(T=10, d=40, L=24, I=16, n=6, k=2, dtype="f32",
                        gate_mode=configs.GATE_SIGMOID, router_f32=1),
+    # decoder wrap: residual-stream norm before the MoE, output norm before the residual gate
+    configs.small_muse(T=12, d=48, L=32, I=24, n=6, k=3, gamma_sigma=0.3, input_norm=1,
+                       post_norm=1),
+    configs.small_muse(T=8, d=40, L=24, I=16, n=5, k=2, dtype="f32", gamma_sigma=0.3,
+                       input_norm=1, post_norm=1, resid_mode=configs.RESID_LITERAL),
 ]
+
+
+def test_post_norm_output_has_unit_rms():
+    """With post_norm, no residual and gamma_post = 0, every output row is R(b): unit RMS."""
+    cfg = configs.small_muse(T=9, d=48, L=32, I=24, n=6, k=2, dtype="f32", post_norm=1,
+                             resid_mode=configs.RESID_NONE, gamma_sigma=0.0, eps_block=0.0,
+                             eps=0.0)
+    res = oracle.layer_forward(cfg, moe_inputs.host_inputs(cfg))
+    np.testing.assert_allclose(np.sqrt(np.mean(res["out"] ** 2, 1)), 1.0, rtol=1e-5)
 
 
 @pytest.mark.parametrize("cfg", BRUTE_CASES, ids=lambda c: f"{c.name}-{c.dtype}-r{c.resid_mode}")
