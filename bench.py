@@ -564,14 +564,15 @@ def main(argv=None) -> int:
             "stage_ms": dres["stage_ms"], "distinct_experts": dres["distinct_experts"],
             "gpu_launches": dres["gpu_launches"], "clocks": dres["clocks"]}
     if not args.no_decode and cfg.name != "muse_decode":
-        # the Muse router as the Muse audit describes it (fp32 weights, sigmoid gate) on decode
-        vcfg = configs.MUSE_DECODE_SIGMOID
-        vres = measure_checked(vcfg, args, device, peaks, rank, local, with_e2e=False)
-        line["variants"] = {vcfg.name: {
-            "value": round(vcfg.T * world / (vres["ms_per_step"] / 1e3), 2), "unit": UNIT,
-            "ms_per_step": round(vres["ms_per_step"], 4),
-            "route_ms": vres["stage_ms"]["route"],
-            "layer_roofline": vres["layer_roofline"], "clocks": vres["clocks"]}}
+        # decode with the Muse router as the Muse audit describes it (fp32 weights, sigmoid
+        # gate), and the decoder layer's whole FFN sub-block (input norm, output norm)
+        line["variants"] = {}
+        for vcfg in (configs.MUSE_DECODE_SIGMOID, configs.MUSE_DECODE_BLOCK):
+            vres = measure_checked(vcfg, args, device, peaks, rank, local, with_e2e=False)
+            line["variants"][vcfg.name] = {
+                "value": round(vcfg.T * world / (vres["ms_per_step"] / 1e3), 2), "unit": UNIT,
+                "ms_per_step": round(vres["ms_per_step"], 4), "stage_ms": vres["stage_ms"],
+                "layer_roofline": vres["layer_roofline"], "clocks": vres["clocks"]}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(cfg, args.cpu_sample or default_cpu_sample(cfg))
     if rank == 0:

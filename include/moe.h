@@ -89,6 +89,12 @@ typedef struct {
   int32_t router_f32;   /* 1: the router weights are fp32, passed as their exact bf16 split
                            [n, 3*d_model] (hi, mid, lo; see moe_router_split_weights) */
   float logit_mult;     /* output_multiplier on the router logits (sigmoid gate) */
+  int32_t input_norm;   /* decoder wrap (bf16): the branch input is u = dtype(C_in(r)), the
+                           residual stream's centred RMSNorm (gain 1+gamma_in, eps_block) */
+  int32_t post_norm;    /* decoder wrap (bf16, latent): the up-projection b goes through the
+                           FFN's input-scaled output norm I_post (gain 1+gamma_post, eps_block)
+                           before the residual gate */
+  float eps_block;      /* epsilon of the two decoder-level norms */
 } moe_config_t;
 
 typedef struct {
@@ -103,6 +109,8 @@ typedef struct {
   const float* resid_g;     /* [d_model] residual gate parameter g (resid_mode != NONE) */
   const float* logit_bias;  /* [n] added to every token's router logits, or NULL */
   const float* correction_bias; /* [n] sigmoid gate: added to the scores for selection only */
+  const float* gamma_in;    /* [d_model] input_norm gain */
+  const float* gamma_post;  /* [d_model] post_norm gain */
 } moe_weights_t;
 
 /* Human-readable name of a status code (static storage). */
@@ -201,11 +209,23 @@ MOE_API moe_status_t moe_latent_down(const moe_config_t* cfg, const void* u, con
 MOE_API moe_status_t moe_latent_up(const moe_config_t* cfg, const void* y, const void* p_up,
                            const void* r, const float* resid_g, void* out, void* stream);
 
-/* The whole layer: route -> latent down (+C_pre) -> dispatch -> experts (+I_gamma prep) ->
- * normalise and combine -> latent up -> residual update.  u: [T, d_model] is the branch input
- * (router and down-projection read it), r: [T, d_model] the residual stream (may equal u;
- * ignored when resid_mode is NONE), out: [T, d_model].  logits_out [T, n], topk_idx_out [T, k]
- * and topk_w_out [T, k] are optional copies of the routing. */
+/* Residual update of the decoder layer's FFN sub-block [MUSE "The complete layer has two
+ * separately normalized residual updates", "Residual gates"]: for each row,
+ *   n = b, or with gamma_post (cfg->post_norm) the input-scaled output norm
+ *   n = dtype(s / sqrt(mean(s^2) + eps_block)), s = dtype((1 + gamma_post) * b);
+ *   out = dtype(alpha*r + beta*n) (MUSE_GATE), dtype(r + g*n) (LITERAL) or n (NONE).
+ * b, r, out: [T, d_model] bf16; gamma_post, resid_g: [d_model] fp32.  bf16 only. */
+MOE_API moe_status_t moe_residual_update(const moe_config_t* cfg, const void* b, const void* r,
+                                         const float* gamma_post, const float* resid_g, void* out,
+                                         void* stream);
+
+/* The whole layer: [input norm] -> route -> latent down (+C_pre) -> dispatch -> experts
+ * (+I_gamma prep) -> normalise and combine -> latent up -> [output norm] -> residual update.
+ * u: [T, d_model] is the branch input (router and down-projection read it; with input_norm it
+ * is computed from r and this argument may be NULL), r: [T, d_model] the residual stream (may
+ * equal u; ignored when resid_mode is NONE and input_norm is off), out: [T, d_model].
+ * logits_out [T, n], topk_idx_out [T, k] and topk_w_out [T, k] are optional copies of the
+ * routing. */
 MOE_API moe_status_t moe_layer_forward(const moe_config_t* cfg, const moe_weights_t* w, const void* u,
                                const void* r, void* out, float* logits_out,
                                int32_t* topk_idx_out, float* topk_w_out, void* workspace,

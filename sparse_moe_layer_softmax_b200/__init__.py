@@ -29,7 +29,7 @@ EXPORTS = ("moe_status_string", "moe_workspace_size", "moe_route", "moe_permute"
            "moe_expert_ffn", "moe_combine", "moe_latent_down", "moe_latent_up",
            "moe_layer_forward", "moe_get_device_status", "moe_profile_begin", "moe_profile_end",
            "moe_launch_count", "moe_permute_static", "moe_selftest_wait_timeout",
-           "moe_router_split_weights")
+           "moe_router_split_weights", "moe_residual_update")
 PROFILE_STAGES = ("route", "latent_down", "dispatch", "expert_gate_up", "expert_down", "combine",
                   "latent_up_resgate")
 
@@ -47,14 +47,16 @@ class Config(ctypes.Structure):
                                               "expert_norm", "resid_mode")] + \
                [(n, ctypes.c_float) for n in ("eps", "tau", "resid_floor", "routed_scale")] + \
                [("gate_mode", ctypes.c_int32), ("router_f32", ctypes.c_int32),
-                ("logit_mult", ctypes.c_float)]
+                ("logit_mult", ctypes.c_float), ("input_norm", ctypes.c_int32),
+                ("post_norm", ctypes.c_int32), ("eps_block", ctypes.c_float)]
 
 
 class Weights(ctypes.Structure):
     """moe_weights_t"""
     _fields_ = [(n, ctypes.c_void_p) for n in ("w_router", "p_down", "p_up", "w_gu", "w_down",
                                                "gamma_pre", "gamma_expert", "resid_g",
-                                               "logit_bias", "correction_bias")]
+                                               "logit_bias", "correction_bias", "gamma_in",
+                                               "gamma_post")]
 
 
 _lib = None
@@ -76,6 +78,7 @@ def lib():
             "moe_workspace_size": [cp, ctypes.POINTER(sz)],
             "moe_route": [cp, vp, vp, vp, vp, vp, vp, vp, vp],
             "moe_router_split_weights": [vp, ctypes.c_int32, ctypes.c_int32, vp, vp],
+            "moe_residual_update": [cp, vp, vp, vp, vp, vp, vp],
             "moe_permute": [cp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp],
             "moe_expert_ffn": [cp, vp, vp, vp, vp, vp, vp, vp, sz, vp],
             "moe_combine": [cp, vp, vp, vp, vp, vp],
@@ -101,12 +104,14 @@ def lib():
 def make_config(T, d_model, n_experts, top_k, d_ff, d_latent=0, dtype=MOE_BF16,
                 expert_act=MOE_ACT_SWIGLU, pre_norm=0, expert_norm=0, resid_mode=MOE_RESID_NONE,
                 eps=1e-6, tau=0.3, resid_floor=1e-3, routed_scale=1.0, gate_mode=MOE_GATE_SOFTMAX,
-                router_f32=0, logit_mult=1.0) -> Config:
+                router_f32=0, logit_mult=1.0, input_norm=0, post_norm=0,
+                eps_block=1e-5) -> Config:
     return Config(T=T, d_model=d_model, d_latent=d_latent, d_ff=d_ff, n_experts=n_experts,
                   top_k=top_k, dtype=dtype, expert_act=expert_act, pre_norm=pre_norm,
                   expert_norm=expert_norm, resid_mode=resid_mode, eps=eps, tau=tau,
                   resid_floor=resid_floor, routed_scale=routed_scale, gate_mode=gate_mode,
-                  router_f32=router_f32, logit_mult=logit_mult)
+                  router_f32=router_f32, logit_mult=logit_mult, input_norm=input_norm,
+                  post_norm=post_norm, eps_block=eps_block)
 
 
 def _ptr(t) -> int | None:
@@ -140,6 +145,12 @@ def moe_route(cfg, u, w_router, logit_bias, logits_out, topk_idx, topk_w, stream
     _check("moe_route", lib().moe_route(ctypes.byref(cfg), _ptr(u), _ptr(w_router),
                                         _ptr(logit_bias), _ptr(correction_bias), _ptr(logits_out),
                                         _ptr(topk_idx), _ptr(topk_w), _stream(stream)))
+
+
+def moe_residual_update(cfg, b, r, gamma_post, resid_g, out, stream=None):
+    _check("moe_residual_update", lib().moe_residual_update(
+        ctypes.byref(cfg), _ptr(b), _ptr(r), _ptr(gamma_post), _ptr(resid_g), _ptr(out),
+        _stream(stream)))
 
 
 def moe_router_split_weights(w, w_split, stream=None):

@@ -433,6 +433,100 @@ __global__ void router_split_kernel(const float* __restrict__ w, size_t count, i
   }
 }
 
+// ------------------------------------------------------------------ decoder-level row kernels
+//
+// One CTA per row of width D (VEC 16-byte vectors per thread, D <= 256*8*VEC).
+
+// Centred RMSNorm of a row: out = dtype((1 + gamma) * x / sqrt(mean(x^2) + eps)).
+template <int VEC>
+__global__ void rownorm_centered_bf16_kernel(const uint16_t* __restrict__ x, int D,
+                                             const float* __restrict__ gamma, float eps,
+                                             uint16_t* __restrict__ out) {
+  __shared__ float red[8];
+  const size_t base = static_cast<size_t>(blockIdx.x) * D;
+  const int nvec = D / 8;
+  uint4 r[VEC];
+  float ss = 0.0f;
+#pragma unroll
+  for (int v = 0; v < VEC; ++v) {
+    const int vi = threadIdx.x + v * blockDim.x;
+    r[v] = vi < nvec ? reinterpret_cast<const uint4*>(x + base)[vi] : make_uint4(0, 0, 0, 0);
+    const uint16_t* h = reinterpret_cast<const uint16_t*>(&r[v]);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) { const float f = bf16_to_f32(h[i]); ss += f * f; }
+  }
+  const float rinv = rsqrtf(block_sum_256(ss, red) / static_cast<float>(D) + eps);
+#pragma unroll
+  for (int v = 0; v < VEC; ++v) {
+    const int vi = threadIdx.x + v * blockDim.x;
+    if (vi >= nvec) continue;
+    const uint16_t* h = reinterpret_cast<const uint16_t*>(&r[v]);
+    uint32_t pk[4];
+#pragma unroll
+    for (int i = 0; i < 8; i += 2)
+      pk[i / 2] = pack_bf16x2((1.0f + gamma[8 * vi + i]) * (bf16_to_f32(h[i]) * rinv),
+                              (1.0f + gamma[8 * vi + i + 1]) * (bf16_to_f32(h[i + 1]) * rinv));
+    reinterpret_cast<uint4*>(out + base)[vi] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+  }
+}
+
+// Residual update of a row with an optional input-scaled output norm:
+//   n = b, or with gamma_post: s = dtype((1 + gamma_post) * b), n = dtype(s / sqrt(mean(s^2) + eps));
+//   out = dtype(alpha * r + beta * n), alpha/beta of the residual gate (MUSE gate), r + g * n
+//   (literal) or n (none).
+template <int VEC>
+__global__ void resid_update_bf16_kernel(const uint16_t* __restrict__ b, const uint16_t* __restrict__ r,
+                                         int D, const float* __restrict__ gamma_post, float eps,
+                                         const float* __restrict__ g, int resid_mode, float tau,
+                                         float floor_, uint16_t* __restrict__ out) {
+  __shared__ float red[8];
+  const size_t base = static_cast<size_t>(blockIdx.x) * D;
+  const int nvec = D / 8;
+  float nv[VEC][8];
+  float ss = 0.0f;
+#pragma unroll
+  for (int v = 0; v < VEC; ++v) {
+    const int vi = threadIdx.x + v * blockDim.x;
+    const uint4 q = vi < nvec ? reinterpret_cast<const uint4*>(b + base)[vi] : make_uint4(0, 0, 0, 0);
+    const uint16_t* h = reinterpret_cast<const uint16_t*>(&q);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      float s = bf16_to_f32(h[i]);
+      if (gamma_post && vi < nvec) s = round_bf16(s * (1.0f + gamma_post[8 * vi + i]));
+      nv[v][i] = s;
+      ss += s * s;
+    }
+  }
+  float rinv = 1.0f;
+  if (gamma_post) rinv = rsqrtf(block_sum_256(ss, red) / static_cast<float>(D) + eps);
+#pragma unroll
+  for (int v = 0; v < VEC; ++v) {
+    const int vi = threadIdx.x + v * blockDim.x;
+    if (vi >= nvec) continue;
+    uint4 rq = make_uint4(0, 0, 0, 0);
+    if (resid_mode != MOE_RESID_NONE) rq = reinterpret_cast<const uint4*>(r + base)[vi];
+    const uint16_t* rh = reinterpret_cast<const uint16_t*>(&rq);
+    float o[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float n = gamma_post ? round_bf16(nv[v][i] * rinv) : nv[v][i];
+      const int col = 8 * vi + i;
+      if (resid_mode == MOE_RESID_MUSE_GATE) {
+        const float beta = sigmoidf_(g[col] / tau);
+        const float alpha = sqrtf(fmaxf(sigmoidf_(-g[col] / tau) * (1.0f + beta), floor_));
+        o[i] = alpha * bf16_to_f32(rh[i]) + beta * n;
+      } else if (resid_mode == MOE_RESID_LITERAL) {
+        o[i] = bf16_to_f32(rh[i]) + g[col] * n;
+      } else {
+        o[i] = n;
+      }
+    }
+    reinterpret_cast<uint4*>(out + base)[vi] =
+        make_uint4(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]), pack_bf16x2(o[4], o[5]),
+                   pack_bf16x2(o[6], o[7]));
+  }
+}
+
 // ------------------------------------------------------------------ failure-detection self-test
 //
 // One thread initialises an mbarrier that expects one arrival which never comes and waits on

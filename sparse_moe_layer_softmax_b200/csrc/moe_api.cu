@@ -200,6 +200,13 @@ moe_status_t check_cfg(const moe_config_t* c) {
   if (c->gate_mode != MOE_GATE_SOFTMAX && c->gate_mode != MOE_GATE_SIGMOID) return MOE_ERR_UNSUPPORTED;
   if (c->router_f32 != 0 && c->router_f32 != 1) return MOE_ERR_INVALID_ARG;
   if (c->gate_mode == MOE_GATE_SIGMOID && !(c->logit_mult == c->logit_mult)) return MOE_ERR_INVALID_ARG;
+  if ((c->input_norm != 0 && c->input_norm != 1) || (c->post_norm != 0 && c->post_norm != 1))
+    return MOE_ERR_INVALID_ARG;
+  if ((c->input_norm || c->post_norm) && !(c->eps_block >= 0.0f)) return MOE_ERR_INVALID_ARG;
+  if ((c->input_norm || c->post_norm) && c->dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
+  if (c->post_norm && c->d_latent == 0) return MOE_ERR_UNSUPPORTED;
+  if (c->input_norm && c->d_model > 8192) return MOE_ERR_UNSUPPORTED;  // row kernels
+  if (c->post_norm && c->d_model > 8192) return MOE_ERR_UNSUPPORTED;
   if (!(c->eps >= 0.0f) || !(c->tau > 0.0f) || !(c->resid_floor >= 0.0f)) return MOE_ERR_INVALID_ARG;
   if (static_cast<long>(c->T) * c->top_k > 0x7fffffffL / 2) return MOE_ERR_UNSUPPORTED;
   if (c->dtype == MOE_BF16) {
@@ -217,7 +224,7 @@ size_t dsize(const moe_config_t& c) { return c.dtype == MOE_BF16 ? 2 : 4; }
 int nchunks(const moe_config_t& c) { return cdiv(c.T, kPermChunk); }
 
 struct Workspace {
-  size_t idx, w, logits, z_raw, offsets, perm, inv, counts, x_perm, act, y, total;
+  size_t idx, w, logits, z_raw, offsets, perm, inv, counts, x_perm, act, y, u_norm, b, total;
 };
 
 Workspace layout(const moe_config_t& c) {
@@ -236,6 +243,8 @@ Workspace layout(const moe_config_t& c) {
   L.x_perm = take(TK * E * ds);
   L.act = take(TK * c.d_ff * ds);
   L.y = take(c.d_latent > 0 ? static_cast<size_t>(c.T) * E * ds : 0);
+  L.u_norm = take(c.input_norm ? static_cast<size_t>(c.T) * c.d_model * ds : 0);
+  L.b = take(c.post_norm ? static_cast<size_t>(c.T) * c.d_model * ds : 0);
   L.total = o;
   return L;
 }
@@ -495,6 +504,49 @@ moe_status_t do_latent_up(const moe_config_t& c, const void* y, const void* p_up
                   c.d_model, p, st);
 }
 
+// Launch shape of the one-CTA-per-row kernels for a row of D bf16 values.
+bool row_launch(int D, int* threads, int* vec) {
+  const int nvec = D / 8;
+  *threads = nvec >= 256 ? 256 : ((nvec + 31) / 32) * 32;
+  *vec = cdiv(nvec, *threads);
+  if (*vec == 3) *vec = 4;
+  return *vec <= 4;
+}
+
+moe_status_t do_input_norm(const moe_config_t& c, const void* r, const float* gamma_in, void* u,
+                           cudaStream_t st) {
+  if (c.T == 0) return MOE_OK;
+  int threads, vec;
+  if (!row_launch(c.d_model, &threads, &vec)) return MOE_ERR_UNSUPPORTED;
+  const uint16_t* x = static_cast<const uint16_t*>(r);
+  uint16_t* o = static_cast<uint16_t*>(u);
+  switch (vec) {
+    case 1: rownorm_centered_bf16_kernel<1><<<c.T, threads, 0, st>>>(x, c.d_model, gamma_in, c.eps_block, o); break;
+    case 2: rownorm_centered_bf16_kernel<2><<<c.T, threads, 0, st>>>(x, c.d_model, gamma_in, c.eps_block, o); break;
+    default: rownorm_centered_bf16_kernel<4><<<c.T, threads, 0, st>>>(x, c.d_model, gamma_in, c.eps_block, o); break;
+  }
+  return last_launch();
+}
+
+moe_status_t do_resid_update(const moe_config_t& c, const void* b, const void* r,
+                             const float* gamma_post, const float* g, void* out, cudaStream_t st) {
+  if (c.T == 0) return MOE_OK;
+  int threads, vec;
+  if (!row_launch(c.d_model, &threads, &vec)) return MOE_ERR_UNSUPPORTED;
+  const uint16_t* bp = static_cast<const uint16_t*>(b);
+  const uint16_t* rp = static_cast<const uint16_t*>(r);
+  uint16_t* o = static_cast<uint16_t*>(out);
+#define RU(V) resid_update_bf16_kernel<V><<<c.T, threads, 0, st>>>(bp, rp, c.d_model, gamma_post, \
+      c.eps_block, g, c.resid_mode, c.tau, c.resid_floor, o)
+  switch (vec) {
+    case 1: RU(1); break;
+    case 2: RU(2); break;
+    default: RU(4); break;
+  }
+#undef RU
+  return last_launch();
+}
+
 }  // namespace
 }  // namespace moe
 
@@ -685,7 +737,10 @@ moe_status_t moe_layer_forward(const moe_config_t* cfg, const moe_weights_t* w, 
   if (!w) return MOE_ERR_INVALID_ARG;
   if (c.T == 0) return MOE_OK;
   const bool latent = c.d_latent > 0;
-  if (!u || !out || !w->w_router || !w->w_gu || !w->w_down) return MOE_ERR_INVALID_ARG;
+  if ((!u && !c.input_norm) || !out || !w->w_router || !w->w_gu || !w->w_down)
+    return MOE_ERR_INVALID_ARG;
+  if (c.input_norm && (!r || !w->gamma_in)) return MOE_ERR_INVALID_ARG;
+  if (c.post_norm && !w->gamma_post) return MOE_ERR_INVALID_ARG;
   if (latent && (!w->p_down || !w->p_up)) return MOE_ERR_INVALID_ARG;
   if (c.pre_norm && !w->gamma_pre) return MOE_ERR_INVALID_ARG;
   if (c.expert_norm && !w->gamma_expert) return MOE_ERR_INVALID_ARG;
@@ -696,7 +751,9 @@ moe_status_t moe_layer_forward(const moe_config_t* cfg, const moe_weights_t* w, 
                         static_cast<const void*>(w->gamma_pre),
                         static_cast<const void*>(w->gamma_expert),
                         static_cast<const void*>(w->resid_g), static_cast<const void*>(w->logit_bias),
-                        static_cast<const void*>(w->correction_bias)})) return MOE_ERR_ALIGNMENT;
+                        static_cast<const void*>(w->correction_bias),
+                        static_cast<const void*>(w->gamma_in),
+                        static_cast<const void*>(w->gamma_post)})) return MOE_ERR_ALIGNMENT;
   const Workspace L = layout(c);
   if (!workspace || workspace_bytes < L.total) return MOE_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -709,6 +766,11 @@ moe_status_t moe_layer_forward(const moe_config_t* cfg, const moe_weights_t* w, 
   void* act = at<void>(workspace, L.act);
 
   prof_mark(st, 0);
+  if (c.input_norm) {  // the branch input is the residual stream's norm (counted in stage 0)
+    void* un = at<void>(workspace, L.u_norm);
+    if ((s = do_input_norm(c, r, w->gamma_in, un, st)) != MOE_OK) return s;
+    u = un;
+  }
   if ((s = do_route(c, u, w->w_router, w->logit_bias, w->correction_bias, logits_out, idx, wt, st,
                     at<float>(workspace, L.logits))) != MOE_OK)
     return s;
@@ -733,10 +795,33 @@ moe_status_t moe_layer_forward(const moe_config_t* cfg, const moe_weights_t* w, 
   void* y = latent ? at<void>(workspace, L.y) : out;
   if ((s = do_combine(c, x_perm, inv, wt, y, st)) != MOE_OK) return s;
   prof_mark(st, 6);
-  if (latent && (s = do_latent_up(c, y, w->p_up, r, w->resid_g, out, st)) != MOE_OK) return s;
+  if (latent && !c.post_norm &&
+      (s = do_latent_up(c, y, w->p_up, r, w->resid_g, out, st)) != MOE_OK)
+    return s;
+  if (c.post_norm) {  // b to the workspace, then output norm + residual gate per row
+    moe_config_t plain = c;
+    plain.resid_mode = MOE_RESID_NONE;
+    void* b = at<void>(workspace, L.b);
+    if ((s = do_latent_up(plain, y, w->p_up, nullptr, nullptr, b, st)) != MOE_OK) return s;
+    if ((s = do_resid_update(c, b, r, w->gamma_post, w->resid_g, out, st)) != MOE_OK) return s;
+  }
   prof_mark(st, 7);
   prof_next_call();
   return MOE_OK;
+}
+
+moe_status_t moe_residual_update(const moe_config_t* cfg, const void* b, const void* r,
+                                 const float* gamma_post, const float* resid_g, void* out,
+                                 void* stream) {
+  moe_status_t s = check_cfg(cfg);
+  if (s != MOE_OK) return s;
+  if (cfg->dtype != MOE_BF16 || cfg->d_model > 8192) return MOE_ERR_UNSUPPORTED;
+  if (cfg->T > 0 && (!b || !out)) return MOE_ERR_INVALID_ARG;
+  if (cfg->T > 0 && cfg->resid_mode != MOE_RESID_NONE && (!r || !resid_g)) return MOE_ERR_INVALID_ARG;
+  if (!all_aligned({b, r, static_cast<const void*>(gamma_post), static_cast<const void*>(resid_g),
+                    static_cast<const void*>(out)}))
+    return MOE_ERR_ALIGNMENT;
+  return do_resid_update(*cfg, b, r, gamma_post, resid_g, out, static_cast<cudaStream_t>(stream));
 }
 
 unsigned long long moe_launch_count(void) { return g_launches.load(); }

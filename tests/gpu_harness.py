@@ -23,7 +23,8 @@ def abi_config(cfg, T: int | None = None):
         dtype=moe.MOE_BF16 if cfg.dtype == "bf16" else moe.MOE_F32, expert_act=cfg.act,
         pre_norm=cfg.pre_norm, expert_norm=cfg.expert_norm, resid_mode=cfg.resid_mode,
         eps=cfg.eps, tau=cfg.tau, resid_floor=cfg.resid_floor, routed_scale=cfg.routed_scale,
-        gate_mode=cfg.gate_mode, router_f32=cfg.router_f32, logit_mult=cfg.logit_mult)
+        gate_mode=cfg.gate_mode, router_f32=cfg.router_f32, logit_mult=cfg.logit_mult,
+        input_norm=cfg.input_norm, post_norm=cfg.post_norm, eps_block=cfg.eps_block)
 
 
 def host_values(a: np.ndarray, dtype: str) -> np.ndarray:
@@ -59,7 +60,14 @@ def logit_atol(cfg, logits: np.ndarray) -> float:
     the output multiplier, so the same bound scaled by the multiplier covers them."""
     K = cfg.d_model * (3 if cfg.router_f32 and cfg.dtype == "bf16" else 1)
     mult = max(1.0, abs(cfg.logit_mult)) if cfg.gate_mode == configs.GATE_SIGMOID else 1.0
-    return 16.0 * np.sqrt(K) * 2.0 ** -24 * mult * max(1.0, float(np.abs(logits).max()))
+    tol = 16.0 * np.sqrt(K) * 2.0 ** -24 * mult * max(1.0, float(np.abs(logits).max()))
+    if cfg.input_norm:
+        # the router input is itself a bf16-rounded norm: fp32 (GPU) and double (oracle) may
+        # round an element of u to neighbouring bf16 values; allow two such flips per row, each
+        # moving the logit by at most |w|max * ulp(|u|max) with |u| < 6 (unit-RMS rows) and
+        # |w| <= 4.9 sigma (the generator's Irwin-Hall bound)
+        tol += mult * 2 * (6.0 * 2.0 ** -7) * 4.9 * cfg.sigma_router()
+    return tol
 
 
 def run_layer(cfg, dev: dict, want_logits: bool = True):

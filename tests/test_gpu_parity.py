@@ -83,6 +83,12 @@ SMALL = [
                        gate_mode=configs.GATE_SIGMOID, corr_sigma=0.2),
     configs.TINY_SHAZEER_F32.replace(T=50, seed=24, gate_mode=configs.GATE_SIGMOID,
                                      logit_mult=0.5, router_gain=1.0),
+    # decoder wrap: residual-stream norm in, FFN output norm before the residual gate
+    configs.small_muse(T=300, d=512, L=256, I=256, n=16, k=4, seed=28, input_norm=1, post_norm=1,
+                       gamma_sigma=0.2),
+    configs.small_muse(T=40, d=256, L=128, I=128, n=64, k=8, seed=29, input_norm=1, post_norm=1,
+                       resid_mode=configs.RESID_LITERAL),
+    configs.small_muse(T=70, d=8192, L=128, I=128, n=8, k=2, seed=30, input_norm=1, post_norm=0),
 ]
 
 
