@@ -270,6 +270,35 @@ def sigmoid_topk_scores_f32(scores: np.ndarray, k: int, correction_bias=None,
     return idx, w
 
 
+def noisy_gate(l: np.ndarray, m: np.ndarray, eps: np.ndarray, k: int):
+    """Noisy top-k gate per row of [rows, n] clean logits l, noise logits m and draws eps:
+    returns H, G (dense), P (smooth load probabilities) and idx [rows, k]."""
+    L = lib()
+    if not hasattr(L, "_noisy_sig"):
+        L.orc_noisy_gate_token.argtypes = [ctypes.c_void_p] * 3 + [ctypes.c_int] * 2 + \
+            [ctypes.c_void_p] * 4
+        L.orc_noisy_gate_token.restype = None
+        L.orc_cv_squared.argtypes = [ctypes.c_void_p, ctypes.c_int]
+        L.orc_cv_squared.restype = ctypes.c_double
+        L._noisy_sig = True
+    rows, n = l.shape
+    l = np.ascontiguousarray(l, np.float64)
+    m = np.ascontiguousarray(m, np.float64)
+    eps = np.ascontiguousarray(eps, np.float64)
+    H, G, P = np.zeros_like(l), np.zeros_like(l), np.zeros_like(l)
+    idx = np.zeros((rows, k), dtype=np.int32)
+    for r in range(rows):
+        L.orc_noisy_gate_token(_p(l[r]), _p(m[r]), _p(eps[r]), n, k, _p(H[r]), _p(G[r]), _p(P[r]),
+                               _p(idx[r]))
+    return H, G, P, idx
+
+
+def cv_squared(v) -> float:
+    noisy_gate(np.zeros((1, 2)), np.zeros((1, 2)), np.zeros((1, 2)), 1)  # binds the signatures
+    v = np.ascontiguousarray(v, np.float64)
+    return float(lib().orc_cv_squared(_p(v), v.size))
+
+
 def rms_normalize(x, eps=0.0):
     x = np.ascontiguousarray(x, np.float64)
     out = np.zeros_like(x)

@@ -462,6 +462,58 @@ void orc_expert_batch(const orc_cfg* c, const void* w_gu_e, const void* w_down_e
   free(jobs);
 }
 
+/* ------------------------------------------------------------------ noisy gate statistics */
+
+static double softplus(double z) { return z > 30.0 ? z : log1p(exp(z)); }
+static double std_normal_cdf(double z) { return 0.5 * erfc(-z / sqrt(2.0)); }
+
+void orc_noisy_gate_token(const double* l, const double* m, const double* eps, int n, int k,
+                          double* H, double* G, double* P, int* idx) {
+  char* taken = (char*)calloc((size_t)n, 1);
+  for (int i = 0; i < n; ++i) {
+    H[i] = l[i] + eps[i] * softplus(m[i]);
+    G[i] = 0.0;
+  }
+  /* KeepTopK: the k largest H (ties to the lower index), then a softmax over them */
+  for (int j = 0; j < k; ++j) {
+    int best = -1;
+    for (int e = 0; e < n; ++e)
+      if (!taken[e] && (best < 0 || H[e] > H[best])) best = e;
+    taken[best] = 1;
+    idx[j] = best;
+  }
+  double mx = H[idx[0]], z = 0.0;
+  for (int j = 0; j < k; ++j) z += exp(H[idx[j]] - mx);
+  for (int j = 0; j < k; ++j) G[idx[j]] = exp(H[idx[j]] - mx) / z;
+  /* kth_excluding(H, k, i): the k-th largest H among the experts other than i */
+  for (int i = 0; i < n; ++i) {
+    int rank = 0; /* how many of the others have been taken so far in descending order */
+    double kth = 0.0;
+    char* used = (char*)calloc((size_t)n, 1);
+    used[i] = 1;
+    while (rank < k) {
+      int best = -1;
+      for (int e = 0; e < n; ++e)
+        if (!used[e] && (best < 0 || H[e] > H[best])) best = e;
+      used[best] = 1;
+      kth = H[best];
+      ++rank;
+    }
+    free(used);
+    P[i] = std_normal_cdf((l[i] - kth) / softplus(m[i]));
+  }
+  free(taken);
+}
+
+double orc_cv_squared(const double* v, int n) {
+  double mean = 0.0, var = 0.0;
+  for (int i = 0; i < n; ++i) mean += v[i];
+  mean /= n;
+  for (int i = 0; i < n; ++i) var += (v[i] - mean) * (v[i] - mean);
+  var /= n;
+  return var / (mean * mean);
+}
+
 /* ------------------------------------------------------------------ permutation */
 
 /* Dispatch "tokens to selected experts" [MUSE "Latent experts"] in the canonical order: count

@@ -120,6 +120,18 @@ void orc_expert_batch(const orc_cfg* c, const void* w_gu_e, const void* w_down_e
                       const float* gamma_expert, const double* z_rows, int nrows, double* n_rows,
                       int nthreads);
 
+/* Shazeer et al.'s noisy top-k gate and its balancing statistics [SHAZEER "The gate", "Keeping the
+ * experts busy"], for one token from its clean logits l = x W_g, noise logits m = x W_noise and
+ * the standard-normal draw eps (all [n]):
+ *   H_i = l_i + eps_i * softplus(m_i);  G = Softmax(KeepTopK(H, k)) (dense [n], zeros off the
+ *   top k; selection by H desc, ties to the lower index; idx gets the k selected in order);
+ *   P_i = Phi((l_i - kth_excluding(H, k, i)) / softplus(m_i)), kth_excluding(H, k, i) being the
+ *   k-th largest of H over the experts other than i. */
+void orc_noisy_gate_token(const double* l, const double* m, const double* eps, int n, int k,
+                          double* H, double* G, double* P, int* idx);
+/* CV(v)^2 = population variance / mean^2 of v[n]. */
+double orc_cv_squared(const double* v, int n);
+
 /* Canonical permutation of routed slots: rows grouped by expert ascending, and within an expert
  * by token ascending.  offsets[n+1], perm_token[T*k] (row -> token), inv_perm[T*k]
  * (slot t*k+j -> row).  Returns 0, or -1 if an index is out of range or repeated in a token. */

@@ -316,6 +316,62 @@ BRUTE_CASES = [
 ]
 
 
+def test_noisy_gate_chart_values():
+    g = gold("noisy_gate_chart.json")
+    # expert 0 has noise pre-activation 0; the bar it must clear is max(H_1, H_2) = 1 (k = 1)
+    sp = math.log(2.0)
+    assert round(sp, 3) == g["softplus_3dp"]
+
+    def p0(l0):
+        l = np.array([[l0, 1.0, -5.0]])
+        _, _, P, _ = oracle.noisy_gate(l, np.zeros((1, 3)), np.zeros((1, 3)), 1)
+        return P[0, 0]
+
+    assert round(100 * p0(0.0), 2) == g["p_one_unit_below_bar_pct_2dp"]   # one unit below
+    h = 1e-5
+    slope = (p0(1.0 + h) - p0(1.0 - h)) / (2 * h)
+    assert round(slope, 3) == g["slope_at_bar_3dp"]
+    assert p0(1.0) == pytest.approx(0.5, abs=1e-15)                    # at the bar
+
+
+def test_noisy_gate_cv_example():
+    g = gold("noisy_gate_chart.json")
+    v = np.array(g["importance_example"], dtype=np.float64)
+    cv2 = oracle.cv_squared(v)
+    assert cv2 == pytest.approx(g["population_variance"] / g["mean"] ** 2, rel=1e-15)
+    assert round(math.sqrt(cv2), 2) == g["cv_2dp"] and round(cv2, 2) == g["cv_squared_2dp"]
+    assert round(g["w_importance"] * cv2, 3) == g["loss_3dp"]
+    assert oracle.cv_squared(np.full(4, 25.0)) == 0.0
+
+
+def test_noisy_gate_against_library_routines():
+    from scipy.stats import norm
+    rng = np.random.default_rng(8)
+    rows, n, k = 30, 12, 3
+    l, m, eps = rng.normal(size=(rows, n)), rng.normal(size=(rows, n)), rng.normal(size=(rows, n))
+    H, G, P, idx = oracle.noisy_gate(l, m, eps, k)
+    sp = np.log1p(np.exp(m))
+    np.testing.assert_allclose(H, l + eps * sp, rtol=1e-14)
+    for r in range(rows):
+        top = np.argsort(-H[r], kind="stable")[:k]
+        assert idx[r].tolist() == top.tolist()
+        e = np.exp(H[r, top] - H[r, top].max())
+        dense = np.zeros(n)
+        dense[top] = e / e.sum()
+        np.testing.assert_allclose(G[r], dense, rtol=1e-13, atol=1e-300)
+        for i in range(n):
+            kth = np.sort(np.delete(H[r], i))[::-1][k - 1]
+            assert P[r, i] == pytest.approx(norm.cdf((l[r, i] - kth) / sp[r, i]), rel=1e-12, abs=1e-300)
+    # without noise the gate is the plain softmax top-k, and P approaches the hard top-k
+    _, G0, P0, idx0 = oracle.noisy_gate(l, np.full((rows, n), -60.0), np.zeros((rows, n)), k)
+    sel, w = oracle.softmax_topk(l, k)
+    np.testing.assert_array_equal(idx0, sel)
+    np.testing.assert_allclose(np.take_along_axis(G0, sel.astype(np.int64), 1), w, rtol=1e-13)
+    hard = np.zeros_like(P0)
+    np.put_along_axis(hard, sel.astype(np.int64), 1.0, 1)
+    np.testing.assert_allclose(P0, hard, atol=1e-12)
+
+
 def test_post_norm_output_has_unit_rms():
     """With post_norm, no residual and gamma_post = 0, every output row is R(b): unit RMS."""
     cfg = configs.small_muse(T=9, d=48, L=32, I=24, n=6, k=2, dtype="f32", post_norm=1,
