@@ -219,6 +219,27 @@ MOE_API moe_status_t moe_residual_update(const moe_config_t* cfg, const void* b,
                                          const float* gamma_post, const float* resid_g, void* out,
                                          void* stream);
 
+/* Shazeer et al.'s noisy top-k gate and its balancing statistics [SHAZEER "The gate", "Keeping the
+ * experts busy"] for a batch of T tokens u [T, d_model]:
+ *   l = u W_router^T, m = u W_noise^T (fp32 accumulation; W_noise [n, d_model] in the router's
+ *   format), H = l + eps * softplus(m) with the standard-normal draws noise_eps [T, n] (fp32,
+ *   supplied by the caller);
+ *   G = Softmax(KeepTopK(H, k)): topk_idx [T, k] (ties to the lower index, descending) and
+ *   topk_w [T, k];
+ *   P_i = Phi((l_i - kth_excluding(H, k, i)) / softplus(m_i)) (optional copy load_prob_out
+ *   [T, n]); importance[n] = sum_t G, load[n] = sum_t P (fp32, deterministic order), cv2[0] =
+ *   CV(importance)^2 and cv2[1] = CV(load)^2 with the population variance.
+ * noisy_logits_out [T, n] (H) and load_prob_out may be NULL.  Needs top_k < n_experts and T > 0;
+ * workspace of moe_noisy_gate_workspace_size bytes.  cfg->gate_mode is ignored (the two logit
+ * passes are plain logits); logit_bias does not apply. */
+MOE_API moe_status_t moe_noisy_gate_workspace_size(const moe_config_t* cfg, size_t* bytes);
+MOE_API moe_status_t moe_noisy_gate(const moe_config_t* cfg, const void* u, const void* w_router,
+                                    const void* w_noise, const float* noise_eps,
+                                    float* noisy_logits_out, int32_t* topk_idx, float* topk_w,
+                                    float* load_prob_out, float* importance, float* load,
+                                    float* cv2, void* workspace, size_t workspace_bytes,
+                                    void* stream);
+
 /* The whole layer: [input norm] -> route -> latent down (+C_pre) -> dispatch -> experts
  * (+I_gamma prep) -> normalise and combine -> latent up -> [output norm] -> residual update.
  * u: [T, d_model] is the branch input (router and down-projection read it; with input_norm it

@@ -180,6 +180,10 @@ def tensor_specs(cfg: MoEConfig):
                                  cfg.gamma_sigma)
     if cfg.gate_mode == configs.GATE_SIGMOID:
         specs["correction_bias"] = ((n,), configs.STREAM_CORR_BIAS, "f32n", cfg.corr_sigma)
+    if cfg.noisy_gate:
+        specs["w_noise"] = ((n, d), configs.STREAM_W_NOISE, "f32n" if cfg.router_f32 else "w",
+                            cfg.sigma_router())
+        specs["noise_eps"] = ((cfg.T, n), configs.STREAM_NOISE_EPS, "f32n", 1.0)
     if cfg.input_norm:
         specs["gamma_in"] = ((d,), configs.STREAM_GAMMA_IN, "f32n", cfg.gamma_sigma)
     if cfg.post_norm:

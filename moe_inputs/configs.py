@@ -48,6 +48,8 @@ GATE_SIGMOID = 1
 STREAM_CORR_BIAS = 13
 STREAM_GAMMA_IN = 14
 STREAM_GAMMA_POST = 15
+STREAM_W_NOISE = 16
+STREAM_NOISE_EPS = 17
 
 # Scale c of the Zipf router bias  bias_e = -c * s * ln(rank_e)  (s = 1.2) for the imbalanced
 # workload.  Calibrated by tests/golden/calibrate_zipf_bias.py, which bisects c with the CPU
@@ -88,6 +90,7 @@ class MoEConfig:
     input_norm: int = 0         # decoder wrap: u = C_in(h), centred RMSNorm of the residual stream
     post_norm: int = 0          # decoder wrap: input-scaled output norm I_post on b before the gate
     eps_block: float = 1e-5     # epsilon of the decoder-level norms (model sheet: 1e-5)
+    noisy_gate: bool = False    # Shazeer's noisy gate: W_noise ~ N(0, router std^2), eps ~ N(0, 1)
 
     @property
     def latent(self) -> bool:
@@ -167,6 +170,11 @@ MUSE_PREFILL_BLOCK = MUSE_PREFILL.replace(name="muse_prefill_block", input_norm=
                                           seed=11)
 VARIANT_CONFIGS = {c.name: c for c in (MUSE_DECODE_SIGMOID, MUSE_PREFILL_SIGMOID,
                                        MUSE_DECODE_BLOCK, MUSE_PREFILL_BLOCK)}
+
+# Shazeer et al.'s noisy gate statistics on the Shazeer-shaped batch (training-time diagnostics
+# computed forward: noisy logits, KeepTopK gate, importance and smooth load with their CV^2).
+SHAZEER_BF16_NOISY = SHAZEER_BF16.replace(name="shazeer_bf16_noisy", noisy_gate=True, seed=12)
+GATE_STAT_CONFIGS = {c.name: c for c in (SHAZEER_BF16_NOISY,)}
 ALL_CONFIGS = {**CONFIGS, **PROFILE_CONFIGS, **VARIANT_CONFIGS}
 
 

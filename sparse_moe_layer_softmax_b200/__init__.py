@@ -29,7 +29,8 @@ EXPORTS = ("moe_status_string", "moe_workspace_size", "moe_route", "moe_permute"
            "moe_expert_ffn", "moe_combine", "moe_latent_down", "moe_latent_up",
            "moe_layer_forward", "moe_get_device_status", "moe_profile_begin", "moe_profile_end",
            "moe_launch_count", "moe_permute_static", "moe_selftest_wait_timeout",
-           "moe_router_split_weights", "moe_residual_update")
+           "moe_router_split_weights", "moe_residual_update", "moe_noisy_gate",
+           "moe_noisy_gate_workspace_size")
 PROFILE_STAGES = ("route", "latent_down", "dispatch", "expert_gate_up", "expert_down", "combine",
                   "latent_up_resgate")
 
@@ -79,6 +80,8 @@ def lib():
             "moe_route": [cp, vp, vp, vp, vp, vp, vp, vp, vp],
             "moe_router_split_weights": [vp, ctypes.c_int32, ctypes.c_int32, vp, vp],
             "moe_residual_update": [cp, vp, vp, vp, vp, vp, vp],
+            "moe_noisy_gate_workspace_size": [cp, ctypes.POINTER(sz)],
+            "moe_noisy_gate": [cp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp],
             "moe_permute": [cp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp],
             "moe_expert_ffn": [cp, vp, vp, vp, vp, vp, vp, vp, sz, vp],
             "moe_combine": [cp, vp, vp, vp, vp, vp],
@@ -151,6 +154,31 @@ def moe_residual_update(cfg, b, r, gamma_post, resid_g, out, stream=None):
     _check("moe_residual_update", lib().moe_residual_update(
         ctypes.byref(cfg), _ptr(b), _ptr(r), _ptr(gamma_post), _ptr(resid_g), _ptr(out),
         _stream(stream)))
+
+
+def noisy_gate(cfg, u, w_router, w_noise, noise_eps, stream=None, want_h=True, want_p=True):
+    """moe_noisy_gate on CUDA tensors; returns a dict of CUDA tensors (H, idx, w, P,
+    importance, load, cv2)."""
+    import torch
+    T, n, k = cfg.T, cfg.n_experts, cfg.top_k
+    dev = u.device
+    out = {"idx": torch.empty((T, k), dtype=torch.int32, device=dev),
+           "w": torch.empty((T, k), dtype=torch.float32, device=dev),
+           "importance": torch.empty(n, dtype=torch.float32, device=dev),
+           "load": torch.empty(n, dtype=torch.float32, device=dev),
+           "cv2": torch.empty(4, dtype=torch.float32, device=dev)}
+    out["H"] = torch.empty((T, n), dtype=torch.float32, device=dev) if want_h else None
+    out["P"] = torch.empty((T, n), dtype=torch.float32, device=dev) if want_p else None
+    nbytes = ctypes.c_size_t()
+    _check("moe_noisy_gate_workspace_size",
+           lib().moe_noisy_gate_workspace_size(ctypes.byref(cfg), ctypes.byref(nbytes)))
+    ws = torch.empty(nbytes.value, dtype=torch.uint8, device=dev)
+    _check("moe_noisy_gate", lib().moe_noisy_gate(
+        ctypes.byref(cfg), _ptr(u), _ptr(w_router), _ptr(w_noise), _ptr(noise_eps),
+        _ptr(out["H"]), _ptr(out["idx"]), _ptr(out["w"]), _ptr(out["P"]), _ptr(out["importance"]),
+        _ptr(out["load"]), _ptr(out["cv2"]), _ptr(ws), nbytes.value, _stream(stream)))
+    out["workspace"] = ws
+    return out
 
 
 def moe_router_split_weights(w, w_split, stream=None):

@@ -527,6 +527,141 @@ __global__ void resid_update_bf16_kernel(const uint16_t* __restrict__ b, const u
   }
 }
 
+// ------------------------------------------------------------------ noisy gate statistics
+//
+// Shazeer et al.'s noisy top-k gate for tokens with clean logits l and noise logits m (both
+// [T, n] fp32) and standard-normal draws eps [T, n]: H = l + eps * softplus(m); the k largest H
+// (ties to the lower index) with weights Softmax over them; the smooth load
+// P_i = Phi((l_i - kth_excluding(H, k, i)) / softplus(m_i)), where kth_excluding is the k-th
+// largest H of the other experts: the (k+1)-th largest overall for a selected expert, the k-th
+// otherwise.  Each warp walks a fixed run of tokens; lane j owns experts j, j+32, ... and adds
+// their G and P in token order into per-warp partial sums (deterministic).
+constexpr int kGateTokensPerWarp = 64;
+
+__device__ __forceinline__ float softplusf_(float z) { return z > 20.0f ? z : log1pf(expf(z)); }
+
+__global__ void noisy_gate_kernel(const float* __restrict__ l, const float* __restrict__ m,
+                                  const float* __restrict__ eps, int T, int n, int k,
+                                  float* __restrict__ H_out, int32_t* __restrict__ topk_idx,
+                                  float* __restrict__ topk_w, float* __restrict__ P_out,
+                                  float* __restrict__ part_imp, float* __restrict__ part_load) {
+  const int lane = threadIdx.x & 31;
+  const int gw = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);  // global warp
+  const int t0 = gw * kGateTokensPerWarp;
+  constexpr int kPer = kMaxExperts / 32;
+  float imp[kPer], load[kPer];
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) { imp[i] = 0.0f; load[i] = 0.0f; }
+  for (int t = t0; t < min(T, t0 + kGateTokensPerWarp); ++t) {
+    float h[kPer], lv[kPer], sp[kPer];
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {
+      const int e = lane + 32 * i;
+      h[i] = -INFINITY;
+      lv[i] = 0.0f;
+      sp[i] = 1.0f;
+      if (e < n) {
+        const size_t o = static_cast<size_t>(t) * n + e;
+        lv[i] = l[o];
+        sp[i] = softplusf_(m[o]);
+        h[i] = lv[i] + eps[o] * sp[i];
+        if (H_out) H_out[o] = h[i];
+      }
+    }
+    // k + 1 rounds of warp argmax: the selected k, then the (k+1)-th largest
+    bool sel[kPer];
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) sel[i] = false;
+    float top_v[kMaxTopK + 1];
+    int top_i[kMaxTopK + 1];
+    for (int j = 0; j <= k && j < n; ++j) {
+      float bv = -INFINITY;
+      int bi = 0x7fffffff;
+#pragma unroll
+      for (int i = 0; i < kPer; ++i) {
+        const int e = lane + 32 * i;
+        if (e < n && !sel[i] && (h[i] > bv || (h[i] == bv && e < bi))) { bv = h[i]; bi = e; }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+        const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+        if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
+      }
+      top_v[j] = bv;
+      top_i[j] = bi;
+      if (j < k) {
+#pragma unroll
+        for (int i = 0; i < kPer; ++i)
+          if (lane + 32 * i == bi) sel[i] = true;
+      }
+    }
+    float z = 0.0f;
+    for (int j = 0; j < k; ++j) z += expf(top_v[j] - top_v[0]);
+    if (lane == 0) {
+      for (int j = 0; j < k; ++j) {
+        topk_idx[static_cast<size_t>(t) * k + j] = top_i[j];
+        topk_w[static_cast<size_t>(t) * k + j] = expf(top_v[j] - top_v[0]) / z;
+      }
+    }
+    const float kth_in = top_v[k];       // bar for a selected expert
+    const float kth_out = top_v[k - 1];  // bar for the others
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {
+      const int e = lane + 32 * i;
+      if (e >= n) continue;
+      const float g = sel[i] ? expf(h[i] - top_v[0]) / z : 0.0f;
+      const float zz = (lv[i] - (sel[i] ? kth_in : kth_out)) / sp[i];
+      const float p = 0.5f * erfcf(-zz * 0.70710678118654752f);
+      if (P_out) P_out[static_cast<size_t>(t) * n + e] = p;
+      imp[i] += g;
+      load[i] += p;
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) {
+    const int e = lane + 32 * i;
+    if (e < n) {
+      part_imp[static_cast<size_t>(gw) * n + e] = imp[i];
+      part_load[static_cast<size_t>(gw) * n + e] = load[i];
+    }
+  }
+}
+
+// One CTA of kMaxExperts threads: importance and load per expert (partials summed in warp order)
+// and CV^2 = population variance / mean^2 of each.
+__global__ void gate_stats_reduce_kernel(const float* __restrict__ part_imp,
+                                         const float* __restrict__ part_load, int nparts, int n,
+                                         float* __restrict__ importance, float* __restrict__ load,
+                                         float* __restrict__ cv2) {
+  __shared__ float si[kMaxExperts], sl[kMaxExperts];
+  const int e = threadIdx.x;
+  float a = 0.0f, b = 0.0f;
+  if (e < n) {
+    for (int q = 0; q < nparts; ++q) {
+      a += part_imp[static_cast<size_t>(q) * n + e];
+      b += part_load[static_cast<size_t>(q) * n + e];
+    }
+    importance[e] = a;
+    load[e] = b;
+  }
+  si[e] = a;
+  sl[e] = b;
+  __syncthreads();
+  if (e == 0) {
+    double mi = 0.0, ml = 0.0, vi = 0.0, vl = 0.0;
+    for (int i = 0; i < n; ++i) { mi += si[i]; ml += sl[i]; }
+    mi /= n;
+    ml /= n;
+    for (int i = 0; i < n; ++i) {
+      vi += (si[i] - mi) * (si[i] - mi);
+      vl += (sl[i] - ml) * (sl[i] - ml);
+    }
+    cv2[0] = static_cast<float>(vi / n / (mi * mi));
+    cv2[1] = static_cast<float>(vl / n / (ml * ml));
+  }
+}
+
 // ------------------------------------------------------------------ failure-detection self-test
 //
 // One thread initialises an mbarrier that expects one arrival which never comes and waits on

@@ -504,6 +504,29 @@ moe_status_t do_latent_up(const moe_config_t& c, const void* y, const void* p_up
                   c.d_model, p, st);
 }
 
+// Workspace of moe_noisy_gate: clean and noise logits, scratch routing of the two logit passes,
+// per-warp partial sums.
+struct GateWorkspace {
+  size_t l, m, idx, w, pi, pl, total;
+  int nparts;
+};
+GateWorkspace gate_layout(const moe_config_t& c) {
+  GateWorkspace L{};
+  const size_t Tn = static_cast<size_t>(c.T) * c.n_experts, Tk = static_cast<size_t>(c.T) * c.top_k;
+  const int warps = cdiv(c.T, kGateTokensPerWarp);
+  L.nparts = cdiv(warps, 4) * 4;
+  size_t o = 0;
+  auto take = [&](size_t bytes) { size_t at = o; o = align_up(o + bytes, 256); return at; };
+  L.l = take(Tn * 4);
+  L.m = take(Tn * 4);
+  L.idx = take(Tk * 4);
+  L.w = take(Tk * 4);
+  L.pi = take(static_cast<size_t>(L.nparts) * c.n_experts * 4);
+  L.pl = take(static_cast<size_t>(L.nparts) * c.n_experts * 4);
+  L.total = o;
+  return L;
+}
+
 // Launch shape of the one-CTA-per-row kernels for a row of D bf16 values.
 bool row_launch(int D, int* threads, int* vec) {
   const int nvec = D / 8;
@@ -822,6 +845,55 @@ moe_status_t moe_residual_update(const moe_config_t* cfg, const void* b, const v
                     static_cast<const void*>(out)}))
     return MOE_ERR_ALIGNMENT;
   return do_resid_update(*cfg, b, r, gamma_post, resid_g, out, static_cast<cudaStream_t>(stream));
+}
+
+moe_status_t moe_noisy_gate_workspace_size(const moe_config_t* cfg, size_t* bytes) {
+  moe_status_t s = check_cfg(cfg);
+  if (s != MOE_OK) return s;
+  if (!bytes) return MOE_ERR_INVALID_ARG;
+  *bytes = gate_layout(*cfg).total;
+  return MOE_OK;
+}
+
+moe_status_t moe_noisy_gate(const moe_config_t* cfg, const void* u, const void* w_router,
+                            const void* w_noise, const float* noise_eps, float* noisy_logits_out,
+                            int32_t* topk_idx, float* topk_w, float* load_prob_out,
+                            float* importance, float* load, float* cv2, void* workspace,
+                            size_t workspace_bytes, void* stream) {
+  moe_status_t s = check_cfg(cfg);
+  if (s != MOE_OK) return s;
+  const moe_config_t& c = *cfg;
+  if (c.top_k >= c.n_experts) return MOE_ERR_UNSUPPORTED;  // kth_excluding needs k < n
+  if (c.T == 0) return MOE_ERR_INVALID_ARG;                 // statistics of an empty batch
+  if (!u || !w_router || !w_noise || !noise_eps || !topk_idx || !topk_w || !importance || !load ||
+      !cv2)
+    return MOE_ERR_INVALID_ARG;
+  if (!all_aligned({u, w_router, w_noise, static_cast<const void*>(noise_eps),
+                    static_cast<const void*>(noisy_logits_out), static_cast<const void*>(topk_idx),
+                    static_cast<const void*>(topk_w), static_cast<const void*>(load_prob_out),
+                    static_cast<const void*>(importance), static_cast<const void*>(load),
+                    static_cast<const void*>(cv2), workspace}))
+    return MOE_ERR_ALIGNMENT;
+  const GateWorkspace L = gate_layout(c);
+  if (!workspace || workspace_bytes < L.total) return MOE_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // the two logit passes are plain logits (softmax-gate router, no bias)
+  moe_config_t plain = c;
+  plain.gate_mode = MOE_GATE_SOFTMAX;
+  float* lb = at<float>(workspace, L.l);
+  float* mb = at<float>(workspace, L.m);
+  int32_t* si = at<int32_t>(workspace, L.idx);
+  float* sw = at<float>(workspace, L.w);
+  if ((s = do_route(plain, u, w_router, nullptr, nullptr, lb, si, sw, st)) != MOE_OK) return s;
+  if ((s = do_route(plain, u, w_noise, nullptr, nullptr, mb, si, sw, st)) != MOE_OK) return s;
+  float* pi = at<float>(workspace, L.pi);
+  float* pl = at<float>(workspace, L.pl);
+  noisy_gate_kernel<<<L.nparts / 4, 128, 0, st>>>(lb, mb, noise_eps, c.T, c.n_experts, c.top_k,
+                                                  noisy_logits_out, topk_idx, topk_w,
+                                                  load_prob_out, pi, pl);
+  gate_stats_reduce_kernel<<<1, kMaxExperts, 0, st>>>(pi, pl, L.nparts, c.n_experts, importance,
+                                                      load, cv2);
+  return last_launch(2);
 }
 
 unsigned long long moe_launch_count(void) { return g_launches.load(); }
