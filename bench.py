@@ -385,6 +385,35 @@ def measure_ours(cfg, steps: int, warmup: int, device, peaks: dict, with_e2e: bo
     return res
 
 
+def measure_gate_stats(cfg, args, device) -> dict:
+    """moe_noisy_gate (noisy logits, KeepTopK gate, importance and smooth load with CV^2) on one
+    batch, timed with CUDA events over the steps."""
+    import torch
+    import moe_inputs
+    import sparse_moe_layer_softmax_b200 as moe
+    from gpu_harness import abi_config
+    dev = moe_inputs.device_inputs(cfg, device=device)
+    c = abi_config(cfg)
+    args_ = (c, dev["u"], dev["w_router"], dev["w_noise"], dev["noise_eps"])
+    for _ in range(args.warmup):
+        moe.noisy_gate(*args_)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    outs = []
+    e0.record()
+    for _ in range(args.steps):
+        outs.append(moe.noisy_gate(*args_, want_h=False, want_p=False))
+    e1.record()
+    torch.cuda.synchronize()
+    ms = reduce_max(e0.elapsed_time(e1) / args.steps, device)
+    cv2 = outs[-1]["cv2"].cpu().tolist()
+    del dev, outs
+    torch.cuda.empty_cache()
+    return {"value": round(cfg.T / (ms / 1e3), 2), "unit": UNIT, "ms_per_step": round(ms, 4),
+            "cv2_importance": cv2[0], "cv2_load": cv2[1],
+            "note": "includes the allocation of each call's outputs and workspace by the binding"}
+
+
 # ------------------------------------------------------------------ the CPU oracle as a baseline
 
 class OracleRunner:
@@ -573,6 +602,9 @@ def main(argv=None) -> int:
                 "value": round(vcfg.T * world / (vres["ms_per_step"] / 1e3), 2), "unit": UNIT,
                 "ms_per_step": round(vres["ms_per_step"], 4), "stage_ms": vres["stage_ms"],
                 "layer_roofline": vres["layer_roofline"], "clocks": vres["clocks"]}
+    if not args.no_decode and cfg.name != "muse_decode":
+        line.setdefault("variants", {})["shazeer_bf16_noisy_gate_stats"] = measure_gate_stats(
+            configs.SHAZEER_BF16_NOISY, args, device)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(cfg, args.cpu_sample or default_cpu_sample(cfg))
     if rank == 0:
