@@ -29,6 +29,8 @@ enum EpiKind : int {
   EPI_ROUTER = 4,   // top-k selection and renormalised weights over the row's logits
 };
 
+enum TileOrder : int { TILE_CHUNK_FASTEST = 0, TILE_FEATURE_FASTEST = 1 };
+
 struct GemmParams {
   const int* seg;   // [G+1] row offsets of the groups in X, or nullptr: one group of M rows
   int G;            // groups
@@ -53,7 +55,15 @@ struct GemmParams {
   const float* sel_bias;     // EPI_ROUTER (sigmoid): selection-only correction bias [Nout]
   int x_k_period;            // > 0: X's k coordinate wraps every x_k_period columns (W's K is
                              // a multiple: the fp32 router weights' hi/mid/lo bf16 parts)
+  int tile_order;            // TILE_CHUNK_FASTEST | TILE_FEATURE_FASTEST
+  int k_rotate;              // 1: each tile starts its reduction at its own k-block
+  int out_tma;               // bf16 epilogues of the normal orientation: 1 = the output tensor
+                             // map is valid and whole-warp row blocks leave by TMA stores
 };
+
+// Shared memory that stages the bf16 output of the normal-orientation epilogues: one 4 KB
+// buffer (32 rows x 128 bytes) per epilogue warp.
+constexpr int kStageOutBytes = 4 * 4096;
 
 template <bool kSwap, int BN, int kEpi>
 struct GemmShape {
@@ -100,17 +110,74 @@ __device__ __forceinline__ bool epilogue_all(bool v) {
   return r != 0;
 }
 
+// Whether a kernel instance stages its output for TMA stores (bf16 epilogues, normal orientation).
+template <bool kSwap, int kEpi>
+__host__ __device__ constexpr bool stages_output() {
+  return !kSwap && kEpi != EPI_ROUTER;
+}
+
 template <bool kSwap, int BN, int kEpi, int kStages>
 constexpr int gemm_smem_bytes() {
-  return kStages * GemmShape<kSwap, BN, kEpi>::kStageBytes + 1024 + kSmemMisc;
+  return kStages * GemmShape<kSwap, BN, kEpi>::kStageBytes +
+         (stages_output<kSwap, kEpi>() ? kStageOutBytes : 0) + 1024 + kSmemMisc;
+}
+
+// Where one epilogue warp's output goes.  A warp whose 32 rows all lie inside the tile stages
+// each 32 x 64 chunk in its shared-memory buffer (128-byte rows, 16-byte units XOR-swizzled by
+// the row: the layout a SWIZZLE_128B tensor map reads, and free of bank conflicts) and stores it
+// with one TMA box store; a warp holding rows past the tile's end (the next group's rows follow
+// in the same matrix) stores its valid rows directly, 16 bytes at a time.
+struct EpiOut {
+  const CUtensorMap* tm;  // output tensor map, or nullptr: direct stores only
+  uint8_t* buf;           // this warp's 4 KB staging buffer (1024-byte aligned)
+  bool whole;             // all 32 rows of this warp lie inside the tile
+};
+
+// Emits one 64-column chunk (8 x 16 bytes per row) of this thread's row at output column x of
+// row block y (the warp's first row); `dst` is the row's address at column x.
+__device__ __forceinline__ void emit_chunk(const EpiOut& eo, const uint4 (&ch)[8], uint16_t* dst,
+                                           bool valid, int x, int y, int lane) {
+  if (eo.tm != nullptr && eo.whole) {
+    if (lane == 0) bulk_wait_read_all();  // the buffer's previous store has read it
+    __syncwarp();
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      *reinterpret_cast<uint4*>(eo.buf + lane * 128 + ((j ^ (lane & 7)) << 4)) = ch[j];
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+      tma_store_2d(eo.tm, eo.buf, x, y);
+      bulk_commit();
+    }
+  } else if (valid) {
+    uint4* d = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) d[j] = ch[j];
+  }
+}
+
+__device__ __forceinline__ void pack8(const float* v, uint4& lo, uint4& hi) {
+  uint32_t pk[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) pk[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
+  lo = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+  hi = make_uint4(pk[4], pk[5], pk[6], pk[7]);
 }
 
 struct TileCoord {
-  int g, ft, row0, nrows;
+  int g, ft, chunk, row0, nrows;
 };
 
+// Tile t's group, feature tile and row chunk.  Within a group the tiles run in one of two orders:
+//   TILE_CHUNK_FASTEST   : (feature tile, row chunk), row chunk fastest.  The CTAs working at one
+//                          time share each weight tile; a group's activation rows are re-read per
+//                          feature tile, from L2 when the group's rows are few (expert GEMMs).
+//   TILE_FEATURE_FASTEST : (row chunk, feature tile).  The CTAs working at one time share each
+//                          activation chunk, so a large activation matrix leaves HBM once and the
+//                          (smaller) weight matrix is the operand re-read from L2 (dense
+//                          projections over many tokens).
 __device__ __forceinline__ TileCoord decode_tile(int t, const int* s_seg, const int* s_pref,
-                                                 int G, int FT, int CH) {
+                                                 int G, int FT, int CH, int order) {
   int lo = 0, hi = G;
   while (lo < hi) {  // last g with s_pref[g] <= t
     int mid = (lo + hi + 1) >> 1;
@@ -118,14 +185,27 @@ __device__ __forceinline__ TileCoord decode_tile(int t, const int* s_seg, const 
   }
   TileCoord c;
   c.g = lo;
-  int chunks = (s_pref[lo + 1] - s_pref[lo]) / FT;
-  int local = t - s_pref[lo];
-  c.ft = local / chunks;
-  int chunk = local - c.ft * chunks;
-  c.row0 = s_seg[lo] + chunk * CH;
+  const int chunks = (s_pref[lo + 1] - s_pref[lo]) / FT;
+  const int local = t - s_pref[lo];
+  if (order == TILE_FEATURE_FASTEST) {
+    c.chunk = local / FT;
+    c.ft = local - c.chunk * FT;
+  } else {
+    c.ft = local / chunks;
+    c.chunk = local - c.ft * chunks;
+  }
+  c.row0 = s_seg[lo] + c.chunk * CH;
   int rem = s_seg[lo + 1] - c.row0;
   c.nrows = rem < CH ? rem : CH;
   return c;
+}
+
+// First k-block of a tile's reduction.  With k rotation on, tile (chunk, ft) starts at k-block
+// (chunk + ft) mod KB and wraps around, so CTAs that work at the same time on one weight tile
+// read different parts of it (no L2 hot spot on one k-block); the sum is the same up to the
+// order of the fp32 additions, and depends only on the tile, not on the CTA that runs it.
+__device__ __forceinline__ int k_start(const TileCoord& c, int KB, int rotate) {
+  return rotate ? (c.chunk + c.ft) % KB : 0;
 }
 
 template <int kMaxK>
@@ -182,10 +262,12 @@ __device__ __forceinline__ void topk_weights(const TopK<kMaxK>& tk, int k, int g
 // if below nrows) and the tile's BN accumulator columns (output features f0 ...).
 template <int BN, int kEpi>
 __device__ __forceinline__ void epilogue_rows(const GemmParams& p, int row0, int nrows, int f0,
-                                              uint32_t tbase, int q, int lane, float* s_coef) {
+                                              uint32_t tbase, int q, int lane, float* s_coef,
+                                              const EpiOut& eo) {
     const int rl = q * 32 + lane;
     const bool valid = rl < nrows;
     const size_t row = static_cast<size_t>(row0 + rl);
+    const int yblk = row0 + q * 32;  // first row of this warp's row block
     if constexpr (kEpi == EPI_ROUTER) {
       TopK<8> tk;
       tk.init();
@@ -232,20 +314,20 @@ __device__ __forceinline__ void epilogue_rows(const GemmParams& p, int row0, int
         }
       }
     } else if constexpr (kEpi == EPI_SWIGLU) {
+      // accumulator columns [0, BN/2) are the gate projection, [BN/2, BN) the up projection
       uint16_t* out = static_cast<uint16_t*>(p.out) + row * p.Nout + f0;
-      for (int c0 = 0; c0 < BN / 2; c0 += 16) {
-        float gv[16], uv[16];
-        tmem_ld16(tbase + c0, gv);
-        tmem_ld16(tbase + BN / 2 + c0, uv);
-        uint32_t pk[8];
+      for (int c0 = 0; c0 < BN / 2; c0 += 64) {
+        uint4 ch[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
-          pk[i] = pack_bf16x2(silu(gv[2 * i]) * uv[2 * i], silu(gv[2 * i + 1]) * uv[2 * i + 1]);
-        if (valid) {
-          uint4* dst = reinterpret_cast<uint4*>(out + c0);
-          dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-          dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+        for (int qq = 0; qq < 4; ++qq) {
+          float gv[16], uv[16];
+          tmem_ld16(tbase + c0 + 16 * qq, gv);
+          tmem_ld16(tbase + BN / 2 + c0 + 16 * qq, uv);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) gv[i] = silu(gv[i]) * uv[i];
+          pack8(gv, ch[2 * qq], ch[2 * qq + 1]);
         }
+        emit_chunk(eo, ch, out + c0, valid, f0 + c0, yblk, lane);
       }
     } else if constexpr (kEpi == EPI_RESGATE) {
       // Per-column coefficients of this tile, computed once by the 128 epilogue threads:
@@ -275,49 +357,42 @@ __device__ __forceinline__ void epilogue_rows(const GemmParams& p, int row0, int
         for (int i = 0; i < 8; ++i)
           hv[i] = (valid && has_r) ? reinterpret_cast<const uint4*>(hrow + c0)[i]
                                    : make_uint4(0, 0, 0, 0);
+        uint4 ch[8];
 #pragma unroll
         for (int qq = 0; qq < 4; ++qq) {
           float v[16];
           tmem_ld16(tbase + c0 + 16 * qq, v);
           const uint16_t* hs = reinterpret_cast<const uint16_t*>(&hv[2 * qq]);
-          uint32_t pk[8];
 #pragma unroll
-          for (int i = 0; i < 16; i += 2) {
+          for (int i = 0; i < 16; ++i) {
             const int col = c0 + 16 * qq + i;
-            const float o0 = s_coef[col] * bf16_to_f32(hs[i]) + s_coef[BN + col] * round_bf16(v[i]);
-            const float o1 =
-                s_coef[col + 1] * bf16_to_f32(hs[i + 1]) + s_coef[BN + col + 1] * round_bf16(v[i + 1]);
-            pk[i / 2] = pack_bf16x2(o0, o1);
+            v[i] = s_coef[col] * bf16_to_f32(hs[i]) + s_coef[BN + col] * round_bf16(v[i]);
           }
-          if (valid) {
-            uint4* dst = reinterpret_cast<uint4*>(out + c0 + 16 * qq);
-            dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-            dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-          }
+          pack8(v, ch[2 * qq], ch[2 * qq + 1]);
         }
+        emit_chunk(eo, ch, out + c0, valid, f0 + c0, yblk, lane);
       }
     } else {
       uint16_t* out = static_cast<uint16_t*>(p.out) + row * p.Nout + f0;
-      for (int c0 = 0; c0 < BN; c0 += 16) {
-        float v[16];
-        tmem_ld16(tbase + c0, v);
-        if constexpr (kEpi == EPI_RELU) {
+      for (int c0 = 0; c0 < BN; c0 += 64) {
+        uint4 ch[8];
 #pragma unroll
-          for (int i = 0; i < 16; ++i) v[i] = fmaxf(v[i], 0.0f);
-        } else if constexpr (kEpi == EPI_STORE) {
-          if (p.gamma) {
+        for (int qq = 0; qq < 4; ++qq) {
+          float v[16];
+          tmem_ld16(tbase + c0 + 16 * qq, v);
+          if constexpr (kEpi == EPI_RELU) {
 #pragma unroll
-            for (int i = 0; i < 16; ++i) v[i] = round_bf16(v[i]) * (1.0f + p.gamma[f0 + c0 + i]);
+            for (int i = 0; i < 16; ++i) v[i] = fmaxf(v[i], 0.0f);
+          } else if constexpr (kEpi == EPI_STORE) {
+            if (p.gamma) {
+#pragma unroll
+              for (int i = 0; i < 16; ++i)
+                v[i] = round_bf16(v[i]) * (1.0f + p.gamma[f0 + c0 + 16 * qq + i]);
+            }
           }
+          pack8(v, ch[2 * qq], ch[2 * qq + 1]);
         }
-        if (valid) {
-          uint32_t pk[8];
-#pragma unroll
-          for (int i = 0; i < 8; ++i) pk[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
-          uint4* dst = reinterpret_cast<uint4*>(out + c0);
-          dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-          dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-        }
+        emit_chunk(eo, ch, out + c0, valid, f0 + c0, yblk, lane);
       }
     }
 }
@@ -325,13 +400,16 @@ __device__ __forceinline__ void epilogue_rows(const GemmParams& p, int row0, int
 template <bool kSwap, int BN, int kEpi, int kStages>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
-                   const GemmParams p) {
+                   const __grid_constant__ CUtensorMap tmO, const GemmParams p) {
   using S = GemmShape<kSwap, BN, kEpi>;
+  constexpr bool kStageOut = stages_output<kSwap, kEpi>();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* tiles = smem;
-  uint64_t* full = reinterpret_cast<uint64_t*>(tiles + kStages * S::kStageBytes);
+  uint8_t* stage_out = tiles + kStages * S::kStageBytes;  // 1024-byte aligned (stage multiple)
+  uint64_t* full =
+      reinterpret_cast<uint64_t*>(stage_out + (kStageOut ? kStageOutBytes : 0));
   uint64_t* empty = full + kStages;
   uint64_t* tfull = empty + kStages;
   uint64_t* tempty = tfull + 2;
@@ -402,14 +480,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     for (int s = 0; s < kStages; ++s) { issued[s] = false; last_parity[s] = 0; }
     bool ok = true;
     for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-      TileCoord c = decode_tile(t, s_seg, s_pref, G, FT, S::kCH);
+      TileCoord c = decode_tile(t, s_seg, s_pref, G, FT, S::kCH, p.tile_order);
       const int wrow = c.g * p.Nw + c.ft * S::kFO;
+      const int kb0 = k_start(c, KB, p.k_rotate);
       for (int kb = 0; kb < KB; ++kb) {
         if (!mbar_wait(&empty[stage], phase ^ 1)) { ok = false; break; }
         uint8_t* sa = tiles + stage * S::kStageBytes;
         uint8_t* sb = sa + S::kABytes;
         mbar_arrive_expect_tx(&full[stage], S::kStageBytes);
-        const int kx = kb * S::kBK;
+        const int kbr = kb + kb0 < KB ? kb + kb0 : kb + kb0 - KB;
+        const int kx = kbr * S::kBK;
         const int kxx = p.x_k_period > 0 ? kx % p.x_k_period : kx;  // X's k coordinate
         if (!kSwap) {
           tma_load_2d(&tmX, &full[stage], sa, kxx, c.row0);
@@ -465,13 +545,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int q = warp & 3;  // TMEM lane quarter this warp may access
     uint32_t acc = 0, acc_phase = 0;
     for (int t = blockIdx.x; t < total; t += gridDim.x) {
-      TileCoord c = decode_tile(t, s_seg, s_pref, G, FT, S::kCH);
+      TileCoord c = decode_tile(t, s_seg, s_pref, G, FT, S::kCH, p.tile_order);
       if (!epilogue_all(mbar_wait(&tfull[acc], acc_phase))) break;
       tc_fence_after();
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * S::kAccCols;
       const int f0 = c.ft * S::kFO;
       if constexpr (!kSwap) {
-        epilogue_rows<BN, kEpi>(p, c.row0, c.nrows, f0, tbase, q, lane, s_coef);
+        const EpiOut eo{(kStageOut && p.out_tma) ? &tmO : nullptr, stage_out + q * 4096,
+                        c.nrows >= q * 32 + 32};
+        epilogue_rows<BN, kEpi>(p, c.row0, c.nrows, f0, tbase, q, lane, s_coef, eo);
       } else {
         // swap orientation: this thread owns output feature f for the BN rows of the chunk
         const int f = f0 + q * 32 + lane;
@@ -519,6 +601,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       mbar_arrive(&tempty[acc]);
       if (++acc == 2) { acc = 0; acc_phase ^= 1; }
     }
+    // The staged stores have completed before the CTA (and its shared memory) goes away.
+    if (kStageOut && lane == 0) bulk_wait_all();
   }
   tc_fence_before();
   __syncthreads();
@@ -560,19 +644,22 @@ struct PairShape {
 
 template <int BN, int kEpi, int kStages>
 constexpr int gemm_pair_smem_bytes() {
-  return kStages * PairShape<BN, kEpi>::kStageBytes + 1024 + kSmemMisc;
+  return kStages * PairShape<BN, kEpi>::kStageBytes + kStageOutBytes + 1024 + kSmemMisc;
 }
 
 template <int BN, int kEpi, int kStages>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     gemm_tc_pair_kernel(const __grid_constant__ CUtensorMap tmX,
-                        const __grid_constant__ CUtensorMap tmW, const GemmParams p) {
+                        const __grid_constant__ CUtensorMap tmW,
+                        const __grid_constant__ CUtensorMap tmO, const GemmParams p) {
   using S = PairShape<BN, kEpi>;
+  static_assert(kEpi != EPI_ROUTER, "the pair kernel has bf16 epilogues only");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* tiles = smem;
-  uint64_t* full = reinterpret_cast<uint64_t*>(tiles + kStages * S::kStageBytes);
+  uint8_t* stage_out = tiles + kStages * S::kStageBytes;  // 1024-byte aligned (stage multiple)
+  uint64_t* full = reinterpret_cast<uint64_t*>(stage_out + kStageOutBytes);
   uint64_t* empty = full + kStages;
   uint64_t* tfull = empty + kStages;
   uint64_t* tempty = tfull + 2;
@@ -646,17 +733,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     for (int s = 0; s < kStages; ++s) { issued[s] = false; last_parity[s] = 0; }
     bool ok = true;
     for (int t = pair; t < total && ok; t += npairs) {
-      TileCoord c = decode_tile(t, s_seg, s_pref, G, FT, S::kCH);
+      TileCoord c = decode_tile(t, s_seg, s_pref, G, FT, S::kCH, p.tile_order);
       const int xrow = c.row0 + 128 * static_cast<int>(rank);
       const int wrow = S::kDual ? c.g * p.Nw + (leader ? 0 : p.Nw / 2) + c.ft * (BN / 2)
                                 : c.g * p.Nw + c.ft * BN + static_cast<int>(rank) * (BN / 2);
+      const int kb0 = k_start(c, KB, p.k_rotate);
       for (int kb = 0; kb < KB; ++kb) {
         if (!mbar_wait(&empty[stage], phase ^ 1)) { ok = false; break; }
         uint8_t* sa = tiles + stage * S::kStageBytes;
         uint8_t* sb = sa + S::kABytes;
         if (leader) mbar_arrive_expect_tx(&full[stage], 2 * S::kStageBytes);
         const uint32_t fb = cluster_addr(&full[stage], 0);
-        const int kx = kb * S::kBK;
+        const int kbr = kb + kb0 < KB ? kb + kb0 : kb + kb0 - KB;
+        const int kx = kbr * S::kBK;
         tma_load_2d_pair(&tmX, fb, sa, kx, xrow);
         tma_load_2d_pair(&tmW, fb, sb, kx, wrow);
         issued[stage] = true;
@@ -702,13 +791,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     uint32_t acc = 0, acc_phase = 0;
     const uint32_t tempty_leader = cluster_addr(&tempty[0], 0);
     for (int t = pair; t < total; t += npairs) {
-      TileCoord c = decode_tile(t, s_seg, s_pref, G, FT, S::kCH);
+      TileCoord c = decode_tile(t, s_seg, s_pref, G, FT, S::kCH, p.tile_order);
       const int row0 = c.row0 + 128 * static_cast<int>(rank);
       const int nrows = max(0, min(128, c.nrows - 128 * static_cast<int>(rank)));
       if (!epilogue_all(mbar_wait(&tfull[acc], acc_phase))) break;
       tc_fence_after();
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * BN;
-      epilogue_rows<BN, kEpi>(p, row0, nrows, c.ft * S::kFO, tbase, q, lane, s_coef);
+      const EpiOut eo{p.out_tma ? &tmO : nullptr, stage_out + q * 4096, nrows >= q * 32 + 32};
+      epilogue_rows<BN, kEpi>(p, row0, nrows, c.ft * S::kFO, tbase, q, lane, s_coef, eo);
       tc_fence_before();
       epilogue_bar();  // all 128 epilogue threads have finished reading this accumulator
       if (threadIdx.x == 64) {
@@ -717,6 +807,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       }
       if (++acc == 2) { acc = 0; acc_phase ^= 1; }
     }
+    if (lane == 0) bulk_wait_all();  // staged stores complete before the CTA leaves
   }
   tc_fence_before();
   __syncthreads();

@@ -99,10 +99,16 @@ moe_status_t launch_gemm(const void* X, long x_rows, const void* W, long w_rows,
     return MOE_ERR_CUDA;
   if (!make_tmap(&tw, W, static_cast<uint64_t>(w_rows), static_cast<uint64_t>(p.K), S::kWBoxRows))
     return MOE_ERR_CUDA;
+  // Output map for the staged epilogue stores (boxes of 32 rows x 64 columns); where the output
+  // cannot be described (unaligned base or row stride) the epilogue stores directly.
+  GemmParams q = p;
+  CUtensorMap to = tx;
+  q.out_tma = stages_output<kSwap, kEpi>() &&
+              make_tmap(&to, p.out, static_cast<uint64_t>(x_rows), static_cast<uint64_t>(p.Nout), 32);
   long grid = device_info().sms;
   if (max_tiles < grid) grid = max_tiles;
   if (grid <= 0) return MOE_OK;
-  kern<<<static_cast<unsigned>(grid), kGemmThreads, smem, st>>>(tx, tw, p);
+  kern<<<static_cast<unsigned>(grid), kGemmThreads, smem, st>>>(tx, tw, to, q);
   return last_launch();
 }
 
@@ -125,10 +131,13 @@ moe_status_t launch_gemm_pair(const void* X, long x_rows, const void* W, long w_
     return MOE_ERR_CUDA;
   if (!make_tmap(&tw, W, static_cast<uint64_t>(w_rows), static_cast<uint64_t>(p.K), BN / 2))
     return MOE_ERR_CUDA;
+  GemmParams q = p;
+  CUtensorMap to = tx;
+  q.out_tma = make_tmap(&to, p.out, static_cast<uint64_t>(x_rows), static_cast<uint64_t>(p.Nout), 32);
   long pairs = device_info().sms / 2;
   if (max_tiles < pairs) pairs = max_tiles;
   if (pairs <= 0) return MOE_OK;
-  kern<<<static_cast<unsigned>(2 * pairs), kGemmThreads, smem, st>>>(tx, tw, p);
+  kern<<<static_cast<unsigned>(2 * pairs), kGemmThreads, smem, st>>>(tx, tw, to, q);
   return last_launch();
 }
 
@@ -286,6 +295,15 @@ Orient dense_orient(int rows, int bn) {
 // GEMM tile would leave most SMs idle while it streams the router weights).
 constexpr int kSmallRouterMaxT = 256;
 
+// Schedule of a dense projection (one group of x_rows rows against Nw weight rows): when the
+// activations outnumber the weight rows, feature tiles run fastest so each activation chunk is
+// read from HBM once while the weights stay in L2; every tile starts its reduction at its own
+// k-block so the CTAs sharing a weight tile do not all read the same k-block at once.
+void dense_schedule(GemmParams& p, long x_rows) {
+  p.tile_order = x_rows > p.Nw ? TILE_FEATURE_FASTEST : TILE_CHUNK_FASTEST;
+  p.k_rotate = 1;
+}
+
 moe_status_t do_route(const moe_config_t& c, const void* u, const void* w_router,
                       const float* bias, const float* sel_bias, float* logits, int32_t* idx,
                       float* w, cudaStream_t st, float* logits_scratch = nullptr) {
@@ -334,6 +352,7 @@ moe_status_t do_route(const moe_config_t& c, const void* u, const void* w_router
   p.gate_mode = c.gate_mode;
   p.logit_mult = mult;
   p.sel_bias = sel_bias;
+  dense_schedule(p, c.T);
   const int bn = c.n_experts <= 32 ? 32 : c.n_experts <= 64 ? 64 : c.n_experts <= 128 ? 128 : 256;
   return run_gemm(EPI_ROUTER, Orient::kNormal, bn, u, c.T, w_router, c.n_experts, p, st);
 }
@@ -479,6 +498,7 @@ moe_status_t do_latent_down(const moe_config_t& c, const void* u, const void* p_
   p.Nw = c.d_latent;
   p.Nout = c.d_latent;
   p.out = z;
+  dense_schedule(p, c.T);
   const int bn = pick_bn_normal(c.d_latent, false);
   return run_gemm(EPI_STORE, dense_orient(c.T, bn), bn, u, c.T, p_down,
                   c.d_latent, p, st);
@@ -499,6 +519,7 @@ moe_status_t do_latent_up(const moe_config_t& c, const void* y, const void* p_up
   p.tau = c.tau;
   p.floor_ = c.resid_floor;
   p.resid_mode = c.resid_mode;
+  dense_schedule(p, c.T);
   const int bn = pick_bn_normal(c.d_model, false);
   return run_gemm(EPI_RESGATE, dense_orient(c.T, bn), bn, y, c.T, p_up,
                   c.d_model, p, st);
