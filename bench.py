@@ -9,7 +9,8 @@ up-projection with the residual gate.  Rank 0 prints one JSON line.
 
 * value: tokens/s over all ranks (each rank processes the full workload: weak scaling, no
   data-path collective), from CUDA events around K steps, max over ranks;
-* e2e: the same through the host-memory API (pinned host input -> device -> layer -> host);
+* e2e: the same through the host-memory API (pinned host input -> device -> layer -> host, one
+  pipelined moe_layer_forward_host call over the steps);
 * roofline: the dominant kernel (expert gate/up GEMM) timed live with the library's stage events;
 * cpu_baseline: the CPU oracle on a bounded token sample of the same workload (rank 0, N=1);
 * decode: the T=64 Muse decode workload measured the same way (secondary line item).
@@ -362,18 +363,17 @@ def measure_ours(cfg, steps: int, warmup: int, device, peaks: dict, with_e2e: bo
            "distinct_experts": distinct, "max_over_mean_load": round(max_over_mean, 3),
            "gpu_launches": int(launches), "clocks": clocks}
 
-    # ---- end to end through the host-memory API: pinned host in, pinned host out
+    # ---- end to end through the host-memory API: pinned host in, pinned host out.  One call
+    # streams `steps` batches; every batch's input copy and output copy is inside the timed
+    # region (the library overlaps them with the neighbouring batches' kernels).
     if with_e2e:
         u_host = u.cpu().pin_memory()
         out_host = torch.empty_like(u_host).pin_memory()
-        u_dev = torch.empty_like(u)
-        for _ in range(2):
-            layer.forward_host(u_host, out_host, u_dev, out)
+        layer.forward_host([u_host] * 2, [out_host] * 2, stream=stream)
         barrier()
         torch.cuda.synchronize()
         e0.record(stream)
-        for _ in range(steps):
-            layer.forward_host(u_host, out_host, u_dev, out)
+        layer.forward_host([u_host] * steps, [out_host] * steps, stream=stream)
         e1.record(stream)
         torch.cuda.synchronize()
         barrier()

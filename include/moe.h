@@ -252,6 +252,32 @@ MOE_API moe_status_t moe_layer_forward(const moe_config_t* cfg, const moe_weight
                                int32_t* topk_idx_out, float* topk_w_out, void* workspace,
                                size_t workspace_bytes, void* stream);
 
+/* Bytes of device staging moe_layer_forward_host needs for this configuration: two input and two
+ * output buffers of T x d_model elements, each rounded up to 256 bytes. */
+MOE_API moe_status_t moe_host_staging_size(const moe_config_t* cfg, size_t* bytes);
+
+/* The whole layer (as moe_layer_forward, with the residual r = u) over n_batches batches held in
+ * HOST memory: batch i's input u_host[i] [T, d_model] is copied to the device, the layer runs on
+ * it and its output is copied back to out_host[i] [T, d_model].  u_host and out_host are host
+ * arrays of n_batches host pointers; the buffers should be page-locked (cudaHostAlloc /
+ * cudaHostRegister), or the copies are not asynchronous.
+ *   - The copies run on two copy streams owned by the library, in double-buffered device staging
+ *     (moe_host_staging_size bytes, caller-owned, 16-byte aligned).  Batch i+1's input copy and
+ *     batch i-1's output copy therefore overlap batch i's kernels, which run on `stream` in order.
+ *   - The copy streams start after the work already queued on `stream`; when `stream` reaches
+ *     the end of the call's work, every output copy has completed.  Synchronise `stream` before
+ *     reading out_host.
+ *   - Batches share the workspace.  Logits and routing copies are not returned.
+ *   - Errors: MOE_ERR_INVALID_ARG for n_batches < 0 or a NULL array or entry, MOE_ERR_WORKSPACE for
+ *     missing or short staging or workspace, MOE_ERR_ALIGNMENT for unaligned staging; any error
+ *     moe_layer_forward returns for the first batch stops the call before it queues anything.
+ *   - Not thread-safe per device: one host pipeline per device at a time. */
+MOE_API moe_status_t moe_layer_forward_host(const moe_config_t* cfg, const moe_weights_t* w,
+                                            int32_t n_batches, const void* const* u_host,
+                                            void* const* out_host, void* staging,
+                                            size_t staging_bytes, void* workspace,
+                                            size_t workspace_bytes, void* stream);
+
 /* Synchronises the stream, returns and clears the device status word of the current device
  * (MOE_OK if no kernel latched an error since the last call). */
 MOE_API moe_status_t moe_get_device_status(void* stream);

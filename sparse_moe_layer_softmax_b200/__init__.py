@@ -30,7 +30,7 @@ EXPORTS = ("moe_status_string", "moe_workspace_size", "moe_route", "moe_permute"
            "moe_layer_forward", "moe_get_device_status", "moe_profile_begin", "moe_profile_end",
            "moe_launch_count", "moe_permute_static", "moe_selftest_wait_timeout",
            "moe_router_split_weights", "moe_residual_update", "moe_noisy_gate",
-           "moe_noisy_gate_workspace_size")
+           "moe_noisy_gate_workspace_size", "moe_host_staging_size", "moe_layer_forward_host")
 PROFILE_STAGES = ("route", "latent_down", "dispatch", "expert_gate_up", "expert_down", "combine",
                   "latent_up_resgate")
 
@@ -88,6 +88,9 @@ def lib():
             "moe_latent_down": [cp, vp, vp, vp, vp],
             "moe_latent_up": [cp, vp, vp, vp, vp, vp, vp],
             "moe_layer_forward": [cp, wp, vp, vp, vp, vp, vp, vp, vp, sz, vp],
+            "moe_host_staging_size": [cp, ctypes.POINTER(ctypes.c_size_t)],
+            "moe_layer_forward_host": [cp, wp, ctypes.c_int32, ctypes.POINTER(vp),
+                                       ctypes.POINTER(vp), vp, sz, vp, sz, vp],
             "moe_get_device_status": [vp],
             "moe_profile_begin": [ctypes.c_int32],
             "moe_profile_end": [vp, vp],
@@ -277,6 +280,12 @@ def profile_end() -> tuple[dict, int]:
     return {k: float(v) for k, v in zip(PROFILE_STAGES, ms)}, calls.value
 
 
+def host_staging_size(cfg: Config) -> int:
+    n = ctypes.c_size_t()
+    _check("moe_host_staging_size", lib().moe_host_staging_size(ctypes.byref(cfg), ctypes.byref(n)))
+    return n.value
+
+
 class MoELayer:
     """A layer instance holding its device weights and a workspace, with a forward() that takes
     device or pinned-host inputs.  Nothing here computes: forward() is one moe_layer_forward."""
@@ -301,14 +310,26 @@ class MoELayer:
                           topk_idx_out, topk_w_out, self.workspace, stream=stream)
         return out
 
-    def forward_host(self, u_host, out_host, u_dev, out_dev, stream=None):
-        """One forward from pinned host memory to pinned host memory: the input is copied to the
-        device, the layer runs, and the output is copied back, all queued on one stream (the
-        residual is the input).  u_dev / out_dev are the device staging buffers."""
+    def forward_host(self, u_hosts, out_hosts, stream=None):
+        """Forwards of batches held in (pinned) host memory, one moe_layer_forward_host call:
+        batch i's input u_hosts[i] (also its residual) goes to the device, through the layer and
+        back to out_hosts[i]; the library overlaps the copies of neighbouring batches with each
+        batch's kernels.  A single tensor stands for a one-batch list.  Synchronise `stream`
+        (default: the current stream) before reading the outputs."""
         import torch
-        s = stream if stream is not None else torch.cuda.current_stream()
-        with torch.cuda.stream(s):
-            u_dev.copy_(u_host, non_blocking=True)
-            self.forward(u_dev, u_dev, out=out_dev, stream=s)
-            out_host.copy_(out_dev, non_blocking=True)
-        return out_host
+        if isinstance(u_hosts, torch.Tensor):
+            u_hosts, out_hosts = [u_hosts], [out_hosts]
+        if len(u_hosts) != len(out_hosts):
+            raise ValueError("u_hosts and out_hosts differ in length")
+        if getattr(self, "_staging", None) is None:
+            self._staging = torch.empty(host_staging_size(self.cfg), dtype=torch.uint8,
+                                        device="cuda")
+        n = len(u_hosts)
+        ins = (ctypes.c_void_p * max(n, 1))(*[t.data_ptr() for t in u_hosts])
+        outs = (ctypes.c_void_p * max(n, 1))(*[t.data_ptr() for t in out_hosts])
+        _check("moe_layer_forward_host",
+               lib().moe_layer_forward_host(ctypes.byref(self.cfg), ctypes.byref(self._w), n, ins,
+                                            outs, self._staging.data_ptr(),
+                                            self._staging.numel(), self.workspace.data_ptr(),
+                                            self.workspace.numel(), _stream(stream)))
+        return out_hosts

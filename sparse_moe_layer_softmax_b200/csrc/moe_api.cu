@@ -591,6 +591,73 @@ moe_status_t do_resid_update(const moe_config_t& c, const void* b, const void* r
   return last_launch();
 }
 
+// Host-side checks of a whole-layer forward (nothing is launched when they fail).  T == 0 passes.
+moe_status_t check_forward(const moe_config_t* cfg, const moe_weights_t* w, const void* u,
+                           const void* r, const void* out, const float* logits_out,
+                           const int32_t* topk_idx_out, const float* topk_w_out,
+                           const void* workspace, size_t workspace_bytes) {
+  moe_status_t s = check_cfg(cfg);
+  if (s != MOE_OK) return s;
+  const moe_config_t& c = *cfg;
+  if (!w) return MOE_ERR_INVALID_ARG;
+  if (c.T == 0) return MOE_OK;
+  const bool latent = c.d_latent > 0;
+  if ((!u && !c.input_norm) || !out || !w->w_router || !w->w_gu || !w->w_down)
+    return MOE_ERR_INVALID_ARG;
+  if (c.input_norm && (!r || !w->gamma_in)) return MOE_ERR_INVALID_ARG;
+  if (c.post_norm && !w->gamma_post) return MOE_ERR_INVALID_ARG;
+  if (latent && (!w->p_down || !w->p_up)) return MOE_ERR_INVALID_ARG;
+  if (c.pre_norm && !w->gamma_pre) return MOE_ERR_INVALID_ARG;
+  if (c.expert_norm && !w->gamma_expert) return MOE_ERR_INVALID_ARG;
+  if (c.resid_mode != MOE_RESID_NONE && (!r || !w->resid_g)) return MOE_ERR_INVALID_ARG;
+  if (!all_aligned({u, r, static_cast<const void*>(out), static_cast<const void*>(logits_out),
+                        static_cast<const void*>(topk_idx_out), static_cast<const void*>(topk_w_out),
+                        workspace, w->w_router, w->p_down, w->p_up, w->w_gu, w->w_down,
+                        static_cast<const void*>(w->gamma_pre),
+                        static_cast<const void*>(w->gamma_expert),
+                        static_cast<const void*>(w->resid_g), static_cast<const void*>(w->logit_bias),
+                        static_cast<const void*>(w->correction_bias),
+                        static_cast<const void*>(w->gamma_in),
+                        static_cast<const void*>(w->gamma_post)})) return MOE_ERR_ALIGNMENT;
+  const Workspace L = layout(c);
+  if (!workspace || workspace_bytes < L.total) return MOE_ERR_WORKSPACE;
+  return MOE_OK;
+}
+
+// Copy streams and events of moe_layer_forward_host, created on first use on each device.
+struct HostPipe {
+  bool ok = false;
+  cudaStream_t h2d = nullptr, d2h = nullptr;
+  cudaEvent_t start = nullptr, done = nullptr;
+  cudaEvent_t in_ready[2] = {}, in_free[2] = {}, out_free[2] = {};
+};
+
+HostPipe* host_pipe() {
+  static std::mutex mu;
+  static HostPipe pipes[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lk(mu);
+  HostPipe& h = pipes[dev];
+  if (!h.ok) {
+    bool good = cudaStreamCreateWithFlags(&h.h2d, cudaStreamNonBlocking) == cudaSuccess &&
+                cudaStreamCreateWithFlags(&h.d2h, cudaStreamNonBlocking) == cudaSuccess;
+    cudaEvent_t* evs[] = {&h.start,       &h.done,       &h.in_ready[0], &h.in_ready[1],
+                          &h.in_free[0],  &h.in_free[1], &h.out_free[0], &h.out_free[1]};
+    for (cudaEvent_t* e : evs)
+      good = good && cudaEventCreateWithFlags(e, cudaEventDisableTiming) == cudaSuccess;
+    if (!good) return nullptr;
+    h.ok = true;
+  }
+  return &h;
+}
+
+// Bytes of one staging buffer (T x d_model elements, rounded up to 256 bytes).
+size_t staging_slot_bytes(const moe_config_t& c) {
+  const size_t b = static_cast<size_t>(c.T) * c.d_model * (c.dtype == MOE_F32 ? 4 : 2);
+  return (b + 255) / 256 * 256;
+}
+
 }  // namespace
 }  // namespace moe
 
@@ -775,31 +842,13 @@ moe_status_t moe_layer_forward(const moe_config_t* cfg, const moe_weights_t* w, 
                                const void* r, void* out, float* logits_out,
                                int32_t* topk_idx_out, float* topk_w_out, void* workspace,
                                size_t workspace_bytes, void* stream) {
-  moe_status_t s = check_cfg(cfg);
+  moe_status_t s = check_forward(cfg, w, u, r, out, logits_out, topk_idx_out, topk_w_out,
+                                 workspace, workspace_bytes);
   if (s != MOE_OK) return s;
   const moe_config_t& c = *cfg;
-  if (!w) return MOE_ERR_INVALID_ARG;
   if (c.T == 0) return MOE_OK;
   const bool latent = c.d_latent > 0;
-  if ((!u && !c.input_norm) || !out || !w->w_router || !w->w_gu || !w->w_down)
-    return MOE_ERR_INVALID_ARG;
-  if (c.input_norm && (!r || !w->gamma_in)) return MOE_ERR_INVALID_ARG;
-  if (c.post_norm && !w->gamma_post) return MOE_ERR_INVALID_ARG;
-  if (latent && (!w->p_down || !w->p_up)) return MOE_ERR_INVALID_ARG;
-  if (c.pre_norm && !w->gamma_pre) return MOE_ERR_INVALID_ARG;
-  if (c.expert_norm && !w->gamma_expert) return MOE_ERR_INVALID_ARG;
-  if (c.resid_mode != MOE_RESID_NONE && (!r || !w->resid_g)) return MOE_ERR_INVALID_ARG;
-  if (!all_aligned({u, r, static_cast<const void*>(out), static_cast<const void*>(logits_out),
-                        static_cast<const void*>(topk_idx_out), static_cast<const void*>(topk_w_out),
-                        workspace, w->w_router, w->p_down, w->p_up, w->w_gu, w->w_down,
-                        static_cast<const void*>(w->gamma_pre),
-                        static_cast<const void*>(w->gamma_expert),
-                        static_cast<const void*>(w->resid_g), static_cast<const void*>(w->logit_bias),
-                        static_cast<const void*>(w->correction_bias),
-                        static_cast<const void*>(w->gamma_in),
-                        static_cast<const void*>(w->gamma_post)})) return MOE_ERR_ALIGNMENT;
   const Workspace L = layout(c);
-  if (!workspace || workspace_bytes < L.total) return MOE_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   int32_t* idx = topk_idx_out ? topk_idx_out : at<int32_t>(workspace, L.idx);
   float* wt = topk_w_out ? topk_w_out : at<float>(workspace, L.w);
@@ -968,6 +1017,66 @@ moe_status_t moe_profile_end(float* stage_ms, int32_t* calls) {
   p.active = false;
   p.calls = p.max_calls = 0;
   return s;
+}
+
+moe_status_t moe_host_staging_size(const moe_config_t* cfg, size_t* bytes) {
+  if (!bytes) return MOE_ERR_INVALID_ARG;
+  moe_status_t s = check_cfg(cfg);
+  if (s != MOE_OK) return s;
+  *bytes = 4 * staging_slot_bytes(*cfg);
+  return MOE_OK;
+}
+
+moe_status_t moe_layer_forward_host(const moe_config_t* cfg, const moe_weights_t* w,
+                                    int32_t n_batches, const void* const* u_host,
+                                    void* const* out_host, void* staging, size_t staging_bytes,
+                                    void* workspace, size_t workspace_bytes, void* stream) {
+  moe_status_t s = check_cfg(cfg);
+  if (s != MOE_OK) return s;
+  if (n_batches < 0 || (n_batches > 0 && (!u_host || !out_host))) return MOE_ERR_INVALID_ARG;
+  for (int32_t i = 0; i < n_batches; ++i)
+    if (!u_host[i] || !out_host[i]) return MOE_ERR_INVALID_ARG;
+  const moe_config_t& c = *cfg;
+  const size_t slot = staging_slot_bytes(c);
+  if (!staging || staging_bytes < 4 * slot) return MOE_ERR_WORKSPACE;
+  if (!all_aligned({staging})) return MOE_ERR_ALIGNMENT;
+  uint8_t* base = static_cast<uint8_t*>(staging);
+  void* in[2] = {base, base + slot};
+  void* outb[2] = {base + 2 * slot, base + 3 * slot};
+  if ((s = check_forward(cfg, w, in[0], in[0], outb[0], nullptr, nullptr, nullptr, workspace,
+                         workspace_bytes)) != MOE_OK)
+    return s;
+  if (n_batches == 0 || c.T == 0) return MOE_OK;
+  HostPipe* hp = host_pipe();
+  if (!hp) return MOE_ERR_CUDA;
+  const size_t bytes = static_cast<size_t>(c.T) * c.d_model * (c.dtype == MOE_F32 ? 4 : 2);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // The copy streams start after what is already queued on the caller's stream.
+  cudaEventRecord(hp->start, st);
+  cudaStreamWaitEvent(hp->h2d, hp->start, 0);
+  cudaStreamWaitEvent(hp->d2h, hp->start, 0);
+  for (int32_t i = 0; i < n_batches && s == MOE_OK; ++i) {
+    const int b = i & 1;
+    // input slot b is free once batch i-2's kernels are done with it
+    if (i >= 2) cudaStreamWaitEvent(hp->h2d, hp->in_free[b], 0);
+    cudaMemcpyAsync(in[b], u_host[i], bytes, cudaMemcpyHostToDevice, hp->h2d);
+    cudaEventRecord(hp->in_ready[b], hp->h2d);
+    cudaStreamWaitEvent(st, hp->in_ready[b], 0);
+    // output slot b is free once batch i-2's output copy has read it
+    if (i >= 2) cudaStreamWaitEvent(st, hp->out_free[b], 0);
+    s = moe_layer_forward(cfg, w, in[b], in[b], outb[b], nullptr, nullptr, nullptr, workspace,
+                          workspace_bytes, stream);
+    cudaEventRecord(hp->in_free[b], st);  // batch i's kernels are done: input read, output ready
+    cudaStreamWaitEvent(hp->d2h, hp->in_free[b], 0);
+    if (s == MOE_OK)
+      cudaMemcpyAsync(out_host[i], outb[b], bytes, cudaMemcpyDeviceToHost, hp->d2h);
+    cudaEventRecord(hp->out_free[b], hp->d2h);
+  }
+  // The caller's stream reaches the end of every copy this call queued.
+  cudaEventRecord(hp->done, hp->d2h);
+  cudaStreamWaitEvent(st, hp->done, 0);
+  if (s != MOE_OK) return s;
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
 moe_status_t moe_get_device_status(void* stream) {

@@ -107,3 +107,28 @@ def test_no_cpu_fallback_in_product_package():
                     src = f.read()
                 assert "oracle" not in src.replace("oracle_", ""), fn
                 assert "moe_inputs" not in src, fn
+
+
+def test_host_pipeline_checks_on_host(lib):
+    c = abi_config(configs.MUSE_PREFILL)
+    n = moe.host_staging_size(c)
+    assert n == 4 * ((c.T * c.d_model * 2 + 255) // 256 * 256)
+    w = moe.Weights(w_router=0x1000, p_down=0x1000, p_up=0x1000, w_gu=0x1000, w_down=0x1000,
+                    gamma_pre=0x1000, gamma_expert=0x1000, resid_g=0x1000)
+    ptrs = (ctypes.c_void_p * 1)(0x1000)
+    code = moe.STATUS_CODES
+    f = lib.moe_layer_forward_host
+    assert f(ctypes.byref(c), ctypes.byref(w), -1, ptrs, ptrs, 0x1000, n, 0x1000, 1 << 34,
+             None) == code["MOE_ERR_INVALID_ARG"]
+    assert f(ctypes.byref(c), ctypes.byref(w), 1, None, ptrs, 0x1000, n, 0x1000, 1 << 34,
+             None) == code["MOE_ERR_INVALID_ARG"]
+    nulls = (ctypes.c_void_p * 1)(None)
+    assert f(ctypes.byref(c), ctypes.byref(w), 1, nulls, ptrs, 0x1000, n, 0x1000, 1 << 34,
+             None) == code["MOE_ERR_INVALID_ARG"]
+    assert f(ctypes.byref(c), ctypes.byref(w), 1, ptrs, ptrs, 0x1000, n - 1, 0x1000, 1 << 34,
+             None) == code["MOE_ERR_WORKSPACE"]
+    assert f(ctypes.byref(c), ctypes.byref(w), 1, ptrs, ptrs, 0x1008, n, 0x1000, 1 << 34,
+             None) == code["MOE_ERR_ALIGNMENT"]
+    # the layer's own checks run before anything is queued: a short workspace
+    assert f(ctypes.byref(c), ctypes.byref(w), 1, ptrs, ptrs, 0x1000, n, 0x1000, 16,
+             None) == code["MOE_ERR_WORKSPACE"]
