@@ -151,7 +151,11 @@ CONFIGS = {c.name: c for c in (TINY_SHAZEER_F32, SHAZEER_BF16, MUSE_DECODE, MUSE
 # decode: 2 per expert), i.e. the same per-tile work in every kernel.
 MUSE_PREFILL_N32 = MUSE_PREFILL.replace(name="muse_prefill_n32", T=2048, n_experts=32, seed=5)
 MUSE_DECODE_N32 = MUSE_DECODE.replace(name="muse_decode_n32", T=8, n_experts=32, seed=6)
-PROFILE_CONFIGS = {c.name: c for c in (MUSE_PREFILL_N32, MUSE_DECODE_N32)}
+# The prefill layer with 128-wide experts: the router, dispatch and combine kernels run at exactly
+# their prefill sizes (T=16384, d=8192, 256 experts, top-8, latent 4096) while the whole case
+# holds about 2.5 GB, small enough for a profiler capture of those kernels.
+MUSE_PREFILL_SMALLFFN = MUSE_PREFILL.replace(name="muse_prefill_smallffn", d_ff=128, seed=7)
+PROFILE_CONFIGS = {c.name: c for c in (MUSE_PREFILL_N32, MUSE_DECODE_N32, MUSE_PREFILL_SMALLFFN)}
 
 # The Muse router as the Muse audit describes it ("Latent experts"): fp32 router weights, sigmoid
 # scores, a selection-only correction bias ~ N(0, 0.05^2) (values not given on the pages),

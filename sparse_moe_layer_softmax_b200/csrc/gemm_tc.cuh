@@ -55,6 +55,9 @@ struct GemmParams {
   const float* sel_bias;     // EPI_ROUTER (sigmoid): selection-only correction bias [Nout]
   int x_k_period;            // > 0: X's k coordinate wraps every x_k_period columns (W's K is
                              // a multiple: the fp32 router weights' hi/mid/lo bf16 parts)
+  int router_select;         // EPI_ROUTER: 1 = select the top-k in the epilogue (logits, if
+                             // stored, are the payloads); 0 = only store the pre-activation
+                             // logits (output_multiplier * acc + bias) for a separate selection
   int tile_order;            // TILE_CHUNK_FASTEST | TILE_FEATURE_FASTEST
   int k_rotate;              // 1: each tile starts its reduction at its own k-block
   int out_tma;               // bf16 epilogues of the normal orientation: 1 = the output tensor
@@ -208,54 +211,27 @@ __device__ __forceinline__ int k_start(const TileCoord& c, int KB, int rotate) {
   return rotate ? (c.chunk + c.ft) % KB : 0;
 }
 
-template <int kMaxK>
-struct TopK {
-  float v[kMaxK];  // selection keys, descending
-  float s[kMaxK];  // payload carried with each key (the sigmoid score, or the logit)
-  int i[kMaxK];
-  __device__ __forceinline__ void init() {
-#pragma unroll
-    for (int j = 0; j < kMaxK; ++j) { v[j] = -INFINITY; s[j] = 0.0f; i[j] = -1; }
+// Router epilogue: selection key and payload of logit accumulator value `acc` at column `col`.
+// Softmax gate: the logit l = acc (+ bias) is both.  Muse sigmoid gate: the score
+// s = sigmoid(output_multiplier * acc (+ bias)) is the payload (what the weights are made of and
+// what logits_out returns in this mode) and s + correction bias (one fp32 addition, selection
+// only) the key.
+__device__ __forceinline__ float router_pre(const GemmParams& p, float acc, int col) {
+  const int c = col < p.Nout ? col : 0;
+  const float m = p.gate_mode == MOE_GATE_SIGMOID ? acc * p.logit_mult : acc;
+  return m + (p.bias ? p.bias[c] : 0.0f);
+}
+__device__ __forceinline__ void router_key(const GemmParams& p, float acc, int col, float& key,
+                                           float& pay) {
+  const int c = col < p.Nout ? col : 0;
+  const float l = router_pre(p, acc, col);
+  if (p.gate_mode == MOE_GATE_SIGMOID) {
+    pay = 1.0f / (1.0f + expf(-l));
+    key = pay + (p.sel_bias ? p.sel_bias[c] : 0.0f);
+  } else {
+    pay = l;
+    key = l;
   }
-  // Columns arrive in ascending index order; strict comparisons keep the lower index first
-  // among equal values.  Insertion into the sorted list of the k best (k <= kMaxK).
-  __device__ __forceinline__ void push(float x, float payload, int idx, int k) {
-    if (i[k - 1] >= 0 && !(x > v[k - 1])) return;
-#pragma unroll
-    for (int j = kMaxK - 1; j >= 0; --j) {
-      if (j >= k) continue;
-      const bool above = (j > 0) && (i[j - 1] < 0 || x > v[j - 1]);
-      if (above) {
-        v[j] = v[j - 1];
-        s[j] = s[j - 1];
-        i[j] = i[j - 1];
-      } else {
-        v[j] = x;
-        s[j] = payload;
-        i[j] = idx;
-        break;
-      }
-    }
-  }
-};
-
-// Routing weights of the selected k: softmax over the kept logits (= softmax over all, then
-// renormalised), or the Muse sigmoid gate's scores / (their sum + 1e-15); times routed_scale.
-template <int kMaxK>
-__device__ __forceinline__ void topk_weights(const TopK<kMaxK>& tk, int k, int gate_mode,
-                                             float routed_scale, float* w) {
-  float sum = 0.0f;
-#pragma unroll
-  for (int j = 0; j < kMaxK; ++j) {
-    float e = 0.0f;
-    if (j < k) e = gate_mode == MOE_GATE_SIGMOID ? tk.s[j] : __expf(tk.s[j] - tk.s[0]);
-    w[j] = e;
-    sum += e;
-  }
-  const float scale = gate_mode == MOE_GATE_SIGMOID ? routed_scale / (sum + 1e-15f)
-                                                    : routed_scale / sum;
-#pragma unroll
-  for (int j = 0; j < kMaxK; ++j) w[j] *= scale;
 }
 
 // Epilogue of the normal orientation: this thread owns row row0 + 32*q + lane of the tile (valid
@@ -269,48 +245,87 @@ __device__ __forceinline__ void epilogue_rows(const GemmParams& p, int row0, int
     const size_t row = static_cast<size_t>(row0 + rl);
     const int yblk = row0 + q * 32;  // first row of this warp's row block
     if constexpr (kEpi == EPI_ROUTER) {
-      TopK<8> tk;
-      tk.init();
-      for (int c0 = 0; c0 < BN; c0 += 16) {
-        float v[16];
-        tmem_ld16(tbase + c0, v);
+      // Logits out (when asked for): one pass over the row's accumulator columns.
+      if (p.logits) {
+        for (int c0 = 0; c0 < BN; c0 += 16) {
+          float v[16];
+          tmem_ld16(tbase + c0, v);
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int col = c0 + i;
-          if (col < p.Nout) {
-            if (p.gate_mode == MOE_GATE_SIGMOID) {
-              // score s = sigmoid(output_multiplier * l (+ bias)); selection key s + correction
-              // bias (one fp32 addition); the score is what the weights are made of and what
-              // logits_out returns in this mode
-              const float l = v[i] * p.logit_mult + (p.bias ? p.bias[col] : 0.0f);
-              const float sc = 1.0f / (1.0f + expf(-l));
-              const float key = sc + (p.sel_bias ? p.sel_bias[col] : 0.0f);
-              v[i] = sc;
-              tk.push(key, sc, col, p.top_k);
+          for (int i = 0; i < 16; ++i) {
+            if (p.router_select) {
+              float key;
+              router_key(p, v[i], c0 + i, key, v[i]);
             } else {
-              const float l = v[i] + (p.bias ? p.bias[col] : 0.0f);
-              v[i] = l;
-              tk.push(l, l, col, p.top_k);
+              v[i] = router_pre(p, v[i], c0 + i);
+            }
+          }
+          if (valid) {
+            float* dst = p.logits + row * p.Nout + c0;
+            if (c0 + 16 <= p.Nout && (p.Nout & 3) == 0) {
+#pragma unroll
+              for (int i = 0; i < 16; i += 4)
+                *reinterpret_cast<float4*>(dst + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+            } else {
+#pragma unroll
+              for (int i = 0; i < 16; ++i)
+                if (c0 + i < p.Nout) dst[i] = v[i];
             }
           }
         }
-        if (valid && p.logits) {
-          float* dst = p.logits + row * p.Nout + c0;
-          if (c0 + 16 <= p.Nout && (p.Nout & 3) == 0) {
+      }
+      // Top-k by k selection passes over the row (re-read from TMEM each pass): pass j takes the
+      // best entry in the order (key descending, column ascending) among those ranked after the
+      // previous pick.  That is the order of a stable descending sort, so ties keep the lower
+      // column first; the state is a few scalars per pass, all in registers.
+      if (!p.router_select) return;
+      float pick_pay[8];
+      int pick_col[8];
+      float prev_key = INFINITY;
+      int prev_col = -1;
 #pragma unroll
-            for (int i = 0; i < 16; i += 4)
-              *reinterpret_cast<float4*>(dst + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
-          } else {
-            for (int i = 0; c0 + i < p.Nout; ++i) dst[i] = v[i];
+      for (int j = 0; j < 8; ++j) {
+        pick_pay[j] = 0.0f;
+        pick_col[j] = -1;
+        if (j >= p.top_k) continue;
+        float bk = -INFINITY, bp = 0.0f;
+        int bc = 0x7fffffff;
+#pragma unroll 1
+        for (int c0 = 0; c0 < BN; c0 += 16) {
+          float v[16];
+          tmem_ld16(tbase + c0, v);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const int col = c0 + i;
+            float key, pay;
+            router_key(p, v[i], col, key, pay);
+            const bool after = key < prev_key || (key == prev_key && col > prev_col);
+            const bool better = key > bk || (key == bk && col < bc);
+            if (col < p.Nout && after && better) { bk = key; bc = col; bp = pay; }
           }
         }
+        pick_pay[j] = bp;
+        pick_col[j] = bc;
+        prev_key = bk;
+        prev_col = bc;
       }
       if (valid) {
-        float w[8];
-        topk_weights(tk, p.top_k, p.gate_mode, p.routed_scale, w);
-        for (int j = 0; j < p.top_k; ++j) {
-          p.topk_idx[row * p.top_k + j] = tk.i[j];
-          p.topk_w[row * p.top_k + j] = w[j];
+        // weights: softmax over the kept logits (= softmax over all, renormalised), or the
+        // sigmoid gate's scores / (their sum + 1e-15); times routed_scale
+        const bool sig = p.gate_mode == MOE_GATE_SIGMOID;
+        float e[8], sum = 0.0f;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          e[j] = 0.0f;
+          if (j < p.top_k) e[j] = sig ? pick_pay[j] : __expf(pick_pay[j] - pick_pay[0]);
+          sum += e[j];
+        }
+        const float scale = sig ? p.routed_scale / (sum + 1e-15f) : p.routed_scale / sum;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          if (j < p.top_k) {
+            p.topk_idx[row * p.top_k + j] = pick_col[j];
+            p.topk_w[row * p.top_k + j] = e[j] * scale;
+          }
         }
       }
     } else if constexpr (kEpi == EPI_SWIGLU) {

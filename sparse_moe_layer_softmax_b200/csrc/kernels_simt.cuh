@@ -179,9 +179,10 @@ __global__ void combine_bf16_kernel(const uint16_t* __restrict__ s, int E, int k
                                     const int32_t* __restrict__ inv_perm,
                                     const float* __restrict__ topk_w, int expert_norm, float eps,
                                     uint16_t* __restrict__ y) {
-  // Two passes over the k rows so that few registers are live and several CTAs share an SM:
-  // pass 1 reduces each row's sum of squares, pass 2 re-reads the rows (now in L1/L2) and
-  // accumulates the weighted, normalised values.
+  // One pass: every thread loads its VEC 16-byte vectors of all k rows at once (k x VEC loads in
+  // flight), keeps them in registers as packed bf16, and both the row norms and the weighted sum
+  // are taken from there.  Sum-of-squares order: per thread (vector, element), then the warp
+  // tree, then the warps in index order; accumulation of y in slot order.
   __shared__ float red[8][kMaxTopK];
   __shared__ int s_row[kMaxTopK];
   __shared__ float s_w[kMaxTopK], s_rinv[kMaxTopK];
@@ -195,23 +196,27 @@ __global__ void combine_bf16_kernel(const uint16_t* __restrict__ s, int E, int k
     s_rinv[j] = 1.0f;
   }
   __syncthreads();
+  uint4 q[kMaxTopK][VEC];
+#pragma unroll
+  for (int j = 0; j < kMaxTopK; ++j) {
+    const int row = s_row[j];
+    const uint4* src = reinterpret_cast<const uint4*>(s + static_cast<size_t>(row < 0 ? 0 : row) * E);
+#pragma unroll
+    for (int v = 0; v < VEC; ++v) {
+      const int vi = threadIdx.x + v * blockDim.x;
+      q[j][v] = (row >= 0 && vi < nvec) ? __ldg(src + vi) : make_uint4(0, 0, 0, 0);
+    }
+  }
   if (expert_norm) {
     float ss[kMaxTopK];
 #pragma unroll
     for (int j = 0; j < kMaxTopK; ++j) {
       ss[j] = 0.0f;
-      const int row = s_row[j];
-      if (row < 0) continue;
-      const uint4* src = reinterpret_cast<const uint4*>(s + static_cast<size_t>(row) * E);
 #pragma unroll
       for (int v = 0; v < VEC; ++v) {
-        const int vi = threadIdx.x + v * blockDim.x;
-        if (vi < nvec) {
-          const uint4 q = src[vi];
-          const uint16_t* h = reinterpret_cast<const uint16_t*>(&q);
+        const uint16_t* h = reinterpret_cast<const uint16_t*>(&q[j][v]);
 #pragma unroll
-          for (int i = 0; i < 8; ++i) { const float f = bf16_to_f32(h[i]); ss[j] += f * f; }
-        }
+        for (int i = 0; i < 8; ++i) { const float f = bf16_to_f32(h[i]); ss[j] += f * f; }
       }
     }
     const int w = threadIdx.x >> 5, nw = blockDim.x >> 5;
@@ -234,11 +239,10 @@ __global__ void combine_bf16_kernel(const uint16_t* __restrict__ s, int E, int k
     const int vi = threadIdx.x + v * blockDim.x;
     if (vi >= nvec) continue;
     float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-    for (int j = 0; j < k; ++j) {
-      const int row = s_row[j];
-      if (row < 0) continue;
-      const uint4 q = reinterpret_cast<const uint4*>(s + static_cast<size_t>(row) * E)[vi];
-      const uint16_t* h = reinterpret_cast<const uint16_t*>(&q);
+#pragma unroll
+    for (int j = 0; j < kMaxTopK; ++j) {
+      if (j >= k || s_row[j] < 0) continue;
+      const uint16_t* h = reinterpret_cast<const uint16_t*>(&q[j][v]);
       const float rj = s_rinv[j], wj = s_w[j];
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
@@ -374,9 +378,15 @@ __global__ void topk_rows_kernel(float* __restrict__ logits, int T, int n, int k
       }
     }
   }
+  // Loops over the k kept entries run to the compile-time bound kMaxTopK with k as a guard, so
+  // the arrays stay in registers.
   float top_s[kMaxTopK];
   int top_i[kMaxTopK];
-  for (int j = 0; j < k; ++j) {
+#pragma unroll
+  for (int j = 0; j < kMaxTopK; ++j) {
+    top_s[j] = 0.0f;
+    top_i[j] = 0;
+    if (j >= k) continue;  // warp-uniform
     float bv = -INFINITY, bs = 0.0f;
     int bi = 0x7fffffff;
 #pragma unroll
@@ -400,13 +410,19 @@ __global__ void topk_rows_kernel(float* __restrict__ logits, int T, int n, int k
   if (lane == 0) {
     float e[kMaxTopK];
     float sum = 0.0f;
-    for (int j = 0; j < k; ++j) {
-      e[j] = gate_mode == MOE_GATE_SIGMOID ? top_s[j] : __expf(top_s[j] - top_s[0]);
-      sum += e[j];
+#pragma unroll
+    for (int j = 0; j < kMaxTopK; ++j) {
+      e[j] = 0.0f;
+      if (j < k) {
+        e[j] = gate_mode == MOE_GATE_SIGMOID ? top_s[j] : __expf(top_s[j] - top_s[0]);
+        sum += e[j];
+      }
     }
     const float scale = gate_mode == MOE_GATE_SIGMOID ? routed_scale / (sum + 1e-15f)
                                                       : routed_scale / sum;
-    for (int j = 0; j < k; ++j) {
+#pragma unroll
+    for (int j = 0; j < kMaxTopK; ++j) {
+      if (j >= k) continue;
       topk_idx[static_cast<size_t>(t) * k + j] = top_i[j];
       topk_w[static_cast<size_t>(t) * k + j] = e[j] * scale;
     }
@@ -712,9 +728,15 @@ __global__ void router_f32_kernel(const float* __restrict__ u, const float* __re
       if (logits_out) logits_out[static_cast<size_t>(t) * n + e] = pay[i];
     }
   }
+  // Loops over the k kept entries run to the compile-time bound kMaxTopK with k as a guard, so
+  // the arrays stay in registers.
   float top_s[kMaxTopK];
   int top_i[kMaxTopK];
-  for (int j = 0; j < k; ++j) {
+#pragma unroll
+  for (int j = 0; j < kMaxTopK; ++j) {
+    top_s[j] = 0.0f;
+    top_i[j] = 0;
+    if (j >= k) continue;  // warp-uniform
     float bv = -INFINITY, bs = 0.0f;
     int bi = 0x7fffffff;
 #pragma unroll
@@ -738,12 +760,18 @@ __global__ void router_f32_kernel(const float* __restrict__ u, const float* __re
   if (lane == 0) {
     float e[kMaxTopK];
     float sum = 0.0f;
-    for (int j = 0; j < k; ++j) {
-      e[j] = gate_mode == MOE_GATE_SIGMOID ? top_s[j] : expf(top_s[j] - top_s[0]);
-      sum += e[j];
+#pragma unroll
+    for (int j = 0; j < kMaxTopK; ++j) {
+      e[j] = 0.0f;
+      if (j < k) {
+        e[j] = gate_mode == MOE_GATE_SIGMOID ? top_s[j] : expf(top_s[j] - top_s[0]);
+        sum += e[j];
+      }
     }
     const float denom = gate_mode == MOE_GATE_SIGMOID ? sum + 1e-15f : sum;
-    for (int j = 0; j < k; ++j) {
+#pragma unroll
+    for (int j = 0; j < kMaxTopK; ++j) {
+      if (j >= k) continue;
       topk_idx[static_cast<size_t>(t) * k + j] = top_i[j];
       topk_w[static_cast<size_t>(t) * k + j] = e[j] / denom * routed_scale;
     }

@@ -336,6 +336,10 @@ moe_status_t do_route(const moe_config_t& c, const void* u, const void* w_router
                                                     c.routed_scale, c.gate_mode, sel_bias, idx, w);
     return last_launch(2);
   }
+  // With a logits buffer (the caller's, or the layer's workspace) the GEMM only stores the
+  // pre-activation logits and a warp per token selects the top-k; without one, the GEMM's
+  // epilogue selects from the accumulators itself (k passes over each row).
+  const bool split = lbuf != nullptr;
   GemmParams p{};
   p.G = 1;
   p.M = c.T;
@@ -343,7 +347,8 @@ moe_status_t do_route(const moe_config_t& c, const void* u, const void* w_router
   p.x_k_period = c.router_f32 ? c.d_model : 0;
   p.Nw = c.n_experts;
   p.Nout = c.n_experts;
-  p.logits = logits;
+  p.logits = split ? lbuf : nullptr;
+  p.router_select = split ? 0 : 1;
   p.topk_idx = idx;
   p.topk_w = w;
   p.bias = bias;
@@ -354,7 +359,11 @@ moe_status_t do_route(const moe_config_t& c, const void* u, const void* w_router
   p.sel_bias = sel_bias;
   dense_schedule(p, c.T);
   const int bn = c.n_experts <= 32 ? 32 : c.n_experts <= 64 ? 64 : c.n_experts <= 128 ? 128 : 256;
-  return run_gemm(EPI_ROUTER, Orient::kNormal, bn, u, c.T, w_router, c.n_experts, p, st);
+  moe_status_t s = run_gemm(EPI_ROUTER, Orient::kNormal, bn, u, c.T, w_router, c.n_experts, p, st);
+  if (s != MOE_OK || !split) return s;
+  topk_rows_kernel<<<cdiv(c.T, 8), 256, 0, st>>>(lbuf, c.T, c.n_experts, c.top_k, c.routed_scale,
+                                                  c.gate_mode, sel_bias, idx, w);
+  return last_launch();
 }
 
 moe_status_t do_permute(const moe_config_t& c, const int32_t* idx, int32_t* offsets,

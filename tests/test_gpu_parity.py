@@ -340,3 +340,43 @@ def test_bounded_wait_runs_out_and_reports():
     # the device still runs work correctly afterwards
     cfg = configs.small_muse(T=40, d=256, L=128, I=128, n=16, k=4, seed=77)
     _check_layer(cfg)
+
+
+ROUTE_CASES = [
+    configs.small_shazeer(T=300, d=256, h=256, n=64, k=4, seed=71),
+    configs.small_muse(T=513, d=256, L=128, I=128, n=256, k=8, seed=72),
+    configs.small_muse(T=400, d=256, L=128, I=128, n=48, k=6, seed=73, gate_mode=configs.GATE_SIGMOID,
+                       logit_mult=1.5),
+    configs.MUSE_IMBALANCED.replace(T=700, seed=74),   # Zipf logit bias on the large-T path
+]
+
+
+@pytest.mark.parametrize("cfg", ROUTE_CASES, ids=lambda c: f"{c.name}-n{c.n_experts}-k{c.top_k}")
+def test_route_without_logits_buffer_matches(cfg):
+    """moe_route beyond the small-batch path: with a logits buffer the GEMM stores logits and a
+    warp per token selects; without one the GEMM epilogue selects from its accumulators.  Both
+    must give the same experts and the same weights, bit for bit, and the selection must be the
+    oracle's on the GPU's logits."""
+    import torch
+    dev = moe_inputs.device_inputs(cfg)
+    c = abi_config(cfg)
+    T, n, k = cfg.T, cfg.n_experts, cfg.top_k
+    bias = dev.get("logit_bias")
+    corr = dev.get("correction_bias")
+    logits = torch.empty((T, n), dtype=torch.float32, device="cuda")
+    idx1 = torch.empty((T, k), dtype=torch.int32, device="cuda")
+    w1 = torch.empty((T, k), dtype=torch.float32, device="cuda")
+    idx2, w2 = torch.empty_like(idx1), torch.empty_like(w1)
+    moe.moe_route(c, dev["u"], dev["w_router"], bias, logits, idx1, w1, correction_bias=corr)
+    moe.moe_route(c, dev["u"], dev["w_router"], bias, None, idx2, w2, correction_bias=corr)
+    torch.cuda.synchronize()
+    assert moe.moe_get_device_status() == 0
+    np.testing.assert_array_equal(idx2.cpu().numpy(), idx1.cpu().numpy())
+    np.testing.assert_array_equal(w2.cpu().numpy().view(np.int32), w1.cpu().numpy().view(np.int32))
+    lg = logits.cpu().numpy()
+    if cfg.gate_mode == configs.GATE_SIGMOID:
+        sel, wsel = oracle.sigmoid_topk_scores_f32(lg, k, corr.cpu().numpy(), cfg.routed_scale)
+    else:
+        sel, wsel = oracle.softmax_topk(lg, k)
+    np.testing.assert_array_equal(idx1.cpu().numpy(), sel)
+    np.testing.assert_allclose(w1.cpu().numpy(), wsel, rtol=2e-6, atol=1e-7)
