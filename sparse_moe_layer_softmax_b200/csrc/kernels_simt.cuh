@@ -174,16 +174,29 @@ __global__ void scatter_rows_f32_kernel(const float* __restrict__ x, int E, int 
 // One CTA per token: for each slot j the expert row s_j = out_perm[inv_perm[t,k+j]] is loaded,
 // its I_gamma denominator sqrt(mean(s_j^2) + eps) reduced in fp32, n_j = dtype(s_j / denom)
 // (when expert_norm), and y = dtype(sum_j w_j n_j) accumulated in fp32 in slot order.
+
+// The two bf16 values of a 32-bit word as floats (exact: a bf16 is the top half of an fp32).
+__device__ __forceinline__ float2 bf16x2_to_f2(uint32_t x) {
+  return make_float2(__uint_as_float(x << 16), __uint_as_float(x & 0xffff0000u));
+}
+// Two floats rounded to bf16 (round to nearest even), packed low/high.
+__device__ __forceinline__ uint32_t f2_to_bf16x2(float2 v) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(v.x, v.y);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+constexpr int kCombineMaxThreads = 512;
+
 template <int VEC>
-__global__ void combine_bf16_kernel(const uint16_t* __restrict__ s, int E, int k,
-                                    const int32_t* __restrict__ inv_perm,
-                                    const float* __restrict__ topk_w, int expert_norm, float eps,
-                                    uint16_t* __restrict__ y) {
+__global__ void __launch_bounds__(kCombineMaxThreads)
+    combine_bf16_kernel(const uint16_t* __restrict__ s, int E, int k,
+                        const int32_t* __restrict__ inv_perm, const float* __restrict__ topk_w,
+                        int expert_norm, float eps, uint16_t* __restrict__ y) {
   // One pass: every thread loads its VEC 16-byte vectors of all k rows at once (k x VEC loads in
-  // flight), keeps them in registers as packed bf16, and both the row norms and the weighted sum
-  // are taken from there.  Sum-of-squares order: per thread (vector, element), then the warp
-  // tree, then the warps in index order; accumulation of y in slot order.
-  __shared__ float red[8][kMaxTopK];
+  // flight) and keeps them as packed bf16; the row norms and the weighted sum both come from
+  // there.  The arithmetic runs on fp32 pairs (Blackwell's two-wide FMA / multiply), so each
+  // thread's sum of squares is two interleaved partial sums added at the end.
+  __shared__ float red[kCombineMaxThreads / 32][kMaxTopK];
   __shared__ int s_row[kMaxTopK];
   __shared__ float s_w[kMaxTopK], s_rinv[kMaxTopK];
   const int t = blockIdx.x;
@@ -211,13 +224,17 @@ __global__ void combine_bf16_kernel(const uint16_t* __restrict__ s, int E, int k
     float ss[kMaxTopK];
 #pragma unroll
     for (int j = 0; j < kMaxTopK; ++j) {
-      ss[j] = 0.0f;
+      float2 acc = make_float2(0.0f, 0.0f);
 #pragma unroll
       for (int v = 0; v < VEC; ++v) {
-        const uint16_t* h = reinterpret_cast<const uint16_t*>(&q[j][v]);
+        const uint32_t* w4 = reinterpret_cast<const uint32_t*>(&q[j][v]);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) { const float f = bf16_to_f32(h[i]); ss[j] += f * f; }
+        for (int i = 0; i < 4; ++i) {
+          const float2 f = bf16x2_to_f2(w4[i]);
+          acc = __ffma2_rn(f, f, acc);
+        }
       }
+      ss[j] = acc.x + acc.y;
     }
     const int w = threadIdx.x >> 5, nw = blockDim.x >> 5;
 #pragma unroll
@@ -238,24 +255,27 @@ __global__ void combine_bf16_kernel(const uint16_t* __restrict__ s, int E, int k
   for (int v = 0; v < VEC; ++v) {
     const int vi = threadIdx.x + v * blockDim.x;
     if (vi >= nvec) continue;
-    float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    float2 acc[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) acc[i] = make_float2(0.0f, 0.0f);
 #pragma unroll
     for (int j = 0; j < kMaxTopK; ++j) {
       if (j >= k || s_row[j] < 0) continue;
-      const uint16_t* h = reinterpret_cast<const uint16_t*>(&q[j][v]);
-      const float rj = s_rinv[j], wj = s_w[j];
+      const uint32_t* w4 = reinterpret_cast<const uint32_t*>(&q[j][v]);
+      const float2 r2 = make_float2(s_rinv[j], s_rinv[j]);
+      const float2 w2 = make_float2(s_w[j], s_w[j]);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const float sv = bf16_to_f32(h[i]);
-        const float nv = expert_norm ? round_bf16(sv * rj) : sv;
-        acc[i] += wj * nv;
+      for (int i = 0; i < 4; ++i) {
+        float2 nv = bf16x2_to_f2(w4[i]);
+        if (expert_norm) nv = bf16x2_to_f2(f2_to_bf16x2(__fmul2_rn(nv, r2)));  // dtype(s / denom)
+        acc[i] = __ffma2_rn(w2, nv, acc[i]);
       }
     }
     uint4 o;
-    o.x = pack_bf16x2(acc[0], acc[1]);
-    o.y = pack_bf16x2(acc[2], acc[3]);
-    o.z = pack_bf16x2(acc[4], acc[5]);
-    o.w = pack_bf16x2(acc[6], acc[7]);
+    o.x = f2_to_bf16x2(acc[0]);
+    o.y = f2_to_bf16x2(acc[1]);
+    o.z = f2_to_bf16x2(acc[2]);
+    o.w = f2_to_bf16x2(acc[3]);
     reinterpret_cast<uint4*>(y + static_cast<size_t>(t) * E)[vi] = o;
   }
 }

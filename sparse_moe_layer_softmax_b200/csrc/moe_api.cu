@@ -483,7 +483,7 @@ moe_status_t do_combine(const moe_config_t& c, const void* s, const int32_t* inv
     return last_launch();
   }
   const int nvec = E / 8;
-  const int threads = nvec >= 256 ? 256 : ((nvec + 31) / 32) * 32;
+  const int threads = nvec >= kCombineMaxThreads ? kCombineMaxThreads : ((nvec + 31) / 32) * 32;
   const int vec = cdiv(nvec, threads);
   const uint16_t* sp = static_cast<const uint16_t*>(s);
   uint16_t* yp = static_cast<uint16_t*>(y);
