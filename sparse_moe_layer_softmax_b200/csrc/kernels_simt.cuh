@@ -55,10 +55,19 @@ __global__ void perm_scan_kernel(int32_t* __restrict__ counts, int nchunks, int 
   const int e = threadIdx.x;
   int run = 0;
   if (e < n) {
-    for (int c = 0; c < nchunks; ++c) {
-      const int v = counts[c * n + e];
-      counts[c * n + e] = run;
-      run += v;
+    // batches of kB independent loads in flight, then the in-place exclusive prefix
+    constexpr int kB = 16;
+    for (int c0 = 0; c0 < nchunks; c0 += kB) {
+      int v[kB];
+#pragma unroll
+      for (int j = 0; j < kB; ++j) v[j] = c0 + j < nchunks ? counts[(c0 + j) * n + e] : 0;
+#pragma unroll
+      for (int j = 0; j < kB; ++j) {
+        if (c0 + j < nchunks) {
+          counts[(c0 + j) * n + e] = run;
+          run += v[j];
+        }
+      }
     }
   }
   // block-wide exclusive scan of run over e
@@ -77,27 +86,38 @@ __global__ void perm_scan_kernel(int32_t* __restrict__ counts, int nchunks, int 
   if (e == n - 1) offsets[n] = base + incl;
 }
 
-__global__ void perm_rank_kernel(const int32_t* __restrict__ idx, int T, int k, int n,
-                                 const int32_t* __restrict__ chunk_base,
-                                 const int32_t* __restrict__ offsets,
-                                 int32_t* __restrict__ perm_token, int32_t* __restrict__ inv_perm) {
-  __shared__ int s_idx[kPermChunk * kMaxTopK];
-  const int t0 = blockIdx.x * kPermChunk;
-  const int cnt = (min(T, t0 + kPermChunk) - t0) * k;
-  for (int i = threadIdx.x; i < cnt; i += blockDim.x) {
-    const int e = idx[static_cast<long>(t0) * k + i];
-    s_idx[i] = e;
-    if (e < 0 || e >= n) inv_perm[static_cast<long>(t0) * k + i] = -1;  // dropped slot
-  }
-  __syncthreads();
-  for (int e = threadIdx.x; e < n; e += blockDim.x) {
-    int row = offsets[e] + chunk_base[blockIdx.x * n + e];
-    for (int i = 0; i < cnt; ++i) {
-      if (s_idx[i] == e) {
-        perm_token[row] = t0 + i / k;
-        inv_perm[static_cast<long>(t0) * k + i] = row;
-        ++row;
-      }
+// One warp per chunk walks the chunk's slots in token-major order, 32 at a time: lanes holding
+// the same expert are ranked among themselves with a warp match, and a per-expert counter in
+// shared memory (starting at the expert's offset plus the rows of earlier chunks) carries the
+// next free row from one window to the next.  Slots with an expert outside [0, n) are dropped
+// (inv_perm = -1; the count kernel has latched MOE_ERR_DEVICE_CHECK).
+__global__ void __launch_bounds__(32)
+    perm_rank_kernel(const int32_t* __restrict__ idx, int T, int k, int n,
+                     const int32_t* __restrict__ chunk_base, const int32_t* __restrict__ offsets,
+                     int32_t* __restrict__ perm_token, int32_t* __restrict__ inv_perm) {
+  __shared__ int s_next[kMaxExperts];
+  const int lane = threadIdx.x;
+  const long t0 = static_cast<long>(blockIdx.x) * kPermChunk;
+  const int cnt = static_cast<int>((min(static_cast<long>(T), t0 + kPermChunk) - t0) * k);
+  for (int e = lane; e < n; e += 32) s_next[e] = offsets[e] + chunk_base[blockIdx.x * n + e];
+  __syncwarp();
+  const unsigned lower = (1u << lane) - 1u;
+  for (int w0 = 0; w0 < cnt; w0 += 32) {
+    const int i = w0 + lane;
+    const bool act = i < cnt;
+    const int e = act ? idx[t0 * k + i] : -1;
+    const bool ok = act && e >= 0 && e < n;
+    const unsigned m = __match_any_sync(0xffffffffu, ok ? e : -1 - lane);
+    int row = 0;
+    if (ok) row = s_next[e] + __popc(m & lower);
+    __syncwarp();
+    if (ok && (m & lower) == 0) s_next[e] += __popc(m);  // the group's first lane advances it
+    __syncwarp();
+    if (ok) {
+      perm_token[row] = static_cast<int32_t>(t0 + i / k);
+      inv_perm[t0 * k + i] = row;
+    } else if (act) {
+      inv_perm[t0 * k + i] = -1;
     }
   }
 }

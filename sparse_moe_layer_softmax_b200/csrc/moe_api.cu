@@ -376,7 +376,7 @@ moe_status_t do_permute(const moe_config_t& c, const int32_t* idx, int32_t* offs
   }
   perm_count_kernel<<<nc, 256, 0, st>>>(idx, c.T, k, n, counts);
   perm_scan_kernel<<<1, kMaxExperts, 0, st>>>(counts, nc, n, offsets);
-  perm_rank_kernel<<<nc, 256, 0, st>>>(idx, c.T, k, n, counts, offsets, perm, inv);
+  perm_rank_kernel<<<nc, 32, 0, st>>>(idx, c.T, k, n, counts, offsets, perm, inv);
   moe_status_t s = last_launch(3);
   if (s != MOE_OK || !x) return s;
   const int E = c.d_latent > 0 ? c.d_latent : c.d_model;
