@@ -229,9 +229,9 @@ def measured_peaks() -> dict:
 # launch scales by the same units: prefill by routed rows and experts (both 8x), decode by routed
 # experts.  Valid only for the kernel source the capture was taken on (fingerprint below).
 TRAFFIC_CAPTURES = {
-    "kernel_sha256_16": "cda9ed45040aa486",
-    "muse_prefill": {"bytes": 2.332767e9 + 0.130547456e9, "experts": 32, "rows": 2048 * 8},
-    "muse_decode": {"bytes": 1.947489e9 + 0.007632384e9, "experts": 29, "rows": 8 * 8},
+    "kernel_sha256_16": "0fd095b46b1c2877",
+    "muse_prefill": {"bytes": 2.331217e9 + 0.131040256e9, "experts": 32, "rows": 2048 * 8},
+    "muse_decode": {"bytes": 1.947527e9 + 0.005481216e9, "experts": 29, "rows": 8 * 8},
 }
 
 
