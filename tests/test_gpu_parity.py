@@ -380,3 +380,54 @@ def test_route_without_logits_buffer_matches(cfg):
         sel, wsel = oracle.softmax_topk(lg, k)
     np.testing.assert_array_equal(idx1.cpu().numpy(), sel)
     np.testing.assert_allclose(w1.cpu().numpy(), wsel, rtol=2e-6, atol=1e-7)
+
+
+STAGED_CASES = [
+    configs.small_muse(T=300, d=256, L=128, I=128, n=16, k=4, seed=81),
+    configs.small_muse(T=1000, d=256, L=256, I=256, n=8, k=2, seed=82),     # several chunks / expert
+    configs.small_shazeer(T=250, d=128, h=256, n=16, k=4, seed=83),         # ReLU, no latent
+    configs.MUSE_IMBALANCED.replace(T=700, seed=84),                        # Zipf-skewed groups
+]
+
+
+@pytest.mark.parametrize("cfg", STAGED_CASES, ids=lambda c: f"{c.name}-n{c.n_experts}")
+def test_layer_equals_staged_entry_points(cfg):
+    """moe_layer_forward against the same layer composed from the staged entry points (route,
+    latent down, permute with the row scatter, expert FFN, combine, latent up): the same output
+    bits (the fused call shares the workspace between stages; nothing else may differ)."""
+    import torch
+    dev = moe_inputs.device_inputs(cfg)
+    c = abi_config(cfg)
+    fused = run_layer(cfg, dev)["out"]
+    T, n, k = cfg.T, cfg.n_experts, cfg.top_k
+    E = cfg.expert_in
+    dt = fused.dtype
+    ws = torch.empty(moe.workspace_size(c), dtype=torch.uint8, device="cuda")
+    logits = torch.empty((T, n), dtype=torch.float32, device="cuda")
+    idx = torch.empty((T, k), dtype=torch.int32, device="cuda")
+    w = torch.empty((T, k), dtype=torch.float32, device="cuda")
+    moe.moe_route(c, dev["u"], dev["w_router"], dev.get("logit_bias"), logits, idx, w)
+    x = dev["u"]
+    if cfg.latent:
+        x = torch.empty((T, E), dtype=dt, device="cuda")
+        moe.moe_latent_down(c, dev["u"], dev["p_down"], x)
+    offsets = torch.empty(n + 1, dtype=torch.int32, device="cuda")
+    perm = torch.empty(T * k, dtype=torch.int32, device="cuda")
+    inv = torch.empty(T * k, dtype=torch.int32, device="cuda")
+    x_perm = torch.empty((T * k, E), dtype=dt, device="cuda")
+    moe.moe_permute(c, idx, offsets, perm, inv, x, dev.get("gamma_pre") if cfg.pre_norm else None,
+                    x_perm, ws)
+    s = torch.empty_like(x_perm)
+    moe.moe_expert_ffn(c, x_perm, offsets, dev["w_gu"], dev["w_down"],
+                       dev.get("gamma_expert") if cfg.expert_norm else None, s, ws)
+    y = torch.empty((T, E), dtype=dt, device="cuda")
+    moe.moe_combine(c, s, inv, w, y)
+    staged = y
+    if cfg.latent:
+        staged = torch.empty_like(fused)
+        moe.moe_latent_up(c, y, dev["p_up"], dev["u"], dev.get("resid_g"), staged)
+    torch.cuda.synchronize()
+    assert moe.moe_get_device_status() == 0
+    a = fused.view(torch.int16).cpu().numpy()
+    b = staged.view(torch.int16).cpu().numpy()
+    np.testing.assert_array_equal(a, b)
