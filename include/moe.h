@@ -184,19 +184,31 @@ MOE_API moe_status_t moe_permute_static(const moe_config_t* cfg, const int32_t* 
  *   SwiGLU: a = SiLU(x W_gate^T) * (x W_up^T) stored in dtype;  ReLU: a = ReLU(x W1^T);
  *   o = a W_down^T stored in dtype;  with expert_norm: out = dtype((1+gamma_expert) * o), the
  *   scaled vector that I_gamma reduces ([MUSE "Two normalization orders"]), else out = o.
- * out_perm: [T*k, E_in].  workspace holds the activation a. */
+ * out_perm: [T*k, E_in].  workspace holds the activation a.
+ * row_sumsq (optional, bf16 with expert_norm only, else ignored): [T*k, P] fp32 with P from
+ * moe_row_sumsq_parts; part p of row r is the sum of squares of out's bf16 values over one fixed
+ * block of its columns (the blocks partition the row), so that I_gamma's reduction
+ * mean(s^2) = (sum_p row_sumsq[r, p]) / E_in needs no second pass over the row (moe_combine). */
 MOE_API moe_status_t moe_expert_ffn(const moe_config_t* cfg, const void* x_perm,
                             const int32_t* expert_offsets, const void* w_gu, const void* w_down,
-                            const float* gamma_expert, void* out_perm, void* workspace,
-                            size_t workspace_bytes, void* stream);
+                            const float* gamma_expert, void* out_perm, float* row_sumsq,
+                            void* workspace, size_t workspace_bytes, void* stream);
+
+/* Number of partial sums of squares per row (P) that moe_expert_ffn writes to row_sumsq for this
+ * configuration (host arithmetic only). */
+MOE_API moe_status_t moe_row_sumsq_parts(const moe_config_t* cfg, int32_t* parts);
 
 /* Normalise and combine [MUSE "Latent experts" (normalise each expert output, then weight and
  * accumulate); SHAZEER "The math"]: for each token t,
  *   y_t = dtype( sum_j topk_w[t,j] * n_j ),  n_j = dtype(s_j / sqrt(mean(s_j^2) + eps)) with
  *   s_j = out_perm[inv_perm[t*k+j]] when expert_norm, else n_j = s_j;  fp32 accumulation in slot
- *   order.  y: [T, E_in]. */
-MOE_API moe_status_t moe_combine(const moe_config_t* cfg, const void* out_perm, const int32_t* inv_perm,
-                         const float* topk_w, void* y, void* stream);
+ *   order.  y: [T, E_in].
+ * row_sumsq (optional, bf16 with expert_norm): the partial sums of squares moe_expert_ffn wrote
+ * for out_perm; mean(s_j^2) is then their sum (in part order) / E_in instead of a reduction over
+ * the row here.  NULL: the reduction is done here. */
+MOE_API moe_status_t moe_combine(const moe_config_t* cfg, const void* out_perm,
+                                 const float* row_sumsq, const int32_t* inv_perm,
+                                 const float* topk_w, void* y, void* stream);
 
 /* Latent down-projection [MUSE "Latent experts"]: z_raw = dtype(u P_down^T), [T, d_latent]. */
 MOE_API moe_status_t moe_latent_down(const moe_config_t* cfg, const void* u, const void* p_down,

@@ -30,7 +30,8 @@ EXPORTS = ("moe_status_string", "moe_workspace_size", "moe_route", "moe_permute"
            "moe_layer_forward", "moe_get_device_status", "moe_profile_begin", "moe_profile_end",
            "moe_launch_count", "moe_permute_static", "moe_selftest_wait_timeout",
            "moe_router_split_weights", "moe_residual_update", "moe_noisy_gate",
-           "moe_noisy_gate_workspace_size", "moe_host_staging_size", "moe_layer_forward_host")
+           "moe_noisy_gate_workspace_size", "moe_host_staging_size", "moe_layer_forward_host",
+           "moe_row_sumsq_parts")
 PROFILE_STAGES = ("route", "latent_down", "dispatch", "expert_gate_up", "expert_down", "combine",
                   "latent_up_resgate")
 
@@ -83,8 +84,9 @@ def lib():
             "moe_noisy_gate_workspace_size": [cp, ctypes.POINTER(sz)],
             "moe_noisy_gate": [cp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp],
             "moe_permute": [cp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp],
-            "moe_expert_ffn": [cp, vp, vp, vp, vp, vp, vp, vp, sz, vp],
-            "moe_combine": [cp, vp, vp, vp, vp, vp],
+            "moe_expert_ffn": [cp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp],
+            "moe_combine": [cp, vp, vp, vp, vp, vp, vp],
+            "moe_row_sumsq_parts": [cp, ctypes.POINTER(ctypes.c_int32)],
             "moe_latent_down": [cp, vp, vp, vp, vp],
             "moe_latent_up": [cp, vp, vp, vp, vp, vp, vp],
             "moe_layer_forward": [cp, wp, vp, vp, vp, vp, vp, vp, vp, sz, vp],
@@ -219,19 +221,27 @@ def moe_permute_static(cfg, topk_idx, expert_offsets, perm_token, inv_perm, x=No
 
 
 def moe_expert_ffn(cfg, x_perm, expert_offsets, w_gu, w_down, gamma_expert, out_perm,
-                   workspace=None, workspace_bytes=0, stream=None):
+                   workspace=None, workspace_bytes=0, stream=None, row_sumsq=None):
     if workspace is not None and not workspace_bytes:
         workspace_bytes = workspace.numel() * workspace.element_size()
     _check("moe_expert_ffn", lib().moe_expert_ffn(ctypes.byref(cfg), _ptr(x_perm),
                                                   _ptr(expert_offsets), _ptr(w_gu), _ptr(w_down),
                                                   _ptr(gamma_expert), _ptr(out_perm),
-                                                  _ptr(workspace), workspace_bytes,
-                                                  _stream(stream)))
+                                                  _ptr(row_sumsq), _ptr(workspace),
+                                                  workspace_bytes, _stream(stream)))
 
 
-def moe_combine(cfg, out_perm, inv_perm, topk_w, y, stream=None):
-    _check("moe_combine", lib().moe_combine(ctypes.byref(cfg), _ptr(out_perm), _ptr(inv_perm),
-                                            _ptr(topk_w), _ptr(y), _stream(stream)))
+def row_sumsq_parts(cfg) -> int:
+    """Partial sums of squares per expert-output row that moe_expert_ffn writes to row_sumsq."""
+    n = ctypes.c_int32()
+    _check("moe_row_sumsq_parts", lib().moe_row_sumsq_parts(ctypes.byref(cfg), ctypes.byref(n)))
+    return n.value
+
+
+def moe_combine(cfg, out_perm, inv_perm, topk_w, y, stream=None, row_sumsq=None):
+    _check("moe_combine", lib().moe_combine(ctypes.byref(cfg), _ptr(out_perm), _ptr(row_sumsq),
+                                            _ptr(inv_perm), _ptr(topk_w), _ptr(y),
+                                            _stream(stream)))
 
 
 def moe_latent_down(cfg, u, p_down, z_raw, stream=None):

@@ -59,6 +59,8 @@ struct GemmParams {
                              // stored, are the payloads); 0 = only store the pre-activation
                              // logits (output_multiplier * acc + bias) for a separate selection
   int tile_order;            // TILE_CHUNK_FASTEST | TILE_FEATURE_FASTEST
+  float* row_ss;             // EPI_STORE (optional): [rows, ss_parts] partial sums of squares of
+  int ss_parts;              // the stored bf16 values, one per row and column block
   int k_rotate;              // 1: each tile starts its reduction at its own k-block
   int out_tma;               // bf16 epilogues of the normal orientation: 1 = the output tensor
                              // map is valid and whole-warp row blocks leave by TMA stores
@@ -389,6 +391,7 @@ __device__ __forceinline__ void epilogue_rows(const GemmParams& p, int row0, int
       }
     } else {
       uint16_t* out = static_cast<uint16_t*>(p.out) + row * p.Nout + f0;
+      float ss = 0.0f;  // EPI_STORE with row_ss: this row's sum of squares over the tile's columns
       for (int c0 = 0; c0 < BN; c0 += 64) {
         uint4 ch[8];
 #pragma unroll
@@ -404,10 +407,20 @@ __device__ __forceinline__ void epilogue_rows(const GemmParams& p, int row0, int
               for (int i = 0; i < 16; ++i)
                 v[i] = round_bf16(v[i]) * (1.0f + p.gamma[f0 + c0 + 16 * qq + i]);
             }
+            if (p.row_ss) {
+#pragma unroll
+              for (int i = 0; i < 16; ++i) {
+                const float b = round_bf16(v[i]);
+                ss = fmaf(b, b, ss);
+              }
+            }
           }
           pack8(v, ch[2 * qq], ch[2 * qq + 1]);
         }
         emit_chunk(eo, ch, out + c0, valid, f0 + c0, yblk, lane);
+      }
+      if constexpr (kEpi == EPI_STORE) {
+        if (p.row_ss && valid) p.row_ss[row * p.ss_parts + f0 / BN] = ss;
       }
     }
 }
@@ -601,7 +614,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
               const size_t row = static_cast<size_t>(c.row0 + j);
               float x = v[i];
               if constexpr (kEpi == EPI_RELU) x = fmaxf(x, 0.0f);
-              if constexpr (kEpi == EPI_STORE) { if (p.gamma) x = round_bf16(x) * gsc; }
+              if constexpr (kEpi == EPI_STORE) {
+                if (p.gamma) x = round_bf16(x) * gsc;
+                if (p.row_ss) {  // sum of squares over this warp's 32 features (fixed tree order)
+                  const float b = round_bf16(x);
+                  float sq = b * b;
+#pragma unroll
+                  for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
+                  if (lane == 0) p.row_ss[row * p.ss_parts + (f0 / 128) * 4 + q] = sq;
+                }
+              }
               if constexpr (kEpi == EPI_RESGATE) {
                 const float b = round_bf16(x);
                 if (p.resid_mode == MOE_RESID_NONE) x = b;

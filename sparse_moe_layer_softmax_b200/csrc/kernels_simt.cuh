@@ -300,6 +300,75 @@ __global__ void __launch_bounds__(kCombineMaxThreads)
   }
 }
 
+// The same combine when the expert GEMM has left each row's partial sums of squares in
+// row_ss [T*k, parts]: no reduction over the row and no block barrier.  In every warp, lane j < k
+// loads slot j's row index and weight and adds up its partials (in part order); the values reach
+// the other lanes by shuffles.
+template <int VEC>
+__global__ void __launch_bounds__(kCombineMaxThreads)
+    combine_bf16_ss_kernel(const uint16_t* __restrict__ s, int E, int k,
+                           const int32_t* __restrict__ inv_perm, const float* __restrict__ topk_w,
+                           const float* __restrict__ row_ss, int parts, float eps,
+                           uint16_t* __restrict__ y) {
+  const int t = blockIdx.x;
+  const int nvec = E / 8;
+  const int lane = threadIdx.x & 31;
+  int my_row = -1;
+  float my_w = 0.0f, my_rinv = 1.0f;
+  if (lane < k) {
+    my_row = __ldg(inv_perm + static_cast<size_t>(t) * k + lane);
+    if (my_row >= 0) {
+      my_w = __ldg(topk_w + static_cast<size_t>(t) * k + lane);
+      const float* ps = row_ss + static_cast<size_t>(my_row) * parts;
+      float tot = 0.0f;
+      for (int i = 0; i < parts; ++i) tot += __ldg(ps + i);
+      my_rinv = rsqrtf(tot / static_cast<float>(E) + eps);
+    }
+  }
+  int rows[kMaxTopK];
+  float wgt[kMaxTopK], rinv[kMaxTopK];
+#pragma unroll
+  for (int j = 0; j < kMaxTopK; ++j) {
+    rows[j] = __shfl_sync(0xffffffffu, my_row, j);
+    wgt[j] = __shfl_sync(0xffffffffu, my_w, j);
+    rinv[j] = __shfl_sync(0xffffffffu, my_rinv, j);
+  }
+#pragma unroll
+  for (int v = 0; v < VEC; ++v) {
+    const int vi = threadIdx.x + v * blockDim.x;
+    if (vi >= nvec) continue;
+    uint4 q[kMaxTopK];
+#pragma unroll
+    for (int j = 0; j < kMaxTopK; ++j) {
+      const int row = rows[j];
+      q[j] = (j < k && row >= 0)
+                 ? __ldg(reinterpret_cast<const uint4*>(s + static_cast<size_t>(row) * E) + vi)
+                 : make_uint4(0, 0, 0, 0);
+    }
+    float2 acc[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) acc[i] = make_float2(0.0f, 0.0f);
+#pragma unroll
+    for (int j = 0; j < kMaxTopK; ++j) {
+      if (j >= k || rows[j] < 0) continue;
+      const uint32_t* w4 = reinterpret_cast<const uint32_t*>(&q[j]);
+      const float2 r2 = make_float2(rinv[j], rinv[j]);
+      const float2 w2 = make_float2(wgt[j], wgt[j]);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float2 nv = bf16x2_to_f2(f2_to_bf16x2(__fmul2_rn(bf16x2_to_f2(w4[i]), r2)));
+        acc[i] = __ffma2_rn(w2, nv, acc[i]);
+      }
+    }
+    uint4 o;
+    o.x = f2_to_bf16x2(acc[0]);
+    o.y = f2_to_bf16x2(acc[1]);
+    o.z = f2_to_bf16x2(acc[2]);
+    o.w = f2_to_bf16x2(acc[3]);
+    reinterpret_cast<uint4*>(y + static_cast<size_t>(t) * E)[vi] = o;
+  }
+}
+
 __global__ void combine_f32_kernel(const float* __restrict__ s, int E, int k,
                                    const int32_t* __restrict__ inv_perm,
                                    const float* __restrict__ topk_w, int expert_norm, float eps,

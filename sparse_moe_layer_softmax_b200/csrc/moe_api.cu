@@ -233,8 +233,11 @@ size_t dsize(const moe_config_t& c) { return c.dtype == MOE_BF16 ? 2 : 4; }
 int nchunks(const moe_config_t& c) { return cdiv(c.T, kPermChunk); }
 
 struct Workspace {
-  size_t idx, w, logits, z_raw, offsets, perm, inv, counts, x_perm, act, y, u_norm, b, total;
+  size_t idx, w, logits, z_raw, offsets, perm, inv, counts, x_perm, act, y, u_norm, b, ss, total;
 };
+
+int sumsq_parts(const moe_config_t& c);
+constexpr int kMaxFusedSsParts = 32;  // moe_layer_forward passes row partials up to this many
 
 Workspace layout(const moe_config_t& c) {
   Workspace L{};
@@ -254,6 +257,7 @@ Workspace layout(const moe_config_t& c) {
   L.y = take(c.d_latent > 0 ? static_cast<size_t>(c.T) * E * ds : 0);
   L.u_norm = take(c.input_norm ? static_cast<size_t>(c.T) * c.d_model * ds : 0);
   L.b = take(c.post_norm ? static_cast<size_t>(c.T) * c.d_model * ds : 0);
+  L.ss = take(c.expert_norm && c.dtype == MOE_BF16 ? TK * sumsq_parts(c) * 4 : 0);
   L.total = o;
   return L;
 }
@@ -271,6 +275,8 @@ bool pair_tiles_enabled() {
 }
 
 // Grouped-GEMM orientation for the experts from the mean rows per expert.
+int expert_in_width(const moe_config_t& c) { return c.d_latent > 0 ? c.d_latent : c.d_model; }
+
 void pick_expert_orient(const moe_config_t& c, int nout, bool dual, Orient* o, int* bn) {
   const double mean_rows = static_cast<double>(c.T) * c.top_k / c.n_experts;
   if (nout % 128 == 0 && mean_rows <= 48.0) {
@@ -285,6 +291,17 @@ void pick_expert_orient(const moe_config_t& c, int nout, bool dual, Orient* o, i
 }
 
 // Dense projections: CTA-pair tiles for at least 256 rows and a 256-wide feature tile.
+// Partial sums of squares per expert-output row that the expert down GEMM writes (row_sumsq):
+// one per 256/128/64-column feature tile in the normal (and CTA-pair) orientation, one per
+// 32-feature warp slice of each 128-feature tile in the swapped orientation.
+int sumsq_parts(const moe_config_t& c) {
+  Orient o;
+  int bn;
+  pick_expert_orient(c, expert_in_width(c), false, &o, &bn);
+  if (bn <= 0) return 1;
+  return o == Orient::kSwap ? expert_in_width(c) / 128 * 4 : expert_in_width(c) / bn;
+}
+
 Orient dense_orient(int rows, int bn) {
   return (pair_tiles_enabled() && bn == 256 && rows >= 256) ? Orient::kPair : Orient::kNormal;
 }
@@ -427,7 +444,8 @@ void prof_next_call() {
 
 moe_status_t do_experts(const moe_config_t& c, const void* x_perm, const int32_t* offsets,
                         const void* w_gu, const void* w_down, const float* gamma_e,
-                        void* out_perm, void* act, cudaStream_t st, bool mark = false) {
+                        void* out_perm, void* act, cudaStream_t st, bool mark = false,
+                        float* row_ss = nullptr) {
   const long TK = static_cast<long>(c.T) * c.top_k;
   if (TK == 0) return MOE_OK;
   const int E = expert_in(c), H = c.d_ff, n = c.n_experts;
@@ -466,6 +484,8 @@ moe_status_t do_experts(const moe_config_t& c, const void* x_perm, const int32_t
   p2.Nout = E;
   p2.out = out_perm;
   p2.gamma = c.expert_norm ? gamma_e : nullptr;
+  p2.row_ss = c.expert_norm ? row_ss : nullptr;
+  p2.ss_parts = sumsq_parts(c);
   Orient o2;
   int bn2;
   pick_expert_orient(c, E, false, &o2, &bn2);
@@ -474,7 +494,7 @@ moe_status_t do_experts(const moe_config_t& c, const void* x_perm, const int32_t
 }
 
 moe_status_t do_combine(const moe_config_t& c, const void* s, const int32_t* inv,
-                        const float* w, void* y, cudaStream_t st) {
+                        const float* w, void* y, cudaStream_t st, const float* row_ss = nullptr) {
   if (c.T == 0) return MOE_OK;
   const int E = expert_in(c);
   if (c.dtype == MOE_F32) {
@@ -487,6 +507,17 @@ moe_status_t do_combine(const moe_config_t& c, const void* s, const int32_t* inv
   const int vec = cdiv(nvec, threads);
   const uint16_t* sp = static_cast<const uint16_t*>(s);
   uint16_t* yp = static_cast<uint16_t*>(y);
+  if (row_ss && c.expert_norm) {
+    const int parts = sumsq_parts(c);
+    switch (vec) {
+      case 1: combine_bf16_ss_kernel<1><<<c.T, threads, 0, st>>>(sp, E, c.top_k, inv, w, row_ss, parts, c.eps, yp); break;
+      case 2: combine_bf16_ss_kernel<2><<<c.T, threads, 0, st>>>(sp, E, c.top_k, inv, w, row_ss, parts, c.eps, yp); break;
+      case 3:
+      case 4: combine_bf16_ss_kernel<4><<<c.T, threads, 0, st>>>(sp, E, c.top_k, inv, w, row_ss, parts, c.eps, yp); break;
+      default: return MOE_ERR_UNSUPPORTED;
+    }
+    return last_launch();
+  }
   switch (vec) {
     case 1: combine_bf16_kernel<1><<<c.T, threads, 0, st>>>(sp, E, c.top_k, inv, w, c.expert_norm, c.eps, yp); break;
     case 2: combine_bf16_kernel<2><<<c.T, threads, 0, st>>>(sp, E, c.top_k, inv, w, c.expert_norm, c.eps, yp); break;
@@ -797,10 +828,18 @@ moe_status_t moe_permute_static(const moe_config_t* cfg, const int32_t* topk_idx
                     scratch, static_cast<cudaStream_t>(stream));
 }
 
+moe_status_t moe_row_sumsq_parts(const moe_config_t* cfg, int32_t* parts) {
+  if (!parts) return MOE_ERR_INVALID_ARG;
+  moe_status_t s = check_cfg(cfg);
+  if (s != MOE_OK) return s;
+  *parts = sumsq_parts(*cfg);
+  return MOE_OK;
+}
+
 moe_status_t moe_expert_ffn(const moe_config_t* cfg, const void* x_perm,
                             const int32_t* expert_offsets, const void* w_gu, const void* w_down,
-                            const float* gamma_expert, void* out_perm, void* workspace,
-                            size_t workspace_bytes, void* stream) {
+                            const float* gamma_expert, void* out_perm, float* row_sumsq,
+                            void* workspace, size_t workspace_bytes, void* stream) {
   moe_status_t s = check_cfg(cfg);
   if (s != MOE_OK) return s;
   const size_t TK = static_cast<size_t>(cfg->T) * cfg->top_k;
@@ -808,22 +847,26 @@ moe_status_t moe_expert_ffn(const moe_config_t* cfg, const void* x_perm,
     return MOE_ERR_INVALID_ARG;
   if (cfg->expert_norm && TK > 0 && !gamma_expert) return MOE_ERR_INVALID_ARG;
   if (!all_aligned({x_perm, static_cast<const void*>(expert_offsets), w_gu, w_down,
-                        static_cast<const void*>(gamma_expert), out_perm, workspace})) return MOE_ERR_ALIGNMENT;
+                        static_cast<const void*>(gamma_expert), out_perm,
+                        static_cast<const void*>(row_sumsq), workspace})) return MOE_ERR_ALIGNMENT;
   const size_t need = TK * cfg->d_ff * dsize(*cfg);
   if (cfg->dtype == MOE_BF16 && TK > 0 && (!workspace || workspace_bytes < need))
     return MOE_ERR_WORKSPACE;
   return do_experts(*cfg, x_perm, expert_offsets, w_gu, w_down, gamma_expert, out_perm, workspace,
-                    static_cast<cudaStream_t>(stream));
+                    static_cast<cudaStream_t>(stream), false,
+                    cfg->dtype == MOE_BF16 ? row_sumsq : nullptr);
 }
 
-moe_status_t moe_combine(const moe_config_t* cfg, const void* out_perm, const int32_t* inv_perm,
-                         const float* topk_w, void* y, void* stream) {
+moe_status_t moe_combine(const moe_config_t* cfg, const void* out_perm, const float* row_sumsq,
+                         const int32_t* inv_perm, const float* topk_w, void* y, void* stream) {
   moe_status_t s = check_cfg(cfg);
   if (s != MOE_OK) return s;
   if (cfg->T > 0 && (!out_perm || !inv_perm || !topk_w || !y)) return MOE_ERR_INVALID_ARG;
-  if (!all_aligned({out_perm, static_cast<const void*>(inv_perm),
-                        static_cast<const void*>(topk_w), static_cast<const void*>(y)})) return MOE_ERR_ALIGNMENT;
-  return do_combine(*cfg, out_perm, inv_perm, topk_w, y, static_cast<cudaStream_t>(stream));
+  if (!all_aligned({out_perm, static_cast<const void*>(row_sumsq),
+                    static_cast<const void*>(inv_perm), static_cast<const void*>(topk_w),
+                    static_cast<const void*>(y)})) return MOE_ERR_ALIGNMENT;
+  return do_combine(*cfg, out_perm, inv_perm, topk_w, y, static_cast<cudaStream_t>(stream),
+                    cfg->dtype == MOE_BF16 ? row_sumsq : nullptr);
 }
 
 moe_status_t moe_latent_down(const moe_config_t* cfg, const void* u, const void* p_down,
@@ -889,13 +932,18 @@ moe_status_t moe_layer_forward(const moe_config_t* cfg, const moe_weights_t* w, 
     return s;
   prof_mark(st, 3);
   // The expert output overwrites the dispatched input rows (no longer needed after GEMM 1).
+  // The down GEMM leaves each row's partial sums of squares for the combine's I_gamma norms when
+  // its tiles are the normal orientation (a few per row); the swapped orientation's many per-warp
+  // partials would cost the combine more than its own reduction.
+  float* row_ss = c.expert_norm && c.dtype == MOE_BF16 && sumsq_parts(c) <= kMaxFusedSsParts
+                      ? at<float>(workspace, L.ss) : nullptr;
   if ((s = do_experts(c, x_perm, offsets, w->w_gu, w->w_down, w->gamma_expert, x_perm, act, st,
-                      true)) != MOE_OK)
+                      true, row_ss)) != MOE_OK)
     return s;
   if (c.dtype == MOE_F32) prof_mark(st, 4);  // one fused kernel: all time in stage 3
   prof_mark(st, 5);
   void* y = latent ? at<void>(workspace, L.y) : out;
-  if ((s = do_combine(c, x_perm, inv, wt, y, st)) != MOE_OK) return s;
+  if ((s = do_combine(c, x_perm, inv, wt, y, st, row_ss)) != MOE_OK) return s;
   prof_mark(st, 6);
   if (latent && !c.post_norm &&
       (s = do_latent_up(c, y, w->p_up, r, w->resid_g, out, st)) != MOE_OK)

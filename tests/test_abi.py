@@ -132,3 +132,17 @@ def test_host_pipeline_checks_on_host(lib):
     # the layer's own checks run before anything is queued: a short workspace
     assert f(ctypes.byref(c), ctypes.byref(w), 1, ptrs, ptrs, 0x1000, n, 0x1000, 16,
              None) == code["MOE_ERR_WORKSPACE"]
+
+
+def test_row_sumsq_parts_is_host_arithmetic(lib):
+    # prefill: normal-orientation down GEMM, one partial per 256-column tile of the 4096-wide row;
+    # decode: swapped orientation, one per 32-feature warp slice of each 128-feature tile
+    assert moe.row_sumsq_parts(abi_config(configs.MUSE_PREFILL)) == 4096 // 256
+    assert moe.row_sumsq_parts(abi_config(configs.MUSE_DECODE)) == 4096 // 128 * 4
+    n = ctypes.c_int32()
+    c = abi_config(configs.MUSE_DECODE)
+    c.top_k = 0
+    assert lib.moe_row_sumsq_parts(ctypes.byref(c), ctypes.byref(n)) == \
+        moe.STATUS_CODES["MOE_ERR_INVALID_ARG"]
+    assert lib.moe_row_sumsq_parts(ctypes.byref(abi_config(configs.MUSE_DECODE)), None) == \
+        moe.STATUS_CODES["MOE_ERR_INVALID_ARG"]

@@ -242,10 +242,18 @@ def test_expert_ffn(cfg, monkeypatch):
     x = torch.from_numpy(xh.view(np.int16)).view(torch.bfloat16).cuda()
     out = torch.empty((T * k, E), dtype=torch.bfloat16, device="cuda")
     ws = torch.empty(moe.workspace_size(c), dtype=torch.uint8, device="cuda")
+    parts = moe.row_sumsq_parts(c)
+    ss = torch.full((T * k, parts), float("nan"), dtype=torch.float32, device="cuda")
     moe.moe_expert_ffn(c, x, torch.from_numpy(off).cuda(), dev["w_gu"], dev["w_down"],
-                       dev.get("gamma_expert"), out, workspace=ws)
+                       dev.get("gamma_expert"), out, workspace=ws,
+                       row_sumsq=ss if cfg.expert_norm else None)
     assert moe.moe_get_device_status() == 0
     got = device_values(out)
+    if cfg.expert_norm:
+        # the partials partition each row: their sum is the row's sum of squares of the stored
+        # bf16 values (fp32 sums of up to 256 terms each)
+        tot = ss.double().sum(1).cpu().numpy()
+        np.testing.assert_allclose(tot, (got * got).sum(1), rtol=2e-5, atol=1e-30)
     oc = oracle.make_cfg(cfg.replace(expert_norm=0))
     xv = host_values(xh, "bf16")
     errs = []
@@ -265,8 +273,11 @@ def test_expert_ffn(cfg, monkeypatch):
     assert np.concatenate(errs).max() <= 2e-2
 
 
+@pytest.mark.parametrize("with_ss", [False, True], ids=["reduce", "row_sumsq"])
 @pytest.mark.parametrize("E,k,norm", [(128, 4, 1), (4096, 8, 1), (512, 4, 0), (1024, 1, 1)])
-def test_combine(E, k, norm):
+def test_combine(E, k, norm, with_ss):
+    """Normalise + combine, with the row norms reduced in the kernel or taken from partial sums
+    of squares (here the host's: the whole row's sum in part 0, zeros in the others)."""
     T, n = 45, 16
     cfg = configs.small_muse(T=T, d=E, L=E, I=128, n=n, k=k, expert_norm=norm)
     c = abi_config(cfg)
@@ -276,8 +287,14 @@ def test_combine(E, k, norm):
     wr = moe_inputs.uniform_host(9, 61, 0, T * k).reshape(T, k).astype(np.float64) + 0.05
     wr = (wr / wr.sum(1, keepdims=True)).astype(np.float32)
     y = torch.empty((T, E), dtype=torch.bfloat16, device="cuda")
+    ss = None
+    if with_ss:
+        sv64 = host_values(sh, "bf16")
+        parts = np.zeros((T * k, moe.row_sumsq_parts(c)), dtype=np.float32)
+        parts[:, 0] = (sv64 * sv64).sum(1)
+        ss = torch.from_numpy(parts).cuda()
     moe.moe_combine(c, torch.from_numpy(sh.view(np.int16)).view(torch.bfloat16).cuda(),
-                    torch.from_numpy(inv).cuda(), torch.from_numpy(wr).cuda(), y)
+                    torch.from_numpy(inv).cuda(), torch.from_numpy(wr).cuda(), y, row_sumsq=ss)
     assert moe.moe_get_device_status() == 0
     sv = host_values(sh, "bf16")
     oc = oracle.make_cfg(cfg)
@@ -393,8 +410,9 @@ STAGED_CASES = [
 @pytest.mark.parametrize("cfg", STAGED_CASES, ids=lambda c: f"{c.name}-n{c.n_experts}")
 def test_layer_equals_staged_entry_points(cfg):
     """moe_layer_forward against the same layer composed from the staged entry points (route,
-    latent down, permute with the row scatter, expert FFN, combine, latent up): the same output
-    bits (the fused call shares the workspace between stages; nothing else may differ)."""
+    latent down, permute with the row scatter, expert FFN with its row partial sums of squares,
+    combine from those partials, latent up): the same output bits (the fused call shares the
+    workspace between stages; nothing else may differ)."""
     import torch
     dev = moe_inputs.device_inputs(cfg)
     c = abi_config(cfg)
@@ -418,10 +436,15 @@ def test_layer_equals_staged_entry_points(cfg):
     moe.moe_permute(c, idx, offsets, perm, inv, x, dev.get("gamma_pre") if cfg.pre_norm else None,
                     x_perm, ws)
     s = torch.empty_like(x_perm)
+    # the fused call takes the row partials when the down GEMM writes at most 32 per row (its
+    # normal-orientation tiles); otherwise the combine reduces the rows itself
+    parts = moe.row_sumsq_parts(c)
+    ss = torch.empty((T * k, parts), dtype=torch.float32, device="cuda") \
+        if cfg.expert_norm and parts <= 32 else None
     moe.moe_expert_ffn(c, x_perm, offsets, dev["w_gu"], dev["w_down"],
-                       dev.get("gamma_expert") if cfg.expert_norm else None, s, ws)
+                       dev.get("gamma_expert") if cfg.expert_norm else None, s, ws, row_sumsq=ss)
     y = torch.empty((T, E), dtype=dt, device="cuda")
-    moe.moe_combine(c, s, inv, w, y)
+    moe.moe_combine(c, s, inv, w, y, row_sumsq=ss)
     staged = y
     if cfg.latent:
         staged = torch.empty_like(fused)
