@@ -229,9 +229,9 @@ def measured_peaks() -> dict:
 # launch scales by the same units: prefill by routed rows and experts (both 8x), decode by routed
 # experts.  Valid only for the kernel source the capture was taken on (fingerprint below).
 TRAFFIC_CAPTURES = {
-    "kernel_sha256_16": "0fd095b46b1c2877",
-    "muse_prefill": {"bytes": 2.331217e9 + 0.131040256e9, "experts": 32, "rows": 2048 * 8},
-    "muse_decode": {"bytes": 1.947527e9 + 0.005481216e9, "experts": 29, "rows": 8 * 8},
+    "kernel_sha256_16": "9756377f992a1bf5",
+    "muse_prefill": {"bytes": 2.339689e9 + 0.130892544e9, "experts": 32, "rows": 2048 * 8},
+    "muse_decode": {"bytes": 1.947338e9 + 0.004237824e9, "experts": 29, "rows": 8 * 8},
 }
 
 
@@ -469,7 +469,9 @@ def default_cpu_sample(cfg) -> int:
     per_token_gmac = (cfg.d_model * cfg.n_experts + cfg.top_k * (cfg.gu_rows * cfg.expert_in +
                       cfg.expert_in * cfg.d_ff) + 2 * cfg.d_model * cfg.d_latent) / 1e9
     cores = os.cpu_count() or 1
-    n = int(15.0 * cores * 0.25 / max(per_token_gmac, 1e-6))  # ~0.25 GMAC/s per core
+    # the staged double-precision oracle does about 0.08 GMAC/s per core (measured: 127 prefill
+    # tokens in 46 s on 16 threads)
+    n = int(15.0 * cores * 0.08 / max(per_token_gmac, 1e-6))
     return int(max(cores, min(n, cfg.T, 4096)))
 
 
