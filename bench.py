@@ -50,6 +50,9 @@ def parse_args(argv=None):
     ap.add_argument("--no-decode", action="store_true", help="skip the secondary decode item")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample", type=int, default=0, help="tokens in the CPU oracle sample")
+    ap.add_argument("--expert-parallel", action="store_true",
+                    help="run the workload expert-parallel over the ranks (NCCL all-to-all): each "
+                         "rank holds n_experts / N experts and its own T tokens")
     a = ap.parse_args(argv)
     if a.warmup < 3:
         ap.error("at least 3 warm-up steps")
@@ -422,6 +425,110 @@ def measure_gate_stats(cfg, args, device) -> dict:
             "note": "includes the allocation of each call's outputs and workspace by the binding"}
 
 
+def ep_ranks(cfg, world: int, device, rank_ids=None):
+    """Expert-parallel ranks of `cfg` (cfg.T tokens per rank): rank r holds experts
+    expert_ranges(n, world)[r] of the whole layer's weights, and tokens [r T, (r+1) T) of a
+    world x T batch.  Returns (ranks, us) for rank_ids (all ranks by default)."""
+    import moe_inputs
+    from gpu_harness import abi_config
+    from sparse_moe_layer_softmax_b200 import expert_parallel as ep
+    dev = moe_inputs.device_inputs(cfg.replace(T=cfg.T * world), device=device)
+    ranges = ep.expert_ranges(cfg.n_experts, world)
+    ranks, us = [], []
+    for r in (range(world) if rank_ids is None else rank_ids):
+        lo, hi = ranges[r]
+        w = {k: v for k, v in dev.items() if k not in ("u", "w_gu", "w_down")}
+        w["w_gu"] = dev["w_gu"][lo:hi].clone()
+        w["w_down"] = dev["w_down"][lo:hi].clone()
+        ranks.append(ep.ExpertParallelRank(abi_config(cfg), w, r, world))
+        us.append(dev["u"][r * cfg.T:(r + 1) * cfg.T].clone())
+    del dev
+    return ranks, us
+
+
+def measure_ep_emulated(cfg, world: int, args, device, peaks: dict) -> dict:
+    """The compute of one rank of a `world`-GPU expert-parallel layer (cfg.T tokens per rank),
+    with every rank run on this GPU (the exchanges become slicing and concatenation).  Each stage
+    of each rank is timed with CUDA events; a rank's step is its dispatch + its experts' compute
+    on the rows all ranks sent it + its finish, and the slowest rank sets the step.  The NVLink
+    exchange is not measured: its lower bound is the rows each rank sends and receives over the
+    measured peer-copy bandwidth."""
+    import torch
+    from sparse_moe_layer_softmax_b200 import expert_parallel as ep
+    ranks, us = ep_ranks(cfg, world, device)
+    stream = torch.cuda.current_stream()
+    log = []
+
+    def timer(stage, r, fn):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        out = fn()
+        b.record(stream)
+        log.append((stage, r, a, b))
+        return out
+    for _ in range(args.warmup):
+        ep.emulated_forward(ranks, us)
+    torch.cuda.synchronize()
+    per_step = []
+    sent = []
+    for _ in range(args.steps):
+        log.clear()
+        ep.emulated_forward(ranks, us, timer=timer)
+        torch.cuda.synchronize()
+        t = np.zeros((3, world))
+        for stage, r, a, b in log:
+            t[("dispatch", "compute", "finish").index(stage), r] += a.elapsed_time(b)
+        per_step.append(t)
+    t = np.mean(per_step, axis=0)
+    rank_ms = t.sum(0)
+    # rows a rank sends to the other ranks (and receives back), one bf16 row of E_in each way
+    E = cfg.d_latent or cfg.d_model
+    xfer = cfg.T * cfg.top_k * (world - 1) / world * E * 2 * 2
+    link = 770e9
+    ms = float(rank_ms.max())
+    del ranks, us
+    torch.cuda.empty_cache()
+    return {"ranks": world, "tokens_per_rank": cfg.T,
+            "value_compute_only": round(cfg.T * world / (ms / 1e3), 2), "unit": UNIT,
+            "rank_compute_ms": round(ms, 4),
+            "stage_ms_max_over_ranks": {"dispatch": round(float(t[0].max()), 4),
+                                        "experts": round(float(t[1].max()), 4),
+                                        "finish": round(float(t[2].max()), 4)},
+            "exchange_bytes_per_rank": int(xfer),
+            "exchange_floor_ms": round(xfer / link * 1e3, 4),
+            "note": "one GPU runs every rank; times include each stage's host bookkeeping (the "
+                    "dispatch reads its expert counts back); the NVLink exchange is not measured "
+                    "(floor at the measured 770 GB/s peer copy)"}
+
+
+def measure_ep_dist(cfg, args, device, rank: int, world: int) -> dict:
+    """One rank of a real expert-parallel layer over torch.distributed (NCCL all-to-all between
+    the GPUs): cfg.T tokens and n_experts / world experts on each rank.  CUDA events around the
+    steps, max over ranks."""
+    import torch
+    from sparse_moe_layer_softmax_b200 import expert_parallel as ep
+    (er,), (u,) = ep_ranks(cfg, world, device, rank_ids=[rank])
+    exchange, counts = ep.dist_exchange(), ep.dist_exchange_counts(world)
+    for _ in range(args.warmup):
+        ep.forward(er, u, exchange, counts)
+    torch.cuda.synchronize()
+    barrier()
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        ep.forward(er, u, exchange, counts)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    ms = reduce_max(e0.elapsed_time(e1) / args.steps, device)
+    import sparse_moe_layer_softmax_b200 as moe
+    status = moe.moe_get_device_status()
+    if status != 0:
+        raise RuntimeError(f"device status {moe.STATUS.get(status, status)}")
+    return {"ms_per_step": ms}
+
+
 # ------------------------------------------------------------------ the CPU oracle as a baseline
 
 class OracleRunner:
@@ -562,6 +669,38 @@ def measure_checked(cfg, args, device, peaks, rank, local, with_e2e=True) -> dic
     return res
 
 
+def main_expert_parallel(cfg, args, device, rank: int, world: int) -> int:
+    """bench.py --expert-parallel: the layer expert-parallel over the ranks."""
+    import datetime
+    import socket
+    import torch.distributed as dist
+    if not dist.is_initialized():
+        # one rank: a one-member NCCL group, so that the same all-to-all path runs
+        with socket.socket() as s_:
+            s_.bind(("127.0.0.1", 0))
+            port = s_.getsockname()[1]
+        dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{port}", rank=0,
+                                world_size=1, timeout=datetime.timedelta(seconds=120))
+    res = measure_ep_dist(cfg, args, device, rank, world)
+    if rank == 0:
+        block = config_block(cfg, world)
+        block["parallelism"] = (f"expert parallel x{world}: each rank holds {cfg.n_experts // world} "
+                                f"experts and routes its own {cfg.T} tokens; NCCL all-to-all "
+                                "dispatch and return")
+        line = {"metric": METRIC, "value": round(cfg.T * world / (res["ms_per_step"] / 1e3), 2),
+                "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": round(res["ms_per_step"], 4), "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+                "data": "synthetic (seeded counter-based generator; random-init weights)",
+                "config": block}
+        print(json.dumps(line), flush=True)
+    import torch.distributed as dist
+    if dist.is_initialized():
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
 def main(argv=None) -> int:
     args = parse_args(argv)
     if args.impl == "reference":
@@ -574,6 +713,8 @@ def main(argv=None) -> int:
     init_dist("nccl")
     peaks = measured_peaks()
     cfg = configs.ALL_CONFIGS[args.workload]
+    if args.expert_parallel:
+        return main_expert_parallel(cfg, args, device, rank, world)
     res = measure_checked(cfg, args, device, peaks, rank, local)
     value = cfg.T * world / (res["ms_per_step"] / 1e3)
     line = {"metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
@@ -615,6 +756,11 @@ def main(argv=None) -> int:
     if not args.no_decode and cfg.name != "muse_decode":
         line.setdefault("variants", {})["shazeer_bf16_noisy_gate_stats"] = measure_gate_stats(
             configs.SHAZEER_BF16_NOISY, args, device)
+    if not args.no_decode and world == 1:
+        # the decode workload as one rank of an 8-GPU expert-parallel layer (64 tokens and 32
+        # experts per rank), every rank emulated on this GPU: the ranks' compute only
+        line.setdefault("variants", {})["muse_decode_ep8_emulated"] = measure_ep_emulated(
+            configs.MUSE_DECODE, 8, args, device, peaks)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(cfg, args.cpu_sample or default_cpu_sample(cfg))
     if rank == 0:

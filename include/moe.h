@@ -290,6 +290,17 @@ MOE_API moe_status_t moe_layer_forward_host(const moe_config_t* cfg, const moe_w
                                             size_t staging_bytes, void* workspace,
                                             size_t workspace_bytes, void* stream);
 
+/* Row gather [SHAZEER "Connecting the dots": the experts' batches pooled across devices], the
+ * data movement of an expert-parallel exchange (regrouping rows received from several ranks by
+ * expert, and back): dst[i, :] = src[rows[i], :] for i < n_rows, each row
+ * row_bytes long (a multiple of 16).  rows[i] < 0 writes a zero row; rows[i] >= src_rows latches
+ * MOE_ERR_DEVICE_CHECK and writes a zero row.  src, rows and dst are device pointers, 16-byte
+ * aligned; dst must not overlap src.  Errors: MOE_ERR_INVALID_ARG (NULL with n_rows > 0,
+ * negative sizes), MOE_ERR_UNSUPPORTED (row_bytes not a positive multiple of 16),
+ * MOE_ERR_ALIGNMENT. */
+MOE_API moe_status_t moe_gather_rows(const void* src, int64_t src_rows, const int32_t* rows,
+                                     int64_t n_rows, int64_t row_bytes, void* dst, void* stream);
+
 /* Synchronises the stream, returns and clears the device status word of the current device
  * (MOE_OK if no kernel latched an error since the last call). */
 MOE_API moe_status_t moe_get_device_status(void* stream);

@@ -31,7 +31,7 @@ EXPORTS = ("moe_status_string", "moe_workspace_size", "moe_route", "moe_permute"
            "moe_launch_count", "moe_permute_static", "moe_selftest_wait_timeout",
            "moe_router_split_weights", "moe_residual_update", "moe_noisy_gate",
            "moe_noisy_gate_workspace_size", "moe_host_staging_size", "moe_layer_forward_host",
-           "moe_row_sumsq_parts")
+           "moe_row_sumsq_parts", "moe_gather_rows")
 PROFILE_STAGES = ("route", "latent_down", "dispatch", "expert_gate_up", "expert_down", "combine",
                   "latent_up_resgate")
 
@@ -87,6 +87,7 @@ def lib():
             "moe_expert_ffn": [cp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp],
             "moe_combine": [cp, vp, vp, vp, vp, vp, vp],
             "moe_row_sumsq_parts": [cp, ctypes.POINTER(ctypes.c_int32)],
+            "moe_gather_rows": [vp, ctypes.c_int64, vp, ctypes.c_int64, ctypes.c_int64, vp, vp],
             "moe_latent_down": [cp, vp, vp, vp, vp],
             "moe_latent_up": [cp, vp, vp, vp, vp, vp, vp],
             "moe_layer_forward": [cp, wp, vp, vp, vp, vp, vp, vp, vp, sz, vp],
@@ -252,6 +253,15 @@ def moe_latent_down(cfg, u, p_down, z_raw, stream=None):
 def moe_latent_up(cfg, y, p_up, r, resid_g, out, stream=None):
     _check("moe_latent_up", lib().moe_latent_up(ctypes.byref(cfg), _ptr(y), _ptr(p_up), _ptr(r),
                                                 _ptr(resid_g), _ptr(out), _stream(stream)))
+
+
+def moe_gather_rows(src, rows, dst, stream=None):
+    """dst[i] = src[rows[i]] (rows of src's last dimension; rows[i] < 0 gives a zero row)."""
+    row_bytes = src.shape[-1] * src.element_size()
+    _check("moe_gather_rows", lib().moe_gather_rows(_ptr(src), src.shape[0], _ptr(rows),
+                                                    rows.numel(), row_bytes, _ptr(dst),
+                                                    _stream(stream)))
+    return dst
 
 
 def make_weights(w: dict) -> Weights:

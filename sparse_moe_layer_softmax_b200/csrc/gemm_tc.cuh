@@ -61,7 +61,6 @@ struct GemmParams {
   int tile_order;            // TILE_CHUNK_FASTEST | TILE_FEATURE_FASTEST
   float* row_ss;             // EPI_STORE (optional): [rows, ss_parts] partial sums of squares of
   int ss_parts;              // the stored bf16 values, one per row and column block
-  int k_rotate;              // 1: each tile starts its reduction at its own k-block
   int out_tma;               // bf16 epilogues of the normal orientation: 1 = the output tensor
                              // map is valid and whole-warp row blocks leave by TMA stores
 };
@@ -203,14 +202,6 @@ __device__ __forceinline__ TileCoord decode_tile(int t, const int* s_seg, const 
   int rem = s_seg[lo + 1] - c.row0;
   c.nrows = rem < CH ? rem : CH;
   return c;
-}
-
-// First k-block of a tile's reduction.  With k rotation on, tile (chunk, ft) starts at k-block
-// (chunk + ft) mod KB and wraps around, so CTAs that work at the same time on one weight tile
-// read different parts of it (no L2 hot spot on one k-block); the sum is the same up to the
-// order of the fp32 additions, and depends only on the tile, not on the CTA that runs it.
-__device__ __forceinline__ int k_start(const TileCoord& c, int KB, int rotate) {
-  return rotate ? (c.chunk + c.ft) % KB : 0;
 }
 
 // Router epilogue: selection key and payload of logit accumulator value `acc` at column `col`.
@@ -402,10 +393,16 @@ __device__ __forceinline__ void epilogue_rows(const GemmParams& p, int row0, int
 #pragma unroll
             for (int i = 0; i < 16; ++i) v[i] = fmaxf(v[i], 0.0f);
           } else if constexpr (kEpi == EPI_STORE) {
-            if (p.gamma) {
+            if (p.gamma) {  // 16 gains as four 16-byte loads (the column offset is a multiple of 16)
+              const float4* g4 = reinterpret_cast<const float4*>(p.gamma + f0 + c0 + 16 * qq);
 #pragma unroll
-              for (int i = 0; i < 16; ++i)
-                v[i] = round_bf16(v[i]) * (1.0f + p.gamma[f0 + c0 + 16 * qq + i]);
+              for (int i4 = 0; i4 < 4; ++i4) {
+                const float4 g = __ldg(g4 + i4);
+                v[4 * i4 + 0] = round_bf16(v[4 * i4 + 0]) * (1.0f + g.x);
+                v[4 * i4 + 1] = round_bf16(v[4 * i4 + 1]) * (1.0f + g.y);
+                v[4 * i4 + 2] = round_bf16(v[4 * i4 + 2]) * (1.0f + g.z);
+                v[4 * i4 + 3] = round_bf16(v[4 * i4 + 3]) * (1.0f + g.w);
+              }
             }
             if (p.row_ss) {
 #pragma unroll
@@ -510,14 +507,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
       TileCoord c = decode_tile(t, s_seg, s_pref, G, FT, S::kCH, p.tile_order);
       const int wrow = c.g * p.Nw + c.ft * S::kFO;
-      const int kb0 = k_start(c, KB, p.k_rotate);
       for (int kb = 0; kb < KB; ++kb) {
         if (!mbar_wait(&empty[stage], phase ^ 1)) { ok = false; break; }
         uint8_t* sa = tiles + stage * S::kStageBytes;
         uint8_t* sb = sa + S::kABytes;
         mbar_arrive_expect_tx(&full[stage], S::kStageBytes);
-        const int kbr = kb + kb0 < KB ? kb + kb0 : kb + kb0 - KB;
-        const int kx = kbr * S::kBK;
+        const int kx = kb * S::kBK;
         const int kxx = p.x_k_period > 0 ? kx % p.x_k_period : kx;  // X's k coordinate
         if (!kSwap) {
           tma_load_2d(&tmX, &full[stage], sa, kxx, c.row0);
@@ -774,15 +769,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       const int xrow = c.row0 + 128 * static_cast<int>(rank);
       const int wrow = S::kDual ? c.g * p.Nw + (leader ? 0 : p.Nw / 2) + c.ft * (BN / 2)
                                 : c.g * p.Nw + c.ft * BN + static_cast<int>(rank) * (BN / 2);
-      const int kb0 = k_start(c, KB, p.k_rotate);
       for (int kb = 0; kb < KB; ++kb) {
         if (!mbar_wait(&empty[stage], phase ^ 1)) { ok = false; break; }
         uint8_t* sa = tiles + stage * S::kStageBytes;
         uint8_t* sb = sa + S::kABytes;
         if (leader) mbar_arrive_expect_tx(&full[stage], 2 * S::kStageBytes);
         const uint32_t fb = cluster_addr(&full[stage], 0);
-        const int kbr = kb + kb0 < KB ? kb + kb0 : kb + kb0 - KB;
-        const int kx = kbr * S::kBK;
+        const int kx = kb * S::kBK;
         tma_load_2d_pair(&tmX, fb, sa, kx, xrow);
         tma_load_2d_pair(&tmW, fb, sb, kx, wrow);
         issued[stage] = true;

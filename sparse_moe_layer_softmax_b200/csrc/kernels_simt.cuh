@@ -122,6 +122,26 @@ __global__ void __launch_bounds__(32)
   }
 }
 
+// ------------------------------------------------------------------ row gather
+//
+// dst[i] = src[rows[i]] in 16-byte vectors, one CTA per row (grid-strided); a negative index
+// gives a zero row, an index past src_rows latches MOE_ERR_DEVICE_CHECK and gives a zero row.
+__global__ void gather_rows_kernel(const uint4* __restrict__ src, long src_rows,
+                                   const int32_t* __restrict__ rows, long n_rows, int row_vec,
+                                   uint4* __restrict__ dst) {
+  for (long i = blockIdx.x; i < n_rows; i += gridDim.x) {
+    int r = rows[i];
+    if (r >= src_rows) {
+      if (threadIdx.x == 0) latch_status(MOE_ERR_DEVICE_CHECK);
+      r = -1;
+    }
+    const uint4* s = src + static_cast<size_t>(r < 0 ? 0 : r) * row_vec;
+    uint4* d = dst + static_cast<size_t>(i) * row_vec;
+    for (int v = threadIdx.x; v < row_vec; v += blockDim.x)
+      d[v] = r >= 0 ? s[v] : make_uint4(0, 0, 0, 0);
+  }
+}
+
 // ------------------------------------------------------------------ row scatter (+ C_pre)
 //
 // One CTA per token: the row is read once, optionally normalised with the output-scaled centred

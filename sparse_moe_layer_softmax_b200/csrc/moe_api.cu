@@ -314,11 +314,10 @@ constexpr int kSmallRouterMaxT = 256;
 
 // Schedule of a dense projection (one group of x_rows rows against Nw weight rows): when the
 // activations outnumber the weight rows, feature tiles run fastest so each activation chunk is
-// read from HBM once while the weights stay in L2; every tile starts its reduction at its own
-// k-block so the CTAs sharing a weight tile do not all read the same k-block at once.
+// read from HBM once while the weights stay in L2.  (Every tile reduces over k in the same
+// order, so a token's result does not depend on where it sits in the batch.)
 void dense_schedule(GemmParams& p, long x_rows) {
   p.tile_order = x_rows > p.Nw ? TILE_FEATURE_FASTEST : TILE_CHUNK_FASTEST;
-  p.k_rotate = 1;
 }
 
 moe_status_t do_route(const moe_config_t& c, const void* u, const void* w_router,
@@ -1134,6 +1133,22 @@ moe_status_t moe_layer_forward_host(const moe_config_t* cfg, const moe_weights_t
   cudaStreamWaitEvent(st, hp->done, 0);
   if (s != MOE_OK) return s;
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+moe_status_t moe_gather_rows(const void* src, int64_t src_rows, const int32_t* rows,
+                             int64_t n_rows, int64_t row_bytes, void* dst, void* stream) {
+  if (n_rows < 0 || src_rows < 0 || row_bytes < 0) return MOE_ERR_INVALID_ARG;
+  if (row_bytes == 0 || row_bytes % 16 != 0) return MOE_ERR_UNSUPPORTED;
+  if (n_rows == 0) return MOE_OK;
+  if (!src || !rows || !dst) return MOE_ERR_INVALID_ARG;
+  if (!all_aligned({src, static_cast<const void*>(rows), dst})) return MOE_ERR_ALIGNMENT;
+  const int row_vec = static_cast<int>(row_bytes / 16);
+  const int threads = row_vec >= 256 ? 256 : ((row_vec + 31) / 32) * 32;
+  const long grid = std::min<long>(n_rows, 148L * 16);
+  gather_rows_kernel<<<static_cast<unsigned>(grid), threads, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint4*>(src), static_cast<long>(src_rows), rows, static_cast<long>(n_rows),
+      row_vec, static_cast<uint4*>(dst));
+  return last_launch();
 }
 
 moe_status_t moe_get_device_status(void* stream) {

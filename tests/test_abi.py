@@ -146,3 +146,15 @@ def test_row_sumsq_parts_is_host_arithmetic(lib):
         moe.STATUS_CODES["MOE_ERR_INVALID_ARG"]
     assert lib.moe_row_sumsq_parts(ctypes.byref(abi_config(configs.MUSE_DECODE)), None) == \
         moe.STATUS_CODES["MOE_ERR_INVALID_ARG"]
+
+
+def test_gather_rows_checks_on_host(lib):
+    code = moe.STATUS_CODES
+    f = lib.moe_gather_rows
+    assert f(0x1000, 4, 0x1000, -1, 64, 0x1000, None) == code["MOE_ERR_INVALID_ARG"]
+    assert f(0x1000, 4, 0x1000, 2, 24, 0x1000, None) == code["MOE_ERR_UNSUPPORTED"]
+    assert f(0x1000, 4, 0x1000, 2, 0, 0x1000, None) == code["MOE_ERR_UNSUPPORTED"]
+    assert f(None, 4, 0x1000, 2, 64, 0x1000, None) == code["MOE_ERR_INVALID_ARG"]
+    assert f(0x1000, 4, 0x1000, 2, 64, 0x1004, None) == code["MOE_ERR_ALIGNMENT"]
+    # nothing to gather: no launch, no pointer needed
+    assert f(None, 0, None, 0, 64, None, None) == code["MOE_OK"]
