@@ -232,9 +232,9 @@ def measured_peaks() -> dict:
 # launch scales by the same units: prefill by routed rows and experts (both 8x), decode by routed
 # experts.  Valid only for the kernel source the capture was taken on (fingerprint below).
 TRAFFIC_CAPTURES = {
-    "kernel_sha256_16": "9756377f992a1bf5",
-    "muse_prefill": {"bytes": 2.339689e9 + 0.130892544e9, "experts": 32, "rows": 2048 * 8},
-    "muse_decode": {"bytes": 1.947338e9 + 0.004237824e9, "experts": 29, "rows": 8 * 8},
+    "kernel_sha256_16": "1628c6b35ded1346",
+    "muse_prefill": {"bytes": 2.337346e9 + 0.131153152e9, "experts": 32, "rows": 2048 * 8},
+    "muse_decode": {"bytes": 1.947535e9 + 0.004344576e9, "experts": 29, "rows": 8 * 8},
 }
 
 
@@ -406,19 +406,21 @@ def measure_gate_stats(cfg, args, device) -> dict:
     dev = moe_inputs.device_inputs(cfg, device=device)
     c = abi_config(cfg)
     args_ = (c, dev["u"], dev["w_router"], dev["w_noise"], dev["noise_eps"])
+    # the same call as timed, so that the allocator's cache holds every buffer size it asks for;
+    # only the last call's outputs stay alive
+    out = None
     for _ in range(args.warmup):
-        moe.noisy_gate(*args_)
+        out = moe.noisy_gate(*args_, want_h=False, want_p=False)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    outs = []
     e0.record()
     for _ in range(args.steps):
-        outs.append(moe.noisy_gate(*args_, want_h=False, want_p=False))
+        out = moe.noisy_gate(*args_, want_h=False, want_p=False)
     e1.record()
     torch.cuda.synchronize()
     ms = reduce_max(e0.elapsed_time(e1) / args.steps, device)
-    cv2 = outs[-1]["cv2"].cpu().tolist()
-    del dev, outs
+    cv2 = out["cv2"].cpu().tolist()
+    del dev, out
     torch.cuda.empty_cache()
     return {"value": round(cfg.T / (ms / 1e3), 2), "unit": UNIT, "ms_per_step": round(ms, 4),
             "cv2_importance": cv2[0], "cv2_load": cv2[1],
