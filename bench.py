@@ -427,6 +427,53 @@ def measure_gate_stats(cfg, args, device) -> dict:
             "note": "includes the allocation of each call's outputs and workspace by the binding"}
 
 
+def measure_graph(cfg, args, device, peaks: dict) -> dict:
+    """The layer forward captured once in a CUDA graph and replayed K times (the host's launch
+    work leaves the step); CUDA events around the replays."""
+    import torch
+    import moe_inputs
+    import sparse_moe_layer_softmax_b200 as moe
+    from gpu_harness import abi_config
+    dev = moe_inputs.device_inputs(cfg, device=device)
+    layer = moe.MoELayer(abi_config(cfg), dev)
+    u = dev["u"]
+    out = torch.empty_like(u)
+    idx = torch.empty((cfg.T, cfg.top_k), dtype=torch.int32, device=device)
+    for _ in range(args.warmup):
+        layer.forward(u, u, out=out, topk_idx_out=idx)
+    torch.cuda.synchronize()
+    distinct = int(torch.unique(idx).numel())
+    g = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream(device=device)
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.graph(g, stream=side):
+        layer.forward(u, u, out=out)
+    torch.cuda.current_stream().wait_stream(side)
+    for _ in range(args.warmup):
+        g.replay()
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        g.replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = reduce_max(e0.elapsed_time(e1) / args.steps, device)
+    status = moe.moe_get_device_status()
+    if status != 0:
+        raise RuntimeError(f"device status {moe.STATUS.get(status, status)}")
+    work = work_model(cfg, distinct)
+    t_roof = max(work["flops"] / (peaks["bf16_tflops_sustained"] * 1e12),
+                 work["bytes"] / (peaks["hbm_gbs"] * 1e9))
+    del g, layer, dev
+    torch.cuda.empty_cache()
+    return {"value": round(cfg.T / (ms / 1e3), 2), "unit": UNIT, "ms_per_step": round(ms, 4),
+            "layer_roofline": {"roofline_ms": round(t_roof * 1e3, 4),
+                               "frac": round(t_roof * 1e3 / ms, 4)},
+            "note": "one forward captured in a CUDA graph, replayed K times"}
+
+
 def ep_ranks(cfg, world: int, device, rank_ids=None):
     """Expert-parallel ranks of `cfg` (cfg.T tokens per rank): rank r holds experts
     expert_ranges(n, world)[r] of the whole layer's weights, and tokens [r T, (r+1) T) of a
@@ -749,12 +796,16 @@ def main(argv=None) -> int:
         # decode with the Muse router as the Muse audit describes it (fp32 weights, sigmoid
         # gate), and the decoder layer's whole FFN sub-block (input norm, output norm)
         line["variants"] = {}
-        for vcfg in (configs.MUSE_DECODE_SIGMOID, configs.MUSE_DECODE_BLOCK):
+        for vcfg in (configs.MUSE_DECODE_SIGMOID, configs.MUSE_DECODE_BLOCK,
+                     configs.SHAZEER_BF16, configs.MUSE_IMBALANCED):
             vres = measure_checked(vcfg, args, device, peaks, rank, local, with_e2e=False)
             line["variants"][vcfg.name] = {
                 "value": round(vcfg.T * world / (vres["ms_per_step"] / 1e3), 2), "unit": UNIT,
                 "ms_per_step": round(vres["ms_per_step"], 4), "stage_ms": vres["stage_ms"],
                 "layer_roofline": vres["layer_roofline"], "clocks": vres["clocks"]}
+    if not args.no_decode and cfg.name != "muse_decode":
+        line["variants"]["muse_decode_cuda_graph"] = measure_graph(configs.MUSE_DECODE, args,
+                                                                   device, peaks)
     if not args.no_decode and cfg.name != "muse_decode":
         line.setdefault("variants", {})["shazeer_bf16_noisy_gate_stats"] = measure_gate_stats(
             configs.SHAZEER_BF16_NOISY, args, device)

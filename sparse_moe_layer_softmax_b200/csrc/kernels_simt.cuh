@@ -334,16 +334,10 @@ __global__ void __launch_bounds__(kCombineMaxThreads)
   const int nvec = E / 8;
   const int lane = threadIdx.x & 31;
   int my_row = -1;
-  float my_w = 0.0f, my_rinv = 1.0f;
+  float my_w = 0.0f;
   if (lane < k) {
     my_row = __ldg(inv_perm + static_cast<size_t>(t) * k + lane);
-    if (my_row >= 0) {
-      my_w = __ldg(topk_w + static_cast<size_t>(t) * k + lane);
-      const float* ps = row_ss + static_cast<size_t>(my_row) * parts;
-      float tot = 0.0f;
-      for (int i = 0; i < parts; ++i) tot += __ldg(ps + i);
-      my_rinv = rsqrtf(tot / static_cast<float>(E) + eps);
-    }
+    my_w = __ldg(topk_w + static_cast<size_t>(t) * k + lane);
   }
   int rows[kMaxTopK];
   float wgt[kMaxTopK], rinv[kMaxTopK];
@@ -351,27 +345,42 @@ __global__ void __launch_bounds__(kCombineMaxThreads)
   for (int j = 0; j < kMaxTopK; ++j) {
     rows[j] = __shfl_sync(0xffffffffu, my_row, j);
     wgt[j] = __shfl_sync(0xffffffffu, my_w, j);
-    rinv[j] = __shfl_sync(0xffffffffu, my_rinv, j);
   }
+  // The row loads go out first; the partial sums (and the norms) are fetched while they are in
+  // flight, so a token waits on two memory latencies, not three.
+  uint4 q[VEC][kMaxTopK];
+#pragma unroll
+  for (int v = 0; v < VEC; ++v) {
+    const int vi = threadIdx.x + v * blockDim.x;
+#pragma unroll
+    for (int j = 0; j < kMaxTopK; ++j) {
+      const int row = rows[j];
+      q[v][j] = (vi < nvec && j < k && row >= 0)
+                    ? __ldg(reinterpret_cast<const uint4*>(s + static_cast<size_t>(row) * E) + vi)
+                    : make_uint4(0, 0, 0, 0);
+    }
+  }
+  float my_rinv = 1.0f;
+  if (lane < k && my_row >= 0) {
+    const float* ps = row_ss + static_cast<size_t>(my_row) * parts;
+    float tot = 0.0f;
+    for (int i = 0; i < parts; ++i) tot += __ldg(ps + i);
+    my_rinv = rsqrtf(tot / static_cast<float>(E) + eps);
+  }
+#pragma unroll
+  for (int j = 0; j < kMaxTopK; ++j) rinv[j] = __shfl_sync(0xffffffffu, my_rinv, j);
 #pragma unroll
   for (int v = 0; v < VEC; ++v) {
     const int vi = threadIdx.x + v * blockDim.x;
     if (vi >= nvec) continue;
-    uint4 q[kMaxTopK];
-#pragma unroll
-    for (int j = 0; j < kMaxTopK; ++j) {
-      const int row = rows[j];
-      q[j] = (j < k && row >= 0)
-                 ? __ldg(reinterpret_cast<const uint4*>(s + static_cast<size_t>(row) * E) + vi)
-                 : make_uint4(0, 0, 0, 0);
-    }
+    const uint4 (&qv)[kMaxTopK] = q[v];
     float2 acc[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) acc[i] = make_float2(0.0f, 0.0f);
 #pragma unroll
     for (int j = 0; j < kMaxTopK; ++j) {
       if (j >= k || rows[j] < 0) continue;
-      const uint32_t* w4 = reinterpret_cast<const uint32_t*>(&q[j]);
+      const uint32_t* w4 = reinterpret_cast<const uint32_t*>(&qv[j]);
       const float2 r2 = make_float2(rinv[j], rinv[j]);
       const float2 w2 = make_float2(wgt[j], wgt[j]);
 #pragma unroll

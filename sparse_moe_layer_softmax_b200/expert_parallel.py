@@ -176,17 +176,26 @@ class ExpertParallelRank:
         import torch
         rows, local_offsets = regroup_rows(recv_counts)
         dev = recv.device
+        n = len(rows)
+        # the whole plan (regroup rows, their inverse, the local expert offsets) crosses to the
+        # device in one asynchronous copy from pinned memory; each part starts on a 16-byte
+        # boundary (the library's alignment rule)
+        m = (n + 3) // 4 * 4
+        plan = torch.zeros(2 * m + self.n_local + 1, dtype=torch.int32, pin_memory=True)
+        pv = plan.numpy()
+        pv[:n] = rows
+        pv[m:m + n] = inverse_rows(rows)
+        pv[2 * m:] = local_offsets
+        plan_d = plan.to(dev, non_blocking=True)
         grouped = torch.empty_like(recv)
-        rows_d = torch.from_numpy(rows).to(dev)
-        moe_gather_rows(recv, rows_d, grouped)
-        c = self._local_cfg(recv.shape[0])
+        moe_gather_rows(recv, plan_d[:n], grouped)
+        c = self._local_cfg(n)
         out = torch.empty_like(grouped)
         ws = torch.empty(workspace_size(c), dtype=torch.uint8, device=dev)
-        moe_expert_ffn(c, grouped, torch.from_numpy(local_offsets.astype(np.int32)).to(dev),
-                       self.weights["w_gu"], self.weights["w_down"],
+        moe_expert_ffn(c, grouped, plan_d[2 * m:], self.weights["w_gu"], self.weights["w_down"],
                        self.weights.get("gamma_expert") if self.cfg.expert_norm else None, out, ws)
         back = torch.empty_like(out)
-        moe_gather_rows(out, torch.from_numpy(inverse_rows(rows)).to(dev), back)
+        moe_gather_rows(out, plan_d[m:m + n], back)
         return back
 
     def finish(self, d: Dispatched, out_perm):
