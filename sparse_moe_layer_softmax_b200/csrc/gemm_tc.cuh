@@ -238,30 +238,32 @@ __device__ __forceinline__ void epilogue_rows(const GemmParams& p, int row0, int
     const size_t row = static_cast<size_t>(row0 + rl);
     const int yblk = row0 + q * 32;  // first row of this warp's row block
     if constexpr (kEpi == EPI_ROUTER) {
-      // Logits out (when asked for): one pass over the row's accumulator columns.
+      // Logits out (when asked for): one pass over the row's accumulator columns.  A tile holds
+      // experts [f0, f0 + BN): all of them when it selects (router_select), else possibly a part.
       if (p.logits) {
         for (int c0 = 0; c0 < BN; c0 += 16) {
           float v[16];
           tmem_ld16(tbase + c0, v);
+          const int g0 = f0 + c0;  // expert of accumulator column c0
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
             if (p.router_select) {
               float key;
-              router_key(p, v[i], c0 + i, key, v[i]);
+              router_key(p, v[i], g0 + i, key, v[i]);
             } else {
-              v[i] = router_pre(p, v[i], c0 + i);
+              v[i] = router_pre(p, v[i], g0 + i);
             }
           }
           if (valid) {
-            float* dst = p.logits + row * p.Nout + c0;
-            if (c0 + 16 <= p.Nout && (p.Nout & 3) == 0) {
+            float* dst = p.logits + row * p.Nout + g0;
+            if (g0 + 16 <= p.Nout && (p.Nout & 3) == 0) {
 #pragma unroll
               for (int i = 0; i < 16; i += 4)
                 *reinterpret_cast<float4*>(dst + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
             } else {
 #pragma unroll
               for (int i = 0; i < 16; ++i)
-                if (c0 + i < p.Nout) dst[i] = v[i];
+                if (g0 + i < p.Nout) dst[i] = v[i];
             }
           }
         }

@@ -96,16 +96,20 @@ __global__ void __launch_bounds__(32)
                      const int32_t* __restrict__ chunk_base, const int32_t* __restrict__ offsets,
                      int32_t* __restrict__ perm_token, int32_t* __restrict__ inv_perm) {
   __shared__ int s_next[kMaxExperts];
+  __shared__ int s_idx[kPermChunk * kMaxTopK];
   const int lane = threadIdx.x;
   const long t0 = static_cast<long>(blockIdx.x) * kPermChunk;
   const int cnt = static_cast<int>((min(static_cast<long>(T), t0 + kPermChunk) - t0) * k);
+  // the chunk's expert indices come in first, all loads in flight together; the ranking loop
+  // below then reads shared memory only
+  for (int i = lane; i < cnt; i += 32) s_idx[i] = idx[t0 * k + i];
   for (int e = lane; e < n; e += 32) s_next[e] = offsets[e] + chunk_base[blockIdx.x * n + e];
   __syncwarp();
   const unsigned lower = (1u << lane) - 1u;
   for (int w0 = 0; w0 < cnt; w0 += 32) {
     const int i = w0 + lane;
     const bool act = i < cnt;
-    const int e = act ? idx[t0 * k + i] : -1;
+    const int e = act ? s_idx[i] : -1;
     const bool ok = act && e >= 0 && e < n;
     const unsigned m = __match_any_sync(0xffffffffu, ok ? e : -1 - lane);
     int row = 0;

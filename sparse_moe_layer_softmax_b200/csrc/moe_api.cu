@@ -374,7 +374,13 @@ moe_status_t do_route(const moe_config_t& c, const void* u, const void* w_router
   p.logit_mult = mult;
   p.sel_bias = sel_bias;
   dense_schedule(p, c.T);
-  const int bn = c.n_experts <= 32 ? 32 : c.n_experts <= 64 ? 64 : c.n_experts <= 128 ? 128 : 256;
+  int bn = c.n_experts <= 32 ? 32 : c.n_experts <= 64 ? 64 : c.n_experts <= 128 ? 128 : 256;
+  // When only storing logits, a batch with few row tiles splits the experts over narrower
+  // tiles, so that more of the SMs take part (the selection that follows sees whole rows).
+  if (split) {
+    const long chunks = cdiv(c.T, 128);
+    while (bn > 32 && chunks * cdiv(c.n_experts, bn) * 2 <= device_info().sms) bn /= 2;
+  }
   moe_status_t s = run_gemm(EPI_ROUTER, Orient::kNormal, bn, u, c.T, w_router, c.n_experts, p, st);
   if (s != MOE_OK || !split) return s;
   topk_rows_kernel<<<cdiv(c.T, 8), 256, 0, st>>>(lbuf, c.T, c.n_experts, c.top_k, c.routed_scale,

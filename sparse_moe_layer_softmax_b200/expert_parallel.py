@@ -53,19 +53,14 @@ def regroup_rows(recv_counts: np.ndarray) -> tuple[np.ndarray, np.ndarray]:
     rows[g]; local_offsets [n_local + 1] are the experts' row offsets in the grouped order."""
     recv_counts = np.asarray(recv_counts, dtype=np.int64)
     world, n_local = recv_counts.shape
-    src_start = np.zeros((world, n_local), dtype=np.int64)  # received index of (src, expert) block
     flat = recv_counts.reshape(-1)
-    starts = np.concatenate([[0], np.cumsum(flat)[:-1]]).reshape(world, n_local)
-    src_start[:] = starts
-    rows = np.empty(int(flat.sum()), dtype=np.int32)
-    local_offsets = np.zeros(n_local + 1, dtype=np.int64)
-    g = 0
-    for e in range(n_local):
-        for s in range(world):
-            c = int(recv_counts[s, e])
-            rows[g:g + c] = np.arange(src_start[s, e], src_start[s, e] + c, dtype=np.int32)
-            g += c
-        local_offsets[e + 1] = g
+    # received index of each (source, expert) block, then the blocks in (expert, source) order
+    starts = (np.cumsum(flat) - flat).reshape(world, n_local).T.reshape(-1)
+    lens = recv_counts.T.reshape(-1)
+    total = int(lens.sum())
+    grouped_starts = np.cumsum(lens) - lens
+    rows = (np.repeat(starts - grouped_starts, lens) + np.arange(total)).astype(np.int32)
+    local_offsets = np.concatenate([[0], np.cumsum(recv_counts.sum(0))]).astype(np.int64)
     return rows, local_offsets
 
 
