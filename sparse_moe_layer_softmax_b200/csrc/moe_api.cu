@@ -37,7 +37,9 @@ DeviceInfo& device_info() {
   cudaGetDevice(&dev);
   std::lock_guard<std::mutex> lk(mu);
   DeviceInfo& d = info[dev & 63];
-  if (d.sms == 0) cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev);
+  if (d.sms <= 0 &&
+      cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    d.sms = 0;  // callers report MOE_ERR_CUDA rather than launch an empty grid
   return d;
 }
 
@@ -105,9 +107,10 @@ moe_status_t launch_gemm(const void* X, long x_rows, const void* W, long w_rows,
   CUtensorMap to = tx;
   q.out_tma = stages_output<kSwap, kEpi>() &&
               make_tmap(&to, p.out, static_cast<uint64_t>(x_rows), static_cast<uint64_t>(p.Nout), 32);
+  if (max_tiles <= 0) return MOE_OK;
   long grid = device_info().sms;
+  if (grid <= 0) return MOE_ERR_CUDA;  // the SM count could not be read
   if (max_tiles < grid) grid = max_tiles;
-  if (grid <= 0) return MOE_OK;
   kern<<<static_cast<unsigned>(grid), kGemmThreads, smem, st>>>(tx, tw, to, q);
   return last_launch();
 }
@@ -134,9 +137,10 @@ moe_status_t launch_gemm_pair(const void* X, long x_rows, const void* W, long w_
   GemmParams q = p;
   CUtensorMap to = tx;
   q.out_tma = make_tmap(&to, p.out, static_cast<uint64_t>(x_rows), static_cast<uint64_t>(p.Nout), 32);
+  if (max_tiles <= 0) return MOE_OK;
   long pairs = device_info().sms / 2;
+  if (pairs <= 0) return MOE_ERR_CUDA;  // the SM count could not be read
   if (max_tiles < pairs) pairs = max_tiles;
-  if (pairs <= 0) return MOE_OK;
   kern<<<static_cast<unsigned>(2 * pairs), kGemmThreads, smem, st>>>(tx, tw, to, q);
   return last_launch();
 }
@@ -517,18 +521,14 @@ moe_status_t do_combine(const moe_config_t& c, const void* s, const int32_t* inv
     switch (vec) {
       case 1: combine_bf16_ss_kernel<1><<<c.T, threads, 0, st>>>(sp, E, c.top_k, inv, w, row_ss, parts, c.eps, yp); break;
       case 2: combine_bf16_ss_kernel<2><<<c.T, threads, 0, st>>>(sp, E, c.top_k, inv, w, row_ss, parts, c.eps, yp); break;
-      case 3:
-      case 4: combine_bf16_ss_kernel<4><<<c.T, threads, 0, st>>>(sp, E, c.top_k, inv, w, row_ss, parts, c.eps, yp); break;
-      default: return MOE_ERR_UNSUPPORTED;
+      default: return MOE_ERR_UNSUPPORTED;  // E <= 8192: at most 2 vectors per thread
     }
     return last_launch();
   }
   switch (vec) {
     case 1: combine_bf16_kernel<1><<<c.T, threads, 0, st>>>(sp, E, c.top_k, inv, w, c.expert_norm, c.eps, yp); break;
     case 2: combine_bf16_kernel<2><<<c.T, threads, 0, st>>>(sp, E, c.top_k, inv, w, c.expert_norm, c.eps, yp); break;
-    case 3:
-    case 4: combine_bf16_kernel<4><<<c.T, threads, 0, st>>>(sp, E, c.top_k, inv, w, c.expert_norm, c.eps, yp); break;
-    default: return MOE_ERR_UNSUPPORTED;
+    default: return MOE_ERR_UNSUPPORTED;  // E <= 8192: at most 2 vectors per thread
   }
   return last_launch();
 }
@@ -753,7 +753,7 @@ moe_status_t moe_router_split_weights(const float* w, int32_t n, int32_t d, void
   if (!all_aligned({static_cast<const void*>(w), static_cast<const void*>(w_split)}))
     return MOE_ERR_ALIGNMENT;
   const size_t count = static_cast<size_t>(n) * d;
-  const unsigned blocks = static_cast<unsigned>(std::min<size_t>((count + 255) / 256, 148 * 16));
+  const unsigned blocks = static_cast<unsigned>(std::min<size_t>((count + 255) / 256, static_cast<size_t>(std::max(device_info().sms, 1)) * 16));
   router_split_kernel<<<blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(
       w, count, d, static_cast<uint16_t*>(w_split));
   return last_launch();
@@ -1150,7 +1150,7 @@ moe_status_t moe_gather_rows(const void* src, int64_t src_rows, const int32_t* r
   if (!all_aligned({src, static_cast<const void*>(rows), dst})) return MOE_ERR_ALIGNMENT;
   const int row_vec = static_cast<int>(row_bytes / 16);
   const int threads = row_vec >= 256 ? 256 : ((row_vec + 31) / 32) * 32;
-  const long grid = std::min<long>(n_rows, 148L * 16);
+  const long grid = std::min<long>(n_rows, static_cast<long>(std::max(device_info().sms, 1)) * 16);
   gather_rows_kernel<<<static_cast<unsigned>(grid), threads, 0, static_cast<cudaStream_t>(stream)>>>(
       static_cast<const uint4*>(src), static_cast<long>(src_rows), rows, static_cast<long>(n_rows),
       row_vec, static_cast<uint4*>(dst));

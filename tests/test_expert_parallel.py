@@ -105,3 +105,61 @@ def test_dispatch_and_return_over_gloo(world):
     for rank, (ok_range, ok_order, ok_offs, ok_back, n) in res.items():
         assert ok_range and ok_order and ok_offs and ok_back, (rank, res[rank])
     assert sum(v[4] for v in res.values()) == world * 40 * 3  # every dispatched row exchanged
+
+
+class _TaggedRank:
+    """A CPU stand-in for ExpertParallelRank with the same dispatch / compute / finish contract:
+    rows are integer tags (source rank, expert, token, slot) and an expert marks the rows it
+    processes, so forward()'s exchanges can be checked row by row on gloo ranks."""
+
+    def __init__(self, rank, world, n_experts, T, k):
+        self.rank, self.world, self.n, self.T, self.k = rank, world, n_experts, T, k
+        self.lo, self.hi = ep.expert_ranges(n_experts, world)[rank]
+
+    def dispatch(self, u):
+        rng = np.random.default_rng(200 + self.rank)
+        experts = np.stack([rng.choice(self.n, size=self.k, replace=False) for _ in range(self.T)])
+        slots = sorted((int(experts[t, j]), t, j) for t in range(self.T) for j in range(self.k))
+        offsets = np.searchsorted([e for e, _, _ in slots], np.arange(self.n + 1))
+        x_perm = torch.tensor([[self.rank, e, t, j] for e, t, j in slots], dtype=torch.int64)
+        return ep.Dispatched(u=u, w=None, inv=None, x_perm=x_perm,
+                             counts=ep.send_counts(offsets, self.world))
+
+    def compute(self, recv, recv_counts):
+        rows, offs = ep.regroup_rows(recv_counts)
+        grouped = recv.index_select(0, torch.from_numpy(rows).long())
+        for e in range(self.hi - self.lo):  # expert lo + e marks its rows
+            seg = grouped[offs[e]:offs[e + 1]]
+            assert bool((seg[:, 1] == self.lo + e).all())
+            seg[:, 3] += 100 * (self.lo + e + 1)
+        return grouped.index_select(0, torch.from_numpy(ep.inverse_rows(rows)).long())
+
+    def finish(self, d, out_perm):
+        return d.x_perm, out_perm
+
+
+def _forward_worker(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    import torch.distributed as dist
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        r = _TaggedRank(rank, world, n_experts=8, T=24, k=2)
+        sent, back = ep.forward(r, torch.zeros(24, 1), ep.dist_exchange(),
+                                ep.dist_exchange_counts(world))
+        s, b = sent.numpy(), back.numpy()
+        out[rank] = bool(np.array_equal(s[:, :3], b[:, :3]) and
+                         np.array_equal(b[:, 3] - 100 * (s[:, 1] + 1), s[:, 3]))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_forward_orchestration_over_gloo():
+    """expert_parallel.forward itself (counts exchange, dispatch, owner compute, return) between
+    two gloo ranks: every dispatched row comes back in its canonical place, processed once by the
+    expert it was routed to."""
+    world = 2
+    with mp.Manager() as m:
+        out = m.dict()
+        mp.spawn(_forward_worker, args=(world, _free_port(), out), nprocs=world, join=True)
+        res = dict(out)
+    assert res == {0: True, 1: True}
