@@ -257,7 +257,13 @@ def moe_latent_up(cfg, y, p_up, r, resid_g, out, stream=None):
 
 def moe_gather_rows(src, rows, dst, stream=None):
     """dst[i] = src[rows[i]] (rows of src's last dimension; rows[i] < 0 gives a zero row)."""
+    import torch
     row_bytes = src.shape[-1] * src.element_size()
+    if rows.dtype != torch.int32 or dst.shape[0] != rows.numel() or \
+            dst.shape[-1] * dst.element_size() != row_bytes or not src.is_contiguous() or \
+            not dst.is_contiguous() or not rows.is_contiguous():
+        raise ValueError("moe_gather_rows: int32 rows, contiguous src/dst with equal row bytes "
+                         "and one dst row per index")
     _check("moe_gather_rows", lib().moe_gather_rows(_ptr(src), src.shape[0], _ptr(rows),
                                                     rows.numel(), row_bytes, _ptr(dst),
                                                     _stream(stream)))
