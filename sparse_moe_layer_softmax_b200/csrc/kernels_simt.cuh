@@ -435,8 +435,10 @@ __global__ void combine_f32_kernel(const float* __restrict__ s, int E, int k,
 // the exact bf16 products are reduced across the warp.  A second kernel selects the top k.
 constexpr int kRouterTok = 8;
 constexpr int kRouterExp = 16;
+constexpr int kRouterThreads = 512;  // one warp per expert of the CTA
+constexpr int kRouterLoads = 4;      // weight vectors each lane keeps in flight
 
-__global__ void __launch_bounds__(256) router_logits_small_kernel(
+__global__ void __launch_bounds__(kRouterThreads, 1) router_logits_small_kernel(
     const uint16_t* __restrict__ u, const uint16_t* __restrict__ w, const float* __restrict__ bias,
     int T, int d, int n, int wk, float mult, float* __restrict__ logits) {
   // w rows have wk = d (bf16 weights) or 3d (hi/mid/lo parts of fp32 weights; u repeats)
@@ -459,19 +461,31 @@ __global__ void __launch_bounds__(256) router_logits_small_kernel(
 #pragma unroll
     for (int tt = 0; tt < kRouterTok; ++tt) acc[tt] = 0.0f;
     const int wvec = wk / 8;
-    for (int vw = lane; vw < wvec; vw += 32) {
-      const int v = vw % nvec;
-      const uint4 wq = wr[vw];
-      const uint16_t* wh = reinterpret_cast<const uint16_t*>(&wq);
-      float wf[8];
+    // kRouterLoads weight vectors per lane in flight at once; each lane still visits its vectors
+    // lane, lane + 32, ... in order, so the sums do not depend on the unrolling
+    for (int vw0 = lane; vw0 < wvec; vw0 += 32 * kRouterLoads) {
+      uint4 wq[kRouterLoads];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) wf[i] = bf16_to_f32(wh[i]);
+      for (int j = 0; j < kRouterLoads; ++j) {
+        const int vw = vw0 + 32 * j;
+        wq[j] = vw < wvec ? __ldg(wr + vw) : make_uint4(0, 0, 0, 0);
+      }
 #pragma unroll
-      for (int tt = 0; tt < kRouterTok; ++tt) {
-        const uint4 uq = s_u[tt * nvec + v];
-        const uint16_t* uh = reinterpret_cast<const uint16_t*>(&uq);
+      for (int j = 0; j < kRouterLoads; ++j) {
+        const int vw = vw0 + 32 * j;
+        if (vw >= wvec) break;
+        const int v = vw % nvec;
+        const uint16_t* wh = reinterpret_cast<const uint16_t*>(&wq[j]);
+        float wf[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) acc[tt] = fmaf(bf16_to_f32(uh[i]), wf[i], acc[tt]);
+        for (int i = 0; i < 8; ++i) wf[i] = bf16_to_f32(wh[i]);
+#pragma unroll
+        for (int tt = 0; tt < kRouterTok; ++tt) {
+          const uint4 uq = s_u[tt * nvec + v];
+          const uint16_t* uh = reinterpret_cast<const uint16_t*>(&uq);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) acc[tt] = fmaf(bf16_to_f32(uh[i]), wf[i], acc[tt]);
+        }
       }
     }
 #pragma unroll

@@ -171,6 +171,7 @@ moe_status_t run_gemm(int epi, Orient o, int bn, const void* X, long x_rows, con
     SW(16, EPI_SWIGLU, 6) SW(32, EPI_SWIGLU, 6) SW(64, EPI_SWIGLU, 5)
     SW(16, EPI_STORE, 10) SW(32, EPI_STORE, 9) SW(64, EPI_STORE, 8)
     SW(16, EPI_RELU, 10) SW(32, EPI_RELU, 9) SW(64, EPI_RELU, 8)
+    SW(16, EPI_RESGATE, 10) SW(32, EPI_RESGATE, 9) SW(64, EPI_RESGATE, 8)
 #undef SW
     return MOE_ERR_UNSUPPORTED;
   }
@@ -310,6 +311,25 @@ Orient dense_orient(int rows, int bn) {
   return (pair_tiles_enabled() && bn == 256 && rows >= 256) ? Orient::kPair : Orient::kNormal;
 }
 
+// Dense projection (latent down / up) over `rows` activation rows into `nout` features.  Up to
+// 256 rows the weight stream decides the time, and the normal orientation would spread it over
+// only Nout/256 tiles per 128-row chunk (16 CTAs for the 4096-wide latent at T=64).  The swapped
+// orientation puts 128 weight rows on the MMA's M side and the activation rows on N: Nout/128
+// tiles per chunk of BN rows.  BN is the widest of 64/32/16 that still gives two thirds of the
+// SMs a tile (narrower chunks re-read each weight tile from L2, not from HBM).
+void pick_dense(int rows, int nout, Orient* o, int* bn) {
+  if (rows <= 256 && nout % 128 == 0) {
+    *o = Orient::kSwap;
+    const long ft = nout / 128;
+    int b = 64;
+    while (b > 16 && (b / 2 >= rows || cdiv(rows, b) * ft * 3 < 2L * device_info().sms)) b /= 2;
+    *bn = b;
+    return;
+  }
+  *bn = pick_bn_normal(nout, false);
+  *o = dense_orient(rows, *bn);
+}
+
 // ------------------------------------------------------------------ steps
 
 // Tokens up to which the router runs as a many-CTA logits kernel + a top-k kernel (a single
@@ -349,7 +369,7 @@ moe_status_t do_route(const moe_config_t& c, const void* u, const void* w_router
     });
     if (attr != cudaSuccess) return MOE_ERR_CUDA;
     dim3 grid(cdiv(c.n_experts, kRouterExp), cdiv(c.T, kRouterTok));
-    router_logits_small_kernel<<<grid, 256, small_smem, st>>>(
+    router_logits_small_kernel<<<grid, kRouterThreads, small_smem, st>>>(
         static_cast<const uint16_t*>(u), static_cast<const uint16_t*>(w_router), bias, c.T,
         c.d_model, c.n_experts, wk, mult, lbuf);
     topk_rows_kernel<<<cdiv(c.T, 8), 256, 0, st>>>(lbuf, c.T, c.n_experts, c.top_k,
@@ -544,9 +564,11 @@ moe_status_t do_latent_down(const moe_config_t& c, const void* u, const void* p_
   p.Nout = c.d_latent;
   p.out = z;
   dense_schedule(p, c.T);
-  const int bn = pick_bn_normal(c.d_latent, false);
-  return run_gemm(EPI_STORE, dense_orient(c.T, bn), bn, u, c.T, p_down,
-                  c.d_latent, p, st);
+  Orient o;
+  int bn;
+  pick_dense(c.T, c.d_latent, &o, &bn);
+  if (bn == 0) return MOE_ERR_UNSUPPORTED;
+  return run_gemm(EPI_STORE, o, bn, u, c.T, p_down, c.d_latent, p, st);
 }
 
 moe_status_t do_latent_up(const moe_config_t& c, const void* y, const void* p_up, const void* r,
@@ -565,9 +587,11 @@ moe_status_t do_latent_up(const moe_config_t& c, const void* y, const void* p_up
   p.floor_ = c.resid_floor;
   p.resid_mode = c.resid_mode;
   dense_schedule(p, c.T);
-  const int bn = pick_bn_normal(c.d_model, false);
-  return run_gemm(EPI_RESGATE, dense_orient(c.T, bn), bn, y, c.T, p_up,
-                  c.d_model, p, st);
+  Orient o;
+  int bn;
+  pick_dense(c.T, c.d_model, &o, &bn);
+  if (bn == 0) return MOE_ERR_UNSUPPORTED;
+  return run_gemm(EPI_RESGATE, o, bn, y, c.T, p_up, c.d_model, p, st);
 }
 
 // Workspace of moe_noisy_gate: clean and noise logits, scratch routing of the two logit passes,
