@@ -232,9 +232,9 @@ def measured_peaks() -> dict:
 # launch scales by the same units: prefill by routed rows and experts (both 8x), decode by routed
 # experts.  Valid only for the kernel source the capture was taken on (fingerprint below).
 TRAFFIC_CAPTURES = {
-    "kernel_sha256_16": "c41c679957b46f75",
-    "muse_prefill": {"bytes": 2.373458e9 + 0.1326848e9, "experts": 32, "rows": 2048 * 8},
-    "muse_decode": {"bytes": 1.947337e9 + 0.00406528e9, "experts": 29, "rows": 8 * 8},
+    "kernel_sha256_16": "e441b6b39278f22f",
+    "muse_prefill": {"bytes": 2.327961e9 + 0.130886912e9, "experts": 32, "rows": 2048 * 8},
+    "muse_decode": {"bytes": 1.947475e9 + 0.004323584e9, "experts": 29, "rows": 8 * 8},
 }
 
 
