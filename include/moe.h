@@ -258,7 +258,10 @@ MOE_API moe_status_t moe_noisy_gate(const moe_config_t* cfg, const void* u, cons
  * is computed from r and this argument may be NULL), r: [T, d_model] the residual stream (may
  * equal u; ignored when resid_mode is NONE and input_norm is off), out: [T, d_model].
  * logits_out [T, n], topk_idx_out [T, k] and topk_w_out [T, k] are optional copies of the
- * routing. */
+ * routing.  The workspace holds every intermediate.  With T <= 64 (bf16, latent) the two latent
+ * projections split their reduction over k ranges and add the fp32 partials in a fixed order,
+ * so their results are deterministic but may differ in the last bit from moe_latent_down /
+ * moe_latent_up, which do not split. */
 MOE_API moe_status_t moe_layer_forward(const moe_config_t* cfg, const moe_weights_t* w, const void* u,
                                const void* r, void* out, float* logits_out,
                                int32_t* topk_idx_out, float* topk_w_out, void* workspace,
