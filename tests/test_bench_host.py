@@ -68,3 +68,19 @@ def test_default_cpu_sample_is_bounded():
     for cfg in configs.CONFIGS.values():
         n = bench.default_cpu_sample(cfg)
         assert 1 <= n <= max(cfg.T, os.cpu_count() or 1)
+
+
+def test_traffic_scales_the_capture_and_goes_null_for_another_kernel(monkeypatch):
+    """The bench's measured-traffic field: the capture case's DRAM bytes scaled by the units a full
+    launch processes (routed rows at prefill, routed experts at decode), and null as soon as the
+    kernel source differs from the one that was captured."""
+    caps = {"kernel_sha256_16": bench.kernel_fingerprint(),
+            "muse_prefill": {"bytes": 1.0e9, "experts": 32, "rows": 2048 * 8},
+            "muse_decode": {"bytes": 2.0e9, "experts": 29, "rows": 8 * 8}}
+    monkeypatch.setattr(bench, "TRAFFIC_CAPTURES", caps)
+    pf = configs.MUSE_PREFILL
+    assert bench.gate_up_traffic(pf, 256) == round(1.0e9 * pf.T * pf.top_k / (2048 * 8))
+    assert bench.gate_up_traffic(configs.MUSE_DECODE, 228) == round(2.0e9 * 228 / 29)
+    assert bench.gate_up_traffic(configs.SHAZEER_BF16, 256) is None  # no capture for it
+    monkeypatch.setitem(caps, "kernel_sha256_16", "0" * 16)
+    assert bench.gate_up_traffic(pf, 256) is None
