@@ -11,7 +11,10 @@ up-projection with the residual gate.  Rank 0 prints one JSON line.
   data-path collective), from CUDA events around K steps, max over ranks;
 * e2e: the same through the host-memory API (pinned host input -> device -> layer -> host, one
   pipelined moe_layer_forward_host call over the steps);
-* roofline: the dominant kernel (expert gate/up GEMM) timed live with the library's stage events;
+* ms_p50 / ms_p90: the median and 90th percentile of the per-step times of that timed region
+  (an event between consecutive steps);
+* roofline: the dominant kernel (expert gate/up GEMM) timed live with the library's stage events,
+  in a second pass of K steps (the headline pass runs the layer without them);
 * cpu_baseline: the CPU oracle on a bounded token sample of the same workload (rank 0, N=1);
 * decode: the T=64 Muse decode workload measured the same way (secondary line item).
 
@@ -228,7 +231,8 @@ def measured_peaks() -> dict:
 # ------------------------------------------------------------------ measured DRAM traffic
 
 # DRAM bytes (read + write) per launch of the expert gate/up GEMM from one ncu capture of each
-# reduced-expert case (profiles/gemm_gateup_muse_*_n32.md), with the units it processed.  A full
+# reduced-expert case (32 experts at the full workload's rows per expert), with the units it
+# processed.  A full
 # launch scales by the same units: prefill by routed rows and experts (both 8x), decode by routed
 # experts.  Valid only for the kernel source the capture was taken on (fingerprint below).
 TRAFFIC_CAPTURES = {
@@ -322,28 +326,37 @@ def measure_ours(cfg, steps: int, warmup: int, device, peaks: dict, with_e2e: bo
     loads = torch.bincount(idx.flatten().long(), minlength=cfg.n_experts)
     max_over_mean = float(loads.max().item()) / (cfg.T * cfg.top_k / cfg.n_experts)
 
-    # ---- device-resident timed region
+    # ---- device-resident timed region: the plain layer (no stage events inside a forward); an
+    # event between consecutive steps gives each step's duration as well as the total
     barrier()
     torch.cuda.synchronize()
     if sampler:
         sampler.start()
     launches0 = moe.launch_count()
-    moe.profile_begin(steps)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(steps):
+    marks = [torch.cuda.Event(enable_timing=True) for _ in range(steps + 1)]
+    marks[0].record(stream)
+    for i in range(steps):
         layer.forward(u, u, out=out, topk_idx_out=idx)
-    e1.record(stream)
+        marks[i + 1].record(stream)
     torch.cuda.synchronize()
-    stage_ms, calls = moe.profile_end()
     launches = moe.launch_count() - launches0
     clocks = sampler.stop() if sampler else None
     barrier()
-    ms = e0.elapsed_time(e1) / steps
+    per_step = [marks[i].elapsed_time(marks[i + 1]) for i in range(steps)]
+    ms = marks[0].elapsed_time(marks[steps]) / steps
     ms_max = reduce_max(ms, device)
+    p50 = reduce_max(float(np.percentile(per_step, 50)), device)
+    p90 = reduce_max(float(np.percentile(per_step, 90)), device)
     status = moe.moe_get_device_status()
     if status != 0:
         raise RuntimeError(f"device status {moe.STATUS.get(status, status)} after timing")
+
+    # ---- stage breakdown in a pass of its own: the library's per-stage events around each stage
+    moe.profile_begin(steps)
+    for _ in range(steps):
+        layer.forward(u, u, out=out, topk_idx_out=idx)
+    torch.cuda.synchronize()
+    stage_ms, calls = moe.profile_end()
 
     work = work_model(cfg, distinct)
     gate_up_s = stage_ms["expert_gate_up"] / max(calls, 1) / 1e3
@@ -361,7 +374,8 @@ def measure_ours(cfg, steps: int, warmup: int, device, peaks: dict, with_e2e: bo
                  work["bytes"] / (peaks["hbm_gbs"] * 1e9))
     t_exp = max(work["experts"]["flops"] / (peaks["bf16_tflops_sustained"] * 1e12),
                 work["experts"]["bytes"] / (peaks["hbm_gbs"] * 1e9))
-    res = {"ms_per_step": ms_max, "tokens_per_step": cfg.T, "roofline": roof,
+    res = {"ms_per_step": ms_max, "ms_p50": round(p50, 4), "ms_p90": round(p90, 4),
+           "tokens_per_step": cfg.T, "roofline": roof,
            "layer_roofline": {"bound": "tensor" if tensor_bound else "hbm",
                               "flops": work["flops"], "bytes": work["bytes"],
                               "roofline_ms": round(t_roof * 1e3, 4),
@@ -383,6 +397,7 @@ def measure_ours(cfg, steps: int, warmup: int, device, peaks: dict, with_e2e: bo
         layer.forward_host([u_host] * 2, [out_host] * 2, stream=stream)
         barrier()
         torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         layer.forward_host([u_host] * steps, [out_host] * steps, stream=stream)
         e1.record(stream)
@@ -655,6 +670,8 @@ def config_block(cfg, world: int) -> dict:
     return {"workload": cfg.name, "T": cfg.T, "d_model": cfg.d_model, "d_latent": cfg.d_latent,
             "d_ff": cfg.d_ff, "n_experts": cfg.n_experts, "top_k": cfg.top_k, "seed": cfg.seed,
             "global_batch": cfg.T * world,
+            "separated_inputs": {"redrawn_tokens": len(cfg.u_redraw),
+                                 "separation": "top-k margin >= 1e-3 rms of the router keys"},
             "parallelism": f"replicas x{world}: every rank runs the full workload",
             "l2": "no flush: every step streams the routed experts' weights (GBs) and activations "
                   "far larger than the 126 MB L2"}
@@ -768,7 +785,8 @@ def main(argv=None) -> int:
     value = cfg.T * world / (res["ms_per_step"] / 1e3)
     line = {"metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": round(res["ms_per_step"], 4), "higher_is_better": True,
+            "ms_per_step": round(res["ms_per_step"], 4),
+            "ms_p50": res["ms_p50"], "ms_p90": res["ms_p90"], "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded counter-based generator; random-init weights)",
             "config": config_block(cfg, world),
@@ -786,7 +804,7 @@ def main(argv=None) -> int:
         line["decode"] = {
             "workload": "muse_decode", "value": round(64 * world / (dres["ms_per_step"] / 1e3), 2),
             "unit": UNIT, "ms_per_step": round(dres["ms_per_step"], 4),
-            "roofline": dres["roofline"], "layer_roofline": dres["layer_roofline"],
+            "ms_p50": dres["ms_p50"], "ms_p90": dres["ms_p90"], "roofline": dres["roofline"], "layer_roofline": dres["layer_roofline"],
             "e2e": {"value": round(64 * world / (dres["e2e_ms"] / 1e3), 2), "unit": UNIT,
                     "h2d_bytes_per_step": dres["h2d_bytes"],
                     "d2h_bytes_per_step": dres["d2h_bytes"]},
@@ -801,7 +819,8 @@ def main(argv=None) -> int:
             vres = measure_checked(vcfg, args, device, peaks, rank, local, with_e2e=False)
             line["variants"][vcfg.name] = {
                 "value": round(vcfg.T * world / (vres["ms_per_step"] / 1e3), 2), "unit": UNIT,
-                "ms_per_step": round(vres["ms_per_step"], 4), "stage_ms": vres["stage_ms"],
+                "ms_per_step": round(vres["ms_per_step"], 4), "ms_p50": vres["ms_p50"],
+                "ms_p90": vres["ms_p90"], "stage_ms": vres["stage_ms"],
                 "layer_roofline": vres["layer_roofline"], "clocks": vres["clocks"]}
     if not args.no_decode and cfg.name != "muse_decode":
         line["variants"]["muse_decode_cuda_graph"] = measure_graph(configs.MUSE_DECODE, args,

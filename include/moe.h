@@ -267,6 +267,35 @@ MOE_API moe_status_t moe_layer_forward(const moe_config_t* cfg, const moe_weight
                                int32_t* topk_idx_out, float* topk_w_out, void* workspace,
                                size_t workspace_bytes, void* stream);
 
+/* Intermediate values of one whole-layer forward, copied out for verification (the intermediates
+ * the precision contract fixes [MUSE "Latent experts: normalization happens before the weighted
+ * sum", "What this means for serving and kernel work"]).  Every pointer is a caller-owned device
+ * buffer, or NULL to skip that value; E_in = d_latent, or d_model without latent projections.
+ *   z        [T, E_in]    each token's expert input as dispatched: dtype(C_pre(z_raw)) with
+ *                         pre_norm, z_raw = dtype(u P_down^T) without, or u (no latent).
+ *   s        [T*k, E_in]  each dispatched row's expert output before its norm: dtype((1+gamma) o)
+ *                         with expert_norm, else o; in dispatch order (token t's slot j is row
+ *                         inv_perm[t*k+j]).
+ *   y        [T, E_in]    the weighted combine y = dtype(sum_j w_j n_j).
+ *   inv_perm [T*k]        the dispatch row of every slot (int32). */
+typedef struct {
+  void* z;
+  void* s;
+  void* y;
+  int32_t* inv_perm;
+} moe_layer_taps_t;
+
+/* moe_layer_forward that also copies the intermediates named in *taps (taps may be NULL, which is
+ * moe_layer_forward itself).  The forward's kernels and their results are those of
+ * moe_layer_forward; each requested value adds one device-to-device copy (z: one gather kernel)
+ * on the stream after the stage that produces it.  Tap buffers must be 16-byte aligned and must not
+ * overlap any other argument. */
+MOE_API moe_status_t moe_layer_forward_taps(const moe_config_t* cfg, const moe_weights_t* w,
+                                            const void* u, const void* r, void* out,
+                                            float* logits_out, int32_t* topk_idx_out,
+                                            float* topk_w_out, const moe_layer_taps_t* taps,
+                                            void* workspace, size_t workspace_bytes, void* stream);
+
 /* Bytes of device staging moe_layer_forward_host needs for this configuration: two input and two
  * output buffers of T x d_model elements, each rounded up to 256 bytes. */
 MOE_API moe_status_t moe_host_staging_size(const moe_config_t* cfg, size_t* bytes);

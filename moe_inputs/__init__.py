@@ -7,6 +7,7 @@ them bit-identically on the CPU and on the GPU.  Nothing here computes any part 
 from __future__ import annotations
 
 import ctypes
+import functools
 import math
 import os
 import subprocess
@@ -193,10 +194,33 @@ def tensor_specs(cfg: MoEConfig):
     return specs
 
 
+@functools.lru_cache(maxsize=64)
+def _redraw_map(redraws: tuple) -> dict:
+    return dict(redraws)
+
+
+def u_row_first(cfg: MoEConfig, row: int) -> int:
+    """Counter index of the first element of row ``row`` of u (its latest redraw, if any)."""
+    g = _redraw_map(cfg.u_redraw).get(int(row), 0)
+    return (g * cfg.T + int(row)) * cfg.d_model
+
+
 def host_rows(cfg: MoEConfig, name: str, rows=None, lead: int | None = None) -> np.ndarray:
     """A generated tensor on the host.  ``rows`` selects rows of a 2-D tensor (e.g. sampled
-    tokens of u); ``lead`` selects one leading slice of a 3-D tensor (one expert's weights)."""
+    tokens of u); ``lead`` selects one leading slice of a 3-D tensor (one expert's weights).
+    Rows of u listed in the workload's redraw list come from their redraw."""
     shape, stream, kind, sigma = tensor_specs(cfg)[name]
+    if name == "u":
+        dt = cfg.dtype
+        width = shape[-1]
+        if rows is None:
+            full = normal_host(cfg.seed, stream, 0, math.prod(shape), sigma, dt).reshape(shape)
+            for t, _ in cfg.u_redraw:
+                full[t] = normal_host(cfg.seed, stream, u_row_first(cfg, t), width, sigma, dt)
+            return full
+        out = [normal_host(cfg.seed, stream, u_row_first(cfg, r), width, sigma, dt) for r in rows]
+        return np.stack(out) if out else np.empty((0, width), dtype=np.uint16 if dt == "bf16"
+                                                   else np.float32)
     if kind == "f32n":
         return normal_host(cfg.seed, stream, 0, math.prod(shape), sigma, "f32").reshape(shape)
     if kind == "f32u":
@@ -235,6 +259,9 @@ def device_inputs(cfg: MoEConfig, device="cuda") -> dict:
             t = torch.empty(shape, dtype=torch.bfloat16 if is_bf16 else torch.float32,
                             device=device)
             normal_device(t, cfg.seed, stream, 0, sigma)
+            if name == "u":
+                for row, _ in cfg.u_redraw:
+                    normal_device(t[row], cfg.seed, stream, u_row_first(cfg, row), sigma)
         out[name] = t
     if cfg.zipf_bias:
         out["logit_bias"] = torch.from_numpy(zipf_bias(cfg)).to(device)

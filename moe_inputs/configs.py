@@ -22,7 +22,9 @@ This module holds no layer arithmetic: only sizes, seeds and distributions.
 from __future__ import annotations
 
 import dataclasses
+import json
 import math
+import os
 
 # Stream identifiers: one independent counter stream per tensor (any distinct integers work).
 STREAM_X = 1
@@ -91,6 +93,10 @@ class MoEConfig:
     post_norm: int = 0          # decoder wrap: input-scaled output norm I_post on b before the gate
     eps_block: float = 1e-5     # epsilon of the decoder-level norms (model sheet: 1e-5)
     noisy_gate: bool = False    # Shazeer's noisy gate: W_noise ~ N(0, router std^2), eps ~ N(0, 1)
+    # Rows of u drawn again so that every token's router logits are separated at the top-k
+    # boundary: ((token, generation), ...).  Row t of generation g is counter elements
+    # [(g*T + t)*d, (g*T + t + 1)*d) of u's stream (generation 0 is the first draw).
+    u_redraw: tuple = ()
 
     @property
     def latent(self) -> bool:
@@ -107,6 +113,9 @@ class MoEConfig:
         return 2 * self.d_ff if self.act == ACT_SWIGLU else self.d_ff
 
     def replace(self, **kw) -> "MoEConfig":
+        """A derived workload.  A redraw list belongs to the one workload it was computed for,
+        so it is dropped unless given again."""
+        kw.setdefault("u_redraw", ())
         return dataclasses.replace(self, **kw)
 
     # ---- std of each generated tensor (N(0, 1/fan_in) weights) ----
@@ -193,3 +202,52 @@ def small_shazeer(T: int = 45, d: int = 128, h: int = 256, n: int = 16, k: int =
                   seed: int = 5, **kw) -> MoEConfig:
     return SHAZEER_BF16.replace(name=f"small_shazeer_T{T}", T=T, d_model=d, d_ff=h, n_experts=n,
                                 top_k=k, seed=seed, x_sigma=1.0 / math.sqrt(d), **kw)
+
+
+# ---------------------------------------------------------------------------------------------
+# Separated router logits.  The named workloads draw again every token of u whose k-th and
+# (k+1)-th router selection keys (the logits, or the sigmoid scores plus the correction bias)
+# are closer than SEPARATION * rms of that token's keys, so that the top-k selection is the same
+# in any summation order.  The redraw lists are computed with the CPU oracle's router by
+# tests/golden/separate_router_logits.py, which writes tests/golden/router_redraws.json; a CPU
+# test recomputes them.
+SEPARATION = 1e-3
+REDRAWS_PATH = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "tests",
+                            "golden", "router_redraws.json")
+
+
+def _load_redraws() -> dict:
+    if not os.path.exists(REDRAWS_PATH):
+        return {}
+    with open(REDRAWS_PATH) as f:
+        data = json.load(f)
+    return {name: tuple((int(t), int(g)) for t, g in w["redraws"])
+            for name, w in data["workloads"].items()}
+
+
+REDRAWS = _load_redraws()
+
+
+def separated(cfg: MoEConfig) -> MoEConfig:
+    """The named workload with its stored redraw list (unchanged if it has none)."""
+    return dataclasses.replace(cfg, u_redraw=REDRAWS.get(cfg.name, ()))
+
+
+TINY_SHAZEER_F32 = separated(TINY_SHAZEER_F32)
+SHAZEER_BF16 = separated(SHAZEER_BF16)
+MUSE_DECODE = separated(MUSE_DECODE)
+MUSE_PREFILL = separated(MUSE_PREFILL)
+MUSE_IMBALANCED = separated(MUSE_IMBALANCED)
+MUSE_DECODE_SIGMOID = separated(MUSE_DECODE_SIGMOID)
+MUSE_PREFILL_SIGMOID = separated(MUSE_PREFILL_SIGMOID)
+MUSE_DECODE_BLOCK = separated(MUSE_DECODE_BLOCK)
+MUSE_PREFILL_BLOCK = separated(MUSE_PREFILL_BLOCK)
+SEPARATED_NAMES = tuple(c.name for c in (TINY_SHAZEER_F32, SHAZEER_BF16, MUSE_DECODE, MUSE_PREFILL,
+                                         MUSE_IMBALANCED, MUSE_DECODE_SIGMOID,
+                                         MUSE_PREFILL_SIGMOID, MUSE_DECODE_BLOCK,
+                                         MUSE_PREFILL_BLOCK))
+CONFIGS = {c.name: c for c in (TINY_SHAZEER_F32, SHAZEER_BF16, MUSE_DECODE, MUSE_PREFILL,
+                               MUSE_IMBALANCED)}
+VARIANT_CONFIGS = {c.name: c for c in (MUSE_DECODE_SIGMOID, MUSE_PREFILL_SIGMOID,
+                                       MUSE_DECODE_BLOCK, MUSE_PREFILL_BLOCK)}
+ALL_CONFIGS = {**CONFIGS, **PROFILE_CONFIGS, **VARIANT_CONFIGS}

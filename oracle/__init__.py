@@ -73,6 +73,11 @@ def lib():
         L.orc_output_token.argtypes = [cp, tp, ctypes.c_int64, vp, vp]
         L.orc_layer_forward.argtypes = [cp, tp, vp, i32, vp, vp, vp, vp, vp, i32]
         L.orc_expert_batch.argtypes = [cp, vp, vp, vp, vp, i32, vp, i32]
+        L.orc_router_batch.argtypes = [cp, tp, vp, i32, vp, vp, vp, i32]
+        L.orc_expert_batch_parts.argtypes = [cp, vp, vp, vp, vp, i32, vp, vp, i32]
+        L.orc_expert_batch_parts.restype = None
+        L.orc_expert_token_scaled.argtypes = [cp, vp, vp, vp, vp, vp]
+        L.orc_input_scaled_vector.argtypes = [cp, vp, vp, i32, vp]
         L.orc_permutation.restype = i32
         L.orc_permutation.argtypes = [i32, i32, i32, vp, vp, vp, vp]
         L.orc_sigmoid_topk.argtypes = [vp, vp, i32, i32, dbl, vp, vp, vp]
@@ -83,7 +88,8 @@ def lib():
                   "orc_softmax_topk", "orc_softmax_topk_f32", "orc_resid_gate_coeffs",
                   "orc_router_token", "orc_expert_input_token", "orc_expert_token",
                   "orc_combine_token", "orc_output_token", "orc_layer_forward",
-                  "orc_expert_batch"):
+                  "orc_expert_batch", "orc_router_batch", "orc_expert_token_scaled",
+                  "orc_input_scaled_vector"):
             getattr(L, f).restype = None
         _lib = L
     return _lib
@@ -175,12 +181,15 @@ def layer_forward(cfg, inp: dict, tokens=None, nthreads: int | None = None) -> d
     return {"out": out, "logits": logits, "idx": idx, "w": w, "y": y, "tokens": tokens}
 
 
-def layer_forward_staged(cfg, tokens, get_inputs, get_expert, nthreads: int | None = None) -> dict:
+def layer_forward_staged(cfg, tokens, get_inputs, get_expert, nthreads: int | None = None,
+                         want_s: bool = False) -> dict:
     """The same per-token arithmetic as ``layer_forward`` with expert weights held one expert at a
     time: route and build expert inputs for every listed token, evaluate each expert on the rows
     routed to it, then combine and project.  ``get_inputs(tokens)`` returns the non-expert
     tensors with ``u`` restricted to those tokens' rows; ``get_expert(e)`` returns
-    (w_gu_e, w_down_e)."""
+    (w_gu_e, w_down_e).  Besides the outputs of ``layer_forward`` it returns the expert inputs
+    z [ntok, E_in] and, with want_s, each slot's expert output before its norm s [ntok, k, E_in]
+    (the vector I_gamma reduces)."""
     tokens = np.asarray(tokens, np.int64)
     nt = len(tokens)
     L = lib()
@@ -197,17 +206,21 @@ def layer_forward_staged(cfg, tokens, get_inputs, get_expert, nthreads: int | No
         L.orc_router_token(ctypes.byref(c), ctypes.byref(x), i, _p(logits[i]), _p(idx[i]), _p(w[i]))
         L.orc_expert_input_token(ctypes.byref(c), ctypes.byref(x), i, _p(z[i]))
     ns = np.zeros((nt, k, E))
+    ss = np.zeros((nt, k, E)) if want_s else None
     gamma = keep.ptr(inp.get("gamma_expert"))
     for e in np.unique(idx):
         rows = np.argwhere(idx == e)
         zr = np.ascontiguousarray(z[rows[:, 0]])
         nr = np.zeros_like(zr)
+        sr = np.zeros_like(zr) if want_s else None
         wg, wd = get_expert(int(e))
         wg = np.ascontiguousarray(wg)
         wd = np.ascontiguousarray(wd)
-        L.orc_expert_batch(ctypes.byref(c), _p(wg), _p(wd), gamma, _p(zr), len(rows), _p(nr),
-                           nthreads or threads())
+        L.orc_expert_batch_parts(ctypes.byref(c), _p(wg), _p(wd), gamma, _p(zr), len(rows),
+                                 _p(sr) if want_s else None, _p(nr), nthreads or threads())
         ns[rows[:, 0], rows[:, 1]] = nr
+        if want_s:
+            ss[rows[:, 0], rows[:, 1]] = sr
     y = np.zeros((nt, E))
     out = np.zeros((nt, d))
     for i in range(nt):
@@ -215,7 +228,52 @@ def layer_forward_staged(cfg, tokens, get_inputs, get_expert, nthreads: int | No
         wi = np.ascontiguousarray(w[i])
         L.orc_combine_token(ctypes.byref(c), _p(nsi), _p(wi), _p(y[i]))
         L.orc_output_token(ctypes.byref(c), ctypes.byref(x), i, _p(y[i]), _p(out[i]))
-    return {"out": out, "logits": logits, "idx": idx, "w": w, "y": y, "tokens": tokens}
+    return {"out": out, "logits": logits, "idx": idx, "w": w, "y": y, "z": z, "s": ss,
+            "tokens": tokens}
+
+
+def router(cfg, inp: dict, rows=None, nthreads: int | None = None) -> dict:
+    """The router step on rows of ``inp['u']`` (all rows by default), threads over rows: logits
+    [rows, n] (the sigmoid scores in that mode), idx [rows, k], w [rows, k].  Only the router's
+    tensors need be in ``inp`` (u, w_router and, as the mode needs, logit_bias, correction_bias,
+    gamma_in)."""
+    nrow = inp["u"].shape[0]
+    rows = np.arange(nrow, dtype=np.int64) if rows is None else np.asarray(rows, np.int64)
+    keep = _Keep()
+    c = make_cfg(cfg, T=nrow)
+    x = make_tensors(cfg, inp, keep, experts={})
+    nt = len(rows)
+    logits = np.zeros((nt, cfg.n_experts))
+    idx = np.zeros((nt, cfg.top_k), dtype=np.int32)
+    w = np.zeros((nt, cfg.top_k))
+    rk = np.ascontiguousarray(rows)
+    lib().orc_router_batch(ctypes.byref(c), ctypes.byref(x), _p(rk), nt, _p(logits), _p(idx),
+                           _p(w), nthreads or threads())
+    return {"logits": logits, "idx": idx, "w": w}
+
+
+def expert_scaled(cfg, w_gu_e, w_down_e, gamma_expert, z):
+    """One expert's output rows before its norm (the vector I_gamma reduces, or o without
+    expert_norm), for input rows z [rows, E_in] (float64)."""
+    z = np.ascontiguousarray(np.atleast_2d(z), np.float64)
+    out = np.zeros_like(z)
+    keep = _Keep()
+    c = make_cfg(cfg)
+    wg, wd = keep.ptr(w_gu_e), keep.ptr(w_down_e)
+    g = keep.ptr(None if gamma_expert is None else np.asarray(gamma_expert, np.float32))
+    for i in range(z.shape[0]):
+        lib().orc_expert_token_scaled(ctypes.byref(c), wg, wd, g, _p(z[i]), _p(out[i]))
+    return out
+
+
+def input_scaled_vector(x, gamma, is_bf16=1):
+    """D_gamma x = (1 + gamma) * x rounded to the storage dtype (is_bf16 as in bf16_round)."""
+    x = np.ascontiguousarray(x, np.float64)
+    g = np.ascontiguousarray(gamma, np.float64)
+    out = np.zeros_like(x)
+    c = OrcCfg(is_bf16=is_bf16)
+    lib().orc_input_scaled_vector(ctypes.byref(c), _p(x), _p(g), x.size, _p(out))
+    return out
 
 
 def permutation(T: int, k: int, n: int, idx: np.ndarray):

@@ -103,11 +103,17 @@ void orc_centered_rmsnorm(const double* x, const double* gamma, int D, double ep
   for (int i = 0; i < D; ++i) out[i] *= 1.0 + gamma[i];
 }
 
+/* D_gamma x = (1 + gamma) * x, rounded to the input dtype: the vector I_gamma reduces. */
+void orc_input_scaled_vector(const orc_cfg* c, const double* x, const double* gamma, int D,
+                             double* s) {
+  for (int i = 0; i < D; ++i) s[i] = orc_round(c, (1.0 + gamma[i]) * x[i]);
+}
+
 /* I_gamma(x) = R_eps(D_gamma x), with D_gamma x rounded to the input dtype before the reduction. */
 void orc_input_scaled_rmsnorm(const orc_cfg* c, const double* x, const double* gamma, int D,
                               double eps, double* out) {
   double* s = (double*)malloc(sizeof(double) * (size_t)D);
-  for (int i = 0; i < D; ++i) s[i] = orc_round(c, (1.0 + gamma[i]) * x[i]);
+  orc_input_scaled_vector(c, x, gamma, D, s);
   orc_rms_normalize(s, D, eps, out);
   free(s);
 }
@@ -277,11 +283,12 @@ void orc_expert_input_token(const orc_cfg* c, const orc_tensors* x, int64_t t, d
   free(ut);
 }
 
-void orc_expert_token(const orc_cfg* c, const void* w_gu_e, const void* w_down_e,
-                      const float* gamma_expert, const double* z, double* nout) {
+/* One expert on one input row: o = dtype(W_d act), act = dtype(SiLU(W_gate z) * W_up z) or
+ * dtype(ReLU(W_1 z)). */
+static void expert_output(const orc_cfg* c, const void* w_gu_e, const void* w_down_e,
+                          const double* z, double* o) {
   int E = expert_in(c), H = c->d_ff;
   double* hid = (double*)malloc(sizeof(double) * (size_t)H);
-  double* o = (double*)malloc(sizeof(double) * (size_t)E);
   for (int i = 0; i < H; ++i) {
     if (c->act == 1) {
       double g = dot_row(w_gu_e, (size_t)i, E, z, c->is_bf16);       /* gate row i */
@@ -293,17 +300,44 @@ void orc_expert_token(const orc_cfg* c, const void* w_gu_e, const void* w_down_e
     }
   }
   for (int j = 0; j < E; ++j) o[j] = orc_round(c, dot_row(w_down_e, (size_t)j, H, hid, c->is_bf16));
+  free(hid);
+}
+
+/* One expert on one row: nout = I_gamma(o) stored in the dtype (or o without expert_norm), and,
+ * if s is not NULL, the vector I_gamma reduces, s = dtype(D_gamma o) (or o). */
+static void expert_token_parts(const orc_cfg* c, const void* w_gu_e, const void* w_down_e,
+                               const float* gamma_expert, const double* z, double* s,
+                               double* nout) {
+  int E = expert_in(c);
+  double* o = (double*)malloc(sizeof(double) * (size_t)E);
+  expert_output(c, w_gu_e, w_down_e, z, o);
   if (c->expert_norm) {
     double* g = (double*)malloc(sizeof(double) * (size_t)E);
+    double* sv = (double*)malloc(sizeof(double) * (size_t)E);
     for (int j = 0; j < E; ++j) g[j] = (double)gamma_expert[j];
-    orc_input_scaled_rmsnorm(c, o, g, E, c->eps, nout);
+    orc_input_scaled_vector(c, o, g, E, sv); /* I_gamma = R_eps(dtype(D_gamma o)) */
+    orc_rms_normalize(sv, E, c->eps, nout);
     for (int j = 0; j < E; ++j) nout[j] = orc_round(c, nout[j]);
+    if (s) memcpy(s, sv, sizeof(double) * (size_t)E);
+    free(sv);
     free(g);
   } else {
     memcpy(nout, o, sizeof(double) * (size_t)E);
+    if (s) memcpy(s, o, sizeof(double) * (size_t)E);
   }
   free(o);
-  free(hid);
+}
+
+void orc_expert_token(const orc_cfg* c, const void* w_gu_e, const void* w_down_e,
+                      const float* gamma_expert, const double* z, double* nout) {
+  expert_token_parts(c, w_gu_e, w_down_e, gamma_expert, z, NULL, nout);
+}
+
+void orc_expert_token_scaled(const orc_cfg* c, const void* w_gu_e, const void* w_down_e,
+                             const float* gamma_expert, const double* z, double* s) {
+  double* n = (double*)malloc(sizeof(double) * (size_t)expert_in(c));
+  expert_token_parts(c, w_gu_e, w_down_e, gamma_expert, z, s, n);
+  free(n);
 }
 
 /* y = sum_j w_j n_j, accumulated in slot order, then stored in the dtype. */
@@ -426,10 +460,48 @@ void orc_layer_forward(const orc_cfg* c, const orc_tensors* x, const int64_t* to
 
 typedef struct {
   const orc_cfg* c;
+  const orc_tensors* x;
+  const int64_t* rows;
+  int lo, hi;
+  double *logits, *w;
+  int* idx;
+} router_job;
+
+static void* router_worker(void* p) {
+  router_job* j = (router_job*)p;
+  int n = j->c->n_experts, k = j->c->top_k;
+  for (int i = j->lo; i < j->hi; ++i)
+    orc_router_token(j->c, j->x, j->rows[i], j->logits + (size_t)i * n, j->idx + (size_t)i * k,
+                     j->w + (size_t)i * k);
+  return NULL;
+}
+
+void orc_router_batch(const orc_cfg* c, const orc_tensors* x, const int64_t* rows, int nrows,
+                      double* logits, int* idx, double* w, int nthreads) {
+  if (nthreads < 1) nthreads = 1;
+  if (nthreads > nrows) nthreads = nrows > 0 ? nrows : 1;
+  router_job* jobs = (router_job*)calloc((size_t)nthreads, sizeof(router_job));
+  pthread_t* tid = (pthread_t*)calloc((size_t)nthreads, sizeof(pthread_t));
+  int* ok = (int*)calloc((size_t)nthreads, sizeof(int));
+  for (int t = 0; t < nthreads; ++t) {
+    jobs[t] = (router_job){c, x, rows, (int)((long)nrows * t / nthreads),
+                           (int)((long)nrows * (t + 1) / nthreads), logits, w, idx};
+    ok[t] = pthread_create(&tid[t], NULL, router_worker, &jobs[t]) == 0;
+    if (!ok[t]) router_worker(&jobs[t]);
+  }
+  for (int t = 0; t < nthreads; ++t)
+    if (ok[t]) pthread_join(tid[t], NULL);
+  free(ok);
+  free(tid);
+  free(jobs);
+}
+
+typedef struct {
+  const orc_cfg* c;
   const void *wg, *wd;
   const float* gamma;
   const double* z;
-  double* nrow;
+  double *srow, *nrow;
   int lo, hi;
 } expert_job;
 
@@ -437,20 +509,27 @@ static void* expert_worker(void* p) {
   expert_job* j = (expert_job*)p;
   int E = expert_in(j->c);
   for (int r = j->lo; r < j->hi; ++r)
-    orc_expert_token(j->c, j->wg, j->wd, j->gamma, j->z + (size_t)r * E, j->nrow + (size_t)r * E);
+    expert_token_parts(j->c, j->wg, j->wd, j->gamma, j->z + (size_t)r * E,
+                       j->srow ? j->srow + (size_t)r * E : NULL, j->nrow + (size_t)r * E);
   return NULL;
 }
 
 void orc_expert_batch(const orc_cfg* c, const void* w_gu_e, const void* w_down_e,
                       const float* gamma_expert, const double* z_rows, int nrows, double* n_rows,
                       int nthreads) {
+  orc_expert_batch_parts(c, w_gu_e, w_down_e, gamma_expert, z_rows, nrows, NULL, n_rows, nthreads);
+}
+
+void orc_expert_batch_parts(const orc_cfg* c, const void* w_gu_e, const void* w_down_e,
+                            const float* gamma_expert, const double* z_rows, int nrows,
+                            double* s_rows, double* n_rows, int nthreads) {
   if (nthreads < 1) nthreads = 1;
   if (nthreads > nrows) nthreads = nrows > 0 ? nrows : 1;
   expert_job* jobs = (expert_job*)calloc((size_t)nthreads, sizeof(expert_job));
   pthread_t* tid = (pthread_t*)calloc((size_t)nthreads, sizeof(pthread_t));
   int* ok = (int*)calloc((size_t)nthreads, sizeof(int));
   for (int t = 0; t < nthreads; ++t) {
-    jobs[t] = (expert_job){c, w_gu_e, w_down_e, gamma_expert, z_rows, n_rows,
+    jobs[t] = (expert_job){c, w_gu_e, w_down_e, gamma_expert, z_rows, s_rows, n_rows,
                            (int)((long)nrows * t / nthreads), (int)((long)nrows * (t + 1) / nthreads)};
     ok[t] = pthread_create(&tid[t], NULL, expert_worker, &jobs[t]) == 0;
     if (!ok[t]) expert_worker(&jobs[t]);

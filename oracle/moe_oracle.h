@@ -77,6 +77,9 @@ void orc_rms_normalize(const double* x, int D, double eps, double* out);
 void orc_centered_rmsnorm(const double* x, const double* gamma, int D, double eps, double* out);
 void orc_input_scaled_rmsnorm(const orc_cfg* c, const double* x, const double* gamma, int D,
                               double eps, double* out);
+/* The vector I_gamma reduces: s = (1 + gamma) * x rounded to the storage dtype. */
+void orc_input_scaled_vector(const orc_cfg* c, const double* x, const double* gamma, int D,
+                             double* s);
 
 /* Softmax over n logits then top-k by (logit desc, index asc); weights renormalised to sum 1
  * and multiplied by routed_scale.  Slot order is the selection order. */
@@ -104,6 +107,10 @@ void orc_router_token(const orc_cfg* c, const orc_tensors* x, int64_t t, double*
 void orc_expert_input_token(const orc_cfg* c, const orc_tensors* x, int64_t t, double* z);
 void orc_expert_token(const orc_cfg* c, const void* w_gu_e, const void* w_down_e,
                       const float* gamma_expert, const double* z, double* nout);
+/* The same expert's output before its norm: s = dtype((1 + gamma_expert) * o) with expert_norm
+ * (the vector I_gamma reduces), else o. */
+void orc_expert_token_scaled(const orc_cfg* c, const void* w_gu_e, const void* w_down_e,
+                             const float* gamma_expert, const double* z, double* s);
 void orc_combine_token(const orc_cfg* c, const double* n_slots, const double* w, double* y);
 void orc_output_token(const orc_cfg* c, const orc_tensors* x, int64_t t, const double* y,
                       double* out);
@@ -115,10 +122,20 @@ void orc_layer_forward(const orc_cfg* c, const orc_tensors* x, const int64_t* to
                        double* out, double* logits, int* idx, double* w, double* y_latent,
                        int nthreads);
 
+/* Router step (orc_router_token) for rows[i] of the tensors, i < nrows, threads over rows:
+ * logits [nrows, n] (the sigmoid scores in that mode), idx [nrows, k], w [nrows, k]. */
+void orc_router_batch(const orc_cfg* c, const orc_tensors* x, const int64_t* rows, int nrows,
+                      double* logits, int* idx, double* w, int nthreads);
+
 /* Expert step for a batch of (token, slot) rows routed to one expert; threads over rows. */
 void orc_expert_batch(const orc_cfg* c, const void* w_gu_e, const void* w_down_e,
                       const float* gamma_expert, const double* z_rows, int nrows, double* n_rows,
                       int nthreads);
+/* The same, also returning each row's pre-norm vector (orc_expert_token_scaled) in s_rows
+ * [nrows, E_in] when it is not NULL. */
+void orc_expert_batch_parts(const orc_cfg* c, const void* w_gu_e, const void* w_down_e,
+                            const float* gamma_expert, const double* z_rows, int nrows,
+                            double* s_rows, double* n_rows, int nthreads);
 
 /* Shazeer et al.'s noisy top-k gate and its balancing statistics [SHAZEER "The gate", "Keeping the
  * experts busy"], for one token from its clean logits l = x W_g, noise logits m = x W_noise and

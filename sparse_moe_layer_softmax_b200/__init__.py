@@ -31,7 +31,7 @@ EXPORTS = ("moe_status_string", "moe_workspace_size", "moe_route", "moe_permute"
            "moe_launch_count", "moe_permute_static", "moe_selftest_wait_timeout",
            "moe_router_split_weights", "moe_residual_update", "moe_noisy_gate",
            "moe_noisy_gate_workspace_size", "moe_host_staging_size", "moe_layer_forward_host",
-           "moe_row_sumsq_parts", "moe_gather_rows")
+           "moe_row_sumsq_parts", "moe_gather_rows", "moe_layer_forward_taps")
 PROFILE_STAGES = ("route", "latent_down", "dispatch", "expert_gate_up", "expert_down", "combine",
                   "latent_up_resgate")
 
@@ -51,6 +51,11 @@ class Config(ctypes.Structure):
                [("gate_mode", ctypes.c_int32), ("router_f32", ctypes.c_int32),
                 ("logit_mult", ctypes.c_float), ("input_norm", ctypes.c_int32),
                 ("post_norm", ctypes.c_int32), ("eps_block", ctypes.c_float)]
+
+
+class Taps(ctypes.Structure):
+    """moe_layer_taps_t"""
+    _fields_ = [(n, ctypes.c_void_p) for n in ("z", "s", "y", "inv_perm")]
 
 
 class Weights(ctypes.Structure):
@@ -91,6 +96,8 @@ def lib():
             "moe_latent_down": [cp, vp, vp, vp, vp],
             "moe_latent_up": [cp, vp, vp, vp, vp, vp, vp],
             "moe_layer_forward": [cp, wp, vp, vp, vp, vp, vp, vp, vp, sz, vp],
+            "moe_layer_forward_taps": [cp, wp, vp, vp, vp, vp, vp, vp,
+                                       ctypes.POINTER(Taps), vp, sz, vp],
             "moe_host_staging_size": [cp, ctypes.POINTER(ctypes.c_size_t)],
             "moe_layer_forward_host": [cp, wp, ctypes.c_int32, ctypes.POINTER(vp),
                                        ctypes.POINTER(vp), vp, sz, vp, sz, vp],
@@ -284,6 +291,20 @@ def moe_layer_forward(cfg, weights: Weights, u, r, out, logits_out=None, topk_id
         _ptr(topk_idx_out), _ptr(topk_w_out), _ptr(workspace), workspace_bytes, _stream(stream)))
 
 
+def moe_layer_forward_taps(cfg, weights: Weights, u, r, out, taps: dict, logits_out=None,
+                           topk_idx_out=None, topk_w_out=None, workspace=None, workspace_bytes=0,
+                           stream=None):
+    """moe_layer_forward that also copies the intermediates named in ``taps`` (device tensors
+    under the keys z, s, y, inv_perm; missing keys are skipped)."""
+    if workspace is not None and not workspace_bytes:
+        workspace_bytes = workspace.numel() * workspace.element_size()
+    t = Taps(**{k: _ptr(taps.get(k)) for k, _ in Taps._fields_})
+    _check("moe_layer_forward_taps", lib().moe_layer_forward_taps(
+        ctypes.byref(cfg), ctypes.byref(weights), _ptr(u), _ptr(r), _ptr(out), _ptr(logits_out),
+        _ptr(topk_idx_out), _ptr(topk_w_out), ctypes.byref(t), _ptr(workspace), workspace_bytes,
+        _stream(stream)))
+
+
 def moe_get_device_status(stream=None) -> int:
     return lib().moe_get_device_status(_stream(stream))
 
@@ -328,12 +349,19 @@ class MoELayer:
         self.workspace = torch.empty(workspace_size(cfg), dtype=torch.uint8, device="cuda")
 
     def forward(self, u, r=None, out=None, logits_out=None, topk_idx_out=None, topk_w_out=None,
-                stream=None):
+                stream=None, taps: dict | None = None):
+        """One moe_layer_forward; with ``taps`` (a dict of device tensors under the keys z, s, y,
+        inv_perm) one moe_layer_forward_taps that also copies those intermediates."""
         import torch
         if out is None:
             out = torch.empty_like(u)
-        moe_layer_forward(self.cfg, self._w, u, r if r is not None else u, out, logits_out,
-                          topk_idx_out, topk_w_out, self.workspace, stream=stream)
+        r = r if r is not None else u
+        if taps is None:
+            moe_layer_forward(self.cfg, self._w, u, r, out, logits_out, topk_idx_out, topk_w_out,
+                              self.workspace, stream=stream)
+        else:
+            moe_layer_forward_taps(self.cfg, self._w, u, r, out, taps, logits_out, topk_idx_out,
+                                   topk_w_out, self.workspace, stream=stream)
         return out
 
     def forward_host(self, u_hosts, out_hosts, stream=None):

@@ -183,13 +183,14 @@ __global__ void dense_split_finish_kernel(const float* __restrict__ partial, int
 
 // ------------------------------------------------------------------ row gather
 //
-// dst[i] = src[rows[i]] in 16-byte vectors, one CTA per row (grid-strided); a negative index
-// gives a zero row, an index past src_rows latches MOE_ERR_DEVICE_CHECK and gives a zero row.
+// dst[i] = src[rows[i * idx_stride]] in 16-byte vectors, one CTA per row (grid-strided); a
+// negative index gives a zero row, an index past src_rows latches MOE_ERR_DEVICE_CHECK and gives a
+// zero row.
 __global__ void gather_rows_kernel(const uint4* __restrict__ src, long src_rows,
-                                   const int32_t* __restrict__ rows, long n_rows, int row_vec,
-                                   uint4* __restrict__ dst) {
+                                   const int32_t* __restrict__ rows, long n_rows, int idx_stride,
+                                   int row_vec, uint4* __restrict__ dst) {
   for (long i = blockIdx.x; i < n_rows; i += gridDim.x) {
-    int r = rows[i];
+    int r = rows[i * idx_stride];
     if (r >= src_rows) {
       if (threadIdx.x == 0) latch_status(MOE_ERR_DEVICE_CHECK);
       r = -1;
@@ -562,6 +563,10 @@ __global__ void __launch_bounds__(kRouterThreads, 1) router_logits_small_kernel(
 // descending order, weights exp(l_j - l_1) / sum_sel exp(l - l_1) * routed_scale.  Sigmoid gate:
 // scores s = sigmoid(l) replace the logits in the buffer, the k largest keys s + sel_bias are
 // selected, weights s_j / (sum_sel s + 1e-15) * routed_scale.
+// Chosen experts leave the candidate set through a per-lane bit mask, so the k indices are
+// distinct even when fewer than k keys are finite (a logit bias of -inf masks an expert: such
+// experts are taken last, lower index first, with weight 0).  A NaN key ranks as -inf and latches
+// MOE_ERR_DEVICE_CHECK, as does a row whose best key is not finite (its weights are undefined).
 __global__ void topk_rows_kernel(float* __restrict__ logits, int T, int n, int k,
                                  float routed_scale, int gate_mode,
                                  const float* __restrict__ sel_bias,
@@ -571,6 +576,7 @@ __global__ void topk_rows_kernel(float* __restrict__ logits, int T, int n, int k
   const int lane = threadIdx.x & 31;
   if (t >= T) return;
   float key[kMaxExperts / 32], pay[kMaxExperts / 32];
+  bool bad = false;
 #pragma unroll
   for (int i = 0; i < kMaxExperts / 32; ++i) {
     const int e = lane + 32 * i;
@@ -587,12 +593,18 @@ __global__ void topk_rows_kernel(float* __restrict__ logits, int T, int n, int k
         key[i] = l;
         pay[i] = l;
       }
+      if (key[i] != key[i]) {  // NaN
+        bad = true;
+        key[i] = -INFINITY;
+        pay[i] = gate_mode == MOE_GATE_SIGMOID ? 0.0f : -INFINITY;
+      }
     }
   }
   // Loops over the k kept entries run to the compile-time bound kMaxTopK with k as a guard, so
   // the arrays stay in registers.
   float top_s[kMaxTopK];
   int top_i[kMaxTopK];
+  unsigned taken = 0u;  // bit i: expert lane + 32 i is already selected
 #pragma unroll
   for (int j = 0; j < kMaxTopK; ++j) {
     top_s[j] = 0.0f;
@@ -603,7 +615,8 @@ __global__ void topk_rows_kernel(float* __restrict__ logits, int T, int n, int k
 #pragma unroll
     for (int i = 0; i < kMaxExperts / 32; ++i) {
       const int e = lane + 32 * i;
-      if (e < n && (key[i] > bv || (key[i] == bv && e < bi))) { bv = key[i]; bi = e; bs = pay[i]; }
+      const bool cand = e < n && !((taken >> i) & 1u);
+      if (cand && (key[i] > bv || (key[i] == bv && e < bi))) { bv = key[i]; bi = e; bs = pay[i]; }
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
@@ -613,11 +626,13 @@ __global__ void topk_rows_kernel(float* __restrict__ logits, int T, int n, int k
       if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; bs = os; }
     }
     top_s[j] = bs;
-    top_i[j] = bi;
+    top_i[j] = bi;  // k <= n: some candidate is always left
 #pragma unroll
     for (int i = 0; i < kMaxExperts / 32; ++i)
-      if (lane + 32 * i == bi) key[i] = -INFINITY;
+      if (lane + 32 * i == bi) taken |= 1u << i;
   }
+  bad = __any_sync(0xffffffffu, bad);
+  if (lane == 0 && (bad || !(fabsf(top_s[0]) <= 3.0e38f))) latch_status(MOE_ERR_DEVICE_CHECK);
   if (lane == 0) {
     float e[kMaxTopK];
     float sum = 0.0f;

@@ -973,10 +973,46 @@ moe_status_t moe_latent_up(const moe_config_t* cfg, const void* y, const void* p
   return do_latent_up(*cfg, y, p_up, r, resid_g, out, static_cast<cudaStream_t>(stream));
 }
 
-moe_status_t moe_layer_forward(const moe_config_t* cfg, const moe_weights_t* w, const void* u,
-                               const void* r, void* out, float* logits_out,
-                               int32_t* topk_idx_out, float* topk_w_out, void* workspace,
-                               size_t workspace_bytes, void* stream) {
+}  // extern "C"
+
+namespace {
+
+// Copies of the intermediates a caller asked for (moe_layer_forward_taps), each queued right
+// after the stage that produces it.
+struct Taps {
+  const moe_layer_taps_t* t = nullptr;
+  moe_status_t inv(const moe_config_t& c, const int32_t* inv, cudaStream_t st) const {
+    if (!t || !t->inv_perm) return MOE_OK;
+    const size_t bytes = static_cast<size_t>(c.T) * c.top_k * sizeof(int32_t);
+    return cudaMemcpyAsync(t->inv_perm, inv, bytes, cudaMemcpyDeviceToDevice, st) == cudaSuccess
+               ? MOE_OK : MOE_ERR_CUDA;
+  }
+  // z[t] = x_perm[inv[t*k]]: every slot of a token carries the same dispatched row
+  moe_status_t z(const moe_config_t& c, const void* x_perm, const int32_t* inv,
+                 cudaStream_t st) const {
+    if (!t || !t->z) return MOE_OK;
+    const long rb = static_cast<long>(expert_in(c)) * static_cast<long>(dsize(c));
+    const int row_vec = static_cast<int>(rb / 16);
+    const int threads = row_vec >= 256 ? 256 : ((row_vec + 31) / 32) * 32;
+    const long grid = std::min<long>(c.T, static_cast<long>(std::max(device_info().sms, 1)) * 16);
+    gather_rows_kernel<<<static_cast<unsigned>(grid), threads, 0, st>>>(
+        static_cast<const uint4*>(x_perm), static_cast<long>(c.T) * c.top_k, inv,
+        static_cast<long>(c.T), c.top_k, row_vec, static_cast<uint4*>(t->z));
+    return last_launch();
+  }
+  moe_status_t copy(void* dst, const void* src, size_t rows, const moe_config_t& c,
+                    cudaStream_t st) const {
+    if (!dst) return MOE_OK;
+    const size_t bytes = rows * static_cast<size_t>(expert_in(c)) * dsize(c);
+    return cudaMemcpyAsync(dst, src, bytes, cudaMemcpyDeviceToDevice, st) == cudaSuccess
+               ? MOE_OK : MOE_ERR_CUDA;
+  }
+};
+
+moe_status_t layer_forward_impl(const moe_config_t* cfg, const moe_weights_t* w, const void* u,
+                                const void* r, void* out, float* logits_out,
+                                int32_t* topk_idx_out, float* topk_w_out, const Taps& taps,
+                                void* workspace, size_t workspace_bytes, void* stream) {
   moe_status_t s = check_forward(cfg, w, u, r, out, logits_out, topk_idx_out, topk_w_out,
                                  workspace, workspace_bytes);
   if (s != MOE_OK) return s;
@@ -1017,6 +1053,7 @@ moe_status_t moe_layer_forward(const moe_config_t* cfg, const moe_weights_t* w, 
   if ((s = do_permute(c, idx, offsets, perm, inv, xin, c.pre_norm ? w->gamma_pre : nullptr, x_perm,
                       at<int32_t>(workspace, L.counts), st)) != MOE_OK)
     return s;
+  if ((s = taps.inv(c, inv, st)) != MOE_OK || (s = taps.z(c, x_perm, inv, st)) != MOE_OK) return s;
   prof_mark(st, 3);
   // The expert output overwrites the dispatched input rows (no longer needed after GEMM 1).
   // The down GEMM leaves each row's partial sums of squares for the combine's I_gamma norms when
@@ -1028,9 +1065,12 @@ moe_status_t moe_layer_forward(const moe_config_t* cfg, const moe_weights_t* w, 
                       true, row_ss)) != MOE_OK)
     return s;
   if (c.dtype == MOE_F32) prof_mark(st, 4);  // one fused kernel: all time in stage 3
+  if (taps.t && (s = taps.copy(taps.t->s, x_perm, static_cast<size_t>(c.T) * c.top_k, c, st)) != MOE_OK)
+    return s;
   prof_mark(st, 5);
   void* y = latent ? at<void>(workspace, L.y) : out;
   if ((s = do_combine(c, x_perm, inv, wt, y, st, row_ss)) != MOE_OK) return s;
+  if (taps.t && (s = taps.copy(taps.t->y, y, static_cast<size_t>(c.T), c, st)) != MOE_OK) return s;
   prof_mark(st, 6);
   if (latent && !c.post_norm &&
       (s = do_latent_up(c, y, w->p_up, r, w->resid_g, out, st, split)) != MOE_OK)
@@ -1045,6 +1085,31 @@ moe_status_t moe_layer_forward(const moe_config_t* cfg, const moe_weights_t* w, 
   prof_mark(st, 7);
   prof_next_call();
   return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+moe_status_t moe_layer_forward(const moe_config_t* cfg, const moe_weights_t* w, const void* u,
+                               const void* r, void* out, float* logits_out,
+                               int32_t* topk_idx_out, float* topk_w_out, void* workspace,
+                               size_t workspace_bytes, void* stream) {
+  return layer_forward_impl(cfg, w, u, r, out, logits_out, topk_idx_out, topk_w_out, Taps{},
+                            workspace, workspace_bytes, stream);
+}
+
+moe_status_t moe_layer_forward_taps(const moe_config_t* cfg, const moe_weights_t* w,
+                                    const void* u, const void* r, void* out, float* logits_out,
+                                    int32_t* topk_idx_out, float* topk_w_out,
+                                    const moe_layer_taps_t* taps, void* workspace,
+                                    size_t workspace_bytes, void* stream) {
+  if (taps && !all_aligned({taps->z, taps->s, taps->y, static_cast<const void*>(taps->inv_perm)}))
+    return MOE_ERR_ALIGNMENT;
+  Taps tp;
+  tp.t = taps;
+  return layer_forward_impl(cfg, w, u, r, out, logits_out, topk_idx_out, topk_w_out, tp,
+                            workspace, workspace_bytes, stream);
 }
 
 moe_status_t moe_residual_update(const moe_config_t* cfg, const void* b, const void* r,
@@ -1235,7 +1300,7 @@ moe_status_t moe_gather_rows(const void* src, int64_t src_rows, const int32_t* r
   const long grid = std::min<long>(n_rows, static_cast<long>(std::max(device_info().sms, 1)) * 16);
   gather_rows_kernel<<<static_cast<unsigned>(grid), threads, 0, static_cast<cudaStream_t>(stream)>>>(
       static_cast<const uint4*>(src), static_cast<long>(src_rows), rows, static_cast<long>(n_rows),
-      row_vec, static_cast<uint4*>(dst));
+      1, row_vec, static_cast<uint4*>(dst));
   return last_launch();
 }
 

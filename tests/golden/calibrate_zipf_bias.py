@@ -24,7 +24,9 @@ from moe_inputs import configs  # noqa: E402
 
 
 def main():
-    cfg = configs.MUSE_IMBALANCED
+    # the calibration sample is the first draw of u (the workload's separation redraws, which
+    # depend on the bias, come after the scale is fixed)
+    cfg = configs.MUSE_IMBALANCED.replace(u_redraw=())
     ncal = 2048
     toks = np.sort(moe_inputs.fisher_yates(cfg.seed, configs.STREAM_SUBSAMPLE, cfg.T, ncal))
     inp = {"u": moe_inputs.host_rows(cfg, "u", rows=toks),

@@ -70,8 +70,11 @@ def logit_atol(cfg, logits: np.ndarray) -> float:
     return tol
 
 
-def run_layer(cfg, dev: dict, want_logits: bool = True):
-    """moe_layer_forward through the C ABI on device inputs; returns torch tensors."""
+def run_layer(cfg, dev: dict, want_logits: bool = True, want_taps: bool = False):
+    """moe_layer_forward through the C ABI on device inputs; returns torch tensors.  With
+    want_taps, moe_layer_forward_taps: the result also holds the intermediates z [T, E_in],
+    s [T*k, E_in] (dispatch order), y [T, E_in] under "taps" and the dispatch rows under "inv"
+    ([T, k])."""
     import torch
     c = abi_config(cfg)
     layer = moe.MoELayer(c, dev)
@@ -81,18 +84,31 @@ def run_layer(cfg, dev: dict, want_logits: bool = True):
         if want_logits else None
     idx = torch.empty((cfg.T, cfg.top_k), dtype=torch.int32, device="cuda")
     w = torch.empty((cfg.T, cfg.top_k), dtype=torch.float32, device="cuda")
-    layer.forward(u, u, out=out, logits_out=logits, topk_idx_out=idx, topk_w_out=w)
+    taps = None
+    if want_taps:
+        E, TK = cfg.expert_in, cfg.T * cfg.top_k
+        taps = {"z": torch.empty((cfg.T, E), dtype=u.dtype, device="cuda"),
+                "s": torch.empty((TK, E), dtype=u.dtype, device="cuda"),
+                "y": torch.empty((cfg.T, E), dtype=u.dtype, device="cuda"),
+                "inv_perm": torch.empty((cfg.T, cfg.top_k), dtype=torch.int32, device="cuda")}
+    layer.forward(u, u, out=out, logits_out=logits, topk_idx_out=idx, topk_w_out=w, taps=taps)
     status = moe.moe_get_device_status()
     assert status == 0, f"device status {moe.STATUS.get(status, status)}"
-    return {"out": out, "logits": logits, "idx": idx, "w": w, "layer": layer}
+    res = {"out": out, "logits": logits, "idx": idx, "w": w, "layer": layer}
+    if taps is not None:
+        res["taps"] = taps
+        res["inv"] = taps["inv_perm"]
+    return res
 
 
-def oracle_reference(cfg, tokens=None):
+def oracle_reference(cfg, tokens=None, want_s: bool = False):
     """Oracle layer outputs for the listed tokens (all by default).  Small workloads hold every
-    tensor on the host; large ones evaluate one expert's weights at a time."""
+    tensor on the host; large ones evaluate one expert's weights at a time.  With want_s the
+    staged evaluation is used at every size, and the result also holds the expert inputs z and
+    each slot's pre-norm expert output s."""
     import oracle
     big = cfg.n_experts * cfg.gu_rows * cfg.expert_in > 64 * 1024 * 1024
-    if not big:
+    if not big and not want_s:
         inp = moe_inputs.host_inputs(cfg)
         return oracle.layer_forward(cfg, inp, tokens=tokens)
     tokens = np.arange(cfg.T) if tokens is None else np.asarray(tokens)
@@ -109,7 +125,7 @@ def oracle_reference(cfg, tokens=None):
     def get_expert(e):
         return (moe_inputs.host_rows(cfg, "w_gu", lead=e), moe_inputs.host_rows(cfg, "w_down", lead=e))
 
-    return oracle.layer_forward_staged(cfg, tokens, get_inputs, get_expert)
+    return oracle.layer_forward_staged(cfg, tokens, get_inputs, get_expert, want_s=want_s)
 
 
 def correction_bias(cfg):
@@ -162,6 +178,33 @@ def compare_selection(idx_gpu: np.ndarray, ref_logits: np.ndarray, ref_idx: np.n
     np.testing.assert_array_equal(idx_gpu[exact], ref_idx[exact])
     np.testing.assert_array_equal(np.sort(idx_gpu[ot], axis=1), np.sort(ref_idx[ot], axis=1))
     return ties
+
+
+def separate(cfg):
+    """`cfg` with its router inputs separated at the top-k boundary: a named workload keeps its
+    stored redraw list; any other configuration gets one computed here with the oracle's router
+    (tests/golden/separate_router_logits.py)."""
+    if cfg.name in configs.SEPARATED_NAMES and cfg == configs.ALL_CONFIGS.get(cfg.name):
+        return cfg
+    import importlib.util
+    import os
+    path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden",
+                        "separate_router_logits.py")
+    spec = importlib.util.spec_from_file_location("separate_router_logits", path)
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    red, _ = mod.redraws_for(cfg)
+    return cfg.replace(u_redraw=red)
+
+
+def key_margins(keys: np.ndarray, k: int) -> np.ndarray:
+    """k-th minus (k+1)-th largest key per row, over the rms of the row's keys (+inf if k = n)."""
+    n = keys.shape[1]
+    if k >= n:
+        return np.full(len(keys), np.inf)
+    s = -np.sort(-keys, axis=1)
+    rms = np.sqrt(np.mean(keys.astype(np.float64) ** 2, axis=1))
+    return (s[:, k - 1] - s[:, k]) / rms
 
 
 def near_tie_tokens(logits_ref: np.ndarray, k: int, rel: float = 1e-4) -> np.ndarray:

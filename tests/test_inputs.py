@@ -73,3 +73,57 @@ def test_zipf_scale_matches_calibration_output():
     path = os.path.join(os.path.dirname(__file__), "golden", "zipf_bias_scale.json")
     with open(path) as f:
         assert json.load(f)["zipf_bias_scale"] == configs.ZIPF_BIAS_SCALE
+
+
+def test_redrawn_rows_come_from_their_generation():
+    cfg = configs.MUSE_DECODE
+    assert cfg.u_redraw, "the decode workload has stored redraws"
+    full = moe_inputs.host_rows(cfg, "u")
+    first = moe_inputs.host_rows(cfg.replace(u_redraw=()), "u")
+    red = dict(cfg.u_redraw)
+    for t in range(cfg.T):
+        g = red.get(t, 0)
+        row = moe_inputs.normal_host(cfg.seed, configs.STREAM_X, (g * cfg.T + t) * cfg.d_model,
+                                     cfg.d_model, cfg.x_sigma, "bf16")
+        np.testing.assert_array_equal(full[t], row)
+        assert np.array_equal(full[t], first[t]) == (g == 0)
+    rows = sorted(red)[:2] + [0]
+    np.testing.assert_array_equal(moe_inputs.host_rows(cfg, "u", rows=rows), full[rows])
+    # deriving a workload drops the list (it belongs to one workload)
+    assert cfg.replace(T=32).u_redraw == () and configs.small_muse().u_redraw == ()
+
+
+def _separation():
+    import importlib.util
+    path = os.path.join(os.path.dirname(__file__), "golden", "separate_router_logits.py")
+    spec = importlib.util.spec_from_file_location("separate_router_logits", path)
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod
+
+
+SMALL_SEPARATED = ("tiny_shazeer_f32", "shazeer_bf16", "muse_decode", "muse_decode_sigmoid",
+                   "muse_decode_block")
+
+
+def test_stored_redraws_recomputed_for_small_workloads():
+    sep = _separation()
+    for name in SMALL_SEPARATED:
+        cfg = configs.ALL_CONFIGS[name]
+        red, _ = sep.redraws_for(cfg)
+        assert red == cfg.u_redraw, name
+
+
+def test_large_workloads_are_separated_on_redrawn_and_sampled_tokens():
+    sep = _separation()
+    for name in configs.SEPARATED_NAMES:
+        if name in SMALL_SEPARATED:
+            continue
+        cfg = configs.ALL_CONFIGS[name]
+        sample = moe_inputs.fisher_yates(cfg.seed + 77, configs.STREAM_SUBSAMPLE, cfg.T, 256)
+        toks = np.union1d(np.array([t for t, _ in cfg.u_redraw], dtype=np.int64), sample)
+        ratio = sep.check_separated(cfg, toks)
+        assert ratio.min() >= 1.0, (name, float(ratio.min()))
+        # and the first draw of those redrawn tokens was not separated
+        red = np.array([t for t, _ in cfg.u_redraw][:64], dtype=np.int64)
+        assert sep.check_separated(cfg.replace(u_redraw=()), red).max() < 1.0, name

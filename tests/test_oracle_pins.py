@@ -39,6 +39,9 @@ def test_norm_worked_example():
     np.testing.assert_allclose(c, g["centered"], rtol=1e-15)
     expect = np.array(g["input_scaled_numerator"]) / math.sqrt(g["input_scaled_divisor_squared"])
     np.testing.assert_allclose(i, expect, rtol=1e-15)
+    # the vector I_gamma reduces is D_gamma x itself (the example's numerator)
+    np.testing.assert_array_equal(oracle.input_scaled_vector(x, gamma, is_bf16=2),
+                                  g["input_scaled_numerator"])
     # the two orders are collinear but not equal (same page)
     assert abs(c[0] * i[1] - c[1] * i[0]) < 1e-15 and not np.allclose(c, i)
 
@@ -259,7 +262,7 @@ def dense_bruteforce(cfg, inp):
     W1 = _val(inp["w_gu"], dt)
     W2 = _val(inp["w_down"], dt)
     I = cfg.d_ff
-    allout = []
+    allout, allpre = [], []
     for e in range(cfg.n_experts):
         a = z @ W1[e].T
         if cfg.act == configs.ACT_SWIGLU:
@@ -268,12 +271,16 @@ def dense_bruteforce(cfg, inp):
         else:
             hid = _rnd(np.maximum(a, 0), dt)
         o = _rnd(hid @ W2[e].T, dt)
+        s = o
         if cfg.expert_norm:
             s = _rnd(o * (1 + inp["gamma_expert"].astype(np.float64)), dt)
             o = _rnd(s / np.sqrt(np.mean(s * s, 1, keepdims=True) + cfg.eps), dt)
         allout.append(o)
+        allpre.append(s)
     allout = np.stack(allout, 1)  # [T, n, E]
     sel = np.take_along_axis(allout, top[:, :, None], 1)
+    dense_bruteforce.last = {"z": z,
+                             "s": np.take_along_axis(np.stack(allpre, 1), top[:, :, None], 1)}
     y = _rnd(np.einsum("tk,tke->te", w, sel), dt)
     if cfg.latent:
         b = _rnd(y @ _val(inp["p_up"], dt).T, dt)
@@ -391,6 +398,26 @@ def test_layer_bruteforce(cfg):
     np.testing.assert_allclose(res["w"], w, rtol=1e-12)
     np.testing.assert_allclose(res["y"], y, rtol=1e-9, atol=1e-12)
     np.testing.assert_allclose(res["out"], out, rtol=1e-9, atol=1e-12)
+
+
+@pytest.mark.parametrize("cfg", [c for c in BRUTE_CASES if c.latent], ids=lambda c: c.name)
+def test_staged_intermediates_bruteforce(cfg):
+    """The staged driver's expert inputs z and per-slot pre-norm expert outputs s (the vector
+    I_gamma reduces) against the dense brute force."""
+    inp = moe_inputs.host_inputs(cfg)
+    toks = np.arange(cfg.T)
+
+    def get_inputs(tokens):
+        d = {k: v for k, v in inp.items() if k not in ("w_gu", "w_down")}
+        d["u"] = inp["u"][tokens]
+        return d
+
+    res = oracle.layer_forward_staged(cfg, toks, get_inputs,
+                                      lambda e: (inp["w_gu"][e], inp["w_down"][e]), want_s=True)
+    dense_bruteforce(cfg, inp)
+    ref = dense_bruteforce.last
+    np.testing.assert_allclose(res["z"], ref["z"], rtol=1e-9, atol=1e-12)
+    np.testing.assert_allclose(res["s"], ref["s"], rtol=1e-9, atol=1e-12)
 
 
 def test_k_equals_n_is_dense_softmax_mixture():

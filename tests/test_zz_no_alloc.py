@@ -1,8 +1,8 @@
 """moe_permute_static: the dispatch permutation for callers that cannot allocate device memory
 (a host that passes only input and output buffers and has no scratch pool to offer).  Its
 scratch is a fixed array inside the library, so the test checks that two calls in a row, of
-different sizes, give the same outputs as moe_permute with a caller workspace, and that a size
-beyond the array is refused before anything runs.
+different sizes, give the same outputs as moe_permute with a caller workspace and the oracle's
+canonical permutation, and that a size beyond the array is refused before anything runs.
 
 Kept in its own file, collected last, so that a failure here cannot hide any other test.
 """
@@ -10,6 +10,7 @@ import numpy as np
 import pytest
 
 import moe_inputs
+import oracle
 from moe_inputs import configs
 
 from gpu_harness import abi_config
@@ -55,13 +56,26 @@ def test_permute_static_matches_workspace_version_twice():
         got = _run(cfg, idx, use_static=True)
         for a, b in zip(got[:3], ref[:3]):
             np.testing.assert_array_equal(a.numpy(), b.numpy())
+        # and both equal the oracle's canonical permutation of the same routing
+        for a, b in zip(got[:3], oracle.permutation(cfg.T, cfg.top_k, cfg.n_experts, idx)):
+            np.testing.assert_array_equal(a.numpy(), b)
         # same kernels on the same inputs: the gathered, normalised rows agree exactly
         np.testing.assert_array_equal(got[3].float().numpy(), ref[3].float().numpy())
 
 
 def test_permute_static_rejects_sizes_beyond_its_scratch():
+    # real input and output buffers of the refused size (no stand-in addresses): the call is
+    # refused on the host, so the outputs keep their fill
     cfg = configs.small_muse(T=32769, n=256, k=8)  # ceil(T/128) * 256 > 65536
     c = abi_config(cfg)
+    T, k, n = cfg.T, cfg.top_k, cfg.n_experts
+    idx = torch.from_numpy(_routing(T, n, k, 63)).cuda()
+    off = torch.full((n + 1,), -5, dtype=torch.int32, device="cuda")
+    perm = torch.full((T * k,), -5, dtype=torch.int32, device="cuda")
+    inv = torch.full((T * k,), -5, dtype=torch.int32, device="cuda")
     with pytest.raises(moe.MoeError) as e:
-        moe.moe_permute_static(c, 0x1000, 0x1000, 0x1000, 0x1000)
+        moe.moe_permute_static(c, idx, off, perm, inv)
     assert e.value.code == moe.STATUS_CODES["MOE_ERR_WORKSPACE"]
+    torch.cuda.synchronize()
+    for t in (off, perm, inv):  # nothing was launched: the outputs still hold their fill
+        assert bool((t == -5).all())
