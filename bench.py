@@ -347,6 +347,7 @@ def measure_ours(cfg, steps: int, warmup: int, device, peaks: dict, with_e2e: bo
     ms_max = reduce_max(ms, device)
     p50 = reduce_max(float(np.percentile(per_step, 50)), device)
     p90 = reduce_max(float(np.percentile(per_step, 90)), device)
+    step_range = (round(min(per_step), 4), round(max(per_step), 4))
     status = moe.moe_get_device_status()
     if status != 0:
         raise RuntimeError(f"device status {moe.STATUS.get(status, status)} after timing")
@@ -375,6 +376,7 @@ def measure_ours(cfg, steps: int, warmup: int, device, peaks: dict, with_e2e: bo
     t_exp = max(work["experts"]["flops"] / (peaks["bf16_tflops_sustained"] * 1e12),
                 work["experts"]["bytes"] / (peaks["hbm_gbs"] * 1e9))
     res = {"ms_per_step": ms_max, "ms_p50": round(p50, 4), "ms_p90": round(p90, 4),
+           "ms_min_max": step_range,
            "tokens_per_step": cfg.T, "roofline": roof,
            "layer_roofline": {"bound": "tensor" if tensor_bound else "hbm",
                               "flops": work["flops"], "bytes": work["bytes"],
@@ -786,7 +788,8 @@ def main(argv=None) -> int:
     line = {"metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(res["ms_per_step"], 4),
-            "ms_p50": res["ms_p50"], "ms_p90": res["ms_p90"], "higher_is_better": True,
+            "ms_p50": res["ms_p50"], "ms_p90": res["ms_p90"], "ms_min_max": res["ms_min_max"],
+            "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded counter-based generator; random-init weights)",
             "config": config_block(cfg, world),

@@ -157,6 +157,16 @@ MOE_API moe_status_t moe_permute(const moe_config_t* cfg, const int32_t* topk_id
                          const void* x, const float* gamma_pre, void* x_perm, void* workspace,
                          size_t workspace_bytes, void* stream);
 
+/* The row half of moe_permute, for a caller that already holds the permutation (for example
+ * after reading the expert offsets back while another kernel runs): x_perm[inv_perm[t*k+j]] =
+ * f(x[t]) with f = C_pre (gain 1+gamma_pre) when gamma_pre is not NULL (bf16 with a latent
+ * width), else the identity [MUSE "Latent experts"].  x: [T, E_in]; x_perm: [T*k, E_in];
+ * inv_perm: [T*k] as moe_permute returns it (a negative entry skips that slot).  Errors as for
+ * moe_permute. */
+MOE_API moe_status_t moe_dispatch_rows(const moe_config_t* cfg, const int32_t* inv_perm,
+                                       const void* x, const float* gamma_pre, void* x_perm,
+                                       void* stream);
+
 /* moe_permute without a workspace argument, for callers that cannot allocate device memory: a
  * plugin or embedding host that hands the library only its input and output buffers (no
  * allocator handle, no scratch pool), or code that may not call cudaMalloc on its path because

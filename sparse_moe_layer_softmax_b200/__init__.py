@@ -31,7 +31,8 @@ EXPORTS = ("moe_status_string", "moe_workspace_size", "moe_route", "moe_permute"
            "moe_launch_count", "moe_permute_static", "moe_selftest_wait_timeout",
            "moe_router_split_weights", "moe_residual_update", "moe_noisy_gate",
            "moe_noisy_gate_workspace_size", "moe_host_staging_size", "moe_layer_forward_host",
-           "moe_row_sumsq_parts", "moe_gather_rows", "moe_layer_forward_taps")
+           "moe_row_sumsq_parts", "moe_gather_rows", "moe_layer_forward_taps",
+           "moe_dispatch_rows")
 PROFILE_STAGES = ("route", "latent_down", "dispatch", "expert_gate_up", "expert_down", "combine",
                   "latent_up_resgate")
 
@@ -105,6 +106,7 @@ def lib():
             "moe_profile_begin": [ctypes.c_int32],
             "moe_profile_end": [vp, vp],
             "moe_permute_static": [cp, vp, vp, vp, vp, vp, vp, vp, vp],
+            "moe_dispatch_rows": [cp, vp, vp, vp, vp, vp],
             "moe_selftest_wait_timeout": [ctypes.c_longlong, vp, vp],
         }
         for name, args in sigs.items():
@@ -226,6 +228,13 @@ def moe_permute_static(cfg, topk_idx, expert_offsets, perm_token, inv_perm, x=No
     _check("moe_permute_static", lib().moe_permute_static(
         ctypes.byref(cfg), _ptr(topk_idx), _ptr(expert_offsets), _ptr(perm_token),
         _ptr(inv_perm), _ptr(x), _ptr(gamma_pre), _ptr(x_perm), _stream(stream)))
+
+
+def moe_dispatch_rows(cfg, inv_perm, x, gamma_pre, x_perm, stream=None):
+    """The row half of moe_permute: x_perm[inv_perm[t*k+j]] = C_pre(x[t]) (or x[t])."""
+    _check("moe_dispatch_rows", lib().moe_dispatch_rows(
+        ctypes.byref(cfg), _ptr(inv_perm), _ptr(x), _ptr(gamma_pre), _ptr(x_perm),
+        _stream(stream)))
 
 
 def moe_expert_ffn(cfg, x_perm, expert_offsets, w_gu, w_down, gamma_expert, out_perm,

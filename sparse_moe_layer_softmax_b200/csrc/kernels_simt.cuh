@@ -458,6 +458,158 @@ __global__ void __launch_bounds__(kCombineMaxThreads)
   }
 }
 
+// The same combine for prefill-sized batches, with the expert rows brought in by bulk copies:
+// one persistent CTA per SM walks its tokens (t = blockIdx.x, + gridDim.x, ...).  A producer
+// warp keeps up to `nst` tokens in flight in a shared-memory ring: its lane j < k reads slot j's
+// dispatch row and weight (the next token's are loaded while the current token's stage frees
+// up), then copies that row's E values and, with expert_norm, its `parts` partial sums of squares
+// into the stage.  Eight consumer warps finish the token at the head of the ring and write y.
+// Every wait is bounded; a timeout latches MOE_ERR_TIMEOUT and the roles stop.
+constexpr int kBulkCombineConsumers = 256;
+
+struct BulkCombineStage {
+  // byte offsets inside one stage
+  int rows, ss, hdr, bytes;
+};
+__host__ __device__ inline BulkCombineStage bulk_combine_stage(int E, int k, int parts) {
+  BulkCombineStage b;
+  b.rows = 0;
+  b.ss = (k * E * 2 + 127) / 128 * 128;
+  b.hdr = b.ss + (k * parts * 4 + 127) / 128 * 128;
+  b.bytes = b.hdr + 128;  // row indices [8] and weights [8]
+  return b;
+}
+
+__global__ void __launch_bounds__(kBulkCombineConsumers + 32, 1)
+    combine_bf16_bulk_kernel(const uint16_t* __restrict__ s, int E, int k,
+                             const int32_t* __restrict__ inv_perm,
+                             const float* __restrict__ topk_w, const float* __restrict__ row_ss,
+                             int parts, int expert_norm, float eps, uint16_t* __restrict__ y,
+                             int T, int nst) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) &
+                                             ~static_cast<uintptr_t>(127));
+  const BulkCombineStage L = bulk_combine_stage(E, k, parts);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + static_cast<size_t>(nst) * L.bytes);
+  uint64_t* empty = full + nst;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  constexpr int kConsumerWarps = kBulkCombineConsumers / 32;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < nst; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], kConsumerWarps); }
+    fence_barrier_init();
+  }
+  __syncthreads();
+  const bool norm = expert_norm != 0;
+  if (warp == kConsumerWarps) {
+    // ------------------------------------------------------------ producer warp
+    int nrow = -1;
+    float nw = 0.0f;
+    int t = blockIdx.x;
+    if (t < T && lane < k) {
+      nrow = __ldg(inv_perm + static_cast<size_t>(t) * k + lane);
+      nw = __ldg(topk_w + static_cast<size_t>(t) * k + lane);
+    }
+    for (int i = 0; t < T; ++i, t += gridDim.x) {
+      const int row = nrow;
+      const float w = nw;
+      const int tn = t + gridDim.x;  // the next token's slots load while this one is placed
+      if (tn < T && lane < k) {
+        nrow = __ldg(inv_perm + static_cast<size_t>(tn) * k + lane);
+        nw = __ldg(topk_w + static_cast<size_t>(tn) * k + lane);
+      }
+      const int st = i % nst;
+      const uint32_t ph = static_cast<uint32_t>(i / nst) & 1u;
+      if (!__all_sync(0xffffffffu, mbar_wait(&empty[st], ph ^ 1u))) break;
+      uint8_t* sb = smem + static_cast<size_t>(st) * L.bytes;
+      int* hrow = reinterpret_cast<int*>(sb + L.hdr);
+      float* hw = reinterpret_cast<float*>(sb + L.hdr + 32);
+      const bool valid = lane < k && row >= 0;
+      if (lane < kMaxTopK) {
+        hrow[lane] = lane < k ? row : -1;
+        hw[lane] = lane < k ? w : 0.0f;
+      }
+      uint32_t bytes = valid ? static_cast<uint32_t>(E * 2 + (norm ? parts * 4 : 0)) : 0u;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) bytes += __shfl_xor_sync(0xffffffffu, bytes, o);
+      __syncwarp();
+      if (lane == 0) mbar_arrive_expect_tx(&full[st], bytes);  // releases the header too
+      __syncwarp();
+      if (valid) {
+        bulk_load(sb + L.rows + static_cast<size_t>(lane) * E * 2, s + static_cast<size_t>(row) * E,
+                  static_cast<uint32_t>(E * 2), &full[st]);
+        if (norm)
+          bulk_load(sb + L.ss + lane * parts * 4, row_ss + static_cast<size_t>(row) * parts,
+                    static_cast<uint32_t>(parts * 4), &full[st]);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ consumer warps
+    const int nvec = E / 8;
+    int i = 0;
+    for (int t = blockIdx.x; t < T; ++i, t += gridDim.x) {
+      const int st = i % nst;
+      const uint32_t ph = static_cast<uint32_t>(i / nst) & 1u;
+      if (!__all_sync(0xffffffffu, mbar_wait(&full[st], ph))) break;
+      const uint8_t* sb = smem + static_cast<size_t>(st) * L.bytes;
+      const int* hrow = reinterpret_cast<const int*>(sb + L.hdr);
+      const float* hw = reinterpret_cast<const float*>(sb + L.hdr + 32);
+      // slot j's I_gamma factor from its partials, in part order (lane j), to every lane
+      float my_rinv = 1.0f;
+      if (norm && lane < k && hrow[lane] >= 0) {
+        const float* ps = reinterpret_cast<const float*>(sb + L.ss) + lane * parts;
+        float tot = 0.0f;
+        for (int p = 0; p < parts; ++p) tot += ps[p];
+        my_rinv = rsqrtf(tot / static_cast<float>(E) + eps);
+      }
+      float rinv[kMaxTopK], wgt[kMaxTopK];
+      bool use[kMaxTopK];
+#pragma unroll
+      for (int j = 0; j < kMaxTopK; ++j) {
+        rinv[j] = __shfl_sync(0xffffffffu, my_rinv, j);
+        use[j] = j < k && hrow[j] >= 0;
+        wgt[j] = hw[j];
+      }
+      for (int v = threadIdx.x; v < nvec; v += kBulkCombineConsumers) {
+        float2 acc[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) acc[q] = make_float2(0.0f, 0.0f);
+#pragma unroll
+        for (int j = 0; j < kMaxTopK; ++j) {
+          if (!use[j]) continue;
+          const uint4 qv = *reinterpret_cast<const uint4*>(sb + L.rows + (static_cast<size_t>(j) * E + v * 8) * 2);
+          const uint32_t* w4 = reinterpret_cast<const uint32_t*>(&qv);
+          const float2 r2 = make_float2(rinv[j], rinv[j]);
+          const float2 w2 = make_float2(wgt[j], wgt[j]);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            float2 nv = bf16x2_to_f2(w4[q]);
+            if (norm) nv = bf16x2_to_f2(f2_to_bf16x2(__fmul2_rn(nv, r2)));  // dtype(s / denom)
+            acc[q] = __ffma2_rn(w2, nv, acc[q]);
+          }
+        }
+        uint4 o;
+        o.x = f2_to_bf16x2(acc[0]);
+        o.y = f2_to_bf16x2(acc[1]);
+        o.z = f2_to_bf16x2(acc[2]);
+        o.w = f2_to_bf16x2(acc[3]);
+        reinterpret_cast<uint4*>(y + static_cast<size_t>(t) * E)[v] = o;
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[st]);
+    }
+  }
+  // No copy is still landing at exit: every stage the producer filled was waited on by the
+  // consumers, except after a timeout; then the producer's last copies are waited for here.
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const int issued = T > static_cast<int>(blockIdx.x)
+                           ? (T - 1 - static_cast<int>(blockIdx.x)) / static_cast<int>(gridDim.x) + 1
+                           : 0;
+    for (int i = issued > nst ? issued - nst : 0; i < issued; ++i)
+      mbar_wait(&full[i % nst], static_cast<uint32_t>(i / nst) & 1u, 1000000ll);
+  }
+}
+
 __global__ void combine_f32_kernel(const float* __restrict__ s, int E, int k,
                                    const int32_t* __restrict__ inv_perm,
                                    const float* __restrict__ topk_w, int expert_norm, float eps,

@@ -9,6 +9,7 @@
 #include <vector>
 
 #include "common.cuh"
+#include "gemm_swap_pair.cuh"
 #include "gemm_tc.cuh"
 #include "kernels_simt.cuh"
 
@@ -150,10 +151,38 @@ moe_status_t launch_gemm_pair(const void* X, long x_rows, const void* W, long w_
   return last_launch();
 }
 
+// Swapped CTA-pair variant (prefill-sized expert groups): grid of whole clusters of 2.
+template <int kEpi, int kStages>
+moe_status_t launch_gemm_swap_pair(const void* X, long x_rows, const void* W, long w_rows,
+                                   const GemmParams& p, long max_tiles, cudaStream_t st) {
+  using S = SwapPairShape<kEpi>;
+  constexpr int smem = gemm_swap_pair_smem_bytes<kEpi, kStages>();
+  static_assert(smem <= 232448, "shared memory budget");
+  auto kern = gemm_swap_pair_kernel<kEpi, kStages>;
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [&] {
+    attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  });
+  if (attr_err != cudaSuccess) return MOE_ERR_CUDA;
+  if (p.x_k_period > 0 || p.k_splits > 1 || !p.seg) return MOE_ERR_UNSUPPORTED;
+  CUtensorMap tx, tw;
+  if (!make_tmap(&tx, X, static_cast<uint64_t>(x_rows), static_cast<uint64_t>(p.K), 128))
+    return MOE_ERR_CUDA;
+  if (!make_tmap(&tw, W, static_cast<uint64_t>(w_rows), static_cast<uint64_t>(p.K), S::kWBoxRows))
+    return MOE_ERR_CUDA;
+  if (max_tiles <= 0) return MOE_OK;
+  long pairs = device_info().sms / 2;
+  if (pairs <= 0) return MOE_ERR_CUDA;  // the SM count could not be read
+  if (max_tiles < pairs) pairs = max_tiles;
+  kern<<<static_cast<unsigned>(2 * pairs), kGemmThreads, smem, st>>>(tx, tw, p);
+  return last_launch();
+}
+
 // Upper bound of the tile count of a grouped GEMM (each group adds at most one partial chunk).
 long tile_bound(long rows, int G, int ch, int ft) { return (static_cast<long>(cdiv(rows, ch)) + G) * ft; }
 
-enum class Orient { kNormal, kSwap, kPair };
+enum class Orient { kNormal, kSwap, kPair, kSwapPair };
 
 // Output-feature tile choice of the normal orientation: the widest of 256/128/64 dividing Nout
 // (for SwiGLU the tile holds gate and up halves, so the output width per tile is BN/2).
@@ -179,6 +208,15 @@ moe_status_t run_gemm(int epi, Orient o, int bn, const void* X, long x_rows, con
     SW(16, EPI_RESGATE, 10) SW(32, EPI_RESGATE, 9) SW(64, EPI_RESGATE, 8)
     SW(64, EPI_PARTIAL, 8)
 #undef SW
+    return MOE_ERR_UNSUPPORTED;
+  }
+  if (o == Orient::kSwapPair) {
+    const int fo = dual ? SwapPairShape<EPI_SWIGLU>::kFO : SwapPairShape<EPI_STORE>::kFO;
+    if (p.Nout % fo) return MOE_ERR_UNSUPPORTED;
+    const long pt = tile_bound(x_rows, p.G, 256, p.Nout / fo);
+    if (epi == EPI_SWIGLU) return launch_gemm_swap_pair<EPI_SWIGLU, 6>(X, x_rows, W, w_rows, p, pt, st);
+    if (epi == EPI_STORE) return launch_gemm_swap_pair<EPI_STORE, 6>(X, x_rows, W, w_rows, p, pt, st);
+    if (epi == EPI_RELU) return launch_gemm_swap_pair<EPI_RELU, 6>(X, x_rows, W, w_rows, p, pt, st);
     return MOE_ERR_UNSUPPORTED;
   }
   const int fo = dual ? bn / 2 : bn;
@@ -292,11 +330,26 @@ bool pair_tiles_enabled() {
 // Grouped-GEMM orientation for the experts from the mean rows per expert.
 int expert_in_width(const moe_config_t& c) { return c.d_latent > 0 ? c.d_latent : c.d_model; }
 
+// Tuning knob: MOE_EXPERT_TILES=swap_pair in the environment puts prefill-sized expert GEMMs on
+// the swapped CTA-pair tiles instead of the 1-SM 128-row activation tiles (same values up to the
+// fp32 summation inside the tensor core).  Off by default: under the 1 kW power cap the pair
+// tiles do more work per clock but spend more energy per launch, so they run at lower clocks and
+// take longer.
+bool swap_pair_enabled() {
+  const char* v = getenv("MOE_EXPERT_TILES");
+  return v && v[0] == 's';
+}
+
 void pick_expert_orient(const moe_config_t& c, int nout, bool dual, Orient* o, int* bn) {
   const double mean_rows = static_cast<double>(c.T) * c.top_k / c.n_experts;
   if (nout % 128 == 0 && mean_rows <= 48.0) {
     *o = Orient::kSwap;
     *bn = mean_rows <= 12.0 ? 16 : (mean_rows <= 24.0 ? 32 : 64);
+  } else if (swap_pair_enabled() && !pair_tiles_enabled() &&
+             nout % (dual ? SwapPairShape<EPI_SWIGLU>::kFO : SwapPairShape<EPI_STORE>::kFO) == 0) {
+    // prefill-sized groups: tokens on the MMA's N side, cut to 16 rows, on CTA pairs
+    *o = Orient::kSwapPair;
+    *bn = 256;
   } else {
     *bn = pick_bn_normal(nout, dual);
     // 256-row CTA-pair tiles once groups are large enough to fill them
@@ -307,13 +360,15 @@ void pick_expert_orient(const moe_config_t& c, int nout, bool dual, Orient* o, i
 
 // Dense projections: CTA-pair tiles for at least 256 rows and a 256-wide feature tile.
 // Partial sums of squares per expert-output row that the expert down GEMM writes (row_sumsq):
-// one per 256/128/64-column feature tile in the normal (and CTA-pair) orientation, one per
-// 32-feature warp slice of each 128-feature tile in the swapped orientation.
+// one per 256/128/64-column feature tile in the normal (and CTA-pair) orientation, one per CTA's
+// 128 features in the swapped CTA-pair orientation, one per 32-feature warp slice of each
+// 128-feature tile in the swapped orientation.
 int sumsq_parts(const moe_config_t& c) {
   Orient o;
   int bn;
   pick_expert_orient(c, expert_in_width(c), false, &o, &bn);
   if (bn <= 0) return 1;
+  if (o == Orient::kSwapPair) return expert_in_width(c) / 128;  // one per CTA's 128 features
   return o == Orient::kSwap ? expert_in_width(c) / 128 * 4 : expert_in_width(c) / bn;
 }
 
@@ -448,6 +503,9 @@ moe_status_t do_route(const moe_config_t& c, const void* u, const void* w_router
   return last_launch();
 }
 
+moe_status_t do_dispatch_rows(const moe_config_t& c, const int32_t* inv, const void* x,
+                              const float* gamma_pre, void* x_perm, cudaStream_t st);
+
 moe_status_t do_permute(const moe_config_t& c, const int32_t* idx, int32_t* offsets,
                         int32_t* perm, int32_t* inv, const void* x, const float* gamma_pre,
                         void* x_perm, int32_t* counts, cudaStream_t st) {
@@ -461,6 +519,12 @@ moe_status_t do_permute(const moe_config_t& c, const int32_t* idx, int32_t* offs
   perm_rank_kernel<<<nc, 32, 0, st>>>(idx, c.T, k, n, counts, offsets, perm, inv);
   moe_status_t s = last_launch(3);
   if (s != MOE_OK || !x) return s;
+  return do_dispatch_rows(c, inv, x, gamma_pre, x_perm, st);
+}
+
+moe_status_t do_dispatch_rows(const moe_config_t& c, const int32_t* inv, const void* x,
+                              const float* gamma_pre, void* x_perm, cudaStream_t st) {
+  const int k = c.top_k;
   const int E = c.d_latent > 0 ? c.d_latent : c.d_model;
   if (c.dtype == MOE_F32) {
     scatter_rows_f32_kernel<float><<<c.T, 128, 0, st>>>(static_cast<const float*>(x), E, k, inv,
@@ -558,6 +622,9 @@ moe_status_t do_experts(const moe_config_t& c, const void* x_perm, const int32_t
   return run_gemm(EPI_STORE, o2, bn2, act, TK, w_down, static_cast<long>(n) * E, p2, st);
 }
 
+constexpr int kBulkCombineMinT = 1024;        // tokens from which the bulk-copy combine runs
+constexpr int kBulkCombineSmem = 220 * 1024;   // its shared-memory ring, at most
+
 moe_status_t do_combine(const moe_config_t& c, const void* s, const int32_t* inv,
                         const float* w, void* y, cudaStream_t st, const float* row_ss = nullptr) {
   if (c.T == 0) return MOE_OK;
@@ -572,6 +639,28 @@ moe_status_t do_combine(const moe_config_t& c, const void* s, const int32_t* inv
   const int vec = cdiv(nvec, threads);
   const uint16_t* sp = static_cast<const uint16_t*>(s);
   uint16_t* yp = static_cast<uint16_t*>(y);
+  // Prefill-sized batches: one persistent CTA per SM with the expert rows (and their partial
+  // sums of squares) brought in by bulk copies, when the row partials are given or no norm is
+  // taken and at least two tokens' rows fit in shared memory.
+  const int parts_b = row_ss && c.expert_norm ? sumsq_parts(c) : 0;
+  if (c.T >= kBulkCombineMinT && (parts_b * 4) % 16 == 0 && (!c.expert_norm || row_ss)) {
+    const BulkCombineStage B = bulk_combine_stage(E, c.top_k, parts_b);
+    const int nst = std::min(8, (kBulkCombineSmem - 128 - 16 * 8) / B.bytes);
+    if (nst >= 2) {
+      const size_t smem = 128 + static_cast<size_t>(nst) * B.bytes + 16 * static_cast<size_t>(nst);
+      static std::once_flag once;
+      static cudaError_t attr = cudaSuccess;
+      std::call_once(once, [] {
+        attr = cudaFuncSetAttribute(combine_bf16_bulk_kernel,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, kBulkCombineSmem);
+      });
+      if (attr != cudaSuccess) return MOE_ERR_CUDA;
+      const int grid = std::min(c.T, std::max(device_info().sms, 1));
+      combine_bf16_bulk_kernel<<<grid, kBulkCombineConsumers + 32, smem, st>>>(
+          sp, E, c.top_k, inv, w, row_ss, parts_b, c.expert_norm, c.eps, yp, c.T, nst);
+      return last_launch();
+    }
+  }
   if (row_ss && c.expert_norm) {
     const int parts = sumsq_parts(c);
     switch (vec) {
@@ -909,6 +998,19 @@ moe_status_t moe_permute_static(const moe_config_t* cfg, const int32_t* topk_idx
   // The count kernel overwrites every histogram entry this call uses, so no clearing is needed.
   return do_permute(*cfg, topk_idx, expert_offsets, perm_token, inv_perm, x, gamma_pre, x_perm,
                     scratch, static_cast<cudaStream_t>(stream));
+}
+
+moe_status_t moe_dispatch_rows(const moe_config_t* cfg, const int32_t* inv_perm, const void* x,
+                               const float* gamma_pre, void* x_perm, void* stream) {
+  moe_status_t s = check_cfg(cfg);
+  if (s != MOE_OK) return s;
+  if (cfg->T > 0 && (!inv_perm || !x || !x_perm)) return MOE_ERR_INVALID_ARG;
+  if (gamma_pre && (cfg->dtype != MOE_BF16 || cfg->d_latent == 0)) return MOE_ERR_UNSUPPORTED;
+  if (!all_aligned({static_cast<const void*>(inv_perm), x, static_cast<const void*>(gamma_pre),
+                    x_perm}))
+    return MOE_ERR_ALIGNMENT;
+  if (cfg->T == 0) return MOE_OK;
+  return do_dispatch_rows(*cfg, inv_perm, x, gamma_pre, x_perm, static_cast<cudaStream_t>(stream));
 }
 
 moe_status_t moe_row_sumsq_parts(const moe_config_t* cfg, int32_t* parts) {

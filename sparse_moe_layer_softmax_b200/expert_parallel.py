@@ -2,9 +2,10 @@
 the experts (a contiguous range) and its own tokens.
 
 Per forward, on every rank:
-  1. route, latent down-projection and dispatch of the rank's own tokens (moe_route,
-     moe_latent_down, moe_permute).  The dispatched rows come out grouped by expert, hence by
-     the rank that owns each expert;
+  1. route, then the dispatch permutation of the rank's own tokens (moe_route, moe_permute);
+     its per-expert offsets go to pinned host memory by an asynchronous copy that overlaps the
+     latent down-projection (moe_latent_down), and the rows are dispatched (moe_dispatch_rows).
+     The dispatched rows come out grouped by expert, hence by the rank that owns each expert;
   2. exchange: the rows for owner rank d are sent to d (all-to-all), with the per-expert counts;
   3. on the owner: the received rows, ordered (source rank, expert, token), are regrouped by
      expert (moe_gather_rows), the rank's experts run on them (moe_expert_ffn), and the outputs
@@ -16,7 +17,10 @@ Per forward, on every rank:
 The exchange is a callable, so that the same stages run over torch.distributed
 (all_to_all_single: NCCL between GPUs, gloo between CPU processes) or with all ranks emulated in
 one process.  Every arithmetic step is one of the library's kernels; this module only plans the
-exchange (integer bookkeeping on the host) and moves rows.
+exchange (integer bookkeeping on the host) and moves rows.  A rank keeps its buffers between
+forwards (the ones whose size depends on the rows received grow when a forward needs more), so a
+steady stream of forwards allocates nothing; the host reads the expert counts once per forward,
+while the latent down-projection runs.
 """
 from __future__ import annotations
 
@@ -24,8 +28,8 @@ import dataclasses
 
 import numpy as np
 
-from . import (Config, moe_combine, moe_expert_ffn, moe_gather_rows, moe_latent_down,
-               moe_latent_up, moe_permute, moe_route, workspace_size, MOE_BF16)
+from . import (Config, moe_combine, moe_dispatch_rows, moe_expert_ffn, moe_gather_rows,
+               moe_latent_down, moe_latent_up, moe_permute, moe_route, workspace_size, MOE_BF16)
 
 
 # ---------------------------------------------------------------- exchange plan (host integers)
@@ -74,15 +78,16 @@ def inverse_rows(rows: np.ndarray) -> np.ndarray:
 # ---------------------------------------------------------------- exchange over torch.distributed
 
 def dist_exchange(group=None):
-    """An exchange callable over torch.distributed: exchange(send, send_splits, recv_splits)
+    """An exchange callable over torch.distributed: exchange(send, send_splits, recv_splits, out)
     sends rows send[sum(send_splits[:d]) : ...] to rank d and returns the rows received, ordered by
-    source rank."""
+    source rank, in `out` (a buffer of exactly sum(recv_splits) rows) or a new tensor."""
     import torch
     import torch.distributed as dist
 
-    def exchange(send, send_splits, recv_splits):
-        recv = torch.empty((int(sum(recv_splits)),) + tuple(send.shape[1:]), dtype=send.dtype,
-                           device=send.device)
+    def exchange(send, send_splits, recv_splits, out=None):
+        rows = int(sum(recv_splits))
+        recv = out if out is not None else torch.empty(
+            (rows,) + tuple(send.shape[1:]), dtype=send.dtype, device=send.device)
         dist.all_to_all_single(recv, send.contiguous(), [int(x) for x in recv_splits],
                                [int(x) for x in send_splits], group=group)
         return recv
@@ -115,6 +120,26 @@ class Dispatched:
     counts: np.ndarray   # [world, n_local] rows for each (owner rank, owner's local expert)
 
 
+class _Grow:
+    """A buffer kept between forwards and reallocated only when a forward needs a larger one."""
+
+    def __init__(self, dtype, device, pin: bool = False):
+        self.dtype, self.device, self.pin = dtype, device, pin
+        self.buf = None
+
+    def get(self, *shape):
+        import math
+        import torch
+        numel = max(1, math.prod(shape))
+        if self.buf is None or self.buf.numel() < numel:
+            numel = max(numel, 2 * (0 if self.buf is None else self.buf.numel()))
+            if self.pin:
+                self.buf = torch.empty(numel, dtype=self.dtype, pin_memory=True)
+            else:
+                self.buf = torch.empty(numel, dtype=self.dtype, device=self.device)
+        return self.buf[:math.prod(shape)].view(*shape)
+
+
 class ExpertParallelRank:
     """One rank of an expert-parallel layer.
 
@@ -122,7 +147,11 @@ class ExpertParallelRank:
     weights: as for MoELayer, except that w_gu and w_down hold only this rank's experts
     ([n_local, ...], experts [lo, hi) of expert_ranges); the router and latent weights are whole.
     Supported: bf16; no decoder wrap (input_norm / post_norm); a router_f32 router must be given
-    as its bf16 split (moe_router_split_weights)."""
+    as its bf16 split (moe_router_split_weights).
+
+    The rank owns its buffers: the dispatch-side ones (fixed by T) are made here, the ones sized
+    by the rows a forward receives grow on demand.  A forward's Dispatched state and its
+    exchanged rows live in these buffers until the next forward."""
 
     def __init__(self, cfg: Config, weights: dict, rank: int, world: int):
         import torch
@@ -133,7 +162,34 @@ class ExpertParallelRank:
         self.n_local = self.hi - self.lo
         if weights["w_gu"].shape[0] != self.n_local or weights["w_down"].shape[0] != self.n_local:
             raise ValueError("w_gu / w_down must hold exactly this rank's experts")
-        self.workspace = torch.empty(workspace_size(cfg), dtype=torch.uint8, device="cuda")
+        dev = weights["w_gu"].device
+        dt = weights["w_gu"].dtype
+        T, k, n = cfg.T, cfg.top_k, cfg.n_experts
+        E = cfg.d_latent if cfg.d_latent > 0 else cfg.d_model
+        self.workspace = torch.empty(workspace_size(cfg), dtype=torch.uint8, device=dev)
+        self.logits = torch.empty((T, n), dtype=torch.float32, device=dev)
+        self.idx = torch.empty((T, k), dtype=torch.int32, device=dev)
+        self.wt = torch.empty((T, k), dtype=torch.float32, device=dev)
+        self.z = torch.empty((T, E), dtype=dt, device=dev) if cfg.d_latent > 0 else None
+        self.offsets = torch.empty(n + 1, dtype=torch.int32, device=dev)
+        self.perm = torch.empty(T * k, dtype=torch.int32, device=dev)
+        self.inv = torch.empty(T * k, dtype=torch.int32, device=dev)
+        self.x_perm = torch.empty((T * k, E), dtype=dt, device=dev)
+        self.y = torch.empty((T, E), dtype=dt, device=dev)
+        self.offsets_host = torch.empty(n + 1, dtype=torch.int32, pin_memory=True)
+        self.offsets_ready = torch.cuda.Event()
+        self.plan_done = torch.cuda.Event()
+        self.plan_done.record()
+        # sized by the rows received (and sent back) in a forward
+        self.recv = _Grow(dt, dev)
+        self.back_recv = _Grow(dt, dev)
+        self.grouped = _Grow(dt, dev)
+        self.expert_out = _Grow(dt, dev)
+        self.back = _Grow(dt, dev)
+        self.plan_host = _Grow(torch.int32, None, pin=True)
+        self.plan_dev = _Grow(torch.int32, dev)
+        self.expert_ws = _Grow(torch.uint8, dev)
+        self.E = E
 
     def _local_cfg(self, rows: int) -> Config:
         """The expert FFN's configuration on this rank: `rows` received rows over n_local experts."""
@@ -141,81 +197,93 @@ class ExpertParallelRank:
         c.T, c.top_k, c.n_experts = rows, 1, self.n_local
         return c
 
+    def recv_buffer(self, rows: int):
+        """Buffer for the rows this rank receives in a forward's dispatch exchange."""
+        return self.recv.get(rows, self.E)
+
+    def return_buffer(self, rows: int):
+        """Buffer for the rows that come back to this rank in a forward's return exchange."""
+        return self.back_recv.get(rows, self.E)
+
     def dispatch(self, u) -> Dispatched:
-        import torch
         c, w = self.cfg, self.weights
-        T, k, n = c.T, c.top_k, c.n_experts
-        dev = u.device
-        logits = torch.empty((T, n), dtype=torch.float32, device=dev)
-        idx = torch.empty((T, k), dtype=torch.int32, device=dev)
-        wt = torch.empty((T, k), dtype=torch.float32, device=dev)
-        moe_route(c, u, w["w_router"], w.get("logit_bias"), logits, idx, wt,
+        moe_route(c, u, w["w_router"], w.get("logit_bias"), self.logits, self.idx, self.wt,
                   correction_bias=w.get("correction_bias"))
+        # the permutation first: its expert offsets cross to the host while the latent
+        # down-projection runs, then the rows are dispatched
+        moe_permute(c, self.idx, self.offsets, self.perm, self.inv, workspace=self.workspace)
+        self.offsets_host.copy_(self.offsets, non_blocking=True)
+        self.offsets_ready.record()
         x = u
         if c.d_latent > 0:
-            x = torch.empty((T, c.d_latent), dtype=u.dtype, device=dev)
-            moe_latent_down(c, u, w["p_down"], x)
-        E = x.shape[1]
-        offsets = torch.empty(n + 1, dtype=torch.int32, device=dev)
-        perm = torch.empty(T * k, dtype=torch.int32, device=dev)
-        inv = torch.empty(T * k, dtype=torch.int32, device=dev)
-        x_perm = torch.empty((T * k, E), dtype=u.dtype, device=dev)
-        moe_permute(c, idx, offsets, perm, inv, x, w.get("gamma_pre") if c.pre_norm else None,
-                    x_perm, self.workspace)
-        return Dispatched(u=u, w=wt, inv=inv, x_perm=x_perm,
-                          counts=send_counts(offsets.cpu().numpy(), self.world))
+            moe_latent_down(c, u, w["p_down"], self.z)
+            x = self.z
+        moe_dispatch_rows(c, self.inv, x, w.get("gamma_pre") if c.pre_norm else None, self.x_perm)
+        self.offsets_ready.synchronize()
+        return Dispatched(u=u, w=self.wt, inv=self.inv, x_perm=self.x_perm,
+                          counts=send_counts(self.offsets_host.numpy(), self.world))
 
     def compute(self, recv, recv_counts: np.ndarray):
         """The rank's experts on the rows it received (source-major, then expert); returns their
         outputs in the same order."""
-        import torch
         rows, local_offsets = regroup_rows(recv_counts)
-        dev = recv.device
         n = len(rows)
         # the whole plan (regroup rows, their inverse, the local expert offsets) crosses to the
         # device in one asynchronous copy from pinned memory; each part starts on a 16-byte
-        # boundary (the library's alignment rule)
+        # boundary (the library's alignment rule).  The pinned buffer is rewritten only after the
+        # previous forward's copy out of it has completed.
         m = (n + 3) // 4 * 4
-        plan = torch.zeros(2 * m + self.n_local + 1, dtype=torch.int32, pin_memory=True)
+        size = 2 * m + self.n_local + 1
+        self.plan_done.synchronize()
+        plan = self.plan_host.get(size)
         pv = plan.numpy()
         pv[:n] = rows
         pv[m:m + n] = inverse_rows(rows)
         pv[2 * m:] = local_offsets
-        plan_d = plan.to(dev, non_blocking=True)
-        grouped = torch.empty_like(recv)
+        plan_d = self.plan_dev.get(size)
+        plan_d.copy_(plan, non_blocking=True)
+        self.plan_done.record()
+        grouped = self.grouped.get(n, self.E)
         moe_gather_rows(recv, plan_d[:n], grouped)
         c = self._local_cfg(n)
-        out = torch.empty_like(grouped)
-        ws = torch.empty(workspace_size(c), dtype=torch.uint8, device=dev)
+        out = self.expert_out.get(n, self.E)
+        ws = self.expert_ws.get(workspace_size(c))
         moe_expert_ffn(c, grouped, plan_d[2 * m:], self.weights["w_gu"], self.weights["w_down"],
                        self.weights.get("gamma_expert") if self.cfg.expert_norm else None, out, ws)
-        back = torch.empty_like(out)
+        back = self.back.get(n, self.E)
         moe_gather_rows(out, plan_d[m:m + n], back)
         return back
 
-    def finish(self, d: Dispatched, out_perm):
+    def finish(self, d: Dispatched, out_perm, out=None):
+        """Combine and latent up-projection of the rank's tokens into `out` (a new tensor when
+        None), from their expert outputs out_perm in dispatch order."""
         import torch
         c, w = self.cfg, self.weights
-        E = out_perm.shape[1]
-        y = torch.empty((c.T, E), dtype=out_perm.dtype, device=out_perm.device)
-        moe_combine(c, out_perm, d.inv, d.w, y)
+        moe_combine(c, out_perm, d.inv, d.w, self.y)
         if c.d_latent == 0:
-            return y
-        out = torch.empty_like(d.u)
-        moe_latent_up(c, y, w["p_up"], d.u, w.get("resid_g"), out)
+            if out is None:
+                return self.y.clone()
+            out.copy_(self.y)
+            return out
+        if out is None:
+            out = torch.empty_like(d.u)
+        moe_latent_up(c, self.y, w["p_up"], d.u, w.get("resid_g"), out)
         return out
 
 
-def forward(rank: ExpertParallelRank, u, exchange, exchange_counts):
-    """One expert-parallel forward of this rank's tokens (every rank calls it together)."""
+def forward(rank: ExpertParallelRank, u, exchange, exchange_counts, out=None):
+    """One expert-parallel forward of this rank's tokens (every rank calls it together); the
+    exchanged rows land in the rank's own buffers."""
     d = rank.dispatch(u)
     recv_counts = exchange_counts(d.counts, u.device)
     send_splits = d.counts.sum(1)
     recv_splits = recv_counts.sum(1)
-    recv = exchange(d.x_perm, send_splits, recv_splits)
+    recv = exchange(d.x_perm, send_splits, recv_splits,
+                    out=rank.recv_buffer(int(recv_splits.sum())))
     back = rank.compute(recv, recv_counts)
-    out_perm = exchange(back, recv_splits, send_splits)
-    return rank.finish(d, out_perm)
+    out_perm = exchange(back, recv_splits, send_splits,
+                        out=rank.return_buffer(int(send_splits.sum())))
+    return rank.finish(d, out_perm, out)
 
 
 def emulated_forward(ranks: list, us: list, timer=None) -> list:

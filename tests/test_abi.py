@@ -135,8 +135,9 @@ def test_host_pipeline_checks_on_host(lib):
 
 
 def test_row_sumsq_parts_is_host_arithmetic(lib):
-    # prefill: normal-orientation down GEMM, one partial per 256-column tile of the 4096-wide row;
-    # decode: swapped orientation, one per 32-feature warp slice of each 128-feature tile
+    # prefill: normal-orientation down GEMM, one partial per 256-column tile of the 4096-wide row
+    # (one per CTA's 128 features with the swapped CTA-pair tiles); decode: swapped orientation,
+    # one per 32-feature warp slice of each 128-feature tile
     assert moe.row_sumsq_parts(abi_config(configs.MUSE_PREFILL)) == 4096 // 256
     assert moe.row_sumsq_parts(abi_config(configs.MUSE_DECODE)) == 4096 // 128 * 4
     n = ctypes.c_int32()

@@ -134,7 +134,13 @@ class _TaggedRank:
             seg[:, 3] += 100 * (self.lo + e + 1)
         return grouped.index_select(0, torch.from_numpy(ep.inverse_rows(rows)).long())
 
-    def finish(self, d, out_perm):
+    def recv_buffer(self, rows):  # the rank's own buffers for the two exchanges
+        return torch.full((rows, 4), -1, dtype=torch.int64)
+
+    def return_buffer(self, rows):
+        return torch.full((rows, 4), -1, dtype=torch.int64)
+
+    def finish(self, d, out_perm, out=None):
         return d.x_perm, out_perm
 
 

@@ -99,6 +99,16 @@ SMALL = [
 
 
 PAIR_CASES = [c for c in SMALL if c.T in (517, 1100)]
+# layers whose expert groups are prefill-sized (more than 48 rows per expert on average)
+PREFILL_GROUP_CASES = [c for c in SMALL if c.T * c.top_k / c.n_experts > 48]
+
+
+@pytest.mark.parametrize("cfg", PREFILL_GROUP_CASES, ids=lambda c: c.name)
+def test_layer_small_swap_pair_expert_tiles(cfg, monkeypatch):
+    """The same layers with the prefill expert GEMMs on the swapped CTA-pair tiles
+    (MOE_EXPERT_TILES=swap_pair) instead of the 1-SM 128-row activation tiles."""
+    monkeypatch.setenv("MOE_EXPERT_TILES", "swap_pair")
+    _check_layer(cfg)
 
 
 @pytest.mark.parametrize("cfg", SMALL, ids=lambda c: f"{c.name}-n{c.n_experts}k{c.top_k}-{c.dtype}"
@@ -261,23 +271,79 @@ def test_expert_ffn(cfg, monkeypatch):
         # bf16 values (fp32 sums of up to 256 terms each)
         tot = ss.double().sum(1).cpu().numpy()
         np.testing.assert_allclose(tot, (got * got).sum(1), rtol=2e-5, atol=1e-30)
-    oc = oracle.make_cfg(cfg.replace(expert_norm=0))
-    xv = host_values(xh, "bf16")
+    errs = _expert_rows_vs_oracle(cfg, off, host_values(xh, "bf16"), got, w_gu, w_dn, gam)
+    assert errs.max() <= 2e-2
+
+
+def _expert_rows_vs_oracle(cfg, off, xv, got, w_gu, w_dn, gam):
+    """Row errors of expert outputs (dispatch order) against the oracle's pre-norm expert output
+    s (the vector I_gamma reduces with expert_norm, else o) on the same input rows."""
+    oc = oracle.make_cfg(cfg)
+    E = cfg.expert_in
+    gp = None if gam is None else np.ascontiguousarray(gam, dtype=np.float32)
     errs = []
-    for e in range(n):
+    for e in range(cfg.n_experts):
         rows = np.arange(off[e], off[e + 1])
         if len(rows) == 0:
             continue
         ref = np.zeros((len(rows), E))
+        nrm = np.zeros((len(rows), E))
         wg = np.ascontiguousarray(w_gu[e])
         wd = np.ascontiguousarray(w_dn[e])
         zr = np.ascontiguousarray(xv[rows])
-        oracle.lib().orc_expert_batch(oracle.ctypes.byref(oc), wg.ctypes.data, wd.ctypes.data, None,
-                                      zr.ctypes.data, len(rows), ref.ctypes.data, 4)
-        if gam is not None:  # the kernel stores dtype((1 + gamma) * o), the vector I_gamma reduces
-            ref = oracle.bf16_round(ref * (1.0 + gam.astype(np.float64)))
+        oracle.lib().orc_expert_batch_parts(oracle.ctypes.byref(oc), wg.ctypes.data,
+                                            wd.ctypes.data, None if gp is None else gp.ctypes.data,
+                                            zr.ctypes.data, len(rows), ref.ctypes.data,
+                                            nrm.ctypes.data, 4)
         errs.append(row_rel_err(got[rows], ref))
-    assert np.concatenate(errs).max() <= 2e-2
+    return np.concatenate(errs)
+
+
+# group sizes around the swapped pair tiles' 16-row and 256-row steps, an empty group and a hot
+# group of many chunks
+PAIR_GROUPS = [0, 1, 15, 16, 17, 255, 256, 257, 511, 513, 1000, 40, 3000]
+
+
+@pytest.mark.parametrize("tiles", ["swap_pair", "normal"])
+@pytest.mark.parametrize("cfg", [
+    configs.small_muse(T=sum(PAIR_GROUPS), d=256, L=256, I=256, n=len(PAIR_GROUPS), k=1, seed=37),
+    configs.small_muse(T=sum(PAIR_GROUPS), d=256, L=128, I=384, n=len(PAIR_GROUPS), k=1, seed=38),
+    configs.small_shazeer(T=sum(PAIR_GROUPS), d=256, h=512, n=len(PAIR_GROUPS), k=1, seed=39),
+], ids=lambda c: f"{c.name}-L{c.expert_in}-I{c.d_ff}-act{c.act}")
+def test_expert_ffn_prefill_tiles(cfg, tiles, monkeypatch):
+    """Prefill-sized expert groups of chosen sizes on the swapped CTA-pair tiles (tokens on the
+    MMA's N side, chunks cut to 16 rows) and on the 1-SM 128-row tiles: each against the oracle,
+    and the row partial sums of squares against the stored rows.  (A 128-wide latent is not a
+    multiple of the pair's 256 down-projection features: that down GEMM keeps the 1-SM tiles.)"""
+    monkeypatch.setenv("MOE_EXPERT_TILES", tiles)
+    c = abi_config(cfg)
+    n, E = cfg.n_experts, cfg.expert_in
+    counts = np.array(PAIR_GROUPS)
+    idx = np.repeat(np.arange(n, dtype=np.int32), counts).reshape(-1, 1)
+    off = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    TK = int(off[-1])
+    xh = moe_inputs.normal_host(cfg.seed, 50, 0, TK * E, 1.0, "bf16").reshape(TK, E)
+    gam = moe_inputs.host_rows(cfg, "gamma_expert") if cfg.expert_norm else None
+    dev = moe_inputs.device_inputs(cfg)
+    x = torch.from_numpy(xh.view(np.int16)).view(torch.bfloat16).cuda()
+    out = torch.empty((TK, E), dtype=torch.bfloat16, device="cuda")
+    ws = torch.empty(moe.workspace_size(c), dtype=torch.uint8, device="cuda")
+    parts = moe.row_sumsq_parts(c)
+    ss = torch.full((TK, parts), float("nan"), dtype=torch.float32, device="cuda")
+    moe.moe_expert_ffn(c, x, torch.from_numpy(off).cuda(), dev["w_gu"], dev["w_down"],
+                       dev.get("gamma_expert"), out, workspace=ws,
+                       row_sumsq=ss if cfg.expert_norm else None)
+    assert moe.moe_get_device_status() == 0
+    got = device_values(out)
+    if cfg.expert_norm:
+        tot = ss.double().sum(1).cpu().numpy()
+        np.testing.assert_allclose(tot, (got * got).sum(1), rtol=2e-5, atol=1e-30)
+    errs = _expert_rows_vs_oracle(cfg, off, host_values(xh, "bf16"),
+                                  got, moe_inputs.host_rows(cfg, "w_gu"),
+                                  moe_inputs.host_rows(cfg, "w_down"), gam)
+    print(f"{tiles}: parts {parts}, max row rel err {errs.max():.3e}")
+    assert errs.max() <= 2e-2
+    del idx
 
 
 @pytest.mark.parametrize("with_ss", [False, True], ids=["reduce", "row_sumsq"])
@@ -314,6 +380,61 @@ def test_combine(E, k, norm, with_ss):
             ns[j] = oracle.bf16_round(oracle.input_scaled_rmsnorm(s, zero, cfg.eps, 1)) if norm else s
         ref = np.zeros(E)
         wj = wr[t].astype(np.float64)
+        oracle.lib().orc_combine_token(oracle.ctypes.byref(oc), np.ascontiguousarray(ns).ctypes.data,
+                                       wj.ctypes.data, ref.ctypes.data)
+        assert row_rel_err(got[t], ref) <= 1e-2
+
+
+@pytest.mark.parametrize("E,k,norm", [(4096, 8, 1), (512, 4, 0), (1024, 2, 1)])
+def test_combine_bulk_matches_per_token(E, k, norm):
+    """The prefill combine (persistent CTAs, expert rows by bulk copies; from 1024 tokens) against
+    the per-token combine on the same rows, bit for bit (two calls of fewer tokens each), and
+    against the oracle on sampled tokens; a few slots are dropped (negative dispatch row)."""
+    T, n = 1500, 16
+    cfg = configs.small_muse(T=T, d=E, L=E, I=128, n=n, k=k, expert_norm=norm)
+    idx = _rand_routing(T, n, k, seed=E + 3 * k)
+    _, _, inv = oracle.permutation(T, k, n, idx)
+    inv = inv.copy()
+    inv[[5, 777 * k + k - 1, (T - 1) * k]] = -1
+    sh = moe_inputs.normal_host(10, 60, 0, T * k * E, 0.8, "bf16").reshape(T * k, E)
+    wr = moe_inputs.uniform_host(10, 61, 0, T * k).reshape(T, k).astype(np.float64) + 0.05
+    wr = (wr / wr.sum(1, keepdims=True)).astype(np.float32)
+    sv = host_values(sh, "bf16")
+    s_d = torch.from_numpy(sh.view(np.int16)).view(torch.bfloat16).cuda()
+    inv_d = torch.from_numpy(inv).cuda()
+    w_d = torch.from_numpy(wr).cuda()
+    c = abi_config(cfg)
+    ss = None
+    if norm:
+        parts = np.zeros((T * k, moe.row_sumsq_parts(c)), dtype=np.float32)
+        parts[:, 0] = (sv * sv).sum(1)
+        parts[:, -1] = 0.0
+        ss = torch.from_numpy(parts).cuda()
+    y = torch.empty((T, E), dtype=torch.bfloat16, device="cuda")
+    moe.moe_combine(c, s_d, inv_d, w_d, y, row_sumsq=ss)
+    h = T // 2  # below the bulk path's threshold: the per-token kernel
+    y2 = torch.empty_like(y)
+    for part in (slice(0, h), slice(h, T)):
+        ch = abi_config(cfg.replace(T=part.stop - part.start))
+        moe.moe_combine(ch, s_d, inv_d[part.start * k:part.stop * k], w_d[part], y2[part],
+                        row_sumsq=ss)
+    torch.cuda.synchronize()
+    assert moe.moe_get_device_status() == 0
+    np.testing.assert_array_equal(y.view(torch.int16).cpu().numpy(),
+                                  y2.view(torch.int16).cpu().numpy())
+    got = device_values(y)
+    oc = oracle.make_cfg(cfg)
+    zero = np.zeros(E)
+    for t in list(range(0, T, 97)) + [777, T - 1]:
+        ns = np.zeros((k, E))
+        for j in range(k):
+            r = inv[t * k + j]
+            if r < 0:
+                continue
+            ns[j] = oracle.bf16_round(oracle.input_scaled_rmsnorm(sv[r], zero, cfg.eps, 1)) \
+                if norm else sv[r]
+        ref = np.zeros(E)
+        wj = wr[t].astype(np.float64) * (inv[t * k:(t + 1) * k] >= 0)
         oracle.lib().orc_combine_token(oracle.ctypes.byref(oc), np.ascontiguousarray(ns).ctypes.data,
                                        wj.ctypes.data, ref.ctypes.data)
         assert row_rel_err(got[t], ref) <= 1e-2
