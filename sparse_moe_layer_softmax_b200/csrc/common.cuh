@@ -18,6 +18,19 @@ __device__ int g_status = 0;
 
 __device__ __forceinline__ void latch_status(int code) { atomicCAS(&g_status, 0, code); }
 
+// ------------------------------------------------------------------ programmatic dependent launch
+//
+// The library launches the kernels of a layer forward so that each may start while the kernel
+// before it on the stream is finishing (programmatic stream serialization).  Every kernel
+// therefore waits, before it touches global memory, until the grids it depends on have completed
+// and their writes are visible (a no-op for a kernel launched without that attribute).
+// Persistent kernels, whose CTAs are all resident at once, let the next kernel launch as soon as
+// they start; the others let it launch when their CTAs exit.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" :::);
+}
+
 // ------------------------------------------------------------------ bf16
 
 __device__ __forceinline__ float bf16_to_f32(uint16_t b) {

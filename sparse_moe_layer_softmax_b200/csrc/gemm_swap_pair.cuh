@@ -119,6 +119,7 @@ template <int kEpi, int kStages>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     gemm_swap_pair_kernel(const __grid_constant__ CUtensorMap tmX,
                           const __grid_constant__ CUtensorMap tmW, const GemmParams p) {
+  pdl_wait();
   using S = SwapPairShape<kEpi>;
   static_assert(kEpi == EPI_SWIGLU || kEpi == EPI_STORE || kEpi == EPI_RELU,
                 "the swapped pair kernel has the expert epilogues");

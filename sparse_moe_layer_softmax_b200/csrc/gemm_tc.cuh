@@ -433,6 +433,7 @@ template <bool kSwap, int BN, int kEpi, int kStages>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
                    const __grid_constant__ CUtensorMap tmO, const GemmParams p) {
+  pdl_wait();
   using S = GemmShape<kSwap, BN, kEpi>;
   constexpr bool kStageOut = stages_output<kSwap, kEpi>();
   extern __shared__ uint8_t smem_raw[];
@@ -710,6 +711,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     gemm_tc_pair_kernel(const __grid_constant__ CUtensorMap tmX,
                         const __grid_constant__ CUtensorMap tmW,
                         const __grid_constant__ CUtensorMap tmO, const GemmParams p) {
+  pdl_wait();
   using S = PairShape<BN, kEpi>;
   static_assert(kEpi != EPI_ROUTER, "the pair kernel has bf16 epilogues only");
   extern __shared__ uint8_t smem_raw[];

@@ -33,6 +33,7 @@ __device__ __forceinline__ float block_sum_256(float v, float* red) {
 
 __global__ void perm_count_kernel(const int32_t* __restrict__ idx, int T, int k, int n,
                                   int32_t* __restrict__ counts) {
+  pdl_wait();
   __shared__ int h[kMaxExperts];
   for (int e = threadIdx.x; e < n; e += blockDim.x) h[e] = 0;
   __syncthreads();
@@ -51,6 +52,7 @@ __global__ void perm_count_kernel(const int32_t* __restrict__ idx, int T, int k,
 // before c; offsets = exclusive scan of the per-expert totals.
 __global__ void perm_scan_kernel(int32_t* __restrict__ counts, int nchunks, int n,
                                  int32_t* __restrict__ offsets) {
+  pdl_wait();
   __shared__ int warp_tot[kMaxExperts / 32];
   const int e = threadIdx.x;
   int run = 0;
@@ -95,6 +97,7 @@ __global__ void __launch_bounds__(32)
     perm_rank_kernel(const int32_t* __restrict__ idx, int T, int k, int n,
                      const int32_t* __restrict__ chunk_base, const int32_t* __restrict__ offsets,
                      int32_t* __restrict__ perm_token, int32_t* __restrict__ inv_perm) {
+  pdl_wait();
   __shared__ int s_next[kMaxExperts];
   __shared__ int s_idx[kPermChunk * kMaxTopK];
   const int lane = threadIdx.x;
@@ -126,6 +129,136 @@ __global__ void __launch_bounds__(32)
   }
 }
 
+// ------------------------------------------------------------------ small-batch dispatch
+//
+// The whole dispatch of a small batch (T*k <= kSmallDispatchSlots) in one launch, one CTA per
+// token.  Every CTA reads all T*k expert indices, builds the per-expert counts and their
+// exclusive scan in shared memory, and ranks its own token's slots: a slot's row is its expert's
+// offset plus the number of slots of that expert before it in token-major order, which is the
+// canonical order the three permutation kernels above produce.  The CTA writes its inv_perm and
+// perm_token entries (CTA 0 also the offsets) and, when x is given, scatters its row, with C_pre
+// when gamma is given, exactly as scatter_rows_bf16_kernel does.  An expert index outside [0, n)
+// latches MOE_ERR_DEVICE_CHECK and its slot is dropped (inv_perm = -1).
+constexpr int kSmallDispatchSlots = 2048;
+
+template <int VEC>
+__global__ void dispatch_small_bf16_kernel(const int32_t* __restrict__ idx, int T, int k, int n,
+                                           const uint16_t* __restrict__ x, int E,
+                                           const float* __restrict__ gamma, float eps,
+                                           int32_t* __restrict__ offsets,
+                                           int32_t* __restrict__ perm_token,
+                                           int32_t* __restrict__ inv_perm,
+                                           uint16_t* __restrict__ x_perm) {
+  pdl_wait();
+  __shared__ int s_idx[kSmallDispatchSlots];
+  __shared__ int s_off[kMaxExperts + 1];  // counts, then their exclusive scan (and the total)
+  __shared__ int s_rank[kMaxTopK];
+  __shared__ int s_row[kMaxTopK];
+  __shared__ float red[8];
+  const int t = blockIdx.x, tid = threadIdx.x;
+  const int TK = T * k;
+  for (int e = tid; e <= n; e += blockDim.x) s_off[e] = 0;
+  if (tid < kMaxTopK) s_rank[tid] = 0;
+  __syncthreads();
+  bool bad = false;
+  for (int i = tid; i < TK; i += blockDim.x) {
+    const int e = idx[i];
+    s_idx[i] = e;
+    if (e >= 0 && e < n) atomicAdd(&s_off[e], 1);
+    else bad = true;
+  }
+  if (bad && t == 0) latch_status(MOE_ERR_DEVICE_CHECK);
+  __syncthreads();
+  if (tid < 32) {  // exclusive scan of the n <= 256 counts: 8 consecutive experts per lane
+    int v[kMaxExperts / 32];
+    int sum = 0;
+#pragma unroll
+    for (int i = 0; i < kMaxExperts / 32; ++i) {
+      const int e = tid * (kMaxExperts / 32) + i;
+      v[i] = e < n ? s_off[e] : 0;
+      sum += v[i];
+    }
+    int incl = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (tid >= o) incl += y;
+    }
+    int run = incl - sum;
+#pragma unroll
+    for (int i = 0; i < kMaxExperts / 32; ++i) {
+      const int e = tid * (kMaxExperts / 32) + i;
+      if (e < n) s_off[e] = run;
+      run += v[i];
+    }
+    if (tid == 31) s_off[n] = incl;
+  }
+  __syncthreads();
+  // ranks of this token's slots among the earlier slots (token-major) of the same expert
+  const int base = t * k;
+  for (int sidx = tid; sidx < base + k; sidx += blockDim.x) {
+    const int es = s_idx[sidx];
+    for (int j = 0; j < k; ++j)
+      if (sidx < base + j && es == s_idx[base + j]) atomicAdd(&s_rank[j], 1);
+  }
+  __syncthreads();
+  if (tid < k) {
+    const int e = s_idx[base + tid];
+    int row = -1;
+    if (e >= 0 && e < n) {
+      row = s_off[e] + s_rank[tid];
+      perm_token[row] = t;
+    }
+    inv_perm[base + tid] = row;
+    s_row[tid] = row;
+  }
+  if (t == 0)
+    for (int e = tid; e <= n; e += blockDim.x) offsets[e] = s_off[e];
+  if (x == nullptr) return;
+  __syncthreads();
+  // the row scatter (+ C_pre) of scatter_rows_bf16_kernel
+  const int nvec = E / 8;
+  const uint4* src = reinterpret_cast<const uint4*>(x + static_cast<size_t>(t) * E);
+  uint4 r[VEC];
+  float ss = 0.0f;
+#pragma unroll
+  for (int v = 0; v < VEC; ++v) {
+    const int vi = tid + v * blockDim.x;
+    r[v] = vi < nvec ? src[vi] : make_uint4(0, 0, 0, 0);
+    if (gamma) {
+      const uint16_t* h = reinterpret_cast<const uint16_t*>(&r[v]);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) { const float f = bf16_to_f32(h[i]); ss += f * f; }
+    }
+  }
+  if (gamma) {
+    const float tot = block_sum_256(ss, red);
+    const float rinv = rsqrtf(tot / static_cast<float>(E) + eps);
+#pragma unroll
+    for (int v = 0; v < VEC; ++v) {
+      const int vi = tid + v * blockDim.x;
+      if (vi < nvec) {
+        uint16_t* h = reinterpret_cast<uint16_t*>(&r[v]);
+        const float4 g0 = reinterpret_cast<const float4*>(gamma)[2 * vi];
+        const float4 g1 = reinterpret_cast<const float4*>(gamma)[2 * vi + 1];
+        const float gg[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+#pragma unroll
+        for (int i = 0; i < 8; ++i) h[i] = f32_to_bf16((1.0f + gg[i]) * (bf16_to_f32(h[i]) * rinv));
+      }
+    }
+  }
+  for (int j = 0; j < k; ++j) {
+    const int row = s_row[j];
+    if (row < 0) continue;
+    uint4* dst = reinterpret_cast<uint4*>(x_perm + static_cast<size_t>(row) * E);
+#pragma unroll
+    for (int v = 0; v < VEC; ++v) {
+      const int vi = tid + v * blockDim.x;
+      if (vi < nvec) dst[vi] = r[v];
+    }
+  }
+}
+
 // ------------------------------------------------------------------ k-split dense finish
 //
 // A dense projection over few rows whose reduction ran as k-split GEMM tiles (EPI_PARTIAL): the
@@ -137,6 +270,7 @@ __global__ void dense_split_finish_kernel(const float* __restrict__ partial, int
                                           int nout, int resgate, const uint16_t* __restrict__ resid,
                                           const float* __restrict__ g, float tau, float floor_,
                                           int resid_mode, uint16_t* __restrict__ out) {
+  pdl_wait();
   const long nv = rows * nout / 8;
   const size_t plane = static_cast<size_t>(rows) * nout;
   for (long i = blockIdx.x * static_cast<long>(blockDim.x) + threadIdx.x; i < nv;
@@ -189,6 +323,7 @@ __global__ void dense_split_finish_kernel(const float* __restrict__ partial, int
 __global__ void gather_rows_kernel(const uint4* __restrict__ src, long src_rows,
                                    const int32_t* __restrict__ rows, long n_rows, int idx_stride,
                                    int row_vec, uint4* __restrict__ dst) {
+  pdl_wait();
   for (long i = blockIdx.x; i < n_rows; i += gridDim.x) {
     int r = rows[i * idx_stride];
     if (r >= src_rows) {
@@ -212,6 +347,7 @@ __global__ void scatter_rows_bf16_kernel(const uint16_t* __restrict__ x, int E, 
                                          const int32_t* __restrict__ inv_perm,
                                          const float* __restrict__ gamma, float eps,
                                          uint16_t* __restrict__ x_perm) {
+  pdl_wait();
   __shared__ float red[8];
   const int t = blockIdx.x;
   const int nvec = E / 8;
@@ -260,6 +396,7 @@ template <typename Tv>
 __global__ void scatter_rows_f32_kernel(const float* __restrict__ x, int E, int k,
                                         const int32_t* __restrict__ inv_perm,
                                         float* __restrict__ x_perm) {
+  pdl_wait();
   const int t = blockIdx.x;
   for (int j = 0; j < k; ++j) {
     const int row = inv_perm[static_cast<size_t>(t) * k + j];
@@ -292,6 +429,7 @@ __global__ void __launch_bounds__(kCombineMaxThreads)
     combine_bf16_kernel(const uint16_t* __restrict__ s, int E, int k,
                         const int32_t* __restrict__ inv_perm, const float* __restrict__ topk_w,
                         int expert_norm, float eps, uint16_t* __restrict__ y) {
+  pdl_wait();
   // One pass: every thread loads its VEC 16-byte vectors of all k rows at once (k x VEC loads in
   // flight) and keeps them as packed bf16; the row norms and the weighted sum both come from
   // there.  The arithmetic runs on fp32 pairs (Blackwell's two-wide FMA / multiply), so each
@@ -390,6 +528,7 @@ __global__ void __launch_bounds__(kCombineMaxThreads)
                            const int32_t* __restrict__ inv_perm, const float* __restrict__ topk_w,
                            const float* __restrict__ row_ss, int parts, float eps,
                            uint16_t* __restrict__ y) {
+  pdl_wait();
   const int t = blockIdx.x;
   const int nvec = E / 8;
   const int lane = threadIdx.x & 31;
@@ -486,6 +625,7 @@ __global__ void __launch_bounds__(kBulkCombineConsumers + 32, 1)
                              const float* __restrict__ topk_w, const float* __restrict__ row_ss,
                              int parts, int expert_norm, float eps, uint16_t* __restrict__ y,
                              int T, int nst) {
+  pdl_wait();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) &
                                              ~static_cast<uintptr_t>(127));
@@ -614,6 +754,7 @@ __global__ void combine_f32_kernel(const float* __restrict__ s, int E, int k,
                                    const int32_t* __restrict__ inv_perm,
                                    const float* __restrict__ topk_w, int expert_norm, float eps,
                                    float* __restrict__ y) {
+  pdl_wait();
   __shared__ float red[8];
   const int t = blockIdx.x;
   for (int c0 = 0; c0 < E; c0 += blockDim.x) {
@@ -649,6 +790,7 @@ constexpr int kRouterLoads = 4;      // weight vectors each lane keeps in flight
 __global__ void __launch_bounds__(kRouterThreads, 1) router_logits_small_kernel(
     const uint16_t* __restrict__ u, const uint16_t* __restrict__ w, const float* __restrict__ bias,
     int T, int d, int n, int wk, float mult, float* __restrict__ logits) {
+  pdl_wait();
   // w rows have wk = d (bf16 weights) or 3d (hi/mid/lo parts of fp32 weights; u repeats)
   extern __shared__ uint4 s_u[];  // [kRouterTok][d/8]
   const int t0 = blockIdx.y * kRouterTok;
@@ -723,6 +865,7 @@ __global__ void topk_rows_kernel(float* __restrict__ logits, int T, int n, int k
                                  float routed_scale, int gate_mode,
                                  const float* __restrict__ sel_bias,
                                  int32_t* __restrict__ topk_idx, float* __restrict__ topk_w) {
+  pdl_wait();
   const int warps = blockDim.x >> 5;
   const int t = blockIdx.x * warps + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
@@ -811,6 +954,7 @@ __global__ void topk_rows_kernel(float* __restrict__ logits, int T, int n, int k
 // hi = bf16(w), mid = bf16(w - hi), lo = bf16(w - hi - mid); both subtractions are exact in fp32.
 __global__ void router_split_kernel(const float* __restrict__ w, size_t count, int d,
                                     uint16_t* __restrict__ out) {
+  pdl_wait();
   const size_t stride = static_cast<size_t>(gridDim.x) * blockDim.x;
   for (size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < count; i += stride) {
     const size_t row = i / d, c = i - row * d;
@@ -836,6 +980,7 @@ template <int VEC>
 __global__ void rownorm_centered_bf16_kernel(const uint16_t* __restrict__ x, int D,
                                              const float* __restrict__ gamma, float eps,
                                              uint16_t* __restrict__ out) {
+  pdl_wait();
   __shared__ float red[8];
   const size_t base = static_cast<size_t>(blockIdx.x) * D;
   const int nvec = D / 8;
@@ -873,6 +1018,7 @@ __global__ void resid_update_bf16_kernel(const uint16_t* __restrict__ b, const u
                                          int D, const float* __restrict__ gamma_post, float eps,
                                          const float* __restrict__ g, int resid_mode, float tau,
                                          float floor_, uint16_t* __restrict__ out) {
+  pdl_wait();
   __shared__ float red[8];
   const size_t base = static_cast<size_t>(blockIdx.x) * D;
   const int nvec = D / 8;
@@ -939,6 +1085,7 @@ __global__ void noisy_gate_kernel(const float* __restrict__ l, const float* __re
                                   float* __restrict__ H_out, int32_t* __restrict__ topk_idx,
                                   float* __restrict__ topk_w, float* __restrict__ P_out,
                                   float* __restrict__ part_imp, float* __restrict__ part_load) {
+  pdl_wait();
   const int lane = threadIdx.x & 31;
   const int gw = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);  // global warp
   const int t0 = gw * kGateTokensPerWarp;
@@ -1028,6 +1175,7 @@ __global__ void gate_stats_reduce_kernel(const float* __restrict__ part_imp,
                                          const float* __restrict__ part_load, int nparts, int n,
                                          float* __restrict__ importance, float* __restrict__ load,
                                          float* __restrict__ cv2) {
+  pdl_wait();
   __shared__ float si[kMaxExperts], sl[kMaxExperts];
   const int e = threadIdx.x;
   float a = 0.0f, b = 0.0f;
@@ -1062,6 +1210,7 @@ __global__ void gate_stats_reduce_kernel(const float* __restrict__ part_imp,
 // it with the same bounded wait the GEMM pipeline uses; the wait runs out after `budget` clocks,
 // latches MOE_ERR_TIMEOUT in the status word and the kernel returns normally.
 __global__ void wait_timeout_selftest_kernel(long long budget, int* gave_up) {
+  pdl_wait();
   __shared__ __align__(8) uint64_t bar;
   if (threadIdx.x != 0) return;
   mbar_init(&bar, 1);
@@ -1080,6 +1229,7 @@ __global__ void router_f32_kernel(const float* __restrict__ u, const float* __re
                                   const float* __restrict__ sel_bias,
                                   float* __restrict__ logits_out,
                                   int32_t* __restrict__ topk_idx, float* __restrict__ topk_w) {
+  pdl_wait();
   const int warps = blockDim.x >> 5;
   const int t = blockIdx.x * warps + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
@@ -1163,6 +1313,7 @@ __global__ void expert_ffn_f32_kernel(const float* __restrict__ x_perm,
                                       const float* __restrict__ w_down,
                                       const float* __restrict__ gamma,
                                       float* __restrict__ out_perm) {
+  pdl_wait();
   extern __shared__ float sm[];  // [E] input row, [H] hidden
   float* xr = sm;
   float* hid = sm + E;

@@ -85,6 +85,25 @@ moe_status_t last_launch(int n = 1) {
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
+// Every kernel is launched with programmatic stream serialization: it may begin while the kernel
+// before it on the stream finishes, and waits (pdl_wait, its first statement) for that kernel's
+// results before touching memory.  Errors surface through last_launch().
+template <typename... KArgs, typename... Args>
+void launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+              Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
 // ------------------------------------------------------------------ GEMM launcher
 
 template <bool kSwap, int BN, int kEpi, int kStages>
@@ -117,7 +136,7 @@ moe_status_t launch_gemm(const void* X, long x_rows, const void* W, long w_rows,
   long grid = device_info().sms;
   if (grid <= 0) return MOE_ERR_CUDA;  // the SM count could not be read
   if (max_tiles < grid) grid = max_tiles;
-  kern<<<static_cast<unsigned>(grid), kGemmThreads, smem, st>>>(tx, tw, to, q);
+  launch_k(kern, static_cast<unsigned>(grid), kGemmThreads, smem, st, tx, tw, to, q);
   return last_launch();
 }
 
@@ -147,7 +166,7 @@ moe_status_t launch_gemm_pair(const void* X, long x_rows, const void* W, long w_
   long pairs = device_info().sms / 2;
   if (pairs <= 0) return MOE_ERR_CUDA;  // the SM count could not be read
   if (max_tiles < pairs) pairs = max_tiles;
-  kern<<<static_cast<unsigned>(2 * pairs), kGemmThreads, smem, st>>>(tx, tw, to, q);
+  launch_k(kern, static_cast<unsigned>(2 * pairs), kGemmThreads, smem, st, tx, tw, to, q);
   return last_launch();
 }
 
@@ -175,7 +194,7 @@ moe_status_t launch_gemm_swap_pair(const void* X, long x_rows, const void* W, lo
   long pairs = device_info().sms / 2;
   if (pairs <= 0) return MOE_ERR_CUDA;  // the SM count could not be read
   if (max_tiles < pairs) pairs = max_tiles;
-  kern<<<static_cast<unsigned>(2 * pairs), kGemmThreads, smem, st>>>(tx, tw, p);
+  launch_k(kern, static_cast<unsigned>(2 * pairs), kGemmThreads, smem, st, tx, tw, p);
   return last_launch();
 }
 
@@ -415,7 +434,7 @@ moe_status_t launch_dense_finish(const float* partial, int splits, long rows, in
                                  const moe_config_t& c, void* out, cudaStream_t st) {
   const long nv = rows * nout / 8;
   const long blocks = std::min<long>((nv + 255) / 256, static_cast<long>(std::max(device_info().sms, 1)) * 8);
-  dense_split_finish_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(
+  launch_k(dense_split_finish_kernel, static_cast<unsigned>(blocks), 256, 0, st,
       partial, splits, rows, nout, resgate ? 1 : 0, static_cast<const uint16_t*>(resid), g, c.tau,
       c.resid_floor, c.resid_mode, static_cast<uint16_t*>(out));
   return last_launch();
@@ -443,7 +462,7 @@ moe_status_t do_route(const moe_config_t& c, const void* u, const void* w_router
   const float mult = sig ? c.logit_mult : 1.0f;
   if (c.dtype == MOE_F32) {
     const int warps = 4;
-    router_f32_kernel<<<cdiv(c.T, warps), 32 * warps, 0, st>>>(
+    launch_k(router_f32_kernel, cdiv(c.T, warps), 32 * warps, 0, st,
         static_cast<const float*>(u), static_cast<const float*>(w_router), bias, c.T, c.d_model,
         c.n_experts, c.top_k, c.routed_scale, c.gate_mode, mult, sel_bias, logits, idx, w);
     return last_launch();
@@ -460,10 +479,10 @@ moe_status_t do_route(const moe_config_t& c, const void* u, const void* w_router
     });
     if (attr != cudaSuccess) return MOE_ERR_CUDA;
     dim3 grid(cdiv(c.n_experts, kRouterExp), cdiv(c.T, kRouterTok));
-    router_logits_small_kernel<<<grid, kRouterThreads, small_smem, st>>>(
+    launch_k(router_logits_small_kernel, grid, kRouterThreads, small_smem, st,
         static_cast<const uint16_t*>(u), static_cast<const uint16_t*>(w_router), bias, c.T,
         c.d_model, c.n_experts, wk, mult, lbuf);
-    topk_rows_kernel<<<cdiv(c.T, 8), 256, 0, st>>>(lbuf, c.T, c.n_experts, c.top_k,
+    launch_k(topk_rows_kernel, cdiv(c.T, 8), 256, 0, st, lbuf, c.T, c.n_experts, c.top_k,
                                                     c.routed_scale, c.gate_mode, sel_bias, idx, w);
     return last_launch(2);
   }
@@ -498,7 +517,7 @@ moe_status_t do_route(const moe_config_t& c, const void* u, const void* w_router
   }
   moe_status_t s = run_gemm(EPI_ROUTER, Orient::kNormal, bn, u, c.T, w_router, c.n_experts, p, st);
   if (s != MOE_OK || !split) return s;
-  topk_rows_kernel<<<cdiv(c.T, 8), 256, 0, st>>>(lbuf, c.T, c.n_experts, c.top_k, c.routed_scale,
+  launch_k(topk_rows_kernel, cdiv(c.T, 8), 256, 0, st, lbuf, c.T, c.n_experts, c.top_k, c.routed_scale,
                                                   c.gate_mode, sel_bias, idx, w);
   return last_launch();
 }
@@ -514,9 +533,29 @@ moe_status_t do_permute(const moe_config_t& c, const int32_t* idx, int32_t* offs
     cudaMemsetAsync(offsets, 0, (n + 1) * sizeof(int32_t), st);
     return last_launch(0);
   }
-  perm_count_kernel<<<nc, 256, 0, st>>>(idx, c.T, k, n, counts);
-  perm_scan_kernel<<<1, kMaxExperts, 0, st>>>(counts, nc, n, offsets);
-  perm_rank_kernel<<<nc, 32, 0, st>>>(idx, c.T, k, n, counts, offsets, perm, inv);
+  if (c.dtype == MOE_BF16 && static_cast<long>(c.T) * k <= kSmallDispatchSlots) {
+    // small batch: indices, offsets and (with x) the row scatter in one launch
+    const int E = c.d_latent > 0 ? c.d_latent : c.d_model;
+    const int nvec = E / 8;
+    const int threads = nvec >= 256 ? 256 : std::max(32, ((nvec + 31) / 32) * 32);
+    const int vec = cdiv(nvec, threads);
+    const uint16_t* xs = static_cast<const uint16_t*>(x);
+    uint16_t* xp = static_cast<uint16_t*>(x_perm);
+#define SD(V) launch_k(dispatch_small_bf16_kernel<V>, c.T, threads, 0, st, idx, c.T, k, n, xs, E, \
+      gamma_pre, c.eps, offsets, perm, inv, xp)
+    switch (vec) {
+      case 1: SD(1); break;
+      case 2: SD(2); break;
+      case 3:
+      case 4: SD(4); break;
+      default: return MOE_ERR_UNSUPPORTED;
+    }
+#undef SD
+    return last_launch();
+  }
+  launch_k(perm_count_kernel, nc, 256, 0, st, idx, c.T, k, n, counts);
+  launch_k(perm_scan_kernel, 1, kMaxExperts, 0, st, counts, nc, n, offsets);
+  launch_k(perm_rank_kernel, nc, 32, 0, st, idx, c.T, k, n, counts, offsets, perm, inv);
   moe_status_t s = last_launch(3);
   if (s != MOE_OK || !x) return s;
   return do_dispatch_rows(c, inv, x, gamma_pre, x_perm, st);
@@ -527,7 +566,7 @@ moe_status_t do_dispatch_rows(const moe_config_t& c, const int32_t* inv, const v
   const int k = c.top_k;
   const int E = c.d_latent > 0 ? c.d_latent : c.d_model;
   if (c.dtype == MOE_F32) {
-    scatter_rows_f32_kernel<float><<<c.T, 128, 0, st>>>(static_cast<const float*>(x), E, k, inv,
+    launch_k(scatter_rows_f32_kernel<float>, c.T, 128, 0, st, static_cast<const float*>(x), E, k, inv,
                                                         static_cast<float*>(x_perm));
     return last_launch();
   }
@@ -537,10 +576,10 @@ moe_status_t do_dispatch_rows(const moe_config_t& c, const int32_t* inv, const v
   const uint16_t* xs = static_cast<const uint16_t*>(x);
   uint16_t* xp = static_cast<uint16_t*>(x_perm);
   switch (vec) {
-    case 1: scatter_rows_bf16_kernel<1><<<c.T, threads, 0, st>>>(xs, E, k, inv, gamma_pre, c.eps, xp); break;
-    case 2: scatter_rows_bf16_kernel<2><<<c.T, threads, 0, st>>>(xs, E, k, inv, gamma_pre, c.eps, xp); break;
+    case 1: launch_k(scatter_rows_bf16_kernel<1>, c.T, threads, 0, st, xs, E, k, inv, gamma_pre, c.eps, xp); break;
+    case 2: launch_k(scatter_rows_bf16_kernel<2>, c.T, threads, 0, st, xs, E, k, inv, gamma_pre, c.eps, xp); break;
     case 3:
-    case 4: scatter_rows_bf16_kernel<4><<<c.T, threads, 0, st>>>(xs, E, k, inv, gamma_pre, c.eps, xp); break;
+    case 4: launch_k(scatter_rows_bf16_kernel<4>, c.T, threads, 0, st, xs, E, k, inv, gamma_pre, c.eps, xp); break;
     default: return MOE_ERR_UNSUPPORTED;
   }
   return last_launch();
@@ -581,7 +620,7 @@ moe_status_t do_experts(const moe_config_t& c, const void* x_perm, const int32_t
   if (c.dtype == MOE_F32) {
     const size_t smem = static_cast<size_t>(E + H) * sizeof(float);
     if (smem > 48 * 1024) return MOE_ERR_UNSUPPORTED;
-    expert_ffn_f32_kernel<<<static_cast<unsigned>(TK), 128, smem, st>>>(
+    launch_k(expert_ffn_f32_kernel, static_cast<unsigned>(TK), 128, smem, st,
         static_cast<const float*>(x_perm), offsets, n, E, H, c.expert_act,
         static_cast<const float*>(w_gu), static_cast<const float*>(w_down),
         c.expert_norm ? gamma_e : nullptr, static_cast<float*>(out_perm));
@@ -624,13 +663,14 @@ moe_status_t do_experts(const moe_config_t& c, const void* x_perm, const int32_t
 
 constexpr int kBulkCombineMinT = 1024;        // tokens from which the bulk-copy combine runs
 constexpr int kBulkCombineSmem = 220 * 1024;   // its shared-memory ring, at most
+constexpr int kBulkCombineMinBytes = 32 * 1024; // expert-row bytes of a token, at least
 
 moe_status_t do_combine(const moe_config_t& c, const void* s, const int32_t* inv,
                         const float* w, void* y, cudaStream_t st, const float* row_ss = nullptr) {
   if (c.T == 0) return MOE_OK;
   const int E = expert_in(c);
   if (c.dtype == MOE_F32) {
-    combine_f32_kernel<<<c.T, 128, 0, st>>>(static_cast<const float*>(s), E, c.top_k, inv, w,
+    launch_k(combine_f32_kernel, c.T, 128, 0, st, static_cast<const float*>(s), E, c.top_k, inv, w,
                                             c.expert_norm, c.eps, static_cast<float*>(y));
     return last_launch();
   }
@@ -639,11 +679,13 @@ moe_status_t do_combine(const moe_config_t& c, const void* s, const int32_t* inv
   const int vec = cdiv(nvec, threads);
   const uint16_t* sp = static_cast<const uint16_t*>(s);
   uint16_t* yp = static_cast<uint16_t*>(y);
-  // Prefill-sized batches: one persistent CTA per SM with the expert rows (and their partial
-  // sums of squares) brought in by bulk copies, when the row partials are given or no norm is
-  // taken and at least two tokens' rows fit in shared memory.
+  // Prefill-sized batches of wide rows: one persistent CTA per SM with the expert rows (and their
+  // partial sums of squares) brought in by bulk copies, when the row partials are given or no norm
+  // is taken and at least two tokens' rows fit in shared memory.  (Narrow rows keep the per-token
+  // kernel: there a token's copies are too small to amortise the ring's per-token handshakes.)
   const int parts_b = row_ss && c.expert_norm ? sumsq_parts(c) : 0;
-  if (c.T >= kBulkCombineMinT && (parts_b * 4) % 16 == 0 && (!c.expert_norm || row_ss)) {
+  if (c.T >= kBulkCombineMinT && static_cast<long>(c.top_k) * E * 2 >= kBulkCombineMinBytes &&
+      (parts_b * 4) % 16 == 0 && (!c.expert_norm || row_ss)) {
     const BulkCombineStage B = bulk_combine_stage(E, c.top_k, parts_b);
     const int nst = std::min(8, (kBulkCombineSmem - 128 - 16 * 8) / B.bytes);
     if (nst >= 2) {
@@ -656,7 +698,7 @@ moe_status_t do_combine(const moe_config_t& c, const void* s, const int32_t* inv
       });
       if (attr != cudaSuccess) return MOE_ERR_CUDA;
       const int grid = std::min(c.T, std::max(device_info().sms, 1));
-      combine_bf16_bulk_kernel<<<grid, kBulkCombineConsumers + 32, smem, st>>>(
+      launch_k(combine_bf16_bulk_kernel, grid, kBulkCombineConsumers + 32, smem, st,
           sp, E, c.top_k, inv, w, row_ss, parts_b, c.expert_norm, c.eps, yp, c.T, nst);
       return last_launch();
     }
@@ -664,15 +706,15 @@ moe_status_t do_combine(const moe_config_t& c, const void* s, const int32_t* inv
   if (row_ss && c.expert_norm) {
     const int parts = sumsq_parts(c);
     switch (vec) {
-      case 1: combine_bf16_ss_kernel<1><<<c.T, threads, 0, st>>>(sp, E, c.top_k, inv, w, row_ss, parts, c.eps, yp); break;
-      case 2: combine_bf16_ss_kernel<2><<<c.T, threads, 0, st>>>(sp, E, c.top_k, inv, w, row_ss, parts, c.eps, yp); break;
+      case 1: launch_k(combine_bf16_ss_kernel<1>, c.T, threads, 0, st, sp, E, c.top_k, inv, w, row_ss, parts, c.eps, yp); break;
+      case 2: launch_k(combine_bf16_ss_kernel<2>, c.T, threads, 0, st, sp, E, c.top_k, inv, w, row_ss, parts, c.eps, yp); break;
       default: return MOE_ERR_UNSUPPORTED;  // E <= 8192: at most 2 vectors per thread
     }
     return last_launch();
   }
   switch (vec) {
-    case 1: combine_bf16_kernel<1><<<c.T, threads, 0, st>>>(sp, E, c.top_k, inv, w, c.expert_norm, c.eps, yp); break;
-    case 2: combine_bf16_kernel<2><<<c.T, threads, 0, st>>>(sp, E, c.top_k, inv, w, c.expert_norm, c.eps, yp); break;
+    case 1: launch_k(combine_bf16_kernel<1>, c.T, threads, 0, st, sp, E, c.top_k, inv, w, c.expert_norm, c.eps, yp); break;
+    case 2: launch_k(combine_bf16_kernel<2>, c.T, threads, 0, st, sp, E, c.top_k, inv, w, c.expert_norm, c.eps, yp); break;
     default: return MOE_ERR_UNSUPPORTED;  // E <= 8192: at most 2 vectors per thread
   }
   return last_launch();
@@ -777,9 +819,9 @@ moe_status_t do_input_norm(const moe_config_t& c, const void* r, const float* ga
   const uint16_t* x = static_cast<const uint16_t*>(r);
   uint16_t* o = static_cast<uint16_t*>(u);
   switch (vec) {
-    case 1: rownorm_centered_bf16_kernel<1><<<c.T, threads, 0, st>>>(x, c.d_model, gamma_in, c.eps_block, o); break;
-    case 2: rownorm_centered_bf16_kernel<2><<<c.T, threads, 0, st>>>(x, c.d_model, gamma_in, c.eps_block, o); break;
-    default: rownorm_centered_bf16_kernel<4><<<c.T, threads, 0, st>>>(x, c.d_model, gamma_in, c.eps_block, o); break;
+    case 1: launch_k(rownorm_centered_bf16_kernel<1>, c.T, threads, 0, st, x, c.d_model, gamma_in, c.eps_block, o); break;
+    case 2: launch_k(rownorm_centered_bf16_kernel<2>, c.T, threads, 0, st, x, c.d_model, gamma_in, c.eps_block, o); break;
+    default: launch_k(rownorm_centered_bf16_kernel<4>, c.T, threads, 0, st, x, c.d_model, gamma_in, c.eps_block, o); break;
   }
   return last_launch();
 }
@@ -792,7 +834,7 @@ moe_status_t do_resid_update(const moe_config_t& c, const void* b, const void* r
   const uint16_t* bp = static_cast<const uint16_t*>(b);
   const uint16_t* rp = static_cast<const uint16_t*>(r);
   uint16_t* o = static_cast<uint16_t*>(out);
-#define RU(V) resid_update_bf16_kernel<V><<<c.T, threads, 0, st>>>(bp, rp, c.d_model, gamma_post, \
+#define RU(V) launch_k(resid_update_bf16_kernel<V>, c.T, threads, 0, st, bp, rp, c.d_model, gamma_post, \
       c.eps_block, g, c.resid_mode, c.tau, c.resid_floor, o)
   switch (vec) {
     case 1: RU(1); break;
@@ -921,7 +963,7 @@ moe_status_t moe_router_split_weights(const float* w, int32_t n, int32_t d, void
     return MOE_ERR_ALIGNMENT;
   const size_t count = static_cast<size_t>(n) * d;
   const unsigned blocks = static_cast<unsigned>(std::min<size_t>((count + 255) / 256, static_cast<size_t>(std::max(device_info().sms, 1)) * 16));
-  router_split_kernel<<<blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+  launch_k(router_split_kernel, blocks, 256, 0, static_cast<cudaStream_t>(stream),
       w, count, d, static_cast<uint16_t*>(w_split));
   return last_launch();
 }
@@ -1097,7 +1139,7 @@ struct Taps {
     const int row_vec = static_cast<int>(rb / 16);
     const int threads = row_vec >= 256 ? 256 : ((row_vec + 31) / 32) * 32;
     const long grid = std::min<long>(c.T, static_cast<long>(std::max(device_info().sms, 1)) * 16);
-    gather_rows_kernel<<<static_cast<unsigned>(grid), threads, 0, st>>>(
+    launch_k(gather_rows_kernel, static_cast<unsigned>(grid), threads, 0, st,
         static_cast<const uint4*>(x_perm), static_cast<long>(c.T) * c.top_k, inv,
         static_cast<long>(c.T), c.top_k, row_vec, static_cast<uint4*>(t->z));
     return last_launch();
@@ -1269,10 +1311,10 @@ moe_status_t moe_noisy_gate(const moe_config_t* cfg, const void* u, const void* 
   if ((s = do_route(plain, u, w_noise, nullptr, nullptr, mb, si, sw, st)) != MOE_OK) return s;
   float* pi = at<float>(workspace, L.pi);
   float* pl = at<float>(workspace, L.pl);
-  noisy_gate_kernel<<<L.nparts / 4, 128, 0, st>>>(lb, mb, noise_eps, c.T, c.n_experts, c.top_k,
+  launch_k(noisy_gate_kernel, L.nparts / 4, 128, 0, st, lb, mb, noise_eps, c.T, c.n_experts, c.top_k,
                                                   noisy_logits_out, topk_idx, topk_w,
                                                   load_prob_out, pi, pl);
-  gate_stats_reduce_kernel<<<1, kMaxExperts, 0, st>>>(pi, pl, L.nparts, c.n_experts, importance,
+  launch_k(gate_stats_reduce_kernel, 1, kMaxExperts, 0, st, pi, pl, L.nparts, c.n_experts, importance,
                                                       load, cv2);
   return last_launch(2);
 }
@@ -1282,7 +1324,7 @@ unsigned long long moe_launch_count(void) { return g_launches.load(); }
 moe_status_t moe_selftest_wait_timeout(long long budget_clocks, int32_t* gave_up, void* stream) {
   if (!gave_up || budget_clocks <= 0 || budget_clocks > kWaitBudgetClocks) return MOE_ERR_INVALID_ARG;
   if (!aligned16(gave_up)) return MOE_ERR_ALIGNMENT;
-  wait_timeout_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(budget_clocks,
+  launch_k(wait_timeout_selftest_kernel, 1, 32, 0, static_cast<cudaStream_t>(stream), budget_clocks,
                                                                                 gave_up);
   return last_launch();
 }
@@ -1400,7 +1442,7 @@ moe_status_t moe_gather_rows(const void* src, int64_t src_rows, const int32_t* r
   const int row_vec = static_cast<int>(row_bytes / 16);
   const int threads = row_vec >= 256 ? 256 : ((row_vec + 31) / 32) * 32;
   const long grid = std::min<long>(n_rows, static_cast<long>(std::max(device_info().sms, 1)) * 16);
-  gather_rows_kernel<<<static_cast<unsigned>(grid), threads, 0, static_cast<cudaStream_t>(stream)>>>(
+  launch_k(gather_rows_kernel, static_cast<unsigned>(grid), threads, 0, static_cast<cudaStream_t>(stream),
       static_cast<const uint4*>(src), static_cast<long>(src_rows), rows, static_cast<long>(n_rows),
       1, row_vec, static_cast<uint4*>(dst));
   return last_launch();

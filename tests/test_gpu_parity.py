@@ -385,9 +385,10 @@ def test_combine(E, k, norm, with_ss):
         assert row_rel_err(got[t], ref) <= 1e-2
 
 
-@pytest.mark.parametrize("E,k,norm", [(4096, 8, 1), (512, 4, 0), (1024, 2, 1)])
+@pytest.mark.parametrize("E,k,norm", [(4096, 8, 1), (4096, 4, 0), (8192, 2, 1)])
 def test_combine_bulk_matches_per_token(E, k, norm):
-    """The prefill combine (persistent CTAs, expert rows by bulk copies; from 1024 tokens) against
+    """The prefill combine (persistent CTAs, expert rows by bulk copies; from 1024 tokens whose k
+    expert rows hold at least 32 KB) against
     the per-token combine on the same rows, bit for bit (two calls of fewer tokens each), and
     against the oracle on sampled tokens; a few slots are dropped (negative dispatch row)."""
     T, n = 1500, 16
