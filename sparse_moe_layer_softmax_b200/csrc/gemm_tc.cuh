@@ -68,6 +68,10 @@ struct GemmParams {
   int k_splits;              // 1-SM kernel: the reduction split into this many equal k ranges,
                              // each a tile of its own (0 or 1: no split; EPI_PARTIAL only)
   float* partial;            // EPI_PARTIAL: [k_splits][M][Nout] fp32
+  int l2_hints;              // 1: weight tiles are loaded as the first lines L2 evicts (each is
+                             // read by the tiles running at the same time, then not again), and
+                             // the staged output stores are kept in L2 ahead of other lines (the
+                             // next GEMM reads them); for layers whose activations fit in L2
 };
 
 // Shared memory that stages the bf16 output of the normal-orientation epilogues: one 4 KB
@@ -140,6 +144,7 @@ struct EpiOut {
   const CUtensorMap* tm;  // output tensor map, or nullptr: direct stores only
   uint8_t* buf;           // this warp's 4 KB staging buffer (1024-byte aligned)
   bool whole;             // all 32 rows of this warp lie inside the tile
+  bool keep;              // store with the L2 evict-last policy
 };
 
 // Emits one 64-column chunk (8 x 16 bytes per row) of this thread's row at output column x of
@@ -155,7 +160,8 @@ __device__ __forceinline__ void emit_chunk(const EpiOut& eo, const uint4 (&ch)[8
     fence_proxy_async_smem();
     __syncwarp();
     if (lane == 0) {
-      tma_store_2d(eo.tm, eo.buf, x, y);
+      if (eo.keep) tma_store_2d_hint(eo.tm, eo.buf, x, y, l2_policy_evict_last());
+      else tma_store_2d(eo.tm, eo.buf, x, y);
       bulk_commit();
     }
   } else if (valid) {
@@ -530,8 +536,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const int kxx = p.x_k_period > 0 ? kx % p.x_k_period : kx;  // X's k coordinate
         if (!kSwap) {
           tma_load_2d(&tmX, &full[stage], sa, kxx, c.row0);
-          tma_load_2d(&tmW, &full[stage], sb, kx, wrow);
-          if (S::kDual) tma_load_2d(&tmW, &full[stage], sb + (BN / 2) * 128, kx, wrow + p.Nw / 2);
+          if (p.l2_hints) {
+            const uint64_t pol = l2_policy_evict_first();
+            tma_load_2d_hint(&tmW, &full[stage], sb, kx, wrow, pol);
+            if (S::kDual)
+              tma_load_2d_hint(&tmW, &full[stage], sb + (BN / 2) * 128, kx, wrow + p.Nw / 2, pol);
+          } else {
+            tma_load_2d(&tmW, &full[stage], sb, kx, wrow);
+            if (S::kDual) tma_load_2d(&tmW, &full[stage], sb + (BN / 2) * 128, kx, wrow + p.Nw / 2);
+          }
         } else {
           tma_load_2d(&tmW, &full[stage], sa, kx, wrow);
           if (S::kDual) tma_load_2d(&tmW, &full[stage], sa + 128 * 128, kx, wrow + p.Nw / 2);
@@ -591,7 +604,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const int f0 = c.ft * S::kFO;
       if constexpr (!kSwap) {
         const EpiOut eo{(kStageOut && p.out_tma) ? &tmO : nullptr, stage_out + q * 4096,
-                        c.nrows >= q * 32 + 32};
+                        c.nrows >= q * 32 + 32, p.l2_hints != 0};
         epilogue_rows<BN, kEpi>(p, c.row0, c.nrows, f0, tbase, q, lane, s_coef, eo);
       } else {
         // swap orientation: this thread owns output feature f for the BN rows of the chunk
@@ -855,7 +868,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       if (!epilogue_all(mbar_wait(&tfull[acc], acc_phase))) break;
       tc_fence_after();
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * BN;
-      const EpiOut eo{p.out_tma ? &tmO : nullptr, stage_out + q * 4096, nrows >= q * 32 + 32};
+      const EpiOut eo{p.out_tma ? &tmO : nullptr, stage_out + q * 4096, nrows >= q * 32 + 32,
+                      p.l2_hints != 0};
       epilogue_rows<BN, kEpi>(p, row0, nrows, c.ft * S::kFO, tbase, q, lane, s_coef, eo);
       tc_fence_before();
       epilogue_bar();  // all 128 epilogue threads have finished reading this accumulator

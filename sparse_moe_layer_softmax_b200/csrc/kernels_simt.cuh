@@ -103,9 +103,22 @@ __global__ void __launch_bounds__(32)
   const int lane = threadIdx.x;
   const long t0 = static_cast<long>(blockIdx.x) * kPermChunk;
   const int cnt = static_cast<int>((min(static_cast<long>(T), t0 + kPermChunk) - t0) * k);
-  // the chunk's expert indices come in first, all loads in flight together; the ranking loop
-  // below then reads shared memory only
-  for (int i = lane; i < cnt; i += 32) s_idx[i] = idx[t0 * k + i];
+  // the chunk's expert indices come in first, all loads in flight together (a register batch
+  // per lane); the ranking loop below then reads shared memory only
+  {
+    constexpr int kPer = kPermChunk * kMaxTopK / 32;
+    int v[kPer];
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) {
+      const int i = lane + 32 * j;
+      v[j] = i < cnt ? __ldg(idx + t0 * k + i) : 0;
+    }
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) {
+      const int i = lane + 32 * j;
+      if (i < cnt) s_idx[i] = v[j];
+    }
+  }
   for (int e = lane; e < n; e += 32) s_next[e] = offsets[e] + chunk_base[blockIdx.x * n + e];
   __syncwarp();
   const unsigned lower = (1u << lane) - 1u;
@@ -349,9 +362,14 @@ __global__ void scatter_rows_bf16_kernel(const uint16_t* __restrict__ x, int E, 
                                          uint16_t* __restrict__ x_perm) {
   pdl_wait();
   __shared__ float red[8];
+  __shared__ int s_rows[kMaxTopK];
   const int t = blockIdx.x;
   const int nvec = E / 8;
   const uint4* src = reinterpret_cast<const uint4*>(x + static_cast<size_t>(t) * E);
+  // the token's dispatch rows load alongside its values
+  if (threadIdx.x < kMaxTopK)
+    s_rows[threadIdx.x] = static_cast<int>(threadIdx.x) < k
+                              ? __ldg(inv_perm + static_cast<size_t>(t) * k + threadIdx.x) : -1;
   uint4 r[VEC];
   float ss = 0.0f;
 #pragma unroll
@@ -380,8 +398,9 @@ __global__ void scatter_rows_bf16_kernel(const uint16_t* __restrict__ x, int E, 
       }
     }
   }
+  __syncthreads();
   for (int j = 0; j < k; ++j) {
-    const int row = inv_perm[static_cast<size_t>(t) * k + j];
+    const int row = s_rows[j];
     if (row < 0) continue;
     uint4* dst = reinterpret_cast<uint4*>(x_perm + static_cast<size_t>(row) * E);
 #pragma unroll
@@ -604,7 +623,7 @@ __global__ void __launch_bounds__(kCombineMaxThreads)
 // up), then copies that row's E values and, with expert_norm, its `parts` partial sums of squares
 // into the stage.  Eight consumer warps finish the token at the head of the ring and write y.
 // Every wait is bounded; a timeout latches MOE_ERR_TIMEOUT and the roles stop.
-constexpr int kBulkCombineConsumers = 256;
+constexpr int kBulkCombineConsumers = 512;
 
 struct BulkCombineStage {
   // byte offsets inside one stage
@@ -695,10 +714,16 @@ __global__ void __launch_bounds__(kBulkCombineConsumers + 32, 1)
       const float* hw = reinterpret_cast<const float*>(sb + L.hdr + 32);
       // slot j's I_gamma factor from its partials, in part order (lane j), to every lane
       float my_rinv = 1.0f;
-      if (norm && lane < k && hrow[lane] >= 0) {
-        const float* ps = reinterpret_cast<const float*>(sb + L.ss) + lane * parts;
+      if (norm && lane < k && hrow[lane] >= 0) {  // parts is a multiple of 4 (16-byte copies)
+        const float4* ps = reinterpret_cast<const float4*>(sb + L.ss + lane * parts * 4);
         float tot = 0.0f;
-        for (int p = 0; p < parts; ++p) tot += ps[p];
+        for (int p4 = 0; p4 < parts / 4; ++p4) {
+          const float4 q4 = ps[p4];
+          tot += q4.x;
+          tot += q4.y;
+          tot += q4.z;
+          tot += q4.w;
+        }
         my_rinv = rsqrtf(tot / static_cast<float>(E) + eps);
       }
       float rinv[kMaxTopK], wgt[kMaxTopK];
@@ -785,7 +810,7 @@ __global__ void combine_f32_kernel(const float* __restrict__ s, int E, int k,
 constexpr int kRouterTok = 8;
 constexpr int kRouterExp = 16;
 constexpr int kRouterThreads = 512;  // one warp per expert of the CTA
-constexpr int kRouterLoads = 4;      // weight vectors each lane keeps in flight
+constexpr int kRouterLoads = 8;      // weight vectors each lane keeps in flight
 
 __global__ void __launch_bounds__(kRouterThreads, 1) router_logits_small_kernel(
     const uint16_t* __restrict__ u, const uint16_t* __restrict__ w, const float* __restrict__ bias,
@@ -793,14 +818,25 @@ __global__ void __launch_bounds__(kRouterThreads, 1) router_logits_small_kernel(
   pdl_wait();
   // w rows have wk = d (bf16 weights) or 3d (hi/mid/lo parts of fp32 weights; u repeats)
   extern __shared__ uint4 s_u[];  // [kRouterTok][d/8]
+  __shared__ uint64_t s_bar;
   const int t0 = blockIdx.y * kRouterTok;
   const int nt = min(kRouterTok, T - t0);
   const int nvec = d / 8;
-  for (int i = threadIdx.x; i < kRouterTok * nvec; i += blockDim.x) {
-    const int tt = i / nvec, v = i - tt * nvec;
-    s_u[i] = tt < nt ? reinterpret_cast<const uint4*>(u + static_cast<size_t>(t0 + tt) * d)[v]
-                     : make_uint4(0, 0, 0, 0);
+  // the CTA's token rows come in by bulk copies (one per row); rows past the batch are zero
+  if (threadIdx.x == 0) {
+    mbar_init(&s_bar, 1);
+    fence_barrier_init();
   }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    mbar_arrive_expect_tx(&s_bar, static_cast<uint32_t>(nt) * static_cast<uint32_t>(d) * 2u);
+    for (int tt = 0; tt < nt; ++tt)
+      bulk_load(s_u + static_cast<size_t>(tt) * nvec, u + static_cast<size_t>(t0 + tt) * d,
+                static_cast<uint32_t>(d) * 2u, &s_bar);
+  }
+  for (int i = nt * nvec + static_cast<int>(threadIdx.x); i < kRouterTok * nvec; i += blockDim.x)
+    s_u[i] = make_uint4(0, 0, 0, 0);
+  mbar_wait(&s_bar, 0);
   __syncthreads();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
   for (int el = warp; el < kRouterExp; el += nwarps) {
