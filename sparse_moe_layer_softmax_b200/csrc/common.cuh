@@ -98,26 +98,6 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
   return true;
 }
 
-// The same bounded wait for a thread that expects to wait long (an epilogue warp waiting for the
-// next accumulator while the tensor pipe works on it): between polls it sleeps, starting at 256 ns
-// and doubling to 4 us, so that a warp waiting tens of microseconds issues a few dozen
-// instructions instead of thousands.
-__device__ __forceinline__ bool mbar_wait_sleepy(uint64_t* bar, uint32_t parity,
-                                                 long long budget = kWaitBudgetClocks) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const long long t0 = clock64();
-  uint32_t ns = 256;
-  while (!mbar_try_wait(bar, parity)) {
-    if (clock64() - t0 > budget) {
-      latch_status(MOE_ERR_TIMEOUT);
-      return false;
-    }
-    __nanosleep(ns);
-    if (ns < 4096) ns <<= 1;
-  }
-  return true;
-}
-
 // ------------------------------------------------------------------ TMA (no multicast)
 
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* m) {

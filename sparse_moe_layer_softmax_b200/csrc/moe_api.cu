@@ -233,9 +233,9 @@ moe_status_t run_gemm(int epi, Orient o, int bn, const void* X, long x_rows, con
     const int fo = dual ? SwapPairShape<EPI_SWIGLU>::kFO : SwapPairShape<EPI_STORE>::kFO;
     if (p.Nout % fo) return MOE_ERR_UNSUPPORTED;
     const long pt = tile_bound(x_rows, p.G, 256, p.Nout / fo);
-    if (epi == EPI_SWIGLU) return launch_gemm_swap_pair<EPI_SWIGLU, 6>(X, x_rows, W, w_rows, p, pt, st);
-    if (epi == EPI_STORE) return launch_gemm_swap_pair<EPI_STORE, 6>(X, x_rows, W, w_rows, p, pt, st);
-    if (epi == EPI_RELU) return launch_gemm_swap_pair<EPI_RELU, 6>(X, x_rows, W, w_rows, p, pt, st);
+    if (epi == EPI_SWIGLU) return launch_gemm_swap_pair<EPI_SWIGLU, 4>(X, x_rows, W, w_rows, p, pt, st);
+    if (epi == EPI_STORE) return launch_gemm_swap_pair<EPI_STORE, 4>(X, x_rows, W, w_rows, p, pt, st);
+    if (epi == EPI_RELU) return launch_gemm_swap_pair<EPI_RELU, 4>(X, x_rows, W, w_rows, p, pt, st);
     return MOE_ERR_UNSUPPORTED;
   }
   const int fo = dual ? bn / 2 : bn;
