@@ -41,6 +41,13 @@ __device__ __forceinline__ uint16_t f32_to_bf16(float f) {
   return *reinterpret_cast<uint16_t*>(&h);
 }
 __device__ __forceinline__ float round_bf16(float f) { return bf16_to_f32(f32_to_bf16(f)); }
+// acc + a * b for bf16 a, b and an fp32 acc in one instruction (sm_100 mixed-precision FMA): the
+// product of two bf16 values is exact in fp32, so this equals fmaf(float(a), float(b), acc).
+__device__ __forceinline__ float fma_bf16_f32(uint16_t a, uint16_t b, float acc) {
+  float d;
+  asm("fma.rn.f32.bf16 %0, %1, %2, %3;" : "=f"(d) : "h"(a), "h"(b), "f"(acc));
+  return d;
+}
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return static_cast<uint32_t>(f32_to_bf16(lo)) | (static_cast<uint32_t>(f32_to_bf16(hi)) << 16);
 }
@@ -119,6 +126,13 @@ __device__ __forceinline__ void tma_load_2d_hint(const CUtensorMap* m, uint64_t*
       " [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(smem_u32(dst)),
       "l"(reinterpret_cast<uint64_t>(m)), "r"(smem_u32(bar)), "r"(x), "r"(y), "l"(policy)
       : "memory");
+}
+// Asks L2 to fetch one box of the tensor ahead of its load (no shared memory, nothing to wait for).
+__device__ __forceinline__ void tma_prefetch_2d(const CUtensorMap* m, int32_t x, int32_t y) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
+                   reinterpret_cast<uint64_t>(m)),
+               "r"(x), "r"(y)
+               : "memory");
 }
 // Untiled bulk copy of `bytes` (a multiple of 16; both addresses 16-byte aligned) from global
 // memory into this CTA's shared memory, completing its bytes on the mbarrier.  No multicast.

@@ -528,6 +528,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       TileCoord c = decode_tile(t - ks * total, s_seg, s_pref, G, FT, S::kCH, p.tile_order);
       const int wrow = c.g * p.Nw + c.ft * S::kFO;
       for (int kb = ks * KBs; kb < (ks + 1) * KBs; ++kb) {
+        // weight-stream-bound layers (l2_hints): L2 fetches the weight k-block one ring ahead, so
+        // more DRAM requests are in flight than the shared-memory ring holds
+        if (!kSwap && p.l2_hints && kb + kStages < (ks + 1) * KBs) {
+          const int kp = (kb + kStages) * S::kBK;
+          tma_prefetch_2d(&tmW, kp, wrow);
+          if (S::kDual) tma_prefetch_2d(&tmW, kp, wrow + p.Nw / 2);
+        }
         if (!mbar_wait(&empty[stage], phase ^ 1)) { ok = false; break; }
         uint8_t* sa = tiles + stage * S::kStageBytes;
         uint8_t* sb = sa + S::kABytes;

@@ -862,15 +862,13 @@ __global__ void __launch_bounds__(kRouterThreads, 1) router_logits_small_kernel(
         if (vw >= wvec) break;
         const int v = vw % nvec;
         const uint16_t* wh = reinterpret_cast<const uint16_t*>(&wq[j]);
-        float wf[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) wf[i] = bf16_to_f32(wh[i]);
 #pragma unroll
         for (int tt = 0; tt < kRouterTok; ++tt) {
           const uint4 uq = s_u[tt * nvec + v];
           const uint16_t* uh = reinterpret_cast<const uint16_t*>(&uq);
+          // fp32 += bf16 x bf16, the product exact, one rounding: one instruction per product
 #pragma unroll
-          for (int i = 0; i < 8; ++i) acc[tt] = fmaf(bf16_to_f32(uh[i]), wf[i], acc[tt]);
+          for (int i = 0; i < 8; ++i) acc[tt] = fma_bf16_f32(uh[i], wh[i], acc[tt]);
         }
       }
     }

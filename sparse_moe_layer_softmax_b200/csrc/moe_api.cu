@@ -1,6 +1,7 @@
 // Host side of the C ABI declared in include/moe.h: argument checks, workspace layout, TMA
 // descriptors and the launch sequence of the MoE-layer forward on the caller's stream.
 #include <cudaTypedefs.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <algorithm>
 #include <atomic>
@@ -602,9 +603,17 @@ Profiler& prof() {
 
 constexpr int kMarks = MOE_PROFILE_STAGES + 1;
 
+// Stage names of the forward, for the NVTX ranges a profiler's timeline shows around each stage's
+// launches (a range per stage, from this mark to the next).
+constexpr const char* kStageNames[MOE_PROFILE_STAGES] = {
+    "moe.route", "moe.latent_down", "moe.dispatch", "moe.expert_gate_up", "moe.expert_down",
+    "moe.combine", "moe.latent_up"};
+
 void prof_mark(cudaStream_t st, int i) {
   Profiler& p = prof();
   if (p.active && p.calls < p.max_calls) cudaEventRecord(p.ev[p.calls * kMarks + i], st);
+  if (i > 0) nvtxRangePop();
+  if (i < MOE_PROFILE_STAGES) nvtxRangePushA(kStageNames[i]);
 }
 
 void prof_next_call() {
