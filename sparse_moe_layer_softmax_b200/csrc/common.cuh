@@ -21,11 +21,12 @@ __device__ __forceinline__ void latch_status(int code) { atomicCAS(&g_status, 0,
 // ------------------------------------------------------------------ programmatic dependent launch
 //
 // The library launches the kernels of a layer forward so that each may start while the kernel
-// before it on the stream is finishing (programmatic stream serialization).  Every kernel
-// therefore waits, before it touches global memory, until the grids it depends on have completed
-// and their writes are visible (a no-op for a kernel launched without that attribute).
-// Persistent kernels, whose CTAs are all resident at once, let the next kernel launch as soon as
-// they start; the others let it launch when their CTAs exit.
+// before it on the stream is finishing (programmatic stream serialization).  Every kernel waits,
+// before it reads anything an earlier kernel writes, until the grids it depends on have completed
+// and their writes are visible (a no-op for a kernel launched without that attribute), and then
+// lets the next kernel launch: that kernel's CTAs take SMs as this kernel's CTAs leave them and do
+// their own setup, and wait in turn.  (The next kernel launches once every CTA of this one has
+// passed that point, so its waiting CTAs never keep one of this kernel's CTAs off an SM.)
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_launch_dependents() {
   asm volatile("griddepcontrol.launch_dependents;" :::);

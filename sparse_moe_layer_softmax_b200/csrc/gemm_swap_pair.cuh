@@ -119,7 +119,6 @@ template <int kEpi, int kStages>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     gemm_swap_pair_kernel(const __grid_constant__ CUtensorMap tmX,
                           const __grid_constant__ CUtensorMap tmW, const GemmParams p) {
-  pdl_wait();
   using S = SwapPairShape<kEpi>;
   static_assert(kEpi == EPI_SWIGLU || kEpi == EPI_STORE || kEpi == EPI_RELU,
                 "the swapped pair kernel has the expert epilogues");
@@ -146,6 +145,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   const int G = p.G;
   const int FT = p.Nout / S::kFO;
   const int KB = p.K / S::kBK;
+
+  // Setup that reads nothing an earlier kernel writes (barriers, TMEM, the tensor-map prefetch)
+  // runs before the dependency wait and overlaps the previous kernel's tail.
+  if (threadIdx.x == 32) {
+    for (int s = 0; s < kStages; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+    for (int a = 0; a < 2; ++a) { mbar_init(&tfull[a], 1); mbar_init(&tempty[a], 2); }
+    mbar_init(done, 1);
+    fence_barrier_init();
+  }
+  if (warp == 1) tmem_alloc_pair(tmem_slot, S::kTmemCols);
+  if (threadIdx.x == 0) {
+    tma_prefetch_desc(&tmX);
+    tma_prefetch_desc(&tmW);
+  }
+  pdl_wait();
+  pdl_launch_dependents();  // every CTA is resident: the next kernel may launch
 
   if (warp == 0) {  // group segments and the per-group tile prefix
     const int per = (G + 31) / 32;
@@ -178,13 +193,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     }
     if (lane == 31) s_pref[G] = incl;
   }
-  if (threadIdx.x == 32) {
-    for (int s = 0; s < kStages; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
-    for (int a = 0; a < 2; ++a) { mbar_init(&tfull[a], 1); mbar_init(&tempty[a], 2); }
-    mbar_init(done, 1);
-    fence_barrier_init();
-  }
-  if (warp == 1) tmem_alloc_pair(tmem_slot, S::kTmemCols);
   tc_fence_before();
   __syncthreads();
   cluster_sync_all();  // the peer's barriers exist before any remote arrive or TMA completion
@@ -194,8 +202,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
 
   if (warp == 0 && lane == 0) {
     // ------------------------------------------------------------ TMA producer (both CTAs)
-    tma_prefetch_desc(&tmX);
-    tma_prefetch_desc(&tmW);
     uint32_t stage = 0, phase = 0;
     uint32_t last_parity[kStages];
     bool issued[kStages];

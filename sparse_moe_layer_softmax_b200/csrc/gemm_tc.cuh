@@ -439,7 +439,6 @@ template <bool kSwap, int BN, int kEpi, int kStages>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
                    const __grid_constant__ CUtensorMap tmO, const GemmParams p) {
-  pdl_wait();
   using S = GemmShape<kSwap, BN, kEpi>;
   constexpr bool kStageOut = stages_output<kSwap, kEpi>();
   extern __shared__ uint8_t smem_raw[];
@@ -462,6 +461,22 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const int G = p.G;
   const int FT = (p.Nout + S::kFO - 1) / S::kFO;  // the router's last tile may be partial
   const int KB = p.K / S::kBK;
+
+  // Setup that reads nothing an earlier kernel writes (barriers, TMEM, the tensor-map prefetch)
+  // runs before the dependency wait and overlaps the previous kernel's tail.
+  if (threadIdx.x == 32) {
+    for (int s = 0; s < kStages; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+    for (int a = 0; a < 2; ++a) { mbar_init(&tfull[a], 1); mbar_init(&tempty[a], 128); }
+    mbar_init(done, 1);
+    fence_barrier_init();
+  }
+  if (warp == 1) tmem_alloc(tmem_slot, S::kTmemCols);
+  if (threadIdx.x == 0) {
+    tma_prefetch_desc(&tmX);
+    tma_prefetch_desc(&tmW);
+  }
+  pdl_wait();
+  pdl_launch_dependents();  // one CTA per SM, all resident: the next kernel may launch
 
   // ---- group segments and the per-group tile prefix (warp 0)
   if (warp == 0) {
@@ -495,13 +510,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
     if (lane == 31) s_pref[G] = incl;
   }
-  if (threadIdx.x == 32) {
-    for (int s = 0; s < kStages; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
-    for (int a = 0; a < 2; ++a) { mbar_init(&tfull[a], 1); mbar_init(&tempty[a], 128); }
-    mbar_init(done, 1);
-    fence_barrier_init();
-  }
-  if (warp == 1) tmem_alloc(tmem_slot, S::kTmemCols);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -515,8 +523,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
   if (warp == 0 && lane == 0) {
     // ------------------------------------------------------------ TMA producer
-    tma_prefetch_desc(&tmX);
-    tma_prefetch_desc(&tmW);
     uint32_t stage = 0, phase = 0;
     uint32_t last_parity[kStages];
     bool issued[kStages];
@@ -731,7 +737,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     gemm_tc_pair_kernel(const __grid_constant__ CUtensorMap tmX,
                         const __grid_constant__ CUtensorMap tmW,
                         const __grid_constant__ CUtensorMap tmO, const GemmParams p) {
-  pdl_wait();
   using S = PairShape<BN, kEpi>;
   static_assert(kEpi != EPI_ROUTER, "the pair kernel has bf16 epilogues only");
   extern __shared__ uint8_t smem_raw[];
@@ -756,6 +761,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   const int G = p.G;
   const int FT = p.Nout / S::kFO;
   const int KB = p.K / S::kBK;
+
+  // Setup that reads nothing an earlier kernel writes (barriers, TMEM, the tensor-map prefetch)
+  // runs before the dependency wait and overlaps the previous kernel's tail.
+  if (threadIdx.x == 32) {
+    for (int s = 0; s < kStages; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+    for (int a = 0; a < 2; ++a) { mbar_init(&tfull[a], 1); mbar_init(&tempty[a], 2); }
+    mbar_init(done, 1);
+    fence_barrier_init();
+  }
+  if (warp == 1) tmem_alloc_pair(tmem_slot, S::kTmemCols);
+  if (threadIdx.x == 0) {
+    tma_prefetch_desc(&tmX);
+    tma_prefetch_desc(&tmW);
+  }
+  pdl_wait();
+  pdl_launch_dependents();  // one CTA per SM, all resident: the next kernel may launch
 
   if (warp == 0) {  // group segments and tile prefix, as in the 1-SM kernel (256-row chunks)
     const int per = (G + 31) / 32;
@@ -788,13 +809,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     }
     if (lane == 31) s_pref[G] = incl;
   }
-  if (threadIdx.x == 32) {
-    for (int s = 0; s < kStages; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
-    for (int a = 0; a < 2; ++a) { mbar_init(&tfull[a], 1); mbar_init(&tempty[a], 2); }
-    mbar_init(done, 1);
-    fence_barrier_init();
-  }
-  if (warp == 1) tmem_alloc_pair(tmem_slot, S::kTmemCols);
   tc_fence_before();
   __syncthreads();
   cluster_sync_all();  // the peer's barriers exist before any remote arrive or TMA completion
@@ -804,8 +818,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
 
   if (warp == 0 && lane == 0) {
     // ------------------------------------------------------------ TMA producer (both CTAs)
-    tma_prefetch_desc(&tmX);
-    tma_prefetch_desc(&tmW);
     uint32_t stage = 0, phase = 0;
     uint32_t last_parity[kStages];
     bool issued[kStages];

@@ -34,6 +34,7 @@ __device__ __forceinline__ float block_sum_256(float v, float* red) {
 __global__ void perm_count_kernel(const int32_t* __restrict__ idx, int T, int k, int n,
                                   int32_t* __restrict__ counts) {
   pdl_wait();
+  pdl_launch_dependents();
   __shared__ int h[kMaxExperts];
   for (int e = threadIdx.x; e < n; e += blockDim.x) h[e] = 0;
   __syncthreads();
@@ -53,6 +54,7 @@ __global__ void perm_count_kernel(const int32_t* __restrict__ idx, int T, int k,
 __global__ void perm_scan_kernel(int32_t* __restrict__ counts, int nchunks, int n,
                                  int32_t* __restrict__ offsets) {
   pdl_wait();
+  pdl_launch_dependents();
   __shared__ int warp_tot[kMaxExperts / 32];
   const int e = threadIdx.x;
   int run = 0;
@@ -98,6 +100,7 @@ __global__ void __launch_bounds__(32)
                      const int32_t* __restrict__ chunk_base, const int32_t* __restrict__ offsets,
                      int32_t* __restrict__ perm_token, int32_t* __restrict__ inv_perm) {
   pdl_wait();
+  pdl_launch_dependents();
   __shared__ int s_next[kMaxExperts];
   __shared__ int s_idx[kPermChunk * kMaxTopK];
   const int lane = threadIdx.x;
@@ -163,6 +166,7 @@ __global__ void dispatch_small_bf16_kernel(const int32_t* __restrict__ idx, int 
                                            int32_t* __restrict__ inv_perm,
                                            uint16_t* __restrict__ x_perm) {
   pdl_wait();
+  pdl_launch_dependents();
   __shared__ int s_idx[kSmallDispatchSlots];
   __shared__ int s_off[kMaxExperts + 1];  // counts, then their exclusive scan (and the total)
   __shared__ int s_rank[kMaxTopK];
@@ -284,6 +288,7 @@ __global__ void dense_split_finish_kernel(const float* __restrict__ partial, int
                                           const float* __restrict__ g, float tau, float floor_,
                                           int resid_mode, uint16_t* __restrict__ out) {
   pdl_wait();
+  pdl_launch_dependents();
   const long nv = rows * nout / 8;
   const size_t plane = static_cast<size_t>(rows) * nout;
   for (long i = blockIdx.x * static_cast<long>(blockDim.x) + threadIdx.x; i < nv;
@@ -337,6 +342,7 @@ __global__ void gather_rows_kernel(const uint4* __restrict__ src, long src_rows,
                                    const int32_t* __restrict__ rows, long n_rows, int idx_stride,
                                    int row_vec, uint4* __restrict__ dst) {
   pdl_wait();
+  pdl_launch_dependents();
   for (long i = blockIdx.x; i < n_rows; i += gridDim.x) {
     int r = rows[i * idx_stride];
     if (r >= src_rows) {
@@ -361,6 +367,7 @@ __global__ void scatter_rows_bf16_kernel(const uint16_t* __restrict__ x, int E, 
                                          const float* __restrict__ gamma, float eps,
                                          uint16_t* __restrict__ x_perm) {
   pdl_wait();
+  pdl_launch_dependents();
   __shared__ float red[8];
   __shared__ int s_rows[kMaxTopK];
   const int t = blockIdx.x;
@@ -416,6 +423,7 @@ __global__ void scatter_rows_f32_kernel(const float* __restrict__ x, int E, int 
                                         const int32_t* __restrict__ inv_perm,
                                         float* __restrict__ x_perm) {
   pdl_wait();
+  pdl_launch_dependents();
   const int t = blockIdx.x;
   for (int j = 0; j < k; ++j) {
     const int row = inv_perm[static_cast<size_t>(t) * k + j];
@@ -449,6 +457,7 @@ __global__ void __launch_bounds__(kCombineMaxThreads)
                         const int32_t* __restrict__ inv_perm, const float* __restrict__ topk_w,
                         int expert_norm, float eps, uint16_t* __restrict__ y) {
   pdl_wait();
+  pdl_launch_dependents();
   // One pass: every thread loads its VEC 16-byte vectors of all k rows at once (k x VEC loads in
   // flight) and keeps them as packed bf16; the row norms and the weighted sum both come from
   // there.  The arithmetic runs on fp32 pairs (Blackwell's two-wide FMA / multiply), so each
@@ -548,6 +557,7 @@ __global__ void __launch_bounds__(kCombineMaxThreads)
                            const float* __restrict__ row_ss, int parts, float eps,
                            uint16_t* __restrict__ y) {
   pdl_wait();
+  pdl_launch_dependents();
   const int t = blockIdx.x;
   const int nvec = E / 8;
   const int lane = threadIdx.x & 31;
@@ -645,6 +655,7 @@ __global__ void __launch_bounds__(kBulkCombineConsumers + 32, 1)
                              int parts, int expert_norm, float eps, uint16_t* __restrict__ y,
                              int T, int nst) {
   pdl_wait();
+  pdl_launch_dependents();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) &
                                              ~static_cast<uintptr_t>(127));
@@ -780,6 +791,7 @@ __global__ void combine_f32_kernel(const float* __restrict__ s, int E, int k,
                                    const float* __restrict__ topk_w, int expert_norm, float eps,
                                    float* __restrict__ y) {
   pdl_wait();
+  pdl_launch_dependents();
   __shared__ float red[8];
   const int t = blockIdx.x;
   for (int c0 = 0; c0 < E; c0 += blockDim.x) {
@@ -816,6 +828,7 @@ __global__ void __launch_bounds__(kRouterThreads, 1) router_logits_small_kernel(
     const uint16_t* __restrict__ u, const uint16_t* __restrict__ w, const float* __restrict__ bias,
     int T, int d, int n, int wk, float mult, float* __restrict__ logits) {
   pdl_wait();
+  pdl_launch_dependents();
   // w rows have wk = d (bf16 weights) or 3d (hi/mid/lo parts of fp32 weights; u repeats)
   extern __shared__ uint4 s_u[];  // [kRouterTok][d/8]
   __shared__ uint64_t s_bar;
@@ -900,6 +913,7 @@ __global__ void topk_rows_kernel(float* __restrict__ logits, int T, int n, int k
                                  const float* __restrict__ sel_bias,
                                  int32_t* __restrict__ topk_idx, float* __restrict__ topk_w) {
   pdl_wait();
+  pdl_launch_dependents();
   const int warps = blockDim.x >> 5;
   const int t = blockIdx.x * warps + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
@@ -989,6 +1003,7 @@ __global__ void topk_rows_kernel(float* __restrict__ logits, int T, int n, int k
 __global__ void router_split_kernel(const float* __restrict__ w, size_t count, int d,
                                     uint16_t* __restrict__ out) {
   pdl_wait();
+  pdl_launch_dependents();
   const size_t stride = static_cast<size_t>(gridDim.x) * blockDim.x;
   for (size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < count; i += stride) {
     const size_t row = i / d, c = i - row * d;
@@ -1015,6 +1030,7 @@ __global__ void rownorm_centered_bf16_kernel(const uint16_t* __restrict__ x, int
                                              const float* __restrict__ gamma, float eps,
                                              uint16_t* __restrict__ out) {
   pdl_wait();
+  pdl_launch_dependents();
   __shared__ float red[8];
   const size_t base = static_cast<size_t>(blockIdx.x) * D;
   const int nvec = D / 8;
@@ -1053,6 +1069,7 @@ __global__ void resid_update_bf16_kernel(const uint16_t* __restrict__ b, const u
                                          const float* __restrict__ g, int resid_mode, float tau,
                                          float floor_, uint16_t* __restrict__ out) {
   pdl_wait();
+  pdl_launch_dependents();
   __shared__ float red[8];
   const size_t base = static_cast<size_t>(blockIdx.x) * D;
   const int nvec = D / 8;
@@ -1120,6 +1137,7 @@ __global__ void noisy_gate_kernel(const float* __restrict__ l, const float* __re
                                   float* __restrict__ topk_w, float* __restrict__ P_out,
                                   float* __restrict__ part_imp, float* __restrict__ part_load) {
   pdl_wait();
+  pdl_launch_dependents();
   const int lane = threadIdx.x & 31;
   const int gw = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);  // global warp
   const int t0 = gw * kGateTokensPerWarp;
@@ -1210,6 +1228,7 @@ __global__ void gate_stats_reduce_kernel(const float* __restrict__ part_imp,
                                          float* __restrict__ importance, float* __restrict__ load,
                                          float* __restrict__ cv2) {
   pdl_wait();
+  pdl_launch_dependents();
   __shared__ float si[kMaxExperts], sl[kMaxExperts];
   const int e = threadIdx.x;
   float a = 0.0f, b = 0.0f;
@@ -1245,6 +1264,7 @@ __global__ void gate_stats_reduce_kernel(const float* __restrict__ part_imp,
 // latches MOE_ERR_TIMEOUT in the status word and the kernel returns normally.
 __global__ void wait_timeout_selftest_kernel(long long budget, int* gave_up) {
   pdl_wait();
+  pdl_launch_dependents();
   __shared__ __align__(8) uint64_t bar;
   if (threadIdx.x != 0) return;
   mbar_init(&bar, 1);
@@ -1264,6 +1284,7 @@ __global__ void router_f32_kernel(const float* __restrict__ u, const float* __re
                                   float* __restrict__ logits_out,
                                   int32_t* __restrict__ topk_idx, float* __restrict__ topk_w) {
   pdl_wait();
+  pdl_launch_dependents();
   const int warps = blockDim.x >> 5;
   const int t = blockIdx.x * warps + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
@@ -1348,6 +1369,7 @@ __global__ void expert_ffn_f32_kernel(const float* __restrict__ x_perm,
                                       const float* __restrict__ gamma,
                                       float* __restrict__ out_perm) {
   pdl_wait();
+  pdl_launch_dependents();
   extern __shared__ float sm[];  // [E] input row, [H] hidden
   float* xr = sm;
   float* hid = sm + E;

@@ -87,8 +87,8 @@ moe_status_t last_launch(int n = 1) {
 }
 
 // Every kernel is launched with programmatic stream serialization: it may begin while the kernel
-// before it on the stream finishes, and waits (pdl_wait, its first statement) for that kernel's
-// results before touching memory.  Errors surface through last_launch().
+// before it on the stream finishes, and waits (pdl_wait) for that kernel's results before it reads
+// anything an earlier kernel writes.  Errors surface through last_launch().
 template <typename... KArgs, typename... Args>
 void launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
               Args... args) {
@@ -350,24 +350,48 @@ bool pair_tiles_enabled() {
 // Grouped-GEMM orientation for the experts from the mean rows per expert.
 int expert_in_width(const moe_config_t& c) { return c.d_latent > 0 ? c.d_latent : c.d_model; }
 
-// Tuning knob: MOE_EXPERT_TILES=swap_pair in the environment puts prefill-sized expert GEMMs on
-// the swapped CTA-pair tiles instead of the 1-SM 128-row activation tiles (same values up to the
-// fp32 summation inside the tensor core).  Off by default: under the 1 kW power cap the pair
-// tiles do more work per clock but spend more energy per launch, so they run at lower clocks and
-// take longer.
-bool swap_pair_enabled() {
+// Expert tilings for groups too large for the swapped 1-SM tiles (more than 48 rows per expert on
+// average).  The 1-SM tiles put 128 token rows on the MMA's M side, so a group's last chunk pays for
+// up to 127 padding rows; the swapped CTA-pair tiles put the tokens on N, cut to 16 rows.  Measured
+// inside the layer:
+//   - at 512 rows per expert (the prefill batch) both GEMMs take about as long either way; the
+//     pair tiles do more work per clock but spend more energy per launch under the 1 kW cap;
+//   - at about 128 rows per expert with 1 MB experts (the Shazeer batch, d 512, hidden 1024: the
+//     128-row chunks do 1.48x the MMA work) the down GEMM is faster on the pair tiles (0.076
+//     against 0.088 ms), while the first GEMM, whose reduction is only 512 deep, is slower (0.094
+//     against 0.081 ms);
+//   - at 64 and 128 rows per expert with the Muse experts (reductions 4096 deep) the pair tiles
+//     are slower for both GEMMs (down 1.69 against 1.41 ms and 1.84 against 1.70 ms): there the
+//     weight stream, not the MMA work, sets the pace.
+// So by default the down GEMM takes the pair tiles from 49 to 256 mean rows per expert when its
+// reduction is at most 1024 deep.  Tuning knob: MOE_EXPERT_TILES=swap_pair (both GEMMs on the pair
+// tiles for every group above 48 rows) or MOE_EXPERT_TILES=normal (neither).  The values are the
+// same up to the fp32 summation inside the tensor core.
+enum class TilePref { kDefault, kSwapPair, kNormal };
+TilePref expert_tile_pref() {
   const char* v = getenv("MOE_EXPERT_TILES");
-  return v && v[0] == 's';
+  if (v && v[0] == 's') return TilePref::kSwapPair;
+  if (v && v[0] == 'n') return TilePref::kNormal;
+  return TilePref::kDefault;
 }
 
-void pick_expert_orient(const moe_config_t& c, int nout, bool dual, Orient* o, int* bn) {
+constexpr double kSwapMaxMeanRows = 48.0;      // swapped 1-SM tiles up to this mean
+constexpr double kDownPairMaxMeanRows = 256.0; // down GEMM on the pair tiles up to this mean
+constexpr int kDownPairMaxK = 1024;            // ... and up to this reduction depth
+
+// `down` selects the rule of the second expert GEMM (a -> o), `dual` the SwiGLU pairing of the first.
+void pick_expert_orient(const moe_config_t& c, int nout, bool dual, bool down, Orient* o, int* bn) {
   const double mean_rows = static_cast<double>(c.T) * c.top_k / c.n_experts;
-  if (nout % 128 == 0 && mean_rows <= 48.0) {
+  const TilePref pref = expert_tile_pref();
+  const int fo = dual ? SwapPairShape<EPI_SWIGLU>::kFO : SwapPairShape<EPI_STORE>::kFO;
+  const bool pair_ok = !pair_tiles_enabled() && nout % fo == 0;
+  if (nout % 128 == 0 && mean_rows <= kSwapMaxMeanRows) {
     *o = Orient::kSwap;
     *bn = mean_rows <= 12.0 ? 16 : (mean_rows <= 24.0 ? 32 : 64);
-  } else if (swap_pair_enabled() && !pair_tiles_enabled() &&
-             nout % (dual ? SwapPairShape<EPI_SWIGLU>::kFO : SwapPairShape<EPI_STORE>::kFO) == 0) {
-    // prefill-sized groups: tokens on the MMA's N side, cut to 16 rows, on CTA pairs
+  } else if (pair_ok && (pref == TilePref::kSwapPair ||
+                         (pref == TilePref::kDefault && down && c.d_ff <= kDownPairMaxK &&
+                          mean_rows <= kDownPairMaxMeanRows))) {
+    // tokens on the MMA's N side, cut to 16 rows, on CTA pairs
     *o = Orient::kSwapPair;
     *bn = 256;
   } else {
@@ -386,7 +410,7 @@ void pick_expert_orient(const moe_config_t& c, int nout, bool dual, Orient* o, i
 int sumsq_parts(const moe_config_t& c) {
   Orient o;
   int bn;
-  pick_expert_orient(c, expert_in_width(c), false, &o, &bn);
+  pick_expert_orient(c, expert_in_width(c), false, true, &o, &bn);
   if (bn <= 0) return 1;
   if (o == Orient::kSwapPair) return expert_in_width(c) / 128;  // one per CTA's 128 features
   return o == Orient::kSwap ? expert_in_width(c) / 128 * 4 : expert_in_width(c) / bn;
@@ -656,7 +680,7 @@ moe_status_t do_experts(const moe_config_t& c, const void* x_perm, const int32_t
   p1.out = act;
   Orient o1;
   int bn1;
-  pick_expert_orient(c, H, swiglu, &o1, &bn1);
+  pick_expert_orient(c, H, swiglu, false, &o1, &bn1);
   if (bn1 == 0) return MOE_ERR_UNSUPPORTED;
   moe_status_t s = run_gemm(swiglu ? EPI_SWIGLU : EPI_RELU, o1, bn1, x_perm, TK, w_gu,
                             static_cast<long>(n) * p1.Nw, p1, st);
@@ -676,7 +700,7 @@ moe_status_t do_experts(const moe_config_t& c, const void* x_perm, const int32_t
   p2.ss_parts = sumsq_parts(c);
   Orient o2;
   int bn2;
-  pick_expert_orient(c, E, false, &o2, &bn2);
+  pick_expert_orient(c, E, false, true, &o2, &bn2);
   if (bn2 == 0) return MOE_ERR_UNSUPPORTED;
   return run_gemm(EPI_STORE, o2, bn2, act, TK, w_down, static_cast<long>(n) * E, p2, st);
 }

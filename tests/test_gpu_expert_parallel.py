@@ -118,12 +118,23 @@ def make_ranks(cfg, dev, world, logit_bias=None):
     return ranks, us
 
 
+def _tiling(mean_rows: float, E: int, H: int) -> tuple:
+    """The expert tilings the library picks from the mean rows per expert: the swapped 1-SM tiles
+    up to 48 rows; above that the down GEMM on the swapped CTA-pair tiles up to 256 rows (when its
+    output width is a multiple of 256 and its reduction at most 1024 deep), the 128-row activation
+    tiles otherwise."""
+    if mean_rows <= 48.0:
+        return ("swap", "swap")
+    return ("normal", "pair" if (E % 256 == 0 and H <= 1024 and mean_rows <= 256.0) else "normal")
+
+
 def owner_orients(cfg, idx, world):
-    """Whether each owner's expert GEMMs take the same orientation as the whole-batch ones: both
-    pick it from the mean rows per expert (at most 48 rows: the swapped orientation)."""
+    """Whether each owner's expert GEMMs take the same tilings as the whole-batch ones (both pick
+    them from the mean rows per expert)."""
     counts = np.bincount(idx.reshape(-1), minlength=cfg.n_experts)
-    whole = counts.sum() / cfg.n_experts <= 48.0
-    return [bool((counts[lo:hi].sum() / (hi - lo) <= 48.0) == whole)
+    E, H = cfg.d_latent or cfg.d_model, cfg.d_ff
+    whole = _tiling(counts.sum() / cfg.n_experts, E, H)
+    return [_tiling(counts[lo:hi].sum() / (hi - lo), E, H) == whole
             for lo, hi in ep.expert_ranges(cfg.n_experts, world)]
 
 

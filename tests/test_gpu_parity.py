@@ -76,6 +76,8 @@ SMALL = [
     # Shazeer structure in bf16 (ReLU experts, no latent, no norm)
     configs.small_shazeer(T=257, d=128, h=256, n=16, k=4, seed=18),
     configs.small_shazeer(T=33, d=256, h=512, n=64, k=2, seed=19),
+    # 49-256 rows per expert with a 256-wide expert output: the down GEMM on the CTA-pair tiles
+    configs.small_shazeer(T=600, d=256, h=512, n=16, k=4, seed=31),
     # fp32 CUDA-core path
     configs.TINY_SHAZEER_F32.replace(T=45, seed=20),
     configs.TINY_SHAZEER_F32.replace(T=64, top_k=8, seed=21),
@@ -108,6 +110,14 @@ def test_layer_small_swap_pair_expert_tiles(cfg, monkeypatch):
     """The same layers with the prefill expert GEMMs on the swapped CTA-pair tiles
     (MOE_EXPERT_TILES=swap_pair) instead of the 1-SM 128-row activation tiles."""
     monkeypatch.setenv("MOE_EXPERT_TILES", "swap_pair")
+    _check_layer(cfg)
+
+
+@pytest.mark.parametrize("cfg", PREFILL_GROUP_CASES, ids=lambda c: c.name)
+def test_layer_small_normal_expert_tiles(cfg, monkeypatch):
+    """The same layers with both expert GEMMs on the 1-SM 128-row activation tiles
+    (MOE_EXPERT_TILES=normal), whatever the rows per expert."""
+    monkeypatch.setenv("MOE_EXPERT_TILES", "normal")
     _check_layer(cfg)
 
 
@@ -200,6 +210,33 @@ def test_permute_empty_and_bad_index():
     assert moe.moe_get_device_status() == 0  # cleared by the read
     assert off.cpu().numpy().tolist() == [0, 2, 3, 4, 5]
     assert inv.cpu().numpy()[3] == -1
+
+
+@pytest.mark.parametrize("T,k,n", [(500, 8, 16), (3000, 4, 256)])
+def test_permute_chunked_bad_index(T, k, n):
+    """The chunked permutation (more than 2048 slots: counts, scan and rank over several chunks)
+    with an expert index out of range: the error is latched, that slot is dropped, and the other
+    slots keep the canonical order (offsets from the valid counts; rows by expert, then token)."""
+    idx_h = _rand_routing(T, n, k, seed=T + n)
+    idx_h[T // 2, 1] = n + 3
+    cfg = configs.small_muse(T=T, n=n, k=k)
+    c = abi_config(cfg)
+    off = torch.zeros(n + 1, dtype=torch.int32, device="cuda")
+    perm = torch.full((T * k,), -9, dtype=torch.int32, device="cuda")
+    inv = torch.zeros(T * k, dtype=torch.int32, device="cuda")
+    ws = torch.empty(moe.workspace_size(c), dtype=torch.uint8, device="cuda")
+    moe.moe_permute(c, torch.from_numpy(idx_h).cuda(), off, perm, inv, workspace=ws)
+    assert moe.moe_get_device_status() == moe.STATUS_CODES["MOE_ERR_DEVICE_CHECK"]
+    flat = idx_h.reshape(-1)
+    valid = flat < n
+    counts = np.bincount(flat[valid], minlength=n)
+    np.testing.assert_array_equal(off.cpu().numpy(), np.concatenate([[0], np.cumsum(counts)]))
+    slots = np.nonzero(valid)[0]
+    order = slots[np.lexsort((slots // k, flat[slots]))]  # expert ascending, then token
+    want_inv = np.full(T * k, -1)
+    want_inv[order] = np.arange(len(order))
+    np.testing.assert_array_equal(inv.cpu().numpy(), want_inv)
+    np.testing.assert_array_equal(perm.cpu().numpy()[:len(order)], order // k)
 
 
 @pytest.mark.parametrize("E,gamma", [(256, True), (4096, True), (512, False), (8192, True)])
