@@ -236,9 +236,9 @@ def measured_peaks() -> dict:
 # launch scales by the same units: prefill by routed rows and experts (both 8x), decode by routed
 # experts.  Valid only for the kernel source the capture was taken on (fingerprint below).
 TRAFFIC_CAPTURES = {
-    "kernel_sha256_16": "e441b6b39278f22f",
-    "muse_prefill": {"bytes": 2.327961e9 + 0.130886912e9, "experts": 32, "rows": 2048 * 8},
-    "muse_decode": {"bytes": 1.947475e9 + 0.004323584e9, "experts": 29, "rows": 8 * 8},
+    "kernel_sha256_16": "9f4daa006e90ef61",
+    "muse_prefill": {"bytes": 2.306629e9 + 0.131756544e9, "experts": 32, "rows": 2048 * 8},
+    "muse_decode": {"bytes": 1.947402e9 + 0.005626368e9, "experts": 29, "rows": 8 * 8},
 }
 
 

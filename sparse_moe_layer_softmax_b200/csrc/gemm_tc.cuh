@@ -72,6 +72,7 @@ struct GemmParams {
                              // read by the tiles running at the same time, then not again), and
                              // the staged output stores are kept in L2 ahead of other lines (the
                              // next GEMM reads them); for layers whose activations fit in L2
+  int tail_m64;              // 1: normal-orientation tiles of at most 64 rows run M = 64 MMAs
 };
 
 // Shared memory that stages the bf16 output of the normal-orientation epilogues: one 4 KB
@@ -96,6 +97,7 @@ struct GemmShape {
   static constexpr int kXBoxRows = kSwap ? BN : 128;
   static constexpr int kWBoxRows = kSwap ? 128 : (kDual ? BN / 2 : BN);
   static constexpr uint32_t kIdesc = idesc_bf16_f32(128, BN);
+  static constexpr uint32_t kIdesc64 = idesc_bf16_f32(64, BN);  // a group's last chunk of <= 64 rows
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "tcgen05 M=128 needs N % 16 == 0");
   static_assert(2 * kAccCols <= 512, "two accumulators must fit in TMEM");
 };
@@ -238,14 +240,16 @@ __device__ __forceinline__ void router_key(const GemmParams& p, float acc, int c
   }
 }
 
-// Epilogue of the normal orientation: this thread owns row row0 + 32*q + lane of the tile (valid
-// if below nrows) and the tile's BN accumulator columns (output features f0 ...).
+// Epilogue of the normal orientation: this thread owns row row0 + rpw*q + lane of the tile (valid
+// if lane < rpw and below nrows) and the tile's BN accumulator columns (output features f0 ...).
+// An M = 128 tile holds row r in TMEM lane r (rpw = 32); an M = 64 tile holds rows 16q .. 16q+15
+// in lanes 32q .. 32q+15 (rpw = 16).
 template <int BN, int kEpi>
 __device__ __forceinline__ void epilogue_rows(const GemmParams& p, int row0, int nrows, int f0,
                                               uint32_t tbase, int q, int lane, float* s_coef,
-                                              const EpiOut& eo) {
-    const int rl = q * 32 + lane;
-    const bool valid = rl < nrows;
+                                              const EpiOut& eo, int rpw = 32) {
+    const int rl = q * rpw + lane;
+    const bool valid = lane < rpw && rl < nrows;
     const size_t row = static_cast<size_t>(row0 + rl);
     const int yblk = row0 + q * 32;  // first row of this warp's row block
     if constexpr (kEpi == EPI_ROUTER) {
@@ -577,6 +581,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     bool ok = true;
     for (int t = blockIdx.x; t < total_all && ok; t += gridDim.x) {
       const int kb0 = (t / total) * KBs;
+      uint32_t idesc = S::kIdesc;
+      if (!kSwap && p.tail_m64) {
+        const TileCoord c = decode_tile(t - (t / total) * total, s_seg, s_pref, G, FT, S::kCH,
+                                        p.tile_order);
+        if (c.nrows <= 64) idesc = S::kIdesc64;
+      }
       if (!mbar_wait(&tempty[acc], acc_phase ^ 1)) break;
       tc_fence_after();
       const uint32_t d = tmem_base + acc * S::kAccCols;
@@ -589,7 +599,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         for (int k = 0; k < S::kBK / 16; ++k) {
           const uint32_t accum = (kb > kb0 || k > 0) ? 1u : 0u;
           const uint64_t bdesc = smem_desc_k128(b_addr + 32 * k);
-          tc_mma_bf16(d, smem_desc_k128(a_addr + 32 * k), bdesc, S::kIdesc, accum);
+          tc_mma_bf16(d, smem_desc_k128(a_addr + 32 * k), bdesc, idesc, accum);
           if (kSwap && S::kDual)
             tc_mma_bf16(d + BN, smem_desc_k128(a_addr + 128 * 128 + 32 * k), bdesc, S::kIdesc,
                         accum);
@@ -616,9 +626,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * S::kAccCols;
       const int f0 = c.ft * S::kFO;
       if constexpr (!kSwap) {
+        const int rpw = (p.tail_m64 && c.nrows <= 64) ? 16 : 32;  // rows per warp (M = 64 / 128)
         const EpiOut eo{(kStageOut && p.out_tma) ? &tmO : nullptr, stage_out + q * 4096,
-                        c.nrows >= q * 32 + 32, p.l2_hints != 0};
-        epilogue_rows<BN, kEpi>(p, c.row0, c.nrows, f0, tbase, q, lane, s_coef, eo);
+                        rpw == 32 && c.nrows >= q * 32 + 32, p.l2_hints != 0};
+        epilogue_rows<BN, kEpi>(p, c.row0, c.nrows, f0, tbase, q, lane, s_coef, eo, rpw);
       } else {
         // swap orientation: this thread owns output feature f for the BN rows of the chunk
         const int f = f0 + q * 32 + lane;

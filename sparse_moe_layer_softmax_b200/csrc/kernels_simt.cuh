@@ -908,6 +908,15 @@ __global__ void __launch_bounds__(kRouterThreads, 1) router_logits_small_kernel(
 // distinct even when fewer than k keys are finite (a logit bias of -inf masks an expert: such
 // experts are taken last, lower index first, with weight 0).  A NaN key ranks as -inf and latches
 // MOE_ERR_DEVICE_CHECK, as does a row whose best key is not finite (its weights are undefined).
+// Each round takes the warp's largest key with one integer max-reduction over the lanes' best
+// keys (fp32 keys mapped onto uint32 in the same order, -0 read as +0) and the lowest expert
+// index holding it with one min-reduction: the order (key descending, index ascending) of the
+// float comparison, in two warp-wide instructions instead of a five-level shuffle tree.
+__device__ __forceinline__ uint32_t ordered_key(float f) {
+  const uint32_t u = __float_as_uint(f + 0.0f);  // -0 + 0 = +0 under round-to-nearest
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
 __global__ void topk_rows_kernel(float* __restrict__ logits, int T, int n, int k,
                                  float routed_scale, int gate_mode,
                                  const float* __restrict__ sel_bias,
@@ -918,61 +927,58 @@ __global__ void topk_rows_kernel(float* __restrict__ logits, int T, int n, int k
   const int t = blockIdx.x * warps + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (t >= T) return;
-  float key[kMaxExperts / 32], pay[kMaxExperts / 32];
+  uint32_t key[kMaxExperts / 32];  // ordered keys; 0 marks no candidate (below every key)
+  float pay[kMaxExperts / 32];
   bool bad = false;
 #pragma unroll
   for (int i = 0; i < kMaxExperts / 32; ++i) {
     const int e = lane + 32 * i;
-    key[i] = -INFINITY;
+    key[i] = 0u;
     pay[i] = 0.0f;
     if (e < n) {
       const float l = logits[static_cast<size_t>(t) * n + e];
+      float kf;
       if (gate_mode == MOE_GATE_SIGMOID) {
-        const float s = 1.0f / (1.0f + expf(-l));
-        logits[static_cast<size_t>(t) * n + e] = s;
-        key[i] = s + (sel_bias ? sel_bias[e] : 0.0f);
-        pay[i] = s;
+        const float sg = 1.0f / (1.0f + expf(-l));
+        logits[static_cast<size_t>(t) * n + e] = sg;
+        kf = sg + (sel_bias ? sel_bias[e] : 0.0f);
+        pay[i] = sg;
       } else {
-        key[i] = l;
+        kf = l;
         pay[i] = l;
       }
-      if (key[i] != key[i]) {  // NaN
+      if (kf != kf) {  // NaN
         bad = true;
-        key[i] = -INFINITY;
+        kf = -INFINITY;
         pay[i] = gate_mode == MOE_GATE_SIGMOID ? 0.0f : -INFINITY;
       }
+      key[i] = ordered_key(kf);
     }
   }
   // Loops over the k kept entries run to the compile-time bound kMaxTopK with k as a guard, so
   // the arrays stay in registers.
   float top_s[kMaxTopK];
   int top_i[kMaxTopK];
-  unsigned taken = 0u;  // bit i: expert lane + 32 i is already selected
 #pragma unroll
   for (int j = 0; j < kMaxTopK; ++j) {
     top_s[j] = 0.0f;
     top_i[j] = 0;
     if (j >= k) continue;  // warp-uniform
-    float bv = -INFINITY, bs = 0.0f;
+    // this lane's best remaining candidate (the lowest index among equal keys)
+    uint32_t bk = 0u;
     int bi = 0x7fffffff;
-#pragma unroll
-    for (int i = 0; i < kMaxExperts / 32; ++i) {
-      const int e = lane + 32 * i;
-      const bool cand = e < n && !((taken >> i) & 1u);
-      if (cand && (key[i] > bv || (key[i] == bv && e < bi))) { bv = key[i]; bi = e; bs = pay[i]; }
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-      const float os = __shfl_xor_sync(0xffffffffu, bs, o);
-      if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; bs = os; }
-    }
-    top_s[j] = bs;
-    top_i[j] = bi;  // k <= n: some candidate is always left
+    float bp = 0.0f;
 #pragma unroll
     for (int i = 0; i < kMaxExperts / 32; ++i)
-      if (lane + 32 * i == bi) taken |= 1u << i;
+      if (key[i] > bk) { bk = key[i]; bi = lane + 32 * i; bp = pay[i]; }
+    const uint32_t m = __reduce_max_sync(0xffffffffu, bk);
+    const uint32_t win = __reduce_min_sync(0xffffffffu, bk == m ? static_cast<uint32_t>(bi)
+                                                                 : 0xffffffffu);
+    top_i[j] = static_cast<int>(win);  // k <= n: some candidate is always left
+    top_s[j] = __shfl_sync(0xffffffffu, bp, static_cast<int>(win & 31u));
+#pragma unroll
+    for (int i = 0; i < kMaxExperts / 32; ++i)
+      if (static_cast<uint32_t>(lane + 32 * i) == win) key[i] = 0u;  // taken
   }
   bad = __any_sync(0xffffffffu, bad);
   if (lane == 0 && (bad || !(fabsf(top_s[0]) <= 3.0e38f))) latch_status(MOE_ERR_DEVICE_CHECK);

@@ -478,8 +478,12 @@ def test_combine_bulk_matches_per_token(E, k, norm):
         assert row_rel_err(got[t], ref) <= 1e-2
 
 
-def test_latent_down_and_up():
-    cfg = configs.small_muse(T=150, d=512, L=256, I=128, n=8, k=2, seed=41)
+@pytest.mark.parametrize("T", [150, 64, 17, 1])
+def test_latent_down_and_up(T):
+    """The standalone latent projections against the oracle: over 64 rows one GEMM; up to 64 rows
+    the reduction split over clusters of 8 (down) and 4 (up) CTAs that add their partial tiles in
+    distributed shared memory."""
+    cfg = configs.small_muse(T=T, d=512, L=256, I=128, n=8, k=2, seed=41)
     c = abi_config(cfg)
     dev = moe_inputs.device_inputs(cfg)
     inp = moe_inputs.host_inputs(cfg)
@@ -600,6 +604,42 @@ def test_route_with_masked_experts(T):
         assert (ih[:, -1] == first_masked).all()
         assert (wh[:, -1] == 0.0).all()
         np.testing.assert_allclose(wh, wsel, rtol=2e-6, atol=1e-7)
+
+
+@pytest.mark.parametrize("T", [40, 300])
+def test_route_exact_ties_take_lower_index(T):
+    """Router weight rows copied between experts give bit-equal logits for every token: the
+    selection must take the lower expert index first wherever such a pair meets at or inside the
+    top k, as the oracle's order on the same logits does, on the few-token router, the
+    warp-per-token top-k after the GEMM router and the GEMM epilogue's own selection."""
+    import torch
+    cfg = configs.small_muse(T=T, d=256, L=128, I=128, n=64, k=8, seed=77)
+    dev = moe_inputs.device_inputs(cfg)
+    c = abi_config(cfg)
+    n, k = cfg.n_experts, cfg.top_k
+    w = dev["w_router"].clone()
+    pairs = [(3, 17), (40, 5), (22, 63), (9, 10), (31, 0), (50, 51), (12, 48), (60, 33)]
+    for a, b in pairs:
+        w[b] = w[a]
+    logits = torch.empty((T, n), dtype=torch.float32, device="cuda")
+    outs = []
+    for lg in (logits, None):
+        idx = torch.empty((T, k), dtype=torch.int32, device="cuda")
+        wt = torch.empty((T, k), dtype=torch.float32, device="cuda")
+        moe.moe_route(c, dev["u"], w, None, lg, idx, wt)
+        outs.append((idx, wt))
+    torch.cuda.synchronize()
+    assert moe.moe_get_device_status() == 0
+    lgh = logits.cpu().numpy()
+    for a, b in pairs:
+        np.testing.assert_array_equal(lgh[:, a].view(np.int32), lgh[:, b].view(np.int32))
+    sel, wsel = oracle.softmax_topk(lgh, k)
+    # the copies meet inside the top k, or at its boundary, on many tokens
+    hit = sum(int(np.isin([a, b], sel[t]).all()) for t in range(T) for a, b in pairs)
+    assert hit >= T // 8
+    for idx, wt in outs:
+        np.testing.assert_array_equal(idx.cpu().numpy(), sel)
+        np.testing.assert_allclose(wt.cpu().numpy(), wsel, rtol=2e-6, atol=1e-7)
 
 
 STAGED_CASES = [
