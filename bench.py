@@ -236,9 +236,9 @@ def measured_peaks() -> dict:
 # launch scales by the same units: prefill by routed rows and experts (both 8x), decode by routed
 # experts.  Valid only for the kernel source the capture was taken on (fingerprint below).
 TRAFFIC_CAPTURES = {
-    "kernel_sha256_16": "9f4daa006e90ef61",
-    "muse_prefill": {"bytes": 2.306629e9 + 0.131756544e9, "experts": 32, "rows": 2048 * 8},
-    "muse_decode": {"bytes": 1.947402e9 + 0.005626368e9, "experts": 29, "rows": 8 * 8},
+    "kernel_sha256_16": "5bf7eea9458d308a",
+    "muse_prefill": {"bytes": 2.355861e9 + 0.130924544e9, "experts": 32, "rows": 2048 * 8},
+    "muse_decode": {"bytes": 1.947568e9 + 0.00495232e9, "experts": 29, "rows": 8 * 8},
 }
 
 

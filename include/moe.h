@@ -220,14 +220,17 @@ MOE_API moe_status_t moe_combine(const moe_config_t* cfg, const void* out_perm,
                                  const float* row_sumsq, const int32_t* inv_perm,
                                  const float* topk_w, void* y, void* stream);
 
-/* Latent down-projection [MUSE "Latent experts"]: z_raw = dtype(u P_down^T), [T, d_latent]. */
+/* Latent down-projection [MUSE "Latent experts"]: z_raw = dtype(u P_down^T), [T, d_latent].
+ * Up to 64 rows the reduction is split over the CTAs of a thread-block cluster, which add their
+ * fp32 partial sums in a fixed order (deterministic; the same bits as moe_layer_forward). */
 MOE_API moe_status_t moe_latent_down(const moe_config_t* cfg, const void* u, const void* p_down,
                              void* z_raw, void* stream);
 
 /* Latent up-projection and residual update [MUSE "Residual gates"; ARCHDB residual field]:
  *   b = dtype(y P_up^T); out = dtype(alpha*r + beta*b) with beta = sigmoid(g/tau),
  *   alpha = sqrt(max(sigmoid(-g/tau)*(1+beta), resid_floor)) per channel (MUSE_GATE), or
- *   dtype(r + g*b) (LITERAL), or b (NONE).  y: [T, d_latent]; r, out: [T, d_model]. */
+ *   dtype(r + g*b) (LITERAL), or b (NONE).  y: [T, d_latent]; r, out: [T, d_model].  Up to 64
+ * rows the reduction is split as in moe_latent_down. */
 MOE_API moe_status_t moe_latent_up(const moe_config_t* cfg, const void* y, const void* p_up,
                            const void* r, const float* resid_g, void* out, void* stream);
 
@@ -269,9 +272,9 @@ MOE_API moe_status_t moe_noisy_gate(const moe_config_t* cfg, const void* u, cons
  * equal u; ignored when resid_mode is NONE and input_norm is off), out: [T, d_model].
  * logits_out [T, n], topk_idx_out [T, k] and topk_w_out [T, k] are optional copies of the
  * routing.  The workspace holds every intermediate.  With T <= 64 (bf16, latent) the two latent
- * projections split their reduction over k ranges and add the fp32 partials in a fixed order,
- * so their results are deterministic but may differ in the last bit from moe_latent_down /
- * moe_latent_up, which do not split. */
+ * projections split their reduction over k ranges and add the fp32 partials in a fixed order (the
+ * same bits as moe_latent_down / moe_latent_up, which split the same way), so their results are
+ * deterministic but may differ in the last bit from a forward of more than 64 tokens. */
 MOE_API moe_status_t moe_layer_forward(const moe_config_t* cfg, const moe_weights_t* w, const void* u,
                                const void* r, void* out, float* logits_out,
                                int32_t* topk_idx_out, float* topk_w_out, void* workspace,
