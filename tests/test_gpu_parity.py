@@ -127,6 +127,33 @@ def test_layer_small(cfg):
     _check_layer(cfg)
 
 
+# batch sizes at the layer's switch points: one token; the split latent projections (T <= 64);
+# the few-token router (T <= 256); the one-launch dispatch (T * k <= 2048 slots)
+EDGE_CASES = [configs.small_muse(T=T, d=512, L=256, I=256, n=16, k=4, seed=200 + T)
+              for T in (1, 2, 63, 64, 65)] + \
+             [configs.small_muse(T=T, d=256, L=128, I=128, n=64, k=8, seed=300 + T)
+              for T in (255, 256, 257)]
+
+
+@pytest.mark.parametrize("cfg", EDGE_CASES, ids=lambda c: f"T{c.T}-n{c.n_experts}k{c.top_k}")
+def test_layer_at_switch_points(cfg):
+    _check_layer(cfg)
+
+
+def test_layer_empty_batch():
+    """T = 0: the forward launches nothing that touches the (empty) buffers and reports success."""
+    import torch
+    cfg = configs.small_muse(T=0, d=256, L=128, I=128, n=16, k=4, seed=399)
+    c = abi_config(cfg)
+    dev = moe_inputs.device_inputs(cfg.replace(T=1))
+    layer = moe.MoELayer(c, dev)
+    u = torch.empty((0, cfg.d_model), dtype=torch.bfloat16, device="cuda")
+    out = torch.empty_like(u)
+    layer.forward(u, u, out=out)
+    torch.cuda.synchronize()
+    assert moe.moe_get_device_status() == 0
+
+
 @pytest.mark.parametrize("cfg", PAIR_CASES, ids=lambda c: c.name)
 def test_layer_small_pair_tiles(cfg, monkeypatch):
     """The same layers with the CTA-pair 256-row GEMM tiles selected (MOE_GEMM_PAIR=1)."""
