@@ -579,9 +579,12 @@ moe_status_t do_route(const moe_config_t& c, const void* u, const void* w_router
   }
   // With a logits buffer (the caller's, or the layer's workspace) the GEMM only stores the
   // pre-activation logits and a warp per token selects the top-k; without one, the GEMM's
-  // epilogue selects from the accumulators itself (k passes over each row).  (Selecting in the
-  // epilogue was also measured with a buffer present: slower, 0.089 against 0.033 ms for the
-  // Shazeer batch.)
+  // epilogue selects from the accumulators itself (k passes over each row).  Selecting in the
+  // epilogue with a buffer present was measured slower, with these k passes (0.089 against 0.033
+  // ms of route for the Shazeer batch) and with a single pass keeping the best k in registers
+  // (0.124 against 0.040 ms; 0.27 against 0.16 ms at prefill: the insertion into the k-list runs
+  // predicated for every column in each thread), while the warp-per-token kernel spreads the
+  // selection over every SM.
   const bool split = lbuf != nullptr;
   GemmParams p{};
   p.G = 1;
