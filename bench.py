@@ -236,9 +236,9 @@ def measured_peaks() -> dict:
 # launch scales by the same units: prefill by routed rows and experts (both 8x), decode by routed
 # experts.  Valid only for the kernel source the capture was taken on (fingerprint below).
 TRAFFIC_CAPTURES = {
-    "kernel_sha256_16": "5bf7eea9458d308a",
-    "muse_prefill": {"bytes": 2.355861e9 + 0.130924544e9, "experts": 32, "rows": 2048 * 8},
-    "muse_decode": {"bytes": 1.947568e9 + 0.00495232e9, "experts": 29, "rows": 8 * 8},
+    "kernel_sha256_16": "e59c35af08759c4a",
+    "muse_prefill": {"bytes": 2.322391e9 + 0.130761216e9, "experts": 32, "rows": 2048 * 8},
+    "muse_decode": {"bytes": 1.947448e9 + 0.004316416e9, "experts": 29, "rows": 8 * 8},
 }
 
 

@@ -45,6 +45,86 @@ __device__ __forceinline__ float4 ld_cluster_f32x4(uint32_t caddr) {
   return v;
 }
 
+// Reduce + epilogue of one CTA of a cluster of NS: CTA `rank` finishes features
+// [rank * 128/NS, (rank + 1) * 128/NS) of feature tile `ft` for every row, in vectors of 8
+// features.  Thread (group g, row lane r) of the 128 epilogue threads takes features g*8 .. g*8+7
+// of that part and rows r, r + nr, ... (8/NS rows); all of its loads (the NS partial tiles through
+// distributed shared memory, the residual rows) are issued before the first sum, and the partials
+// are added in the order s = 0, 1, ..., NS-1.
+template <int kEpi, int NS>
+__device__ __forceinline__ void splitk_reduce(const GemmParams& p, const float* part, uint32_t rank,
+                                              int ft) {
+  constexpr int kFs = 128 / NS, kGroups = kFs / 8, kNr = 128 / kGroups, kRows = kSplitBN / kNr;
+  static_assert(kRows * kNr == kSplitBN && kGroups * 8 == kFs, "reduce layout");
+  const int et = static_cast<int>(threadIdx.x) - 64;
+  const int g = et % kGroups, r0 = et / kGroups;
+  const int fl = static_cast<int>(rank) * kFs + g * 8;  // first feature within the tile
+  const int col = ft * 128 + fl;
+  float4 cur[NS][kRows][2];
+#pragma unroll
+  for (int s = 0; s < NS; ++s) {
+    const uint32_t base = cluster_addr(part, static_cast<uint32_t>(s));
+#pragma unroll
+    for (int q = 0; q < kRows; ++q) {
+      const int row = r0 + q * kNr;
+      if (row < p.M) {
+        const uint32_t off = base + static_cast<uint32_t>((row * 128 + fl) * 4);
+        cur[s][q][0] = ld_cluster_f32x4(off);
+        cur[s][q][1] = ld_cluster_f32x4(off + 16);
+      }
+    }
+  }
+  const bool has_r = kEpi == EPI_RESGATE && p.resid_mode != MOE_RESID_NONE;
+  uint4 rv[kRows];
+#pragma unroll
+  for (int q = 0; q < kRows; ++q) {
+    const int row = r0 + q * kNr;
+    rv[q] = make_uint4(0, 0, 0, 0);
+    if (row < p.M && has_r)
+      rv[q] = __ldg(reinterpret_cast<const uint4*>(p.resid + static_cast<size_t>(row) * p.Nout + col));
+  }
+  float a[8], b[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    a[j] = 0.0f;
+    b[j] = 1.0f;
+    if constexpr (kEpi == EPI_RESGATE) {
+      const float gg = p.gparam ? p.gparam[col + j] : 0.0f;
+      if (p.resid_mode == MOE_RESID_MUSE_GATE) {
+        b[j] = sigmoidf_(gg / p.tau);
+        a[j] = sqrtf(fmaxf(sigmoidf_(-gg / p.tau) * (1.0f + b[j]), p.floor_));
+      } else if (p.resid_mode == MOE_RESID_LITERAL) {
+        a[j] = 1.0f;
+        b[j] = gg;
+      }
+    }
+  }
+  uint16_t* out = static_cast<uint16_t*>(p.out);
+#pragma unroll
+  for (int q = 0; q < kRows; ++q) {
+    const int row = r0 + q * kNr;
+    if (row >= p.M) continue;
+    float v[8] = {cur[0][q][0].x, cur[0][q][0].y, cur[0][q][0].z, cur[0][q][0].w,
+                  cur[0][q][1].x, cur[0][q][1].y, cur[0][q][1].z, cur[0][q][1].w};
+#pragma unroll
+    for (int s = 1; s < NS; ++s) {
+      v[0] += cur[s][q][0].x; v[1] += cur[s][q][0].y; v[2] += cur[s][q][0].z; v[3] += cur[s][q][0].w;
+      v[4] += cur[s][q][1].x; v[5] += cur[s][q][1].y; v[6] += cur[s][q][1].z; v[7] += cur[s][q][1].w;
+    }
+    const uint16_t* rh = reinterpret_cast<const uint16_t*>(&rv[q]);
+    uint4 o;
+    uint16_t* oh = reinterpret_cast<uint16_t*>(&o);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      float x = v[j];
+      if constexpr (kEpi == EPI_RESGATE)
+        x = __fmaf_rn(a[j], bf16_to_f32(rh[j]), __fmul_rn(b[j], round_bf16(x)));
+      oh[j] = f32_to_bf16(x);
+    }
+    *reinterpret_cast<uint4*>(out + static_cast<size_t>(row) * p.Nout + col) = o;
+  }
+}
+
 // kEpi: EPI_STORE (out = dtype(sum)) or EPI_RESGATE (out = dtype(alpha r + beta dtype(sum))).
 // Grid: (Nout / 128) * S CTAs in clusters of S (2 <= S <= 8, S divides K / 64); rows p.M <= kSplitBN.
 template <int kEpi>
@@ -146,88 +226,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
   if (warp >= 2) {
     // ------------------------------------------------------------ reduce + epilogue
-    // CTA `rank` finishes features [rank * fs, (rank + 1) * fs) of the tile for every row, in
-    // vectors of 8 features: thread (group g, row lane r) takes features g*8 .. g*8+7 of its part
-    // and rows r, r + nr, ...; every load of a thread is issued before the first sum.
-    const int fs = 128 / ns;
-    const int groups = fs / 8;
-    const int nr = 128 / groups;
-    const int et = static_cast<int>(threadIdx.x) - 64;
-    const int g = et % groups, r0 = et / groups;
-    const int fl = static_cast<int>(rank) * fs + g * 8;  // first feature within the tile
-    const int col = ft * 128 + fl;
-    float a[8], b[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      a[j] = 0.0f;
-      b[j] = 1.0f;
-      if constexpr (kEpi == EPI_RESGATE) {
-        const float gg = p.gparam ? p.gparam[col + j] : 0.0f;
-        if (p.resid_mode == MOE_RESID_MUSE_GATE) {
-          b[j] = sigmoidf_(gg / p.tau);
-          a[j] = sqrtf(fmaxf(sigmoidf_(-gg / p.tau) * (1.0f + b[j]), p.floor_));
-        } else if (p.resid_mode == MOE_RESID_LITERAL) {
-          a[j] = 1.0f;
-          b[j] = gg;
-        }
-      }
-    }
-    // rows per thread: kSplitBN / nr = 8 / ns, at most 4 (clusters of at least 2)
-    constexpr int kMaxRowsPerThread = 4;
-    uint4 rv[kMaxRowsPerThread];
-    float4 pv[kMaxRowsPerThread][2];
-    const bool has_r = kEpi == EPI_RESGATE && p.resid_mode != MOE_RESID_NONE;
-#pragma unroll
-    for (int q = 0; q < kMaxRowsPerThread; ++q) {
-      const int row = r0 + q * nr;
-      rv[q] = make_uint4(0, 0, 0, 0);
-      if (row < p.M && has_r)
-        rv[q] = __ldg(reinterpret_cast<const uint4*>(p.resid + static_cast<size_t>(row) * p.Nout +
-                                                     col));
-    }
-    // partial sums in the order s = 0, 1, ..., S-1
-    for (int s = 0; s < ns; ++s) {
-      const uint32_t base = cluster_addr(part, static_cast<uint32_t>(s));
-      float4 cur[kMaxRowsPerThread][2];
-#pragma unroll
-      for (int q = 0; q < kMaxRowsPerThread; ++q) {
-        const int row = r0 + q * nr;
-        if (row < p.M) {
-          const uint32_t off = base + static_cast<uint32_t>((row * 128 + fl) * 4);
-          cur[q][0] = ld_cluster_f32x4(off);
-          cur[q][1] = ld_cluster_f32x4(off + 16);
-        }
-      }
-#pragma unroll
-      for (int q = 0; q < kMaxRowsPerThread; ++q) {
-        if (s == 0) {
-          pv[q][0] = cur[q][0];
-          pv[q][1] = cur[q][1];
-        } else {
-          pv[q][0].x += cur[q][0].x; pv[q][0].y += cur[q][0].y;
-          pv[q][0].z += cur[q][0].z; pv[q][0].w += cur[q][0].w;
-          pv[q][1].x += cur[q][1].x; pv[q][1].y += cur[q][1].y;
-          pv[q][1].z += cur[q][1].z; pv[q][1].w += cur[q][1].w;
-        }
-      }
-    }
-    uint16_t* out = static_cast<uint16_t*>(p.out);
-#pragma unroll
-    for (int q = 0; q < kMaxRowsPerThread; ++q) {
-      const int row = r0 + q * nr;
-      if (row >= p.M) continue;
-      float v[8] = {pv[q][0].x, pv[q][0].y, pv[q][0].z, pv[q][0].w,
-                    pv[q][1].x, pv[q][1].y, pv[q][1].z, pv[q][1].w};
-      const uint16_t* rh = reinterpret_cast<const uint16_t*>(&rv[q]);
-      uint4 o;
-      uint16_t* oh = reinterpret_cast<uint16_t*>(&o);
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        float x = v[j];
-        if constexpr (kEpi == EPI_RESGATE) x = __fmaf_rn(a[j], bf16_to_f32(rh[j]), __fmul_rn(b[j], round_bf16(x)));
-        oh[j] = f32_to_bf16(x);
-      }
-      *reinterpret_cast<uint4*>(out + static_cast<size_t>(row) * p.Nout + col) = o;
+    switch (ns) {
+      case 2: splitk_reduce<kEpi, 2>(p, part, rank, ft); break;
+      case 4: splitk_reduce<kEpi, 4>(p, part, rank, ft); break;
+      default: splitk_reduce<kEpi, 8>(p, part, rank, ft); break;
     }
   }
   __syncthreads();

@@ -27,8 +27,6 @@ enum EpiKind : int {
   EPI_SWIGLU = 2,   // dtype(SiLU(gate) * up), gate/up W rows paired (rows c and Nw/2 + c)
   EPI_RESGATE = 3,  // residual update of the latent up-projection
   EPI_ROUTER = 4,   // top-k selection and renormalised weights over the row's logits
-  EPI_PARTIAL = 5,  // swapped orientation, dense: the fp32 sums of one k-split,
-                    // partial[split][row][col], reduced and finished by a separate kernel
 };
 
 enum TileOrder : int { TILE_CHUNK_FASTEST = 0, TILE_FEATURE_FASTEST = 1 };
@@ -65,9 +63,6 @@ struct GemmParams {
   int ss_parts;              // the stored bf16 values, one per row and column block
   int out_tma;               // bf16 epilogues of the normal orientation: 1 = the output tensor
                              // map is valid and whole-warp row blocks leave by TMA stores
-  int k_splits;              // 1-SM kernel: the reduction split into this many equal k ranges,
-                             // each a tile of its own (0 or 1: no split; EPI_PARTIAL only)
-  float* partial;            // EPI_PARTIAL: [k_splits][M][Nout] fp32
   int l2_hints;              // 1: weight tiles are loaded as the first lines L2 evicts (each is
                              // read by the tiles running at the same time, then not again), and
                              // the staged output stores are kept in L2 ahead of other lines (the
@@ -519,11 +514,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const int total = s_pref[G];
-  // k-split tiles: tile t covers base tile t % total over k-blocks [ks * KBs, (ks + 1) * KBs)
-  // with ks = t / total (the host makes KB a multiple of the split count)
-  const int KS = p.k_splits > 1 ? p.k_splits : 1;
-  const int KBs = KB / KS;
-  const int total_all = total * KS;
 
   if (warp == 0 && lane == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -533,14 +523,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
     for (int s = 0; s < kStages; ++s) { issued[s] = false; last_parity[s] = 0; }
     bool ok = true;
-    for (int t = blockIdx.x; t < total_all && ok; t += gridDim.x) {
-      const int ks = t / total;
-      TileCoord c = decode_tile(t - ks * total, s_seg, s_pref, G, FT, S::kCH, p.tile_order);
+    for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+      TileCoord c = decode_tile(t, s_seg, s_pref, G, FT, S::kCH, p.tile_order);
       const int wrow = c.g * p.Nw + c.ft * S::kFO;
-      for (int kb = ks * KBs; kb < (ks + 1) * KBs; ++kb) {
+      for (int kb = 0; kb < KB; ++kb) {
         // weight-stream-bound layers (l2_hints): L2 fetches the weight k-block one ring ahead, so
         // more DRAM requests are in flight than the shared-memory ring holds
-        if (!kSwap && p.l2_hints && kb + kStages < (ks + 1) * KBs) {
+        if (!kSwap && p.l2_hints && kb + kStages < KB) {
           const int kp = (kb + kStages) * S::kBK;
           tma_prefetch_2d(&tmW, kp, wrow);
           if (S::kDual) tma_prefetch_2d(&tmW, kp, wrow + p.Nw / 2);
@@ -579,25 +568,23 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     // ------------------------------------------------------------ MMA issuer
     uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
     bool ok = true;
-    for (int t = blockIdx.x; t < total_all && ok; t += gridDim.x) {
-      const int kb0 = (t / total) * KBs;
+    for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
       uint32_t idesc = S::kIdesc;
       if (!kSwap && p.tail_m64) {
-        const TileCoord c = decode_tile(t - (t / total) * total, s_seg, s_pref, G, FT, S::kCH,
-                                        p.tile_order);
+        const TileCoord c = decode_tile(t, s_seg, s_pref, G, FT, S::kCH, p.tile_order);
         if (c.nrows <= 64) idesc = S::kIdesc64;
       }
       if (!mbar_wait(&tempty[acc], acc_phase ^ 1)) break;
       tc_fence_after();
       const uint32_t d = tmem_base + acc * S::kAccCols;
-      for (int kb = kb0; kb < kb0 + KBs; ++kb) {
+      for (int kb = 0; kb < KB; ++kb) {
         if (!mbar_wait(&full[stage], phase)) { ok = false; break; }
         tc_fence_after();
         const uint32_t a_addr = smem_u32(tiles + stage * S::kStageBytes);
         const uint32_t b_addr = a_addr + S::kABytes;
 #pragma unroll
         for (int k = 0; k < S::kBK / 16; ++k) {
-          const uint32_t accum = (kb > kb0 || k > 0) ? 1u : 0u;
+          const uint32_t accum = (kb > 0 || k > 0) ? 1u : 0u;
           const uint64_t bdesc = smem_desc_k128(b_addr + 32 * k);
           tc_mma_bf16(d, smem_desc_k128(a_addr + 32 * k), bdesc, idesc, accum);
           if (kSwap && S::kDual)
@@ -618,9 +605,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;  // TMEM lane quarter this warp may access
     uint32_t acc = 0, acc_phase = 0;
-    for (int t = blockIdx.x; t < total_all; t += gridDim.x) {
-      const int ks = t / total;
-      TileCoord c = decode_tile(t - ks * total, s_seg, s_pref, G, FT, S::kCH, p.tile_order);
+    for (int t = blockIdx.x; t < total; t += gridDim.x) {
+      TileCoord c = decode_tile(t, s_seg, s_pref, G, FT, S::kCH, p.tile_order);
       if (!epilogue_all(mbar_wait(&tfull[acc], acc_phase))) break;
       tc_fence_after();
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * S::kAccCols;
@@ -646,17 +632,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
         }
         uint16_t* out = static_cast<uint16_t*>(p.out);
-        if constexpr (kEpi == EPI_PARTIAL) {
-          // this k-split's fp32 sums; a warp writes 128 contiguous bytes per row
-          float* dst = p.partial + static_cast<size_t>(ks) * p.M * p.Nout + f;
-          for (int j0 = 0; j0 < BN; j0 += 16) {
-            float v[16];
-            tmem_ld16(tbase + j0, v);
-#pragma unroll
-            for (int i = 0; i < 16; ++i)
-              if (j0 + i < c.nrows) dst[static_cast<size_t>(c.row0 + j0 + i) * p.Nout] = v[i];
-          }
-        } else
         for (int j0 = 0; j0 < BN; j0 += 16) {
           float v[16];
           tmem_ld16(tbase + j0, v);

@@ -278,61 +278,6 @@ __global__ void dispatch_small_bf16_kernel(const int32_t* __restrict__ idx, int 
 
 // ------------------------------------------------------------------ k-split dense finish
 //
-// A dense projection over few rows whose reduction ran as k-split GEMM tiles (EPI_PARTIAL): the
-// fp32 partials partial[split][row][col] are added in split order, then finished as the GEMM
-// epilogue would: out = dtype(v), or with the residual gate out = dtype(alpha * r + beta * dtype(v))
-// (MUSE gate: beta = sigmoid(g/tau), alpha = sqrt(max(sigmoid(-g/tau)(1+beta), floor)); literal:
-// alpha = 1, beta = g; none: dtype(v)).  One thread per 8 consecutive outputs.
-__global__ void dense_split_finish_kernel(const float* __restrict__ partial, int splits, long rows,
-                                          int nout, int resgate, const uint16_t* __restrict__ resid,
-                                          const float* __restrict__ g, float tau, float floor_,
-                                          int resid_mode, uint16_t* __restrict__ out) {
-  pdl_wait();
-  pdl_launch_dependents();
-  const long nv = rows * nout / 8;
-  const size_t plane = static_cast<size_t>(rows) * nout;
-  for (long i = blockIdx.x * static_cast<long>(blockDim.x) + threadIdx.x; i < nv;
-       i += static_cast<long>(gridDim.x) * blockDim.x) {
-    const size_t e0 = static_cast<size_t>(i) * 8;
-    const int col = static_cast<int>(e0 % static_cast<size_t>(nout));
-    float v[8];
-    {
-      const float4 a = __ldg(reinterpret_cast<const float4*>(partial + e0));
-      const float4 b = __ldg(reinterpret_cast<const float4*>(partial + e0 + 4));
-      v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
-    }
-    for (int sp = 1; sp < splits; ++sp) {
-      const float4 a = __ldg(reinterpret_cast<const float4*>(partial + sp * plane + e0));
-      const float4 b = __ldg(reinterpret_cast<const float4*>(partial + sp * plane + e0 + 4));
-      v[0] += a.x; v[1] += a.y; v[2] += a.z; v[3] += a.w;
-      v[4] += b.x; v[5] += b.y; v[6] += b.z; v[7] += b.w;
-    }
-    if (resgate) {
-      const bool has_r = resid_mode != MOE_RESID_NONE;
-      uint4 rv = has_r ? __ldg(reinterpret_cast<const uint4*>(resid + e0)) : make_uint4(0, 0, 0, 0);
-      const uint16_t* rh = reinterpret_cast<const uint16_t*>(&rv);
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const float gg = g ? g[col + j] : 0.0f;
-        float a = 0.0f, b = 1.0f;
-        if (resid_mode == MOE_RESID_MUSE_GATE) {
-          b = sigmoidf_(gg / tau);
-          a = sqrtf(fmaxf(sigmoidf_(-gg / tau) * (1.0f + b), floor_));
-        } else if (resid_mode == MOE_RESID_LITERAL) {
-          a = 1.0f;
-          b = gg;
-        }
-        v[j] = a * bf16_to_f32(rh[j]) + b * round_bf16(v[j]);
-      }
-    }
-    uint4 o;
-    uint16_t* oh = reinterpret_cast<uint16_t*>(&o);
-#pragma unroll
-    for (int j = 0; j < 8; ++j) oh[j] = f32_to_bf16(v[j]);
-    reinterpret_cast<uint4*>(out + e0)[0] = o;
-  }
-}
-
 // ------------------------------------------------------------------ row gather
 //
 // dst[i] = src[rows[i * idx_stride]] in 16-byte vectors, one CTA per row (grid-strided); a

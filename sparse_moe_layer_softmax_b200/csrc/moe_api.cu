@@ -216,7 +216,7 @@ moe_status_t launch_gemm_swap_pair(const void* X, long x_rows, const void* W, lo
     attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   });
   if (attr_err != cudaSuccess) return MOE_ERR_CUDA;
-  if (p.x_k_period > 0 || p.k_splits > 1 || !p.seg) return MOE_ERR_UNSUPPORTED;
+  if (p.x_k_period > 0 || !p.seg) return MOE_ERR_UNSUPPORTED;
   CUtensorMap tx, tw;
   if (!make_tmap(&tx, X, static_cast<uint64_t>(x_rows), static_cast<uint64_t>(p.K), 128))
     return MOE_ERR_CUDA;
@@ -250,14 +250,13 @@ moe_status_t run_gemm(int epi, Orient o, int bn, const void* X, long x_rows, con
   const bool dual = epi == EPI_SWIGLU;
   if (o == Orient::kSwap) {
     const int ft = p.Nout / 128;
-    const long mt = tile_bound(x_rows, p.G, bn, ft) * std::max(1, p.k_splits);
+    const long mt = tile_bound(x_rows, p.G, bn, ft);
 #define SW(BN_, E_, ST_) \
   if (bn == BN_ && epi == E_) return launch_gemm<true, BN_, E_, ST_>(X, x_rows, W, w_rows, p, mt, st);
     SW(16, EPI_SWIGLU, 6) SW(32, EPI_SWIGLU, 6) SW(64, EPI_SWIGLU, 5)
     SW(16, EPI_STORE, 10) SW(32, EPI_STORE, 9) SW(64, EPI_STORE, 8)
     SW(16, EPI_RELU, 10) SW(32, EPI_RELU, 9) SW(64, EPI_RELU, 8)
     SW(16, EPI_RESGATE, 10) SW(32, EPI_RESGATE, 9) SW(64, EPI_RESGATE, 8)
-    SW(64, EPI_PARTIAL, 8)
 #undef SW
     return MOE_ERR_UNSUPPORTED;
   }
@@ -333,7 +332,7 @@ size_t dsize(const moe_config_t& c) { return c.dtype == MOE_BF16 ? 2 : 4; }
 int nchunks(const moe_config_t& c) { return cdiv(c.T, kPermChunk); }
 
 struct Workspace {
-  size_t idx, w, logits, z_raw, offsets, perm, inv, counts, x_perm, act, y, u_norm, b, ss, dp, total;
+  size_t idx, w, logits, z_raw, offsets, perm, inv, counts, x_perm, act, y, u_norm, b, ss, total;
 };
 
 int sumsq_parts(const moe_config_t& c);
@@ -358,10 +357,6 @@ Workspace layout(const moe_config_t& c) {
   L.u_norm = take(c.input_norm ? static_cast<size_t>(c.T) * c.d_model * ds : 0);
   L.b = take(c.post_norm ? static_cast<size_t>(c.T) * c.d_model * ds : 0);
   L.ss = take(c.expert_norm && c.dtype == MOE_BF16 ? TK * sumsq_parts(c) * 4 : 0);
-  // fp32 partials of the k-split latent projections (at most kMaxDenseSplits of them)
-  L.dp = take(c.d_latent > 0 && c.dtype == MOE_BF16 && c.T <= kMaxSplitRows
-                  ? static_cast<size_t>(kMaxDenseSplits) * c.T * std::max(c.d_latent, c.d_model) * 4
-                  : 0);
   L.total = o;
   return L;
 }
@@ -470,11 +465,11 @@ void pick_dense(int rows, int nout, Orient* o, int* bn) {
   *o = dense_orient(rows, *bn);
 }
 
-// Dense projections over at most 64 rows split their reduction: with S k-ranges the swapped GEMM
-// has Nout/128 * S tiles, each streaming 1/S of a weight tile, and the fp32 partials are added in
-// split order, by the CTAs of a cluster or by a second kernel (split_in_cluster), before the
-// epilogue.  S is the largest power of two up to kMaxDenseSplits whose tiles still fit on the SMs
-// at once and divides the k-blocks.
+// Dense projections over at most 64 rows split their reduction: with S k-ranges the swapped tiles
+// number Nout/128 * S, each streaming 1/S of a weight tile, and the S CTAs of a feature tile (one
+// thread-block cluster) add their fp32 partial tiles in split order in distributed shared memory
+// before the epilogue.  S is the largest power of two up to kMaxDenseSplits whose tiles still fit
+// on the SMs at once and divides the k-blocks.
 int dense_k_splits(int rows, int nout, int K) {
   if (rows > kMaxSplitRows || nout % 128 != 0) return 1;
   const long ft = nout / 128;
@@ -482,18 +477,6 @@ int dense_k_splits(int rows, int nout, int K) {
   int sp = 1;
   while (sp < kMaxDenseSplits && ft * sp * 2 <= device_info().sms && kb % (sp * 2) == 0) sp *= 2;
   return sp;
-}
-
-// The k-split finish kernel over rows x nout outputs.
-moe_status_t launch_dense_finish(const float* partial, int splits, long rows, int nout,
-                                 bool resgate, const void* resid, const float* g,
-                                 const moe_config_t& c, void* out, cudaStream_t st) {
-  const long nv = rows * nout / 8;
-  const long blocks = std::min<long>((nv + 255) / 256, static_cast<long>(std::max(device_info().sms, 1)) * 8);
-  launch_k(dense_split_finish_kernel, static_cast<unsigned>(blocks), 256, 0, st,
-      partial, splits, rows, nout, resgate ? 1 : 0, static_cast<const uint16_t*>(resid), g, c.tau,
-      c.resid_floor, c.resid_mode, static_cast<uint16_t*>(out));
-  return last_launch();
 }
 
 // Dense projection of at most kMaxSplitRows rows with its reduction split over clusters of
@@ -522,14 +505,6 @@ moe_status_t launch_gemm_splitk(const void* X, long x_rows, const void* W, long 
                    st, tx, tw, p);
   return last_launch();
 }
-
-// Which way a split dense projection adds its partial sums.  A cluster of two CTAs adds them in
-// distributed shared memory faster than a finish kernel does through global memory (latent up at
-// T=64: 0.028 against 0.032 ms per call); from four splits on, each CTA's sequential reads of its
-// peers' tiles cost more than the finish kernel, which spreads the sums over every SM (latent
-// down, four splits: 0.0276 against 0.0257 ms).  Calls without a workspace for the partials (the
-// standalone projections) always add them in the cluster.  Both give the same bits.
-bool split_in_cluster(int splits, const float* scratch) { return splits == 2 || scratch == nullptr; }
 
 // ------------------------------------------------------------------ steps
 
@@ -834,7 +809,7 @@ moe_status_t do_combine(const moe_config_t& c, const void* s, const int32_t* inv
 }
 
 moe_status_t do_latent_down(const moe_config_t& c, const void* u, const void* p_down, void* z,
-                            cudaStream_t st, float* split_scratch = nullptr) {
+                            cudaStream_t st) {
   if (c.T == 0) return MOE_OK;
   GemmParams p{};
   p.G = 1;
@@ -845,16 +820,7 @@ moe_status_t do_latent_down(const moe_config_t& c, const void* u, const void* p_
   p.out = z;
   dense_schedule(p, c.T);
   const int splits = dense_k_splits(c.T, c.d_latent, c.d_model);
-  if (splits > 1 && split_in_cluster(splits, split_scratch))
-    return launch_gemm_splitk<EPI_STORE>(u, c.T, p_down, c.d_latent, p, splits, st);
-  if (splits > 1) {
-    p.k_splits = splits;
-    p.partial = split_scratch;
-    moe_status_t s = run_gemm(EPI_PARTIAL, Orient::kSwap, 64, u, c.T, p_down, c.d_latent, p, st);
-    if (s != MOE_OK) return s;
-    return launch_dense_finish(split_scratch, splits, c.T, c.d_latent, false, nullptr, nullptr, c,
-                               z, st);
-  }
+  if (splits > 1) return launch_gemm_splitk<EPI_STORE>(u, c.T, p_down, c.d_latent, p, splits, st);
   Orient o;
   int bn;
   pick_dense(c.T, c.d_latent, &o, &bn);
@@ -863,8 +829,7 @@ moe_status_t do_latent_down(const moe_config_t& c, const void* u, const void* p_
 }
 
 moe_status_t do_latent_up(const moe_config_t& c, const void* y, const void* p_up, const void* r,
-                          const float* g, void* out, cudaStream_t st,
-                          float* split_scratch = nullptr) {
+                          const float* g, void* out, cudaStream_t st) {
   if (c.T == 0) return MOE_OK;
   GemmParams p{};
   p.G = 1;
@@ -880,15 +845,7 @@ moe_status_t do_latent_up(const moe_config_t& c, const void* y, const void* p_up
   p.resid_mode = c.resid_mode;
   dense_schedule(p, c.T);
   const int splits = dense_k_splits(c.T, c.d_model, c.d_latent);
-  if (splits > 1 && split_in_cluster(splits, split_scratch))
-    return launch_gemm_splitk<EPI_RESGATE>(y, c.T, p_up, c.d_model, p, splits, st);
-  if (splits > 1) {
-    p.k_splits = splits;
-    p.partial = split_scratch;
-    moe_status_t s = run_gemm(EPI_PARTIAL, Orient::kSwap, 64, y, c.T, p_up, c.d_model, p, st);
-    if (s != MOE_OK) return s;
-    return launch_dense_finish(split_scratch, splits, c.T, c.d_model, true, r, g, c, out, st);
-  }
+  if (splits > 1) return launch_gemm_splitk<EPI_RESGATE>(y, c.T, p_up, c.d_model, p, splits, st);
   Orient o;
   int bn;
   pick_dense(c.T, c.d_model, &o, &bn);
@@ -1300,14 +1257,10 @@ moe_status_t layer_forward_impl(const moe_config_t* cfg, const moe_weights_t* w,
                     at<float>(workspace, L.logits))) != MOE_OK)
     return s;
   prof_mark(st, 1);
-  // k-split partials of the latent projections (decode-sized batches; the region is empty
-  // otherwise and the projections do not split)
-  float* split = latent && c.dtype == MOE_BF16 && c.T <= kMaxSplitRows
-                     ? at<float>(workspace, L.dp) : nullptr;
   const void* xin = u;
   if (latent) {
     void* z = at<void>(workspace, L.z_raw);
-    if ((s = do_latent_down(c, u, w->p_down, z, st, split)) != MOE_OK) return s;
+    if ((s = do_latent_down(c, u, w->p_down, z, st)) != MOE_OK) return s;
     xin = z;
   }
   prof_mark(st, 2);
@@ -1334,13 +1287,13 @@ moe_status_t layer_forward_impl(const moe_config_t* cfg, const moe_weights_t* w,
   if (taps.t && (s = taps.copy(taps.t->y, y, static_cast<size_t>(c.T), c, st)) != MOE_OK) return s;
   prof_mark(st, 6);
   if (latent && !c.post_norm &&
-      (s = do_latent_up(c, y, w->p_up, r, w->resid_g, out, st, split)) != MOE_OK)
+      (s = do_latent_up(c, y, w->p_up, r, w->resid_g, out, st)) != MOE_OK)
     return s;
   if (c.post_norm) {  // b to the workspace, then output norm + residual gate per row
     moe_config_t plain = c;
     plain.resid_mode = MOE_RESID_NONE;
     void* b = at<void>(workspace, L.b);
-    if ((s = do_latent_up(plain, y, w->p_up, nullptr, nullptr, b, st, split)) != MOE_OK) return s;
+    if ((s = do_latent_up(plain, y, w->p_up, nullptr, nullptr, b, st)) != MOE_OK) return s;
     if ((s = do_resid_update(c, b, r, w->gamma_post, w->resid_g, out, st)) != MOE_OK) return s;
   }
   prof_mark(st, 7);
