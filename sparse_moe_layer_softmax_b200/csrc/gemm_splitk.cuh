@@ -203,8 +203,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       if (++stage == kSplitStages) { stage = 0; phase ^= 1; }
     }
     // Arrives when every MMA issued above has finished (and with them every operand load the
-    // producer issued, each of which an MMA waited for), so the ring may be overwritten.
+    // producer issued, each of which an MMA waited for), so the ring may be overwritten; the
+    // issuer waits for it too, so no MMA is in flight when TMEM is released.
     tc_commit(tfull);
+    mbar_wait(tfull, 0);
   } else if (warp >= 2) {
     // ------------------------------------------------------------ partial tile to shared memory
     const int q = warp & 3;  // TMEM lane quarter: features 32q .. 32q + 31
