@@ -122,7 +122,20 @@ __global__ void __launch_bounds__(32)
       if (i < cnt) s_idx[i] = v[j];
     }
   }
-  for (int e = lane; e < n; e += 32) s_next[e] = offsets[e] + chunk_base[blockIdx.x * n + e];
+  {
+    // every lane's offset and chunk-base loads in flight together (a loop of load-then-store
+    // waited on each pair in turn)
+    int ov[kMaxExperts / 32], cv[kMaxExperts / 32];
+#pragma unroll
+    for (int j = 0; j < kMaxExperts / 32; ++j) {
+      const int e = lane + 32 * j;
+      ov[j] = e < n ? offsets[e] : 0;
+      cv[j] = e < n ? chunk_base[blockIdx.x * n + e] : 0;
+    }
+#pragma unroll
+    for (int j = 0; j < kMaxExperts / 32; ++j)
+      if (lane + 32 * j < n) s_next[lane + 32 * j] = ov[j] + cv[j];
+  }
   __syncwarp();
   const unsigned lower = (1u << lane) - 1u;
   for (int w0 = 0; w0 < cnt; w0 += 32) {
