@@ -364,14 +364,22 @@ Workspace layout(const moe_config_t& c) {
 template <typename T>
 T* at(void* base, size_t off) { return reinterpret_cast<T*>(static_cast<char*>(base) + off); }
 
-// Tuning knob: MOE_GEMM_PAIR=1 in the environment selects CTA-pair 256-row tiles for large groups
-// and dense projections (same values as the 1-SM tiles).  Off by default: on this power-capped
-// part the pair kernel keeps the tensor pipe busier per clock but runs at lower clocks and reads
-// more DRAM, and its steps measured slower than the 1-SM 128 x 256 tiles.
-bool pair_tiles_enabled() {
+// CTA-pair 256-row tiles (same values as the 1-SM tiles).  For expert groups they are off by
+// default: groups are ragged, a group's last 256-row tile is mostly padding, and under the power
+// cap those steps measured slower than the 1-SM 128 x 256 tiles.  Dense projections over at least
+// kDensePairMinRows rows have no such tails, and there the pair tiles read a third fewer operand
+// bytes per MMA from L2: at prefill latent down took 0.89-0.92 against 0.96-0.98 ms and latent up
+// 0.91-0.94 against 1.02-1.04 ms, with the same bits.  Tuning knob: MOE_GEMM_PAIR=1 in the
+// environment also puts large expert groups and dense projections from 256 rows on the pair
+// tiles; MOE_GEMM_PAIR=0 puts nothing on them.
+constexpr long kDensePairMinRows = 2048;
+int pair_tiles_knob() {  // 1: on everywhere, 0: off everywhere, -1: default
   const char* v = getenv("MOE_GEMM_PAIR");
-  return v && v[0] == '1';
+  if (v && v[0] == '1') return 1;
+  if (v && v[0] == '0') return 0;
+  return -1;
 }
+bool pair_tiles_enabled() { return pair_tiles_knob() == 1; }
 
 // Grouped-GEMM orientation for the experts from the mean rows per expert.
 int expert_in_width(const moe_config_t& c) { return c.d_latent > 0 ? c.d_latent : c.d_model; }
@@ -428,7 +436,6 @@ void pick_expert_orient(const moe_config_t& c, int nout, bool dual, bool down, O
   }
 }
 
-// Dense projections: CTA-pair tiles for at least 256 rows and a 256-wide feature tile.
 // Partial sums of squares per expert-output row that the expert down GEMM writes (row_sumsq):
 // one per 256/128/64-column feature tile in the normal (and CTA-pair) orientation, one per CTA's
 // 128 features in the swapped CTA-pair orientation, one per 32-feature warp slice of each
@@ -442,8 +449,13 @@ int sumsq_parts(const moe_config_t& c) {
   return o == Orient::kSwap ? expert_in_width(c) / 128 * 4 : expert_in_width(c) / bn;
 }
 
+// Dense projections: CTA-pair tiles for a 256-wide feature tile over at least kDensePairMinRows
+// rows (from 256 rows with MOE_GEMM_PAIR=1).
 Orient dense_orient(int rows, int bn) {
-  return (pair_tiles_enabled() && bn == 256 && rows >= 256) ? Orient::kPair : Orient::kNormal;
+  if (bn != 256) return Orient::kNormal;
+  const int knob = pair_tiles_knob();
+  if (knob == 1) return rows >= 256 ? Orient::kPair : Orient::kNormal;
+  return (knob == -1 && rows >= kDensePairMinRows) ? Orient::kPair : Orient::kNormal;
 }
 
 // Dense projection (latent down / up) over `rows` activation rows into `nout` features.  Up to

@@ -140,6 +140,22 @@ def test_layer_at_switch_points(cfg):
     _check_layer(cfg)
 
 
+def test_dense_pair_tiles_at_prefill_size(monkeypatch):
+    """From 2048 rows the latent projections run on CTA-pair 256-row tiles by default: the layer
+    matches the oracle, and gives the same bits as with every GEMM on the 1-SM tiles
+    (MOE_GEMM_PAIR=0)."""
+    import torch
+    raw = configs.small_muse(T=2304, d=512, L=256, I=128, n=16, k=4, seed=310)
+    _check_layer(raw)
+    cfg = separate(raw)
+    dev = moe_inputs.device_inputs(cfg)
+    a = run_layer(cfg, dev, want_logits=False)["out"]
+    monkeypatch.setenv("MOE_GEMM_PAIR", "0")
+    b = run_layer(cfg, dev, want_logits=False)["out"]
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(a.view(torch.int16).cpu().numpy(), b.view(torch.int16).cpu().numpy())
+
+
 def test_layer_empty_batch():
     """T = 0: the forward launches nothing that touches the (empty) buffers and reports success."""
     import torch
